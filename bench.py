@@ -1,0 +1,514 @@
+#!/usr/bin/env python3
+"""Decode throughput of one DeepSeek-V4 CSA + HCA attention layer pair at a
+1,048,576-token context (default workload: 16 sequences), on B200.
+
+A step is one decode token per sequence through both layers, every stage
+included: pooling of the group that closes at this token (CSA m = 4 and HCA
+m = 128), the window-ring write, FP4 indexer scoring, exact top-1024,
+sparse attention over 1024 entries + 128 window rows + sink (CSA), and
+dense attention over 8192 entries + window + sink (HCA).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl lcsc|reference]
+
+Prints ONE JSON line on rank 0.  Multi-GPU (torchrun): every rank runs its
+own sequences (weak scaling, no data-path collective); the timed region is
+bracketed by a barrier and synchronisation, and the time is the max over
+ranks.  ``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from long_context_sparse_compress_b200 import lib as L  # noqa: E402
+from long_context_sparse_compress_b200 import synth, workloads  # noqa: E402
+
+METRIC = "CSA/HCA decode queries/s at 128K-1M ctx; % HBM roofline; prefill % tensor peak"
+DEFAULT_WORKLOAD = workloads.PAIR_DECODE_1M_B16.name
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        d["source"] = "measured"
+        return d
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS)
+
+
+# --------------------------------------------------------------- inputs
+
+class Layer:
+    """Device state of one layer for B sequences: caches filled with seeded
+    synthetic entries (the recipe of ``synth``, drawn on the device), the
+    window ring, raw tail rows, queries and gates."""
+
+    def __init__(self, wl, seed, device):
+        self.wl, self.dev = wl, device
+        g = torch.Generator(device=device)
+        g.manual_seed(seed)
+        B, T, D, m = wl.B, wl.T, wl.D, wl.m
+        self.p = L.params(wl)
+        rope = wl.rope_dim if wl.kv_fmt == "kv" else 0
+        xdt = torch.bfloat16 if wl.x_dtype == "bf16" else torch.float32
+        qdt = torch.bfloat16 if wl.q_dtype == "bf16" else torch.float32
+        rn = lambda shape, std: torch.randn(shape, generator=g, device=device) * std
+        self.n_max = wl.L // m
+        n_cap = self.n_max + 1
+        n_old = (wl.L - T) // m
+        csa = wl.kind == "csa"
+        self.q = rn((B, T, wl.H, D), D ** -0.5).to(qdt)
+        self.q_idx = rn((B, T, wl.H_I, wl.d_I), wl.d_I ** -0.5).to(qdt) if csa else None
+        self.w_idx = (rn((B, T, wl.H_I), 1.0).abs() * wl.H_I ** -0.5) if csa else None
+        self.sink = rn((wl.H,), 1.0)
+        self.w_kv = rn((D, D), 0.02).to(xdt)
+        self.b_kv = rn((wl.G, D), 1.0)
+        self.w_ik = rn((wl.d_I, wl.d_I), 0.02).to(xdt) if csa else None
+        self.b_ik = rn((wl.G, wl.d_I), 1.0) if csa else None
+        self.kv = L.DeviceCache(B, n_cap, wl.kv_fmt, D, rope, device)
+        self.idx = L.DeviceCache(B, n_cap, wl.idx_fmt, wl.d_I, 0, device) if csa else None
+        self.win = L.DeviceCache(B, wl.win_cap, wl.kv_fmt, D, rope, device)
+        R = synth.tail_rows(wl)
+        tail_kv = rn((B, R, D), D ** -0.5).to(xdt)
+        tail_ik = rn((B, R, wl.d_I), wl.d_I ** -0.5).to(xdt) if csa else None
+        self.x_kv = tail_kv[:, R - (T + wl.G - 1):].contiguous()
+        self.x_ik = tail_ik[:, R - (T + wl.G - 1):].contiguous() if csa else None
+        self.planted = []
+        for b in range(B):
+            u_kv = self.q[b].float().mean(dim=(0, 1))
+            u_kv = u_kv / u_kv.norm()
+            vals = rn((n_old, D), D ** -0.5)
+            n_pl = min(wl.n_planted, n_old)
+            pl = None
+            if n_pl:
+                n_lim = max(n_pl, min(n_old, (wl.L - T - wl.w) // m))
+                pl = torch.randperm(n_lim, generator=g, device=device)[:n_pl]
+                vals[pl] = u_kv[None] + rn((n_pl, D), 0.1 * D ** -0.5)
+            L.encode_rows(self.p, "kv", vals[None].contiguous(), 0, self.kv.seq(b))
+            del vals
+            if csa:
+                v = (self.w_idx[b][..., None] * self.q_idx[b].float()).sum(dim=1).mean(dim=0)
+                v = v / v.norm()
+                ik = rn((n_old, wl.d_I), wl.d_I ** -0.5)
+                if pl is not None:
+                    ik[pl] = v[None] + rn((n_pl, wl.d_I), 0.1 * wl.d_I ** -0.5)
+                L.encode_rows(self.p, "idx", ik[None].contiguous(), 0, self.idx.seq(b))
+                del ik
+            self.planted.append(pl)
+            # the window ring: raw rows of positions L - T - w + 1 .. L - T - 1
+            ring = torch.zeros((wl.win_cap, D), device=device)
+            for pos in range(max(0, wl.L - T - wl.w + 1), wl.L - T):
+                ring[pos % wl.win_cap] = tail_kv[b, pos - (wl.L - R)].float()
+            L.encode_rows(self.p, "kv", ring[None].contiguous(), 0, self.win.seq(b))
+        self.ctx_len = torch.full((B,), wl.L, dtype=torch.int32, device=device)
+        self.out = torch.empty((B, T, wl.H, wl.Dv), dtype=qdt, device=device)
+        self.lse = torch.empty((B, T, wl.H), dtype=torch.float32, device=device)
+        self.sel = torch.empty((B, T, wl.k), dtype=torch.int32, device=device) if csa else None
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.ws = L.workspace(L.step_workspace(self.p, csa, B, T, self.n_max), device)
+        self.step = L.make_step(B, T, self.n_max, self.ctx_len, self.x_kv, None, self.x_ik, self.w_kv,
+                                self.b_kv, None, None, self.w_ik, self.b_ik, self.kv, None, self.idx,
+                                self.win, None, self.q, self.q_idx, self.w_idx, self.sink, self.out,
+                                self.lse, self.sel, None)
+        self._ev_arr = None
+
+    def set_events(self, events):
+        self._ev_arr = L.set_step_events(self.step, events)
+
+    def clear_events(self):
+        self.step.events = None
+        self.step.n_events = 0
+        self._ev_arr = None
+
+    def run(self, stream=None):
+        L.decode_step(self.p, self.step, self.wl.kind == "csa", self.ws, self.status, stream)
+
+    # host-side copies for the end-to-end measurement
+    def host_inputs(self):
+        ts = [self.x_kv, self.q, self.ctx_len] + ([self.x_ik, self.q_idx, self.w_idx]
+                                                   if self.wl.kind == "csa" else [])
+        return [(t, t.cpu().pin_memory()) for t in ts]
+
+    def host_output(self):
+        return self.out, torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+
+
+def kernels_per_step(wl):
+    """Kernels of this library one step launches (memsets excluded):
+    CSA: pool + store for the KV latent and for the indexer keys (4), query
+    quantisation + scoring (2), three top-k passes (3), attention partial +
+    combine (2); HCA: pool + store (2), attention partial + combine (2)."""
+    if wl.kind == "pair":
+        return 11 + 4
+    return 11 if wl.kind == "csa" else 4
+
+
+# ------------------------------------------------------------ measurement
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples of one GPU while it runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.samples, self.proc = [], None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.target = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.target = str(device_index)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.target, "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self, t0, t1):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        self.proc.wait()
+        self.thread.join(timeout=2)
+        rows = [s for t, s in self.samples if t0 <= t <= t1] or [s for _, s in self.samples]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def source_sha(*names):
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "long_context_sparse_compress_b200", "csrc", n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload, sha):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path))[kernel]
+    except (OSError, ValueError, KeyError):
+        return None
+    if rec.get("source_sha") != sha or rec.get("workload") != workload:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws == 1:
+        return 1, 0, 0
+    import datetime
+    import torch.distributed as dist
+    rank, local = int(os.environ["RANK"]), int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(ws, x):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_lcsc(args):
+    ws, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    L.load()
+    wl = workloads.ALL[args.workload]
+    layers_wl = [wl.layer("csa"), wl.layer("hca")] if wl.kind == "pair" else [wl]
+    layers = [Layer(lw, synth.SEED + 1000 * rank + i, dev) for i, lw in enumerate(layers_wl)]
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for ly in layers:
+            ly.run(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    for ly in layers:
+        if int(ly.status.item()) != 0:
+            raise RuntimeError(f"device status {int(ly.status.item())} in {ly.wl.name}")
+
+    # ---- timed region: K steps, inputs resident in HBM (working set > L2)
+    csa = layers[0] if layers[0].wl.kind == "csa" else None
+    n_ev = 5
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    for evs in events:
+        for e in evs:
+            e.record(stream)  # creates the events
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        if csa is not None:
+            csa.set_events(events[i])
+        step()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    t1 = time.time()
+    time.sleep(0.25)
+    clocks = sampler.stop(t0, t1)
+    if csa is not None:
+        csa.clear_events()
+    ms_total = max_over_ranks(ws, start.elapsed_time(stop))
+    ms_step = ms_total / args.steps
+    queries = wl.B * wl.T * ws * args.steps
+    value = queries / (ms_total / 1e3)
+
+    # ---- dominant kernel: the CSA indexer scoring (events 1 -> 2 of each step)
+    roof = None
+    if csa is not None:
+        score_ms = float(np.mean([evs[1].elapsed_time(evs[2]) for evs in events]))
+        stage_ms = {name: float(np.mean([evs[a].elapsed_time(evs[b]) for evs in events]))
+                    for name, a, b in (("compress", 0, 1), ("index_score", 1, 2), ("topk", 2, 3),
+                                       ("sparse_attn", 3, 4))}
+        cw = csa.wl
+        key_b = L.row_bytes(cw.idx_fmt, cw.d_I) + (cw.d_I // 16 if cw.idx_fmt == "fp4" else 4)
+        n_keys = cw.B * cw.n_entries()
+        q_b = cw.B * cw.T * cw.H_I * (cw.d_I * 2 + 4)
+        alg_bytes = n_keys * (key_b + 4) + q_b  # keys read + scores written + queries
+        peaks = measured_peaks()
+        peak = float(peaks["hbm_gbs"])
+        achieved = alg_bytes / (score_ms / 1e3) / 1e9
+        sha = source_sha("indexer.cu", "common.cuh")
+        traffic = recorded_traffic("score_kernel", wl.name, sha)
+        roof = {"bound": "hbm", "kernel": "indexer score_kernel", "achieved": round(achieved, 1),
+                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                "traffic": traffic, "algorithmic_bytes": alg_bytes, "ms_per_launch": round(score_ms, 4),
+                "peak_source": peaks["source"] + " hbm_gbs",
+                "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()}}
+
+    # ---- end to end: pinned host inputs -> device, step, output -> host
+    e2e = None
+    if args.e2e_steps > 0:
+        pairs = [p for ly in layers for p in ly.host_inputs()]
+        outs = [ly.host_output() for ly in layers]
+        h2d = sum(h.numel() * h.element_size() for _, h in pairs)
+        d2h = sum(h.numel() * h.element_size() for _, h in outs)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(ws)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for d, h in pairs:
+                d.copy_(h, non_blocking=True)
+            step()
+            for d, h in outs:
+                h.copy_(d, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(ws, e0.elapsed_time(e1))
+        e2e = {"value": round(wl.B * wl.T * ws * args.e2e_steps / (e2e_ms / 1e3), 2), "unit": "queries/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "queries/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 (indexer codes e2m1/e4m3, KV e4m3+bf16, dequantised to f32)",
+        "data": "synthetic (seeded Gaussian entries with planted relevant blocks, drawn on device)",
+        "config": {"workload": wl.name, "layers": [lw.name for lw in layers_wl], "batch_per_gpu": wl.B,
+                   "context": wl.L, "heads": wl.H, "kv_dim": wl.D, "top_k": wl.k, "window": wl.w,
+                   "csa_entries": wl.L // wl.m, "hca_entries": wl.L // wl.m_hca if wl.kind == "pair" else None,
+                   "l2": "inputs larger than L2 (working set per step > 126 MB)"},
+        "roofline": roof, "e2e": e2e, "gpu_launches": kernels_per_step(wl) * args.steps, "clocks": clocks,
+    }
+    if args.cpu_baseline and ws == 1:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_queries)
+    return line
+
+
+# ------------------------------------------------------- CPU oracle legs
+
+def oracle_sequence(wl_layer, b, seed):
+    """Oracle state of one sequence (test-infrastructure oracle, CPU)."""
+    from oracle import storage
+    P = synth.layer_params(wl_layer, seed)
+    inp = synth.sequence_inputs(wl_layer, b, seed)
+    n_cap = wl_layer.L // wl_layer.m + 1
+    rope = wl_layer.rope_dim if wl_layer.kv_fmt == "kv" else 0
+
+    def stored(vals, fmt, r):
+        st = storage.encode(fmt, vals, r)
+        pay = np.zeros((n_cap,) + st.payload.shape[1:], st.payload.dtype)
+        pay[:vals.shape[0]] = st.payload
+        sc = None
+        if st.scale is not None:
+            sc = np.zeros((n_cap,) + st.scale.shape[1:], st.scale.dtype)
+            sc[:vals.shape[0]] = st.scale
+        return storage.Stored(fmt, pay, sc, vals.shape[1], r)
+
+    kv = stored(inp.pop("e_kv"), wl_layer.kv_fmt, rope)
+    idx = stored(inp.pop("e_idx"), wl_layer.idx_fmt, 0) if wl_layer.kind == "csa" else None
+    cap = wl_layer.win_cap
+    R = synth.tail_rows(wl_layer)
+    ring = storage.encode(wl_layer.kv_fmt, np.zeros((cap, wl_layer.D), np.float32), rope)
+    for pos in range(max(0, wl_layer.L - wl_layer.T - wl_layer.w + 1), wl_layer.L - wl_layer.T):
+        one = storage.encode(wl_layer.kv_fmt, inp["x_kv"][pos - (wl_layer.L - R)][None], rope)
+        ring.payload[pos % cap] = one.payload[0]
+        if ring.scale is not None:
+            ring.scale[pos % cap] = one.scale[0]
+    return P, inp, kv, idx, ring
+
+
+def oracle_step(wl_layer, P, inp, kv, idx, ring):
+    from oracle.step import layer_step
+    w = wl_layer
+    tail = lambda a: None if a is None else a[a.shape[0] - (w.T + w.G - 1):]
+    return layer_step(w.kind, m=w.m, G=w.G, w=w.w, k=w.k, sm_scale=w.sm_scale, kv_fmt=w.kv_fmt,
+                      rope_dim=w.rope_dim, idx_fmt=w.idx_fmt, L=w.L, T=w.T, kv=kv, v=None, idx=idx,
+                      ring_kv=ring, ring_v=None, x_kv=tail(inp["x_kv"]), x_v=None,
+                      x_idx=tail(inp.get("x_idx")), W_kv=P["W_kv"], B_kv=P["B_kv"], W_v=None, B_v=None,
+                      W_idx=P.get("W_idx"), B_idx=P.get("B_idx"), q=inp["q"], q_idx=inp.get("q_idx"),
+                      w_idx=inp.get("w_idx"), sink=P["sink"])
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, n_queries):
+    """The oracle, as it stands, on a bounded sample: ``n_queries`` decode
+    queries of sequence 0 through every layer of the workload."""
+    layers_wl = [wl.layer("csa"), wl.layer("hca")] if wl.kind == "pair" else [wl]
+    states = [oracle_sequence(lw.with_(B=1), 0, synth.SEED) for lw in layers_wl]
+    t0 = time.perf_counter()
+    for _ in range(n_queries):
+        for lw, st in zip(layers_wl, states):
+            oracle_step(lw.with_(B=1), *st)
+    dt = time.perf_counter() - t0
+    return {"value": round(n_queries * wl.T / dt, 5), "unit": "queries/s", "cores": blas_threads(),
+            "kind": "oracle", "cpu": _cpu_model(),
+            "sample": f"{n_queries} decode step(s) of 1 sequence (T={wl.T}) through "
+                      f"{'+'.join(x.name for x in layers_wl)}, full context, fp64 numpy oracle"}
+
+
+def _cpu_model():
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def run_reference(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    wl = workloads.ALL[args.workload]
+    layers_wl = [wl.layer("csa"), wl.layer("hca")] if wl.kind == "pair" else [wl]
+    states = [oracle_sequence(lw.with_(B=1), 0, synth.SEED) for lw in layers_wl]
+    for _ in range(args.warmup):
+        for lw, st in zip(layers_wl, states):
+            oracle_step(lw.with_(B=1), *st)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for lw, st in zip(layers_wl, states):
+            oracle_step(lw.with_(B=1), *st)
+    dt = time.perf_counter() - t0
+    value = args.steps * wl.T / dt
+    sample = (f"each step: 1 decode query of 1 sequence (of {wl.B}) through "
+              f"{'+'.join(x.name for x in layers_wl)} at full context")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "queries/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, numpy generator)",
+        "config": {"workload": wl.name, "layers": [lw.name for lw in layers_wl], "context": wl.L},
+        "cpu_baseline": {"value": round(value, 5), "unit": "queries/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 5), "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.ALL))
+    ap.add_argument("--impl", default="lcsc", choices=["lcsc", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-queries", type=int, default=2)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
+    line = run_reference(args) if args.impl == "reference" else run_lcsc(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1 and args.impl != "reference":
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,268 @@
+/*
+ * lcsc.h -- C ABI of the B200 (sm_100a) compressed sparse attention library.
+ *
+ * One attention layer of DeepSeek-V4's hybrid compressed attention:
+ *   CSA: groups of m = 4 tokens are pooled into compressed entries, a
+ *        low-precision lightning indexer scores every entry, and exact
+ *        attention runs over the top-k entries, a sliding window of raw
+ *        tokens and a per-head attention sink.
+ *   HCA: groups of m = 128 tokens are pooled and attended densely, with
+ *        the same window and sink.
+ * Sources: "DeepSeek V4 Architecture Explained" (researchpapers.dev), section
+ * "How compress-then-sparsify attention works" and its Key numbers table;
+ * "Inside DeepSeek-V4" (llmbytes.dev), sections 1 and 2; "How DeepSeek V4
+ * Handles 1M Token Context" (docs.bswen.com), Components 2 and 3.
+ *
+ * Conventions for every call
+ *  - Pointers marked (dev) are device pointers owned by the caller; the
+ *    library never allocates device memory and keeps no state between
+ *    calls.  Pointers marked (host) are read before the call returns.
+ *  - Every call enqueues its kernels on `stream` (a cudaStream_t) and
+ *    returns without synchronising.
+ *  - On a non-zero return nothing has been enqueued.
+ *  - Data-dependent anomalies found on the device (an index in `idx` that
+ *    is out of range, a window ring too small for the query positions) never
+ *    trap: the offending row is skipped and a bit is OR-ed into `*status`
+ *    (dev, nullable, int32): LCSC_DEV_BAD_INDEX, LCSC_DEV_BAD_LENGTH.
+ *  - Batched arrays are dense: sequence b of a [B][n][...] array starts at
+ *    b * n * (row bytes).  Every pointer must be 16-byte aligned.
+ *  - Sequence lengths: `ctx_len` (dev, int32 [B]) gives, per sequence, the
+ *    length L after the T new tokens of the step; the step's queries sit at
+ *    positions p = L - T + i, i < T.
+ *  - Entry g of a tensor pools the tokens [g*m + m - G, g*m + m) (positions
+ *    below 0 are left out); a query at position p sees the entries
+ *    g < N(p) = floor((p + 1) / m) and the raw window rows of positions
+ *    max(0, p - w + 1) .. p.
+ */
+#ifndef LCSC_H_
+#define LCSC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LCSC_ABI_VERSION 1
+
+/* Return codes. */
+#define LCSC_OK 0
+#define LCSC_ERR_INVALID_ARG 1     /* null / misaligned pointer, bad size or parameter */
+#define LCSC_ERR_UNSUPPORTED 2     /* a format / dimension combination that is not built */
+#define LCSC_ERR_CUDA 3            /* a launch failed; see lcsc_last_cuda_error() */
+#define LCSC_ERR_WORKSPACE 4       /* workspace smaller than the *_workspace_size() answer */
+
+/* Bits OR-ed into *status on the device. */
+#define LCSC_DEV_BAD_INDEX 1       /* an index outside [0, N(p)) was skipped */
+#define LCSC_DEV_BAD_LENGTH 2      /* a ctx_len smaller than T, or a window larger than the ring */
+
+/* Row storage formats ("DeepSeek V4 Architecture Explained", Key numbers,
+ * row "KV storage precision"; "Inside DeepSeek-V4", section 1, FP4 indexer).
+ *  LCSC_FMT_F32: dim float32 values.                         row = 4*dim bytes
+ *  LCSC_FMT_KV:  (dim - rope_dim) E4M3 values then rope_dim BF16 values;
+ *                E4M3 part scaled by one float32 per row:
+ *                s = amax / 448 (1 if amax = 0), code = E4M3_rne_sat(c / s).
+ *                                                            row = dim + rope_dim bytes
+ *  LCSC_FMT_FP8: dim E4M3 values, same per-row float32 scale rule.  row = dim bytes
+ *  LCSC_FMT_FP4: dim E2M1 values, element 2i in the low nibble of byte i;
+ *                one E4M3 scale byte per 16 values: b = amax / 6,
+ *                scale = E4M3_rne_sat(b), code = E2M1_rne_sat(c / scale)
+ *                (all-zero codes when the scale byte decodes to 0).
+ *                                                            row = dim / 2 bytes
+ * All encode decisions are taken in float32 with IEEE division. */
+#define LCSC_FMT_F32 0
+#define LCSC_FMT_KV 1
+#define LCSC_FMT_FP8 2
+#define LCSC_FMT_FP4 3
+
+/* Element types of raw rows, gate weights, queries and outputs. */
+#define LCSC_DT_F32 0
+#define LCSC_DT_BF16 1
+
+/* Which compressed tensor a compress / encode call writes. */
+#define LCSC_TENSOR_KV 0    /* the shared KV latent (or K when V is separate) */
+#define LCSC_TENSOR_V 1     /* a separate V */
+#define LCSC_TENSOR_IDX 2   /* the indexer keys (CSA only) */
+
+/* Layer parameters.  The pages fix m, k and w ("Inside DeepSeek-V4",
+ * sections 1-2); the rest are this library's readings, kept as parameters. */
+typedef struct lcsc_params {
+  int32_t m;           /* compression ratio = entry stride: 4 (CSA), 128 (HCA) */
+  int32_t group_len;   /* G, tokens pooled per entry: m, or 2m (overlapping groups) */
+  int32_t window;      /* w, sliding-window length (raw tokens, query included) */
+  int32_t top_k;       /* k, entries kept per query (CSA; <= 2048) */
+  float sm_scale;      /* softmax scale of q.K (e.g. 1/sqrt(D)) */
+  int32_t n_heads;     /* H query heads, all attending to one shared KV */
+  int32_t head_dim;    /* D, query and key row length */
+  int32_t rope_dim;    /* trailing dims stored BF16 in LCSC_FMT_KV */
+  int32_t v_dim;       /* Dv: = D when V is the shared latent */
+  int32_t idx_heads;   /* H_I indexer heads */
+  int32_t idx_dim;     /* d_I indexer query / key length */
+  int32_t kv_format;   /* LCSC_FMT_F32 or LCSC_FMT_KV (entries, V and the window ring) */
+  int32_t idx_format;  /* LCSC_FMT_F32, LCSC_FMT_FP8 or LCSC_FMT_FP4 */
+  int32_t x_dtype;     /* LCSC_DT_*: raw token rows and gate weights W */
+  int32_t q_dtype;     /* LCSC_DT_*: queries, indexer queries and the output */
+} lcsc_params;
+
+/* Stored rows of one tensor for B sequences (dev pointers).
+ *   data:  [B][capacity][row bytes of the format]
+ *   scale: [B][capacity] float32 (KV, FP8) or [B][capacity][dim/16] uint8
+ *          (FP4); NULL for F32.
+ * Compressed entries use row g for entry g.  A window ring uses row
+ * (position mod capacity). */
+typedef struct lcsc_cache {
+  void* data;
+  void* scale;
+  int64_t capacity;
+} lcsc_cache;
+
+/* ---------------------------------------------------------------- misc */
+
+int32_t lcsc_abi_version(void);
+/* cudaError_t of the last LCSC_ERR_CUDA returned on this host thread. */
+int32_t lcsc_last_cuda_error(void);
+const char* lcsc_status_string(int32_t status);
+/* Bytes of one stored row for a format and dimension (0 if invalid). */
+int64_t lcsc_row_bytes(int32_t format, int32_t dim, int32_t rope_dim);
+
+/* ------------------------------------------------------- compression (a1, a2)
+ * lcsc_csa_compress / lcsc_hca_compress: softmax-gated pooling ("DeepSeek V4
+ * Architecture Explained", "How compress-then-sparsify attention works":
+ * trainable compression weights, a softmax over the group, learnable
+ * positional biases).  For each entry g in [tok_begin/m, tok_end/m) and
+ * each channel c:
+ *     z_j[c] = sum_d x_j[d] W[d][c] + Bpos[j - (g*m + m - G)][c]
+ *     e_g[c] = sum_j softmax_j(z[c])_j * x_j[c]
+ * over the tokens j of the group; e_g is stored in the tensor's format.
+ *   tensor:   LCSC_TENSOR_KV, _V or _IDX (IDX only for CSA); fixes the row
+ *             length (D, Dv, d_I) and the format (kv_format / idx_format).
+ *   x (dev):  [B][n_x][dim] x_dtype raw rows of positions
+ *             tok_begin - (G - m) .. tok_end - 1, n_x = tok_end - tok_begin + G - m
+ *             (rows at negative positions are never read).
+ *   tok_begin % m == 0; every group that ends before tok_end is written.
+ *   w_gate (dev): [dim][dim] x_dtype.  b_pos (dev): [G][dim] float32.
+ *   entries: written rows; window (nullable): the window ring, which also
+ *   receives the raw rows of positions max(tok_begin, tok_end - capacity) ..
+ *   tok_end - 1 (KV / V only).
+ *   workspace: lcsc_compress_workspace_size() bytes (dev). */
+int32_t lcsc_compress_workspace_size(const lcsc_params* p, int64_t B, int64_t n_tokens,
+                                     size_t* bytes);
+int32_t lcsc_csa_compress(const lcsc_params* p, int32_t tensor, const void* x, int64_t B,
+                          int64_t tok_begin, int64_t tok_end, const void* w_gate,
+                          const float* b_pos, const lcsc_cache* entries, const lcsc_cache* window,
+                          void* workspace, size_t workspace_bytes, int32_t* status,
+                          void* stream);
+int32_t lcsc_hca_compress(const lcsc_params* p, int32_t tensor, const void* x, int64_t B,
+                          int64_t tok_begin, int64_t tok_end, const void* w_gate,
+                          const float* b_pos, const lcsc_cache* entries, const lcsc_cache* window,
+                          void* workspace, size_t workspace_bytes, int32_t* status,
+                          void* stream);
+
+/* Store already-pooled float32 rows in a tensor's format, no pooling:
+ * rows [B][n][dim] (dev, float32) go to rows row0 .. row0 + n - 1 of `out`.
+ * For building caches from precomputed entry values and for tests. */
+int32_t lcsc_encode_rows(const lcsc_params* p, int32_t tensor, const float* rows, int64_t B,
+                         int64_t n, int64_t row0, const lcsc_cache* out, void* stream);
+
+/* ---------------------------------------------------- indexer + top-k (a3, a4)
+ * Lightning indexer ("DeepSeek V4 Architecture Explained", same section;
+ * "How DeepSeek V4 Handles 1M Token Context", Component 3): every indexer
+ * query row (t, h) is stored in the key format (FP8: per-row scale; FP4:
+ * per-16 block scales; F32: as is), then for every visible entry g < N(p)
+ *     s[g] = sum_h w[h] * ReLU(q~[h] . k~[g])
+ * and the min(k, N(p)) entries with the largest s are kept.
+ *   q_idx (dev): [B][T][H_I][d_I] q_dtype;  w_idx (dev): [B][T][H_I] float32.
+ *   idx_keys: the stored indexer keys (idx_format, d_I).
+ *   out_idx (dev): [B][T][k] int32; the set is unordered; rows beyond
+ *   min(k, N(p)) are -1.  out_score (dev, nullable): [B][T][k] float32, the
+ *   score of each kept index (-inf in padded rows). */
+int32_t lcsc_index_topk_workspace_size(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max,
+                                       size_t* bytes);
+int32_t lcsc_csa_index_topk(const lcsc_params* p, const void* q_idx, const float* w_idx,
+                            const lcsc_cache* idx_keys, const int32_t* ctx_len, int64_t B,
+                            int64_t T, int64_t n_max, int32_t* out_idx, float* out_score,
+                            void* workspace, size_t workspace_bytes, int32_t* status,
+                            void* stream);
+
+/* --------------------------------------------------------- attention (a5-a7)
+ * One joint softmax per query head over a row set S (entries plus window
+ * rows), with a per-head sink logit sigma[h] that only adds exp(sigma) to
+ * the denominator ("an attention-sink term that lets a head's attention
+ * scores sum to less than one"):
+ *     l_j = sm_scale * q[h] . K_j
+ *     o[h] = sum_j e^{l_j - M} V_j / (e^{sigma[h] - M} + sum_j e^{l_j - M})
+ * K_j, V_j are dequantised stored rows; V = K unless `v` is given.
+ *   q (dev): [B][T][H][D] q_dtype.   out (dev): [B][T][H][Dv] q_dtype.
+ *   lse (dev, nullable): [B][T][H] float32 = M + log(denominator).
+ *   sink (dev, nullable): [H] float32; NULL means no sink.
+ *   kv, v (v nullable): stored entries; win_kv, win_v (win_v nullable): the
+ *   window rings, which must hold positions max(0, p - w + 1) .. p.
+ * lcsc_csa_sparse_attn: S = {idx[b][t][j] >= 0} U window (idx (dev):
+ *   [B][T][k] int32, e.g. from lcsc_csa_index_topk).
+ * lcsc_hca_dense_attn: S = {all g < N(p)} U window. */
+int32_t lcsc_attn_workspace_size(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max,
+                                 int32_t dense, size_t* bytes);
+int32_t lcsc_csa_sparse_attn(const lcsc_params* p, const void* q, const lcsc_cache* kv,
+                             const lcsc_cache* v, const lcsc_cache* win_kv,
+                             const lcsc_cache* win_v, const int32_t* idx, const float* sink,
+                             const int32_t* ctx_len, int64_t B, int64_t T, void* out, float* lse,
+                             void* workspace, size_t workspace_bytes, int32_t* status,
+                             void* stream);
+int32_t lcsc_hca_dense_attn(const lcsc_params* p, const void* q, const lcsc_cache* kv,
+                            const lcsc_cache* v, const lcsc_cache* win_kv, const lcsc_cache* win_v,
+                            const float* sink, const int32_t* ctx_len, int64_t B, int64_t T,
+                            int64_t n_max, void* out, float* lse, void* workspace,
+                            size_t workspace_bytes, int32_t* status, void* stream);
+
+/* ------------------------------------------------------------ fused steps
+ * One decode (T = 1) or chunked-prefill (T > 1) step of a layer: pool every
+ * group that closes inside the T new tokens (entries
+ * [floor((L - T) / m), floor(L / m))), store the T new raw rows in the
+ * window rings, then (CSA) score + select + attend, or (HCA) attend densely.
+ * Every sequence must have L >= T; raw rows x_* (dev) are
+ * [B][T + G - 1][dim] x_dtype for positions L - (T + G - 1) .. L - 1.
+ * The caches must already hold every entry below floor((L - T) / m) and the
+ * rings the rows of positions L - T - w + 1 .. L - T - 1; the rings need at
+ * least T + w - 1 rows. */
+typedef struct lcsc_step {
+  int64_t B, T;
+  int64_t n_max;                /* >= floor(L / m) for every sequence */
+  const int32_t* ctx_len;       /* [B] L after the step */
+  const void* x_kv;             /* raw rows of the KV latent (or K) */
+  const void* x_v;              /* raw rows of a separate V, or NULL */
+  const void* x_idx;            /* raw rows of the indexer keys (CSA) */
+  const void* w_kv;  const float* b_kv;    /* gates of each tensor: W [dim][dim], Bpos [G][dim] */
+  const void* w_v;   const float* b_v;
+  const void* w_idx; const float* b_idx;
+  lcsc_cache kv, v, idx_keys;   /* entries (v.data NULL when V = K) */
+  lcsc_cache win_kv, win_v;     /* window rings (win_v.data NULL when V = K) */
+  const void* q;                /* [B][T][H][D] */
+  const void* q_idx;            /* [B][T][H_I][d_I] (CSA) */
+  const float* w_heads;         /* [B][T][H_I] indexer head weights (CSA) */
+  const float* sink;            /* [H] or NULL */
+  void* out;                    /* [B][T][H][Dv] */
+  float* lse;                   /* [B][T][H] or NULL */
+  int32_t* out_idx;             /* [B][T][k] selected entries (CSA), or NULL */
+  float* out_score;             /* [B][T][k] their scores (CSA), or NULL */
+  /* Optional stage timing (host array of cudaEvent_t, or NULL): event i is
+   * recorded on `stream` at stage boundary i while i < n_events.
+   * CSA: 0 start, 1 after compression, 2 after indexer scoring, 3 after
+   * top-k, 4 after attention.  HCA: 0 start, 1 after compression, 2 after
+   * attention. */
+  void* const* events;
+  int32_t n_events;
+} lcsc_step;
+
+int32_t lcsc_step_workspace_size(const lcsc_params* p, int32_t csa, int64_t B, int64_t T,
+                                 int64_t n_max, size_t* bytes);
+int32_t lcsc_csa_decode(const lcsc_params* p, const lcsc_step* s, void* workspace,
+                        size_t workspace_bytes, int32_t* status, void* stream);
+int32_t lcsc_hca_decode(const lcsc_params* p, const lcsc_step* s, void* workspace,
+                        size_t workspace_bytes, int32_t* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LCSC_H_ */

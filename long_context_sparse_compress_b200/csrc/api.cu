@@ -1,0 +1,558 @@
+// The C ABI (include/lcsc.h): argument validation, workspace planning and
+// the launch sequence of every call.  No device memory is allocated here.
+#include <string.h>
+
+#include "kernels.cuh"
+
+namespace lcsc {
+namespace {
+
+thread_local int32_t g_last_cuda_error = 0;
+
+int32_t cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int32_t)e;
+  return LCSC_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Bump allocator over the caller's workspace.
+struct Carve {
+  uint8_t* base;
+  size_t used = 0;
+  template <class T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + used) : nullptr;
+    used += align_up(sizeof(T) * count);
+    return p;
+  }
+};
+
+bool valid_format(int fmt) { return fmt >= LCSC_FMT_F32 && fmt <= LCSC_FMT_FP4; }
+
+int32_t check_params(const lcsc_params* p) {
+  if (!p) return LCSC_ERR_INVALID_ARG;
+  if (p->m < 1 || p->group_len < p->m || p->group_len > 2 * p->m) return LCSC_ERR_INVALID_ARG;
+  if (p->window < 0 || p->top_k < 0 || p->top_k > 2048) return LCSC_ERR_INVALID_ARG;
+  if (p->n_heads < 1 || p->head_dim < 1 || p->v_dim < 1) return LCSC_ERR_INVALID_ARG;
+  if (p->rope_dim < 0 || p->rope_dim > p->head_dim) return LCSC_ERR_INVALID_ARG;
+  if (!valid_format(p->kv_format) || !valid_format(p->idx_format)) return LCSC_ERR_INVALID_ARG;
+  if (p->kv_format != LCSC_FMT_F32 && p->kv_format != LCSC_FMT_KV) return LCSC_ERR_INVALID_ARG;
+  if (p->idx_format == LCSC_FMT_KV) return LCSC_ERR_INVALID_ARG;
+  if (p->x_dtype != LCSC_DT_F32 && p->x_dtype != LCSC_DT_BF16) return LCSC_ERR_INVALID_ARG;
+  if (p->q_dtype != LCSC_DT_F32 && p->q_dtype != LCSC_DT_BF16) return LCSC_ERR_INVALID_ARG;
+  if (!(p->sm_scale == p->sm_scale)) return LCSC_ERR_INVALID_ARG;
+  return LCSC_OK;
+}
+
+// The (format, dim) pairs the kernels are built for.
+bool kv_supported(const lcsc_params* p) {
+  if (p->kv_format == LCSC_FMT_F32) return p->head_dim == 128 && p->v_dim == 128 && p->n_heads % 8 == 0;
+  return p->head_dim == 512 && p->v_dim == 512 && p->rope_dim % 16 == 0 && p->n_heads % 16 == 0;
+}
+
+bool idx_supported(const lcsc_params* p) {
+  if (p->idx_format == LCSC_FMT_F32) return p->idx_dim == 32 && p->idx_heads == 4;
+  return (p->idx_format == LCSC_FMT_FP8 || p->idx_format == LCSC_FMT_FP4) && p->idx_dim == 128 &&
+         p->idx_heads == 64;
+}
+
+int32_t tensor_fmt(const lcsc_params* p, int32_t tensor, RowFmt* f) {
+  switch (tensor) {
+    case LCSC_TENSOR_KV: *f = {p->kv_format, p->head_dim, p->rope_dim, 0}; break;
+    case LCSC_TENSOR_V: *f = {p->kv_format, p->v_dim, p->rope_dim, 0}; break;
+    case LCSC_TENSOR_IDX: *f = {p->idx_format, p->idx_dim, 0, 0}; break;
+    default: return LCSC_ERR_INVALID_ARG;
+  }
+  if (f->fmt != LCSC_FMT_KV) f->rope = 0;
+  f->row_bytes = row_bytes_of(f->fmt, f->dim, f->rope);
+  if (f->dim != 32 && f->dim != 128 && f->dim != 512) return LCSC_ERR_UNSUPPORTED;
+  if (f->fmt == LCSC_FMT_KV && ((f->dim - f->rope) % (f->dim / 32) != 0)) return LCSC_ERR_UNSUPPORTED;
+  if (f->fmt == LCSC_FMT_FP4 && f->dim % 16 != 0) return LCSC_ERR_UNSUPPORTED;
+  return LCSC_OK;
+}
+
+int32_t make_view(const lcsc_cache* c, const RowFmt& f, bool need_scale, CacheView* v) {
+  if (!c || !c->data || c->capacity < 1 || !aligned16(c->data)) return LCSC_ERR_INVALID_ARG;
+  if (need_scale && (!c->scale || ((uintptr_t)c->scale & 3u))) return LCSC_ERR_INVALID_ARG;
+  v->data = reinterpret_cast<uint8_t*>(c->data);
+  v->scale = c->scale;
+  v->capacity = c->capacity;
+  v->f = f;
+  return LCSC_OK;
+}
+
+bool needs_scale(int fmt) { return fmt != LCSC_FMT_F32; }
+
+// ---------------------------------------------------------- workspace plans
+
+void plan_index(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max, Carve& cv,
+                IndexLaunch* L) {
+  const int64_t lists = B * T;
+  const int64_t qrows = lists * p->idx_heads;
+  const int rb = row_bytes_of(p->idx_format, p->idx_dim, 0);
+  uint8_t* qdata = cv.take<uint8_t>((size_t)qrows * rb);
+  void* qscale = nullptr;
+  if (p->idx_format == LCSC_FMT_FP8) qscale = cv.take<float>((size_t)qrows);
+  else if (p->idx_format == LCSC_FMT_FP4) qscale = cv.take<uint8_t>((size_t)qrows * (p->idx_dim / 16));
+  float* scores = cv.take<float>((size_t)lists * n_max);
+  uint32_t* hist = cv.take<uint32_t>((size_t)lists * 2 * 4096);
+  uint32_t* ctr = cv.take<uint32_t>((size_t)lists * 4);
+  uint32_t* cand = cv.take<uint32_t>((size_t)lists * n_max);
+  if (L) {
+    L->q_store.data = qdata;
+    L->q_store.scale = qscale;
+    L->q_store.capacity = T * p->idx_heads;
+    L->q_store.f = {p->idx_format, p->idx_dim, 0, rb};
+    L->scores = scores;
+    L->hist = hist;
+    L->counters = ctr;
+    L->cand = cand;
+  }
+}
+
+void plan_attn(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max, bool dense, Carve& cv,
+               AttnLaunch* L) {
+  const int64_t max_rows = (dense ? n_max : p->top_k) + p->window;
+  const int hpc = p->kv_format == LCSC_FMT_F32 ? 8 : 16;
+  int splits, rps;
+  attention_splits(max_rows, B * T * (p->n_heads / hpc), &splits, &rps);
+  float* po = cv.take<float>((size_t)B * T * splits * p->n_heads * p->v_dim);
+  float* pml = cv.take<float>((size_t)B * T * splits * p->n_heads * 2);
+  if (L) {
+    L->splits = splits;
+    L->rows_per_split = rps;
+    L->part_o = po;
+    L->part_ml = pml;
+  }
+}
+
+
+// Max entries one call pools per sequence.
+int64_t new_entries_max(int64_t T, int m) { return T / m + 1; }
+
+void plan_compress(const lcsc_params* p, int64_t B, int64_t n_new, int dim, Carve& cv, float** pooled) {
+  float* pl = cv.take<float>((size_t)B * (n_new > 0 ? n_new : 1) * dim);
+  if (pooled) *pooled = pl;
+}
+
+}  // namespace
+}  // namespace lcsc
+
+using namespace lcsc;
+
+extern "C" {
+
+int32_t lcsc_abi_version(void) { return LCSC_ABI_VERSION; }
+
+int32_t lcsc_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* lcsc_status_string(int32_t s) {
+  switch (s) {
+    case LCSC_OK: return "ok";
+    case LCSC_ERR_INVALID_ARG: return "invalid argument";
+    case LCSC_ERR_UNSUPPORTED: return "unsupported format or dimension";
+    case LCSC_ERR_CUDA: return "CUDA launch error";
+    case LCSC_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+int64_t lcsc_row_bytes(int32_t format, int32_t dim, int32_t rope_dim) {
+  if (!valid_format(format) || dim < 1) return 0;
+  return row_bytes_of(format, dim, format == LCSC_FMT_KV ? rope_dim : 0);
+}
+
+// ------------------------------------------------------------- compression
+
+int32_t lcsc_compress_workspace_size(const lcsc_params* p, int64_t B, int64_t n_tokens,
+                                     size_t* bytes) {
+  int32_t st = check_params(p);
+  if (st) return st;
+  if (!bytes || B < 1 || n_tokens < 0) return LCSC_ERR_INVALID_ARG;
+  Carve cv{nullptr};
+  const int dim = p->head_dim > p->v_dim ? p->head_dim : p->v_dim;
+  plan_compress(p, B, new_entries_max(n_tokens, p->m), dim > p->idx_dim ? dim : p->idx_dim, cv,
+                nullptr);
+  *bytes = cv.used;
+  return LCSC_OK;
+}
+
+static int32_t compress_impl(const lcsc_params* p, int32_t tensor, const void* x, int64_t B,
+                             int64_t tok_begin, int64_t tok_end, const void* w_gate,
+                             const float* b_pos, const lcsc_cache* entries,
+                             const lcsc_cache* window, void* ws, size_t ws_bytes, int32_t* status,
+                             void* stream, bool hca) {
+  int32_t st = check_params(p);
+  if (st) return st;
+  if (hca && tensor == LCSC_TENSOR_IDX) return LCSC_ERR_INVALID_ARG;
+  RowFmt f;
+  if ((st = tensor_fmt(p, tensor, &f))) return st;
+  if (p->group_len > 128 || (p->group_len - p->m) + p->m > 128) return LCSC_ERR_UNSUPPORTED;
+  if (p->x_dtype == LCSC_DT_BF16 && f.dim == 32) return LCSC_ERR_UNSUPPORTED;
+  if (p->x_dtype == LCSC_DT_F32 && f.dim == 512) return LCSC_ERR_UNSUPPORTED;
+  if (!x || !w_gate || !b_pos || B < 1 || B > 65535) return LCSC_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_gate) || !aligned16(b_pos)) return LCSC_ERR_INVALID_ARG;
+  if (tok_begin < 0 || tok_end < tok_begin || tok_begin % p->m) return LCSC_ERR_INVALID_ARG;
+  CompressLaunch L;
+  memset(&L, 0, sizeof(L));
+  if ((st = make_view(entries, f, needs_scale(f.fmt), &L.entries))) return st;
+  if (window) {
+    if (tensor == LCSC_TENSOR_IDX) return LCSC_ERR_INVALID_ARG;
+    if ((st = make_view(window, f, needs_scale(f.fmt), &L.window))) return st;
+  }
+  const int64_t g_lo = tok_begin / p->m, g_hi = tok_end / p->m;
+  if (g_hi > entries->capacity) return LCSC_ERR_INVALID_ARG;
+  const int64_t n_new = g_hi - g_lo;
+  Carve cv{reinterpret_cast<uint8_t*>(ws)};
+  plan_compress(p, B, n_new, f.dim, cv, &L.pooled);
+  if (n_new > 0 && (!ws || ws_bytes < cv.used)) return LCSC_ERR_WORKSPACE;
+  if (ws && !aligned16(ws)) return LCSC_ERR_INVALID_ARG;
+  L.x = x;
+  L.x_dtype = p->x_dtype;
+  L.n_x = tok_end - tok_begin + p->group_len - p->m;
+  L.w = w_gate;
+  L.bpos = b_pos;
+  L.dim = f.dim;
+  L.B = (int)B;
+  L.span = {nullptr, 0, tok_begin, tok_end, p->m, p->group_len};
+  L.n_new_max = (int)n_new;
+  int64_t n_win = 0;
+  if (window) {
+    const int64_t lo = tok_end - window->capacity > tok_begin ? tok_end - window->capacity : tok_begin;
+    n_win = tok_end - lo;
+  }
+  L.n_win_max = (int)n_win;
+  L.status = status;
+  cudaError_t e = launch_compress(L, (cudaStream_t)stream);
+  return e == cudaSuccess ? LCSC_OK : cuda_fail(e);
+}
+
+int32_t lcsc_csa_compress(const lcsc_params* p, int32_t tensor, const void* x, int64_t B,
+                          int64_t tok_begin, int64_t tok_end, const void* w_gate,
+                          const float* b_pos, const lcsc_cache* entries, const lcsc_cache* window,
+                          void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+  return compress_impl(p, tensor, x, B, tok_begin, tok_end, w_gate, b_pos, entries, window, ws,
+                       ws_bytes, status, stream, false);
+}
+
+int32_t lcsc_hca_compress(const lcsc_params* p, int32_t tensor, const void* x, int64_t B,
+                          int64_t tok_begin, int64_t tok_end, const void* w_gate,
+                          const float* b_pos, const lcsc_cache* entries, const lcsc_cache* window,
+                          void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+  return compress_impl(p, tensor, x, B, tok_begin, tok_end, w_gate, b_pos, entries, window, ws,
+                       ws_bytes, status, stream, true);
+}
+
+int32_t lcsc_encode_rows(const lcsc_params* p, int32_t tensor, const float* rows, int64_t B,
+                         int64_t n, int64_t row0, const lcsc_cache* out, void* stream) {
+  int32_t st = check_params(p);
+  if (st) return st;
+  RowFmt f;
+  if ((st = tensor_fmt(p, tensor, &f))) return st;
+  if (!rows || !aligned16(rows) || B < 1 || B > 65535 || n < 0 || row0 < 0) return LCSC_ERR_INVALID_ARG;
+  CacheView v;
+  if ((st = make_view(out, f, needs_scale(f.fmt), &v))) return st;
+  if (row0 + n > out->capacity) return LCSC_ERR_INVALID_ARG;
+  cudaError_t e = launch_encode_rows(rows, (int)B, n, row0, v, (cudaStream_t)stream);
+  return e == cudaSuccess ? LCSC_OK : cuda_fail(e);
+}
+
+// ---------------------------------------------------------- indexer + top-k
+
+int32_t lcsc_index_topk_workspace_size(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max,
+                                       size_t* bytes) {
+  int32_t st = check_params(p);
+  if (st) return st;
+  if (!bytes || B < 1 || T < 1 || n_max < 0) return LCSC_ERR_INVALID_ARG;
+  Carve cv{nullptr};
+  plan_index(p, B, T, n_max, cv, nullptr);
+  *bytes = cv.used;
+  return LCSC_OK;
+}
+
+static int32_t index_setup(const lcsc_params* p, const void* q_idx, const float* w_idx,
+                           const lcsc_cache* idx_keys, const int32_t* ctx_len, int64_t B, int64_t T,
+                           int64_t n_max, int32_t* out_idx, float* out_score, Carve& cv,
+                           size_t ws_bytes, int32_t* status, IndexLaunch* L) {
+  if (!idx_supported(p)) return LCSC_ERR_UNSUPPORTED;
+  if (p->top_k < 1) return LCSC_ERR_INVALID_ARG;
+  if (!q_idx || !w_idx || !ctx_len || !out_idx) return LCSC_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(w_idx) || !aligned16(out_idx)) return LCSC_ERR_INVALID_ARG;
+  if (out_score && !aligned16(out_score)) return LCSC_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || B * T > 65535 || n_max < 0) return LCSC_ERR_INVALID_ARG;
+  RowFmt f;
+  int32_t st;
+  if ((st = tensor_fmt(p, LCSC_TENSOR_IDX, &f))) return st;
+  memset(L, 0, sizeof(*L));
+  if ((st = make_view(idx_keys, f, needs_scale(f.fmt), &L->keys))) return st;
+  if (n_max > idx_keys->capacity) return LCSC_ERR_INVALID_ARG;
+  plan_index(p, B, T, n_max, cv, L);
+  if (!cv.base || !aligned16(cv.base) || ws_bytes < cv.used) return LCSC_ERR_WORKSPACE;
+  L->q_idx = q_idx;
+  L->q_dtype = p->q_dtype;
+  L->w_idx = w_idx;
+  L->ctx_len = ctx_len;
+  L->B = (int)B;
+  L->T = (int)T;
+  L->H_I = p->idx_heads;
+  L->d_I = p->idx_dim;
+  L->m = p->m;
+  L->k = p->top_k;
+  L->n_max = n_max;
+  L->out_idx = out_idx;
+  L->out_score = out_score;
+  L->status = status;
+  return LCSC_OK;
+}
+
+int32_t lcsc_csa_index_topk(const lcsc_params* p, const void* q_idx, const float* w_idx,
+                            const lcsc_cache* idx_keys, const int32_t* ctx_len, int64_t B,
+                            int64_t T, int64_t n_max, int32_t* out_idx, float* out_score, void* ws,
+                            size_t ws_bytes, int32_t* status, void* stream) {
+  int32_t st = check_params(p);
+  if (st) return st;
+  Carve cv{reinterpret_cast<uint8_t*>(ws)};
+  IndexLaunch L;
+  if ((st = index_setup(p, q_idx, w_idx, idx_keys, ctx_len, B, T, n_max, out_idx, out_score, cv,
+                        ws_bytes, status, &L)))
+    return st;
+  cudaError_t e = launch_index_topk(L, (cudaStream_t)stream);
+  return e == cudaSuccess ? LCSC_OK : cuda_fail(e);
+}
+
+// -------------------------------------------------------------- attention
+
+int32_t lcsc_attn_workspace_size(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max,
+                                 int32_t dense, size_t* bytes) {
+  int32_t st = check_params(p);
+  if (st) return st;
+  if (!bytes || B < 1 || T < 1 || n_max < 0) return LCSC_ERR_INVALID_ARG;
+  Carve cv{nullptr};
+  plan_attn(p, B, T, n_max, dense != 0, cv, nullptr);
+  *bytes = cv.used;
+  return LCSC_OK;
+}
+
+static int32_t attn_setup(const lcsc_params* p, const void* q, const lcsc_cache* kv,
+                          const lcsc_cache* v, const lcsc_cache* win_kv, const lcsc_cache* win_v,
+                          const int32_t* idx, const float* sink, const int32_t* ctx_len, int64_t B,
+                          int64_t T, int64_t n_max, void* out, float* lse, Carve& cv,
+                          size_t ws_bytes, int32_t* status, AttnLaunch* L) {
+  if (!kv_supported(p)) return LCSC_ERR_UNSUPPORTED;
+  if (!q || !ctx_len || !out || !aligned16(q) || !aligned16(out)) return LCSC_ERR_INVALID_ARG;
+  if (lse && !aligned16(lse)) return LCSC_ERR_INVALID_ARG;
+  if (sink && ((uintptr_t)sink & 3u)) return LCSC_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || B * T > 65535 || n_max < 0) return LCSC_ERR_INVALID_ARG;
+  const bool sep = v && v->data;
+  if (sep != (win_v && win_v->data)) return LCSC_ERR_INVALID_ARG;
+  if (sep && p->kv_format != LCSC_FMT_F32) return LCSC_ERR_UNSUPPORTED;
+  if (!sep && p->v_dim != p->head_dim) return LCSC_ERR_INVALID_ARG;
+  RowFmt fk, fv;
+  int32_t st;
+  if ((st = tensor_fmt(p, LCSC_TENSOR_KV, &fk))) return st;
+  if ((st = tensor_fmt(p, LCSC_TENSOR_V, &fv))) return st;
+  memset(L, 0, sizeof(*L));
+  const bool ns = needs_scale(fk.fmt);
+  if ((st = make_view(kv, fk, ns, &L->kv))) return st;
+  if ((st = make_view(win_kv, fk, ns, &L->win_kv))) return st;
+  if (sep) {
+    if ((st = make_view(v, fv, ns, &L->v))) return st;
+    if ((st = make_view(win_v, fv, ns, &L->win_v))) return st;
+    if (win_v->capacity != win_kv->capacity) return LCSC_ERR_INVALID_ARG;
+  }
+  if (n_max > kv->capacity) return LCSC_ERR_INVALID_ARG;
+  if (p->window > 0 && win_kv->capacity < T + p->window - 1) return LCSC_ERR_INVALID_ARG;
+  plan_attn(p, B, T, n_max, idx == nullptr, cv, L);
+  if (!cv.base || !aligned16(cv.base) || ws_bytes < cv.used) return LCSC_ERR_WORKSPACE;
+  L->q = q;
+  L->q_dtype = p->q_dtype;
+  L->idx = idx;
+  L->sink = sink;
+  L->ctx_len = ctx_len;
+  L->B = (int)B;
+  L->T = (int)T;
+  L->H = p->n_heads;
+  L->D = p->head_dim;
+  L->Dv = p->v_dim;
+  L->m = p->m;
+  L->w = p->window;
+  L->k = p->top_k;
+  L->n_max = n_max;
+  L->sm_scale = p->sm_scale;
+  L->out = out;
+  L->lse = lse;
+  L->status = status;
+  return LCSC_OK;
+}
+
+int32_t lcsc_csa_sparse_attn(const lcsc_params* p, const void* q, const lcsc_cache* kv,
+                             const lcsc_cache* v, const lcsc_cache* win_kv,
+                             const lcsc_cache* win_v, const int32_t* idx, const float* sink,
+                             const int32_t* ctx_len, int64_t B, int64_t T, void* out, float* lse,
+                             void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+  int32_t st = check_params(p);
+  if (st) return st;
+  if (!idx || !aligned16(idx) || p->top_k < 1) return LCSC_ERR_INVALID_ARG;
+  Carve cv{reinterpret_cast<uint8_t*>(ws)};
+  AttnLaunch L;
+  if ((st = attn_setup(p, q, kv, v, win_kv, win_v, idx, sink, ctx_len, B, T, kv ? kv->capacity : 0,
+                       out, lse, cv, ws_bytes, status, &L)))
+    return st;
+  cudaError_t e = launch_attention(L, (cudaStream_t)stream);
+  return e == cudaSuccess ? LCSC_OK : cuda_fail(e);
+}
+
+int32_t lcsc_hca_dense_attn(const lcsc_params* p, const void* q, const lcsc_cache* kv,
+                            const lcsc_cache* v, const lcsc_cache* win_kv, const lcsc_cache* win_v,
+                            const float* sink, const int32_t* ctx_len, int64_t B, int64_t T,
+                            int64_t n_max, void* out, float* lse, void* ws, size_t ws_bytes,
+                            int32_t* status, void* stream) {
+  int32_t st = check_params(p);
+  if (st) return st;
+  Carve cv{reinterpret_cast<uint8_t*>(ws)};
+  AttnLaunch L;
+  if ((st = attn_setup(p, q, kv, v, win_kv, win_v, nullptr, sink, ctx_len, B, T, n_max, out, lse,
+                       cv, ws_bytes, status, &L)))
+    return st;
+  cudaError_t e = launch_attention(L, (cudaStream_t)stream);
+  return e == cudaSuccess ? LCSC_OK : cuda_fail(e);
+}
+
+// ------------------------------------------------------------ fused steps
+
+int32_t lcsc_step_workspace_size(const lcsc_params* p, int32_t csa, int64_t B, int64_t T,
+                                 int64_t n_max, size_t* bytes) {
+  int32_t st = check_params(p);
+  if (st) return st;
+  if (!bytes || B < 1 || T < 1 || n_max < 0) return LCSC_ERR_INVALID_ARG;
+  Carve cv{nullptr};
+  const int64_t n_new = new_entries_max(T, p->m);
+  plan_compress(p, B, n_new, p->head_dim, cv, nullptr);
+  plan_compress(p, B, n_new, p->v_dim, cv, nullptr);
+  if (csa) {
+    plan_compress(p, B, n_new, p->idx_dim, cv, nullptr);
+    cv.take<int32_t>((size_t)B * T * (p->top_k > 0 ? p->top_k : 1));
+    plan_index(p, B, T, n_max, cv, nullptr);
+  }
+  plan_attn(p, B, T, n_max, !csa, cv, nullptr);
+  *bytes = cv.used;
+  return LCSC_OK;
+}
+
+static int32_t step_compress(const lcsc_params* p, const lcsc_step* s, int32_t tensor,
+                             const void* x, const void* w, const float* bpos,
+                             const lcsc_cache* ent, const lcsc_cache* win, Carve& cv,
+                             int32_t* status, CompressLaunch* L) {
+  RowFmt f;
+  int32_t st;
+  if ((st = tensor_fmt(p, tensor, &f))) return st;
+  if (!x || !w || !bpos || !aligned16(x) || !aligned16(w) || !aligned16(bpos)) return LCSC_ERR_INVALID_ARG;
+  if (p->x_dtype == LCSC_DT_BF16 && f.dim == 32) return LCSC_ERR_UNSUPPORTED;
+  if (p->x_dtype == LCSC_DT_F32 && f.dim == 512) return LCSC_ERR_UNSUPPORTED;
+  memset(L, 0, sizeof(*L));
+  if ((st = make_view(ent, f, needs_scale(f.fmt), &L->entries))) return st;
+  if (win && (st = make_view(win, f, needs_scale(f.fmt), &L->window))) return st;
+  if (s->n_max > ent->capacity) return LCSC_ERR_INVALID_ARG;
+  const int64_t n_new = new_entries_max(s->T, p->m);
+  plan_compress(p, s->B, n_new, f.dim, cv, &L->pooled);
+  L->x = x;
+  L->x_dtype = p->x_dtype;
+  L->n_x = s->T + p->group_len - 1;
+  L->w = w;
+  L->bpos = bpos;
+  L->dim = f.dim;
+  L->B = (int)s->B;
+  L->span = {s->ctx_len, (int)s->T, 0, 0, p->m, p->group_len};
+  L->n_new_max = (int)n_new;
+  L->n_win_max = win ? (int)s->T : 0;
+  L->status = status;
+  return LCSC_OK;
+}
+
+static int32_t step_impl(const lcsc_params* p, const lcsc_step* s, void* ws, size_t ws_bytes,
+                         int32_t* status, void* stream, bool csa) {
+  int32_t st = check_params(p);
+  if (st) return st;
+  if (!s || s->B < 1 || s->T < 1 || s->B * s->T > 65535 || s->n_max < 0 || !s->ctx_len)
+    return LCSC_ERR_INVALID_ARG;
+  if (p->group_len > 128) return LCSC_ERR_UNSUPPORTED;
+  if (csa && (!idx_supported(p) || p->top_k < 1)) return csa && p->top_k < 1 ? LCSC_ERR_INVALID_ARG : LCSC_ERR_UNSUPPORTED;
+  if (!kv_supported(p)) return LCSC_ERR_UNSUPPORTED;
+  if (!ws || !aligned16(ws)) return LCSC_ERR_WORKSPACE;
+  const bool sep = s->v.data != nullptr;
+  if (sep != (s->win_v.data != nullptr) || sep != (s->x_v != nullptr)) return LCSC_ERR_INVALID_ARG;
+  if (p->window > 0 && s->win_kv.capacity < s->T + p->window - 1) return LCSC_ERR_INVALID_ARG;
+
+  Carve cv{reinterpret_cast<uint8_t*>(ws)};
+  CompressLaunch ck, cvv, ci;
+  if ((st = step_compress(p, s, LCSC_TENSOR_KV, s->x_kv, s->w_kv, s->b_kv, &s->kv, &s->win_kv, cv,
+                          status, &ck)))
+    return st;
+  if (sep) {
+    if ((st = step_compress(p, s, LCSC_TENSOR_V, s->x_v, s->w_v, s->b_v, &s->v, &s->win_v, cv, status,
+                            &cvv)))
+      return st;
+  } else {
+    plan_compress(p, s->B, new_entries_max(s->T, p->m), p->v_dim, cv, nullptr);
+  }
+  IndexLaunch il;
+  int32_t* sel = nullptr;
+  if (csa) {
+    if ((st = step_compress(p, s, LCSC_TENSOR_IDX, s->x_idx, s->w_idx, s->b_idx, &s->idx_keys,
+                            nullptr, cv, status, &ci)))
+      return st;
+    // the selection buffer: the caller's out_idx, else workspace (planned either way)
+    int32_t* sel_ws = cv.take<int32_t>((size_t)s->B * s->T * p->top_k);
+    sel = s->out_idx ? s->out_idx : sel_ws;
+    // workspace bounds are checked once the whole plan is known
+    if ((st = index_setup(p, s->q_idx, s->w_heads, &s->idx_keys, s->ctx_len, s->B, s->T, s->n_max,
+                          sel, s->out_score, cv, (size_t)-1, status, &il)))
+      return st;
+  }
+  AttnLaunch al;
+  if ((st = attn_setup(p, s->q, &s->kv, sep ? &s->v : nullptr, &s->win_kv, sep ? &s->win_v : nullptr,
+                       sel, s->sink, s->ctx_len, s->B, s->T, s->n_max, s->out, s->lse, cv,
+                       (size_t)-1, status, &al)))
+    return st;
+  if (ws_bytes < cv.used) return LCSC_ERR_WORKSPACE;
+
+  if (s->n_events < 0 || (s->n_events > 0 && !s->events)) return LCSC_ERR_INVALID_ARG;
+
+  cudaStream_t strm = (cudaStream_t)stream;
+  cudaError_t e;
+  int stage = 0;
+  auto mark = [&]() -> cudaError_t {
+    const int i = stage++;
+    if (i < s->n_events && s->events[i]) return cudaEventRecord((cudaEvent_t)s->events[i], strm);
+    return cudaSuccess;
+  };
+  if ((e = mark()) != cudaSuccess) return cuda_fail(e);
+  if ((e = launch_compress(ck, strm)) != cudaSuccess) return cuda_fail(e);
+  if (sep && (e = launch_compress(cvv, strm)) != cudaSuccess) return cuda_fail(e);
+  if (csa && (e = launch_compress(ci, strm)) != cudaSuccess) return cuda_fail(e);
+  if ((e = mark()) != cudaSuccess) return cuda_fail(e);
+  if (csa) {
+    if ((e = launch_index_scores(il, strm)) != cudaSuccess) return cuda_fail(e);
+    if ((e = mark()) != cudaSuccess) return cuda_fail(e);
+    if ((e = launch_topk(il, strm)) != cudaSuccess) return cuda_fail(e);
+    if ((e = mark()) != cudaSuccess) return cuda_fail(e);
+  }
+  if ((e = launch_attention(al, strm)) != cudaSuccess) return cuda_fail(e);
+  if ((e = mark()) != cudaSuccess) return cuda_fail(e);
+  return LCSC_OK;
+}
+
+int32_t lcsc_csa_decode(const lcsc_params* p, const lcsc_step* s, void* ws, size_t ws_bytes,
+                        int32_t* status, void* stream) {
+  return step_impl(p, s, ws, ws_bytes, status, stream, true);
+}
+
+int32_t lcsc_hca_decode(const lcsc_params* p, const lcsc_step* s, void* ws, size_t ws_bytes,
+                        int32_t* status, void* stream) {
+  return step_impl(p, s, ws, ws_bytes, status, stream, false);
+}
+
+}  // extern "C"

@@ -1,0 +1,337 @@
+// Softmax-gated pooling of token groups into compressed entries, and the
+// storing of pooled / raw rows in the cache formats.
+//
+// Method: "DeepSeek V4 Architecture Explained" (researchpapers.dev), "How
+// compress-then-sparsify attention works" -- every group of m consecutive
+// tokens' keys/values becomes one entry via trainable compression weights, a
+// softmax over the group and learnable positional biases; per channel c:
+//   z_j[c] = sum_d x_j[d] W[d][c] + Bpos[j_rel][c],  e[c] = sum_j softmax_j(z[c]) x_j[c].
+//
+// Kernel design: a CTA owns up to 128 consecutive token rows (E whole groups
+// plus the G - m rows of history an overlapping group needs) and 64 output
+// channels.  The gate logits z = x W are a [128 x dim] x [dim x 64] GEMM
+// (bf16 tensor-core mma for bf16 rows, FP32 FMA for fp32 rows); the group
+// softmax and the weighted sum run on the tile in shared memory, and the
+// pooled fp32 rows go to scratch.  A second kernel stores each pooled row
+// (whole row needed for the FP8 amax) and the raw window rows.
+#include <type_traits>
+
+#include "kernels.cuh"
+
+namespace lcsc {
+namespace {
+
+constexpr int kRows = 128;   // token rows per CTA
+constexpr int kThreads = 256;
+
+struct SeqSpan {
+  int64_t g_lo, g_hi;   // entries written
+  int64_t x_pos0;       // position of raw row 0
+  int64_t w_lo, w_hi;   // window positions written
+  bool ok;
+};
+
+// `cap` is the entries' capacity: a context length whose entries would not
+// fit makes the sequence invalid (nothing is written; the status flags it).
+__device__ __forceinline__ SeqSpan seq_span(const Span& s, int b, int64_t win_cap, int64_t cap) {
+  SeqSpan r;
+  if (s.ctx_len) {
+    const int64_t L = s.ctx_len[b];
+    r.ok = L >= s.T && L / s.m <= cap;
+    r.g_lo = r.ok ? (L - s.T) / s.m : 0;
+    r.g_hi = r.ok ? L / s.m : 0;
+    r.x_pos0 = L - (s.T + s.G - 1);
+    r.w_lo = r.ok ? L - s.T : 0;
+    r.w_hi = r.ok ? L : 0;
+  } else {
+    r.ok = true;
+    r.g_lo = s.tok_begin / s.m;
+    r.g_hi = s.tok_end / s.m;
+    r.x_pos0 = s.tok_begin - (s.G - s.m);
+    r.w_lo = s.tok_end - win_cap > s.tok_begin ? s.tok_end - win_cap : s.tok_begin;
+    r.w_hi = s.tok_end;
+  }
+  return r;
+}
+
+// ------------------------------------------------------------ mma helpers
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// ------------------------------------------------------------ pool kernel
+// grid: (ceil(n_new_max / E), dim / NC, B); block 256.
+template <bool kBf16, int DIM, int NC>
+__global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E) {
+  using Elem = typename std::conditional<kBf16, uint16_t, float>::type;
+  constexpr int XS = kBf16 ? DIM + 8 : DIM + 1;   // x tile row stride (elements)
+  constexpr int WS = kBf16 ? NC + 8 : NC + 1;     // W chunk row stride
+  constexpr int ZS = NC + 1;                      // z tile row stride (floats)
+  extern __shared__ __align__(16) uint8_t smem[];
+  Elem* xs = reinterpret_cast<Elem*>(smem);
+  Elem* ws = reinterpret_cast<Elem*>(smem + sizeof(Elem) * kRows * XS);
+  float* zs = reinterpret_cast<float*>(ws);  // reuses the W chunk after the GEMM
+
+  const int b = blockIdx.z;
+  const int c0 = blockIdx.y * NC;
+  const SeqSpan sp = seq_span(a.span, b, a.window.capacity, a.entries.capacity);
+  const int64_t n_e = sp.g_hi - sp.g_lo;
+  const int64_t e0 = (int64_t)blockIdx.x * E;
+  if (!sp.ok || e0 >= n_e) return;
+  const int m = a.span.m, G = a.span.G;
+  const int E_cta = (int)(n_e - e0 < E ? n_e - e0 : E);
+  const int R = E_cta * m + G - m;
+  const int64_t first_pos = (sp.g_lo + e0) * m + m - G;
+  const int tid = threadIdx.x;
+
+  // ---- x tile: rows of positions first_pos .. first_pos + R - 1 (zero past R or < 0)
+  const Elem* xb = reinterpret_cast<const Elem*>(a.x) + (int64_t)b * a.n_x * DIM;
+  constexpr int VEC = 16 / sizeof(Elem);
+  for (int i = tid; i < kRows * (DIM / VEC); i += kThreads) {
+    const int r = i / (DIM / VEC), cv = (i % (DIM / VEC)) * VEC;
+    const int64_t pos = first_pos + r;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (r < R && pos >= 0) val = *reinterpret_cast<const uint4*>(xb + (pos - sp.x_pos0) * DIM + cv);
+    Elem* d = xs + r * XS + cv;
+    if constexpr (kBf16) {
+      *reinterpret_cast<uint4*>(d) = val;  // XS*2 bytes is a multiple of 16
+    } else {
+      const float* f = reinterpret_cast<const float*>(&val);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) d[j] = f[j];
+    }
+  }
+  // ---- W chunk: columns c0 .. c0 + NC of W [DIM][DIM]
+  const Elem* wg = reinterpret_cast<const Elem*>(a.w);
+  for (int i = tid; i < DIM * (NC / VEC); i += kThreads) {
+    const int k = i / (NC / VEC), cv = (i % (NC / VEC)) * VEC;
+    uint4 val = *reinterpret_cast<const uint4*>(wg + (int64_t)k * DIM + c0 + cv);
+    Elem* d = ws + k * WS + cv;
+    if constexpr (kBf16) {
+      *reinterpret_cast<uint4*>(d) = val;
+    } else {
+      const float* f = reinterpret_cast<const float*>(&val);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) d[j] = f[j];
+    }
+  }
+  __syncthreads();
+
+  // ---- z = x W for the 128 x NC tile
+  if constexpr (kBf16) {
+    const int warp = tid / kWarp, lane = tid % kWarp;
+    float acc[NC / 8][4];
+#pragma unroll
+    for (int j = 0; j < NC / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+#pragma unroll 4
+    for (int ks = 0; ks < DIM / 16; ++ks) {
+      uint32_t af[4];
+      ldsm_x4(af, xs + (warp * 16 + (lane % 16)) * XS + ks * 16 + (lane / 16) * 8);
+#pragma unroll
+      for (int j = 0; j < NC / 8; j += 2) {
+        uint32_t bf[4];
+        ldsm_x4_t(bf, ws + (ks * 16 + (lane % 8) + ((lane / 8) % 2) * 8) * WS + j * 8 + (lane / 16) * 8);
+        mma_bf16(acc[j], af, bf[0], bf[1]);
+        mma_bf16(acc[j + 1], af, bf[2], bf[3]);
+      }
+    }
+    __syncthreads();  // the W chunk is dead: z reuses it
+    const int g = lane / 4, t = lane % 4;
+#pragma unroll
+    for (int j = 0; j < NC / 8; ++j) {
+      const int col = j * 8 + 2 * t;
+      zs[(warp * 16 + g) * ZS + col] = acc[j][0];
+      zs[(warp * 16 + g) * ZS + col + 1] = acc[j][1];
+      zs[(warp * 16 + g + 8) * ZS + col] = acc[j][2];
+      zs[(warp * 16 + g + 8) * ZS + col + 1] = acc[j][3];
+    }
+  } else {
+    constexpr int RG = kThreads / NC;          // row groups
+    constexpr int RPT = kRows / RG;            // rows per thread
+    const int c = tid % NC, rg = tid / NC;
+    float acc[RPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) acc[i] = 0.f;
+    for (int k = 0; k < DIM; ++k) {
+      const float wv = ws[k * WS + c];
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) acc[i] = fmaf(xs[(rg + i * RG) * XS + k], wv, acc[i]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) zs[(rg + i * RG) * ZS + c] = acc[i];
+  }
+  __syncthreads();
+
+  // ---- group softmax over tokens and weighted sum, per (entry, channel)
+  // TP threads share one (entry, channel) pair, each taking every TP-th token.
+  int TP = kThreads / (E_cta * NC);
+  TP = TP < 1 ? 1 : (TP > 32 ? 32 : TP);
+  while (TP > 1 && (G % TP != 0)) TP >>= 1;
+  {
+    int p2 = 1;
+    while (p2 * 2 <= TP) p2 *= 2;
+    TP = p2;
+  }
+  const int n_pairs = E_cta * NC;
+  const int pairs_per_pass = kThreads / TP;
+  for (int pb = 0; pb < n_pairs; pb += pairs_per_pass) {
+    const int pair = pb + tid / TP;
+    const int sub = tid % TP;
+    const bool active = pair < n_pairs;
+    const int e = active ? pair / NC : 0, c = active ? pair % NC : 0;
+    float mx = -INFINITY;
+    if (active) {
+      for (int j = sub; j < G; j += TP) {
+        const int r = e * m + j;
+        if (first_pos + r < 0) continue;
+        mx = fmaxf(mx, zs[r * ZS + c] + a.bpos[j * DIM + c0 + c]);
+      }
+    }
+    mx = group_max(mx, TP);
+    float den = 0.f, num = 0.f;
+    if (active) {
+      for (int j = sub; j < G; j += TP) {
+        const int r = e * m + j;
+        if (first_pos + r < 0) continue;
+        const float p = expf(zs[r * ZS + c] + a.bpos[j * DIM + c0 + c] - mx);
+        float xv;
+        if constexpr (kBf16) xv = bf16_val(xs[r * XS + c0 + c]);
+        else xv = xs[r * XS + c0 + c];
+        den += p;
+        num = fmaf(p, xv, num);
+      }
+    }
+    for (int o = TP >> 1; o > 0; o >>= 1) {
+      den += __shfl_xor_sync(0xffffffffu, den, o);
+      num += __shfl_xor_sync(0xffffffffu, num, o);
+    }
+    if (active && sub == 0)
+      a.pooled[((int64_t)b * a.n_new_max + e0 + e) * DIM + c0 + c] = num / den;
+  }
+}
+
+// ------------------------------------------------------------ store kernel
+// grid: (ceil((n_new_max + n_win_max) / 8), B); one warp per row.
+template <int VPL>
+__global__ void __launch_bounds__(256) store_kernel(CompressLaunch a) {
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+  const int64_t i = (int64_t)blockIdx.x * 8 + warp;
+  const SeqSpan sp = seq_span(a.span, b, a.window.capacity, a.entries.capacity);
+  if (!sp.ok) {
+    if (i == 0 && lane == 0 && a.status) atomicOr(a.status, LCSC_DEV_BAD_LENGTH);
+    return;
+  }
+  const int64_t n_e = sp.g_hi - sp.g_lo;
+  const int64_t n_w = a.window.data ? sp.w_hi - sp.w_lo : 0;
+  constexpr int DIM = VPL * 32;
+  float v[VPL];
+  if (i < n_e) {
+    const float* src = a.pooled + ((int64_t)b * a.n_new_max + i) * DIM + lane * VPL;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) v[j] = src[j];
+    store_row_warp<VPL>(a.entries, b, sp.g_lo + i, v, lane);
+  } else if (i < n_e + n_w) {
+    const int64_t pos = sp.w_lo + (i - n_e);
+    const int64_t xr = pos - sp.x_pos0;
+    const int64_t base = ((int64_t)b * a.n_x + xr) * DIM + lane * VPL;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) v[j] = load_elem(a.x, base + j, a.x_dtype);
+    store_row_warp<VPL>(a.window, b, pos % a.window.capacity, v, lane);
+  }
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(256) encode_rows_kernel(const float* rows, int64_t n, int64_t row0,
+                                                          CacheView out) {
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+  const int64_t i = (int64_t)blockIdx.x * 8 + warp;
+  if (i >= n) return;
+  constexpr int DIM = VPL * 32;
+  const float* src = rows + ((int64_t)b * n + i) * DIM + lane * VPL;
+  float v[VPL];
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) v[j] = src[j];
+  store_row_warp<VPL>(out, b, row0 + i, v, lane);
+}
+
+template <bool kBf16, int DIM, int NC>
+cudaError_t launch_pool(const CompressLaunch& a, int E, cudaStream_t stream) {
+  using Elem = typename std::conditional<kBf16, uint16_t, float>::type;
+  constexpr int XS = kBf16 ? DIM + 8 : DIM + 1;
+  constexpr int WS = kBf16 ? NC + 8 : NC + 1;
+  size_t smem = sizeof(Elem) * kRows * XS;
+  size_t wz = sizeof(Elem) * DIM * WS;
+  const size_t zbytes = sizeof(float) * kRows * (NC + 1);
+  smem += wz > zbytes ? wz : zbytes;
+  auto kern = pool_kernel<kBf16, DIM, NC>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((a.n_new_max + E - 1) / E), DIM / NC, a.B);
+  kern<<<grid, kThreads, smem, stream>>>(a, E);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_compress(const CompressLaunch& a, cudaStream_t stream) {
+  const int m = a.span.m, G = a.span.G;
+  const int E = (kRows - (G - m)) / m;
+  cudaError_t e = cudaSuccess;
+  if (a.n_new_max > 0) {
+    const bool bf = a.x_dtype == LCSC_DT_BF16;
+    if (bf && a.dim == 512) e = launch_pool<true, 512, 64>(a, E, stream);
+    else if (bf && a.dim == 128) e = launch_pool<true, 128, 64>(a, E, stream);
+    else if (!bf && a.dim == 128) e = launch_pool<false, 128, 64>(a, E, stream);
+    else if (!bf && a.dim == 32) e = launch_pool<false, 32, 32>(a, E, stream);
+    else return cudaErrorInvalidValue;
+    if (e != cudaSuccess) return e;
+  }
+  const int rows = a.n_new_max + (a.window.data ? a.n_win_max : 0);
+  if (rows == 0) return cudaSuccess;
+  dim3 grid((unsigned)((rows + 7) / 8), a.B);
+  switch (a.dim) {
+    case 512: store_kernel<16><<<grid, 256, 0, stream>>>(a); break;
+    case 128: store_kernel<4><<<grid, 256, 0, stream>>>(a); break;
+    case 32: store_kernel<1><<<grid, 256, 0, stream>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_encode_rows(const float* rows, int B, int64_t n, int64_t row0,
+                               const CacheView& out, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  dim3 grid((unsigned)((n + 7) / 8), B);
+  switch (out.f.dim) {
+    case 512: encode_rows_kernel<16><<<grid, 256, 0, stream>>>(rows, n, row0, out); break;
+    case 128: encode_rows_kernel<4><<<grid, 256, 0, stream>>>(rows, n, row0, out); break;
+    case 32: encode_rows_kernel<1><<<grid, 256, 0, stream>>>(rows, n, row0, out); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace lcsc

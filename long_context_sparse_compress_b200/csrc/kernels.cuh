@@ -1,0 +1,95 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernel
+// translation units.  Every launcher enqueues on `stream` and returns the
+// launch's cudaError_t.
+#pragma once
+
+#include "common.cuh"
+
+namespace lcsc {
+
+// Entry range of one call, per sequence:
+//   fused step (ctx_len != nullptr): L = ctx_len[b], entries
+//     [floor((L - T) / m), floor(L / m)), raw rows start at L - (T + G - 1),
+//     window rows L - T .. L - 1;
+//   bulk call (ctx_len == nullptr): entries [tok_begin / m, tok_end / m),
+//     raw rows start at tok_begin - (G - m), window rows
+//     max(tok_begin, tok_end - capacity) .. tok_end - 1.
+struct Span {
+  const int32_t* ctx_len;
+  int T;
+  int64_t tok_begin, tok_end;
+  int m, G;
+};
+
+struct CompressLaunch {
+  const void* x;        // [B][n_x][dim] raw rows
+  int x_dtype;
+  int64_t n_x;
+  const void* w;        // [dim][dim]
+  const float* bpos;    // [G][dim]
+  int dim;
+  int B;
+  Span span;
+  int n_new_max;        // max entries per sequence in this call
+  float* pooled;        // [B][n_new_max][dim] scratch
+  CacheView entries;
+  CacheView window;     // data == nullptr: no window write
+  int n_win_max;        // max window rows per sequence
+  int32_t* status;
+};
+
+cudaError_t launch_compress(const CompressLaunch& a, cudaStream_t stream);
+
+cudaError_t launch_encode_rows(const float* rows, int B, int64_t n, int64_t row0,
+                               const CacheView& out, cudaStream_t stream);
+
+struct IndexLaunch {
+  const void* q_idx;    // [B][T][H_I][d_I] q_dtype
+  int q_dtype;
+  const float* w_idx;   // [B][T][H_I]
+  CacheView keys;       // idx_format, d_I
+  CacheView q_store;    // workspace rows: [B][T*H_I] in the key format
+  const int32_t* ctx_len;
+  int B, T, H_I, d_I, m, k;
+  int64_t n_max;
+  float* scores;        // [B*T][n_max]
+  // top-k workspace
+  uint32_t* hist;       // [B*T][2][4096]
+  uint32_t* counters;   // [B*T][4]
+  uint32_t* cand;       // [B*T][n_max]
+  int32_t* out_idx;     // [B*T][k]
+  float* out_score;     // [B*T][k] or nullptr
+  int32_t* status;
+};
+
+// Indexer scoring (query quantisation + scores) and top-k selection; the
+// stand-alone call runs both.
+cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream);
+cudaError_t launch_topk(const IndexLaunch& a, cudaStream_t stream);
+cudaError_t launch_index_topk(const IndexLaunch& a, cudaStream_t stream);
+
+struct AttnLaunch {
+  const void* q;        // [B][T][H][D]
+  int q_dtype;
+  CacheView kv, v, win_kv, win_v;  // v / win_v data == nullptr: V = K
+  const int32_t* idx;   // [B][T][k] or nullptr (dense)
+  const float* sink;    // [H] or nullptr
+  const int32_t* ctx_len;
+  int B, T, H, D, Dv, m, w, k;
+  int64_t n_max;
+  float sm_scale;
+  int splits;           // row splits per query
+  int rows_per_split;
+  float* part_o;        // [B*T][splits][H][Dv]
+  float* part_ml;       // [B*T][splits][H][2]
+  void* out;            // [B][T][H][Dv] q_dtype
+  float* lse;           // [B][T][H] or nullptr
+  int32_t* status;
+};
+
+cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream);
+
+// Attention split geometry for a call (rows per split and split count).
+void attention_splits(int64_t max_rows, int64_t n_lists, int* splits, int* rows_per_split);
+
+}  // namespace lcsc

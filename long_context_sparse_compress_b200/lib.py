@@ -1,0 +1,282 @@
+"""ctypes binding of liblcsc.so (include/lcsc.h): argument marshalling only.
+
+Every computation happens in the CUDA library.  ``load()`` raises when the
+library is missing or was built for another ABI: there is no fallback.
+Tensors are torch device tensors; pointers are passed as integers.
+"""
+import ctypes
+import os
+
+import torch
+
+from . import workloads
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblcsc.so")
+ABI_VERSION = 1
+
+FMT = {"f32": 0, "kv": 1, "fp8": 2, "fp4": 3}
+DT = {"f32": 0, "bf16": 1}
+TENSOR = {"kv": 0, "v": 1, "idx": 2}
+DEV_BAD_INDEX = 1
+DEV_BAD_LENGTH = 2
+
+c_i32, c_i64, c_f32, c_vp, c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("m", c_i32), ("group_len", c_i32), ("window", c_i32), ("top_k", c_i32),
+                ("sm_scale", c_f32), ("n_heads", c_i32), ("head_dim", c_i32), ("rope_dim", c_i32),
+                ("v_dim", c_i32), ("idx_heads", c_i32), ("idx_dim", c_i32), ("kv_format", c_i32),
+                ("idx_format", c_i32), ("x_dtype", c_i32), ("q_dtype", c_i32)]
+
+
+class Cache(ctypes.Structure):
+    _fields_ = [("data", c_vp), ("scale", c_vp), ("capacity", c_i64)]
+
+
+class Step(ctypes.Structure):
+    _fields_ = [("B", c_i64), ("T", c_i64), ("n_max", c_i64), ("ctx_len", c_vp),
+                ("x_kv", c_vp), ("x_v", c_vp), ("x_idx", c_vp),
+                ("w_kv", c_vp), ("b_kv", c_vp), ("w_v", c_vp), ("b_v", c_vp),
+                ("w_idx", c_vp), ("b_idx", c_vp),
+                ("kv", Cache), ("v", Cache), ("idx_keys", Cache), ("win_kv", Cache), ("win_v", Cache),
+                ("q", c_vp), ("q_idx", c_vp), ("w_heads", c_vp), ("sink", c_vp),
+                ("out", c_vp), ("lse", c_vp), ("out_idx", c_vp), ("out_score", c_vp),
+                ("events", ctypes.POINTER(c_vp)), ("n_events", c_i32)]
+
+
+_SIGS = {
+    "lcsc_abi_version": (c_i32, []),
+    "lcsc_last_cuda_error": (c_i32, []),
+    "lcsc_status_string": (ctypes.c_char_p, [c_i32]),
+    "lcsc_row_bytes": (c_i64, [c_i32, c_i32, c_i32]),
+    "lcsc_compress_workspace_size": (c_i32, [c_vp, c_i64, c_i64, c_vp]),
+    "lcsc_csa_compress": (c_i32, [c_vp, c_i32, c_vp, c_i64, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp,
+                                  c_vp, c_sz, c_vp, c_vp]),
+    "lcsc_hca_compress": (c_i32, [c_vp, c_i32, c_vp, c_i64, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp,
+                                  c_vp, c_sz, c_vp, c_vp]),
+    "lcsc_encode_rows": (c_i32, [c_vp, c_i32, c_vp, c_i64, c_i64, c_i64, c_vp, c_vp]),
+    "lcsc_index_topk_workspace_size": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp]),
+    "lcsc_csa_index_topk": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_vp, c_vp,
+                                    c_vp, c_sz, c_vp, c_vp]),
+    "lcsc_attn_workspace_size": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_i32, c_vp]),
+    "lcsc_csa_sparse_attn": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i64,
+                                     c_i64, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
+    "lcsc_hca_dense_attn": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64,
+                                    c_i64, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
+    "lcsc_step_workspace_size": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, c_vp]),
+    "lcsc_csa_decode": (c_i32, [c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
+    "lcsc_hca_decode": (c_i32, [c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
+}
+
+EXPORTS = tuple(_SIGS)
+_lib = None
+
+
+class LcscError(RuntimeError):
+    pass
+
+
+def load(path=LIB_PATH):
+    """Load the library (once).  Raises if it is missing: nothing runs without it."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise LcscError(f"{path} is missing: build it with `python -m long_context_sparse_compress_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if lib.lcsc_abi_version() != ABI_VERSION:
+        raise LcscError("liblcsc.so ABI version mismatch: rebuild it")
+    _lib = lib
+    return lib
+
+
+def check(status):
+    if status != 0:
+        lib = load()
+        msg = lib.lcsc_status_string(status).decode()
+        if status == 3:
+            msg += f" (cudaError {lib.lcsc_last_cuda_error()})"
+        raise LcscError(f"lcsc call failed: {msg}")
+
+
+def ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def ref(s):
+    return None if s is None else ctypes.byref(s)
+
+
+def stream_handle(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def params(wl):
+    """lcsc_params of a single-layer workload."""
+    return Params(m=wl.m, group_len=wl.G, window=wl.w, top_k=wl.k if wl.kind == "csa" else 0,
+                  sm_scale=wl.sm_scale, n_heads=wl.H, head_dim=wl.D,
+                  rope_dim=wl.rope_dim if wl.kv_fmt == "kv" else 0, v_dim=wl.Dv, idx_heads=wl.H_I,
+                  idx_dim=wl.d_I, kv_format=FMT[wl.kv_fmt], idx_format=FMT[wl.idx_fmt],
+                  x_dtype=DT[wl.x_dtype], q_dtype=DT[wl.q_dtype])
+
+
+def row_bytes(fmt, dim, rope=0):
+    return {"f32": 4 * dim, "kv": dim + rope, "fp8": dim, "fp4": dim // 2}[fmt]
+
+
+class DeviceCache:
+    """Stored rows of one tensor for B sequences, in device memory."""
+
+    def __init__(self, B, capacity, fmt, dim, rope=0, device="cuda"):
+        self.B, self.capacity, self.fmt, self.dim, self.rope = B, capacity, fmt, dim, rope
+        if fmt == "f32":
+            self.data = torch.zeros((B, capacity, dim), dtype=torch.float32, device=device)
+            self.scale = None
+        else:
+            self.data = torch.zeros((B, capacity, row_bytes(fmt, dim, rope)), dtype=torch.uint8, device=device)
+            if fmt == "fp4":
+                self.scale = torch.zeros((B, capacity, dim // 16), dtype=torch.uint8, device=device)
+            else:
+                self.scale = torch.ones((B, capacity), dtype=torch.float32, device=device)
+
+    def c(self):
+        return Cache(data=self.data.data_ptr(), scale=None if self.scale is None else self.scale.data_ptr(),
+                     capacity=self.capacity)
+
+    def seq(self, b):
+        """A one-sequence view (sequence b) usable wherever a cache is."""
+        return _SeqView(self, b)
+
+
+class _SeqView:
+    def __init__(self, cache, b):
+        self.cache, self.b, self.capacity = cache, b, cache.capacity
+
+    def c(self):
+        c = self.cache
+        return Cache(data=c.data[self.b].data_ptr(),
+                     scale=None if c.scale is None else c.scale[self.b].data_ptr(), capacity=c.capacity)
+
+
+def null_cache():
+    return Cache(data=None, scale=None, capacity=0)
+
+
+# ------------------------------------------------------------------ calls
+
+def _ws_size(fn, *args):
+    out = c_sz(0)
+    check(fn(*args, ctypes.byref(out)))
+    return out.value
+
+
+def workspace(nbytes, device="cuda"):
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def compress(p, tensor, x, B, tok_begin, tok_end, w, bpos, entries, window=None, status=None,
+             hca=False, stream=None):
+    lib = load()
+    n_tok = tok_end - tok_begin
+    ws = workspace(_ws_size(lib.lcsc_compress_workspace_size, ctypes.byref(p), B, n_tok), x.device)
+    fn = lib.lcsc_hca_compress if hca else lib.lcsc_csa_compress
+    win = window.c() if window is not None else None
+    check(fn(ctypes.byref(p), TENSOR[tensor], ptr(x), B, tok_begin, tok_end, ptr(w), ptr(bpos),
+             ctypes.byref(entries.c()), ref(win), ptr(ws), ws.numel(), ptr(status), stream_handle(stream)))
+    return ws
+
+
+def encode_rows(p, tensor, rows, row0, out, stream=None):
+    lib = load()
+    B, n = rows.shape[0], rows.shape[1]
+    check(lib.lcsc_encode_rows(ctypes.byref(p), TENSOR[tensor], ptr(rows), B, n, row0,
+                               ctypes.byref(out.c()), stream_handle(stream)))
+
+
+def index_topk_workspace(p, B, T, n_max):
+    return _ws_size(load().lcsc_index_topk_workspace_size, ctypes.byref(p), B, T, n_max)
+
+
+def index_topk(p, q_idx, w_idx, keys, ctx_len, n_max, out_idx, out_score=None, ws=None, status=None,
+               stream=None):
+    lib = load()
+    B, T = q_idx.shape[0], q_idx.shape[1]
+    if ws is None:
+        ws = workspace(index_topk_workspace(p, B, T, n_max), q_idx.device)
+    check(lib.lcsc_csa_index_topk(ctypes.byref(p), ptr(q_idx), ptr(w_idx), ctypes.byref(keys.c()),
+                                  ptr(ctx_len), B, T, n_max, ptr(out_idx), ptr(out_score), ptr(ws),
+                                  ws.numel(), ptr(status), stream_handle(stream)))
+    return ws
+
+
+def attn_workspace(p, B, T, n_max, dense):
+    return _ws_size(load().lcsc_attn_workspace_size, ctypes.byref(p), B, T, n_max, int(dense))
+
+
+def sparse_attn(p, q, kv, v, win_kv, win_v, idx, sink, ctx_len, out, lse=None, ws=None, status=None,
+                stream=None):
+    lib = load()
+    B, T = q.shape[0], q.shape[1]
+    if ws is None:
+        ws = workspace(attn_workspace(p, B, T, kv.capacity, False), q.device)
+    check(lib.lcsc_csa_sparse_attn(
+        ctypes.byref(p), ptr(q), ctypes.byref(kv.c()), ref(v.c() if v else None),
+        ctypes.byref(win_kv.c()), ref(win_v.c() if win_v else None), ptr(idx), ptr(sink), ptr(ctx_len),
+        B, T, ptr(out), ptr(lse), ptr(ws), ws.numel(), ptr(status), stream_handle(stream)))
+    return ws
+
+
+def dense_attn(p, q, kv, v, win_kv, win_v, sink, ctx_len, n_max, out, lse=None, ws=None, status=None,
+               stream=None):
+    lib = load()
+    B, T = q.shape[0], q.shape[1]
+    if ws is None:
+        ws = workspace(attn_workspace(p, B, T, n_max, True), q.device)
+    check(lib.lcsc_hca_dense_attn(
+        ctypes.byref(p), ptr(q), ctypes.byref(kv.c()), ref(v.c() if v else None),
+        ctypes.byref(win_kv.c()), ref(win_v.c() if win_v else None), ptr(sink), ptr(ctx_len), B, T, n_max,
+        ptr(out), ptr(lse), ptr(ws), ws.numel(), ptr(status), stream_handle(stream)))
+    return ws
+
+
+def step_workspace(p, csa, B, T, n_max):
+    return _ws_size(load().lcsc_step_workspace_size, ctypes.byref(p), int(csa), B, T, n_max)
+
+
+def make_step(B, T, n_max, ctx_len, x_kv, x_v, x_idx, w_kv, b_kv, w_v, b_v, w_idx, b_idx, kv, v, idx_keys,
+              win_kv, win_v, q, q_idx, w_heads, sink, out, lse=None, out_idx=None, out_score=None):
+    """An lcsc_step struct over device tensors / caches (None -> NULL)."""
+    cc = lambda c: c.c() if c is not None else null_cache()
+    s = Step(B=B, T=T, n_max=n_max)
+    for name, t in dict(ctx_len=ctx_len, x_kv=x_kv, x_v=x_v, x_idx=x_idx, w_kv=w_kv, b_kv=b_kv, w_v=w_v,
+                        b_v=b_v, w_idx=w_idx, b_idx=b_idx, q=q, q_idx=q_idx, w_heads=w_heads, sink=sink,
+                        out=out, lse=lse, out_idx=out_idx, out_score=out_score).items():
+        setattr(s, name, None if t is None else t.data_ptr())
+    s.kv, s.v, s.idx_keys, s.win_kv, s.win_v = cc(kv), cc(v), cc(idx_keys), cc(win_kv), cc(win_v)
+    return s
+
+
+def set_step_events(step, events):
+    """Attach stage-boundary events (torch.cuda.Event, already created) to a
+    step struct; the returned array must outlive the call."""
+    arr = (c_vp * len(events))(*[e.cuda_event for e in events])
+    step.events = ctypes.cast(arr, ctypes.POINTER(c_vp))
+    step.n_events = len(events)
+    return arr
+
+
+def decode_step(p, step, csa, ws, status=None, stream=None):
+    lib = load()
+    fn = lib.lcsc_csa_decode if csa else lib.lcsc_hca_decode
+    check(fn(ctypes.byref(p), ctypes.byref(step), ptr(ws), ws.numel(), ptr(status), stream_handle(stream)))
+
+
+__all__ = ["load", "params", "DeviceCache", "compress", "encode_rows", "index_topk", "sparse_attn",
+           "dense_attn", "make_step", "decode_step", "workloads"]

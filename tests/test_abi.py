@@ -1,0 +1,77 @@
+"""The C-ABI library loads, exports every function include/lcsc.h declares,
+and rejects bad arguments on the host before any launch (CPU only: no
+call below reaches the GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_sparse_compress_b200 import lib as L
+from long_context_sparse_compress_b200 import workloads as W
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "lcsc.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lcsc_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_context_sparse_compress_b200 import build
+    if not os.path.exists(L.LIB_PATH):
+        build.build()
+    return L.load()
+
+
+def test_every_declared_function_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(L.EXPORTS) == set(names)
+
+
+def test_abi_version_and_strings(lib):
+    assert lib.lcsc_abi_version() == L.ABI_VERSION
+    for code in range(5):
+        assert lib.lcsc_status_string(code)
+    assert lib.lcsc_row_bytes(L.FMT["kv"], 512, 64) == 576
+    assert lib.lcsc_row_bytes(L.FMT["fp8"], 128, 0) == 128
+    assert lib.lcsc_row_bytes(L.FMT["fp4"], 128, 0) == 64
+    assert lib.lcsc_row_bytes(L.FMT["f32"], 128, 0) == 512
+
+
+def test_workspace_sizes_are_host_only(lib):
+    p = L.params(W.PAIR_DECODE_1M_B16.layer("csa"))
+    out = ctypes.c_size_t(0)
+    assert lib.lcsc_index_topk_workspace_size(ctypes.byref(p), 16, 1, 262144, ctypes.byref(out)) == 0
+    assert out.value >= 16 * 262144 * 8
+    assert lib.lcsc_step_workspace_size(ctypes.byref(p), 1, 16, 1, 262144, ctypes.byref(out)) == 0
+    assert lib.lcsc_attn_workspace_size(ctypes.byref(p), 16, 1, 8192, 1, ctypes.byref(out)) == 0
+
+
+def test_bad_arguments_are_rejected_before_launch(lib):
+    p = L.params(W.CSA_DECODE_128K)
+    null = None
+    # null params
+    assert lib.lcsc_csa_decode(null, null, null, 0, null, null) == 1
+    # null step
+    assert lib.lcsc_csa_decode(ctypes.byref(p), null, null, 0, null, null) == 1
+    # k beyond 2048
+    bad = L.params(W.CSA_DECODE_128K.with_(k=4096))
+    out = ctypes.c_size_t(0)
+    assert lib.lcsc_index_topk_workspace_size(ctypes.byref(bad), 1, 1, 10, ctypes.byref(out)) == 1
+    # group length beyond 2m
+    bad = L.params(W.CSA_DECODE_128K.with_(G=12))
+    assert lib.lcsc_index_topk_workspace_size(ctypes.byref(bad), 1, 1, 10, ctypes.byref(out)) == 1
+    # a dimension the kernels are not built for
+    odd = L.params(W.CSA_DECODE_128K.with_(d_I=96))
+    s = L.Step(B=1, T=1, n_max=10, ctx_len=16)
+    ws = ctypes.create_string_buffer(64)
+    assert lib.lcsc_csa_decode(ctypes.byref(odd), ctypes.byref(s), ws, 64, null, null) == 2
+    # misaligned pointer in encode_rows
+    assert lib.lcsc_encode_rows(ctypes.byref(p), 0, 3, 1, 1, 0, null, null) == 1

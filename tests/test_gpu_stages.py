@@ -1,0 +1,294 @@
+"""Per-stage parity of the CUDA library against the oracle (small shapes that
+still span several tiles and ragged tails).  Every input is seeded; every
+expected value comes from ``oracle/``."""
+import numpy as np
+import pytest
+import torch
+
+from long_context_sparse_compress_b200 import lib as L
+from long_context_sparse_compress_b200 import workloads as W
+from oracle import storage
+from oracle.compress import compress_entries
+from oracle.indexer import quantize_query, scores as oracle_scores, topk as oracle_topk
+from oracle.attention import joint_attention, window_positions
+from tests.gpu_harness import TORCH_DT, dev, download, upload
+from tests.harness import max_abs, rel_l2, topk_set_ok
+
+pytestmark = pytest.mark.gpu
+
+ATTN_RTOL, ATTN_ATOL = 1e-2, 2e-2
+FP32_RTOL, Q_RTOL = 1e-5, 1e-2
+
+
+def _rows(rng, n, d, scale=None):
+    scale = d ** -0.5 if scale is None else scale
+    return (rng.standard_normal((n, d)) * scale).astype(np.float32)
+
+
+def _wl_for(fmt_kv="kv", fmt_idx="fp8"):
+    if fmt_kv == "f32":
+        return W.CSA_DECODE_4K_F32
+    return W.CSA_DECODE_128K.with_(idx_fmt=fmt_idx)
+
+
+# ------------------------------------------------------------------ encode
+
+@pytest.mark.parametrize("fmt,dim,rope", [("kv", 512, 64), ("fp8", 128, 0), ("fp4", 128, 0),
+                                          ("f32", 128, 0), ("f32", 32, 0)])
+def test_encode_rows_bit_exact(cuda_lib, fmt, dim, rope):
+    rng = np.random.default_rng(11)
+    B, n = 2, 300
+    rows = _rows(rng, B * n, dim).reshape(B, n, dim)
+    rows[0, 0] = 0.0                                  # zero row
+    rows[0, 1] *= 1e4                                 # large values
+    rows[0, 2] *= 1e-6                                # tiny values (subnormal codes)
+    rows[1, 3, ::3] = 0.0
+    if fmt == "f32":
+        wl = W.CSA_DECODE_4K_F32.with_(d_I=dim) if dim == 32 else W.CSA_DECODE_4K_F32
+        tensor = "idx" if dim == 32 else "kv"
+    else:
+        wl = W.CSA_DECODE_128K.with_(idx_fmt=fmt if fmt != "kv" else "fp8")
+        tensor = "kv" if fmt == "kv" else "idx"
+    p = L.params(wl)
+    out = L.DeviceCache(B, n + 5, fmt, dim, rope)
+    L.encode_rows(p, tensor, dev(rows), 5, out)
+    torch.cuda.synchronize()
+    for b in range(B):
+        st = storage.encode(fmt, rows[b], rope)
+        d, s = download(out, b)
+        assert np.array_equal(d[5:], st.payload), f"payload mismatch b={b}"
+        if s is not None:
+            assert np.array_equal(s[5:], st.scale), f"scale mismatch b={b}"
+
+
+# ---------------------------------------------------------------- compress
+
+COMPRESS_CASES = {
+    "f32_k_m4": ("f32", "kv", 4, 4, 128, "f32"),
+    "f32_idx_m4": ("f32", "idx", 4, 4, 32, "f32"),
+    "kv512_m4": ("kv", "kv", 4, 4, 512, "bf16"),
+    "fp8idx_m4": ("fp8", "idx", 4, 4, 128, "bf16"),
+    "fp4idx_m4": ("fp4", "idx", 4, 4, 128, "bf16"),
+    "kv512_m128": ("kv", "kv", 128, 128, 512, "bf16"),
+    "kv512_m4_overlap8": ("kv", "kv", 4, 8, 512, "bf16"),
+    "f32_k_m4_overlap8": ("f32", "kv", 4, 8, 128, "f32"),
+}
+
+
+@pytest.mark.parametrize("case", sorted(COMPRESS_CASES))
+@pytest.mark.parametrize("with_window", [False, True])
+def test_compress_matches_oracle(cuda_lib, case, with_window):
+    fmt, tensor, m, G, dim, xdt = COMPRESS_CASES[case]
+    rng = np.random.default_rng(hash(case) % 2 ** 31)
+    B = 3
+    tok_begin = 0 if m == 128 else 8 * m
+    n_entries = 5 if m == 128 else 70            # > 2 CTAs of 32 entries, ragged
+    tok_end = tok_begin + n_entries * m + (m // 2)  # a trailing partial group (not pooled)
+    n_x = tok_end - tok_begin + G - m
+    x = _rows(rng, B * n_x, dim).reshape(B, n_x, dim)
+    if xdt == "bf16":
+        x = torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+    Wg = (rng.standard_normal((dim, dim)) * 0.02).astype(np.float32)
+    if xdt == "bf16":
+        Wg = torch.from_numpy(Wg).to(torch.bfloat16).float().numpy()
+    Bp = rng.standard_normal((G, dim)).astype(np.float32)
+    if fmt == "f32":
+        wl = W.CSA_DECODE_4K_F32.with_(m=m, G=G)
+    else:
+        wl = W.CSA_DECODE_128K.with_(m=m, G=G, idx_fmt=fmt if tensor == "idx" else "fp8")
+    p = L.params(wl)
+    rope = wl.rope_dim if fmt == "kv" else 0
+    n_cap = tok_end // m + 3
+    ent = L.DeviceCache(B, n_cap, fmt, dim, rope)
+    win = L.DeviceCache(B, 64, fmt, dim, rope) if (with_window and tensor != "idx") else None
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.compress(p, tensor, dev(x, TORCH_DT[xdt]), B, tok_begin, tok_end, dev(Wg, TORCH_DT[xdt]), dev(Bp),
+               ent, win, status, hca=(m == 128))
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    g_lo, g_hi = tok_begin // m, tok_end // m
+    x_pos0 = tok_begin - (G - m)
+    for b in range(B):
+        want = compress_entries(x[b], x_pos0, Wg, Bp, m, G, range(g_lo, g_hi))
+        d, s = download(ent, b)
+        got = storage.Stored(fmt, d[g_lo:g_hi], None if s is None else s[g_lo:g_hi], dim, rope)
+        got_v = storage.decode(got)
+        if fmt == "f32":
+            assert rel_l2(got_v, want) <= FP32_RTOL
+        else:
+            assert rel_l2(got_v, want) <= Q_RTOL
+            # codes are decided in float32 on both sides: nearly all agree
+            st = storage.encode(fmt, want, rope)
+            same = np.mean(np.all(st.payload == got.payload, axis=1))
+            assert same > 0.9, f"only {same:.3f} of rows identical"
+        # untouched rows stay zero
+        assert not np.any(d[:g_lo]) and not np.any(d[g_hi:])
+        if win is not None:
+            wd, ws_ = download(win, b)
+            lo = max(tok_begin, tok_end - 64)
+            for pos in range(lo, tok_end):
+                st = storage.encode(fmt, x[b][pos - x_pos0][None], rope)
+                assert np.array_equal(wd[pos % 64], st.payload[0])
+
+
+# ----------------------------------------------------------- index + top-k
+
+@pytest.mark.parametrize("fmt", ["f32", "fp8", "fp4"])
+def test_index_topk_matches_oracle(cuda_lib, fmt):
+    rng = np.random.default_rng(21)
+    if fmt == "f32":
+        wl = W.CSA_DECODE_4K_F32.with_(k=64)
+    else:
+        wl = W.CSA_DECODE_128K.with_(idx_fmt=fmt, k=300)
+    H_I, d_I, m = wl.H_I, wl.d_I, wl.m
+    T = 3
+    lengths = [4 * 5000 + 3, 4 * 37, 4 * 2100 + 1]  # one list shorter than k
+    B = len(lengths)
+    n_cap = max(lengths) // m + 1
+    keys_v = _rows(rng, B * n_cap, d_I).reshape(B, n_cap, d_I)
+    keys_v[0, 100:110] = keys_v[0, 99]                 # a run of equal keys
+    qi = (rng.standard_normal((B, T, H_I, d_I)) * d_I ** -0.5).astype(np.float32)
+    if wl.q_dtype == "bf16":
+        qi = torch.from_numpy(qi).to(torch.bfloat16).float().numpy()
+    wi = (np.abs(rng.standard_normal((B, T, H_I))) * H_I ** -0.5).astype(np.float32)
+    wi[2] *= np.where(rng.random(H_I) < 0.3, -1, 1).astype(np.float32)  # signed weights
+    p = L.params(wl)
+    keys = L.DeviceCache(B, n_cap, fmt, d_I)
+    sts = []
+    for b in range(B):
+        st = storage.encode(fmt, keys_v[b])
+        sts.append(st)
+        upload(keys, b, st)
+    ctx = torch.tensor(lengths, dtype=torch.int32, device="cuda")
+    out_idx = torch.full((B, T, wl.k), -5, dtype=torch.int32, device="cuda")
+    out_sc = torch.zeros((B, T, wl.k), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.index_topk(p, dev(qi, TORCH_DT[wl.q_dtype]), dev(wi), keys, ctx, n_cap, out_idx, out_sc, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    oi, osc = out_idx.cpu().numpy(), out_sc.cpu().numpy()
+    for b in range(B):
+        k_all = storage.decode(sts[b])
+        for t in range(T):
+            p_pos = lengths[b] - T + t
+            n = (p_pos + 1) // m
+            s = oracle_scores(quantize_query(qi[b, t], fmt), wi[b, t], k_all[:n])
+            ok, msg = topk_set_ok(oi[b, t], s, wl.k)
+            assert ok, f"b={b} t={t}: {msg}"
+            k_eff = min(wl.k, n)
+            assert np.all(oi[b, t, k_eff:] == -1)
+            sel = oi[b, t, :k_eff]
+            assert np.allclose(osc[b, t, :k_eff], s[sel], rtol=1e-5, atol=1e-6 * np.abs(s).max())
+
+
+# -------------------------------------------------------------- attention
+
+def _attn_case(kind, fmt_kv, rng):
+    if fmt_kv == "f32":
+        wl = W.CSA_DECODE_4K_F32.with_(k=64, w=40)
+    else:
+        wl = W.CSA_DECODE_128K.with_(k=200, w=100)
+    if kind == "hca":
+        wl = wl.with_(kind="hca", m=16, G=16)
+    return wl
+
+
+@pytest.mark.parametrize("kind", ["csa", "hca"])
+@pytest.mark.parametrize("fmt_kv", ["f32", "kv"])
+def test_attention_matches_oracle(cuda_lib, kind, fmt_kv):
+    rng = np.random.default_rng(31)
+    wl = _attn_case(kind, fmt_kv, rng)
+    T = 2
+    lengths = [3000, 30, 1500]                 # one context shorter than the window
+    B = len(lengths)
+    wl = wl.with_(T=T)
+    m, D, Dv, H = wl.m, wl.D, wl.Dv, wl.H
+    rope = wl.rope_dim if fmt_kv == "kv" else 0
+    n_cap = max(lengths) // m + 1
+    cap = wl.win_cap
+    sep = wl.separate_v
+    kv = L.DeviceCache(B, n_cap, fmt_kv, D, rope)
+    v = L.DeviceCache(B, n_cap, fmt_kv, Dv, rope) if sep else None
+    wk = L.DeviceCache(B, cap, fmt_kv, D, rope)
+    wv = L.DeviceCache(B, cap, fmt_kv, Dv, rope) if sep else None
+    st = {}
+    for b in range(B):
+        st[b] = {"kv": storage.encode(fmt_kv, _rows(rng, n_cap, D), rope),
+                 "wk": storage.encode(fmt_kv, _rows(rng, cap, D), rope)}
+        upload(kv, b, st[b]["kv"])
+        upload(wk, b, st[b]["wk"])
+        if sep:
+            st[b]["v"] = storage.encode(fmt_kv, _rows(rng, n_cap, Dv), rope)
+            st[b]["wv"] = storage.encode(fmt_kv, _rows(rng, cap, Dv), rope)
+            upload(v, b, st[b]["v"])
+            upload(wv, b, st[b]["wv"])
+    q = (rng.standard_normal((B, T, H, D)) * D ** -0.5 * 8).astype(np.float32)
+    if wl.q_dtype == "bf16":
+        q = torch.from_numpy(q).to(torch.bfloat16).float().numpy()
+    sink = rng.standard_normal(H).astype(np.float32)
+    ctx = torch.tensor(lengths, dtype=torch.int32, device="cuda")
+    out = torch.zeros((B, T, H, Dv), dtype=TORCH_DT[wl.q_dtype], device="cuda")
+    lse = torch.zeros((B, T, H), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    p = L.params(wl)
+    idx = None
+    if kind == "csa":
+        idx = np.full((B, T, wl.k), -1, dtype=np.int32)
+        for b in range(B):
+            for t in range(T):
+                n = (lengths[b] - T + t + 1) // m
+                k_eff = min(wl.k, n)
+                idx[b, t, :k_eff] = rng.permutation(n)[:k_eff]
+        L.sparse_attn(p, dev(q, TORCH_DT[wl.q_dtype]), kv, v, wk, wv, dev(idx, torch.int32), dev(sink), ctx,
+                      out, lse, status=status)
+    else:
+        L.dense_attn(p, dev(q, TORCH_DT[wl.q_dtype]), kv, v, wk, wv, dev(sink), ctx, n_cap, out, lse,
+                     status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    o_gpu, lse_gpu = out.float().cpu().numpy(), lse.cpu().numpy()
+    for b in range(B):
+        K_all = storage.decode(st[b]["kv"])
+        V_all = storage.decode(st[b]["v"]) if sep else K_all
+        WK = storage.decode(st[b]["wk"])
+        WV = storage.decode(st[b]["wv"]) if sep else WK
+        for t in range(T):
+            pp = lengths[b] - T + t
+            n = (pp + 1) // m
+            ent = idx[b, t][idx[b, t] >= 0] if kind == "csa" else np.arange(n)
+            wpos = window_positions(pp, wl.w) % cap
+            Kr = np.concatenate([K_all[ent], WK[wpos]])
+            Vr = np.concatenate([V_all[ent], WV[wpos]])
+            o, ls = joint_attention(q[b, t], Kr, Vr, sink, wl.sm_scale)
+            assert rel_l2(o_gpu[b, t], o) <= ATTN_RTOL, (b, t, rel_l2(o_gpu[b, t], o))
+            assert max_abs(o_gpu[b, t], o) <= ATTN_ATOL
+            assert np.allclose(lse_gpu[b, t], ls, rtol=1e-4, atol=1e-4)
+
+
+def test_attention_flags_out_of_range_index(cuda_lib):
+    rng = np.random.default_rng(41)
+    wl = W.CSA_DECODE_4K_F32.with_(k=8, w=4)
+    B, T, H, D = 1, 1, wl.H, wl.D
+    n_cap = 64
+    kv = L.DeviceCache(B, n_cap, "f32", D)
+    v = L.DeviceCache(B, n_cap, "f32", D)
+    wk = L.DeviceCache(B, wl.win_cap, "f32", D)
+    wv = L.DeviceCache(B, wl.win_cap, "f32", D)
+    for c in (kv, v, wk, wv):
+        c.data.copy_(torch.from_numpy(_rows(rng, c.capacity, D)).cuda()[None])
+    ctx = torch.tensor([40], dtype=torch.int32, device="cuda")  # N = 10 visible entries
+    idx = torch.tensor([[[0, 3, 9, 10, 500, -1, -3, 2]]], dtype=torch.int32, device="cuda")
+    q = dev(_rows(rng, H, D)[None, None])
+    out = torch.zeros((B, T, H, D), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.sparse_attn(L.params(wl), q, kv, v, wk, wv, idx, None, ctx, out, None, status=status)
+    torch.cuda.synchronize()
+    assert status.item() & L.DEV_BAD_INDEX
+    # the result equals attention over the valid indices alone
+    Kn, Vn = kv.data[0].cpu().double().numpy(), v.data[0].cpu().double().numpy()
+    Wk, Wv = wk.data[0].cpu().double().numpy(), wv.data[0].cpu().double().numpy()
+    wpos = window_positions(39, 4) % wl.win_cap
+    ent = [0, 3, 9, 2]
+    o, _ = joint_attention(q[0, 0].cpu().double().numpy(), np.concatenate([Kn[ent], Wk[wpos]]),
+                           np.concatenate([Vn[ent], Wv[wpos]]), np.full(H, -np.inf), wl.sm_scale)
+    assert rel_l2(out[0, 0].cpu().numpy(), o) < 1e-5

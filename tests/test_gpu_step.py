@@ -1,0 +1,84 @@
+"""Parity of the fused decode / chunked-prefill steps (lcsc_csa_decode,
+lcsc_hca_decode) with the oracle's step, on scaled-down workloads with
+ragged batches (different context lengths per sequence)."""
+import numpy as np
+import pytest
+import torch
+
+from long_context_sparse_compress_b200 import workloads as W
+from oracle import storage
+from tests.gpu_harness import GpuBatch, download, make_seqs
+from tests.harness import max_abs, rel_l2, topk_set_ok
+from oracle.indexer import quantize_query, scores as oracle_scores
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    # name: (workload, per-sequence context lengths)
+    "csa_f32_decode": (W.CSA_DECODE_4K_F32.with_(B=3), [4096, 1000, 101]),
+    "csa_fp8_decode": (W.CSA_DECODE_128K.with_(B=3), [8192, 4100, 300]),
+    "csa_fp4_decode": (W.PAIR_DECODE_1M_B1.layer("csa").with_(B=2, n_planted=16), [16384, 6000]),
+    "hca_decode": (W.HCA_DECODE_64K.with_(B=3), [4096, 1024 + 128, 100]),
+    "csa_fp8_prefill": (W.CSA_PREFILL_256K.with_(B=2, T=40, n_planted=8), [4096 + 40, 2002]),
+    "hca_prefill": (W.HCA_DECODE_64K.with_(B=1, T=130), [4096 + 130]),
+    "csa_overlap_decode": (W.CSA_DECODE_128K.with_(B=2, G=8), [8192, 1001]),
+}
+
+
+def check_step(name, wl, lengths, query_sample=None):
+    seqs = make_seqs(wl, lengths)
+    gb = GpuBatch(seqs)
+    gb.run_step()
+    assert gb.status.item() == 0
+    o_gpu = gb.out.float().cpu().numpy()
+    lse_gpu = gb.lse.cpu().numpy()
+    sel_gpu = gb.out_idx.cpu().numpy() if gb.out_idx is not None else None
+    for b, s in enumerate(seqs):
+        qs = query_sample if query_sample is not None else list(range(wl.T))
+        ref = s.step(queries=qs)
+        # new entries and window rows were stored like the oracle stores them
+        g_lo, g_hi = ref["new_entries"]
+        d, sc = download(gb.kv, b)
+        if g_hi > g_lo:
+            got = storage.decode(storage.Stored(s.kv.fmt, d[g_lo:g_hi], None if sc is None else sc[g_lo:g_hi],
+                                                s.kv.dim, s.kv.rope_dim))
+            want = storage.decode(s.kv.rows(slice(g_lo, g_hi)))
+            assert rel_l2(got, want) <= (1e-5 if s.kv.fmt == "f32" else 1e-2)
+        wd, _ = download(gb.win_kv, b)
+        for pos in range(s.wl.L - wl.T, s.wl.L):
+            r = pos % wl.win_cap
+            if s.kv.fmt == "f32":
+                assert np.array_equal(wd[r], s.ring_kv.payload[r])
+            else:
+                assert np.array_equal(wd[r], s.ring_kv.payload[r]), f"ring row {pos}"
+        for j, i in enumerate(qs):
+            o = ref["o"][j]
+            assert rel_l2(o_gpu[b, i], o) <= 1e-2, (name, b, i, rel_l2(o_gpu[b, i], o))
+            assert max_abs(o_gpu[b, i], o) <= 2e-2
+            assert np.allclose(lse_gpu[b, i], ref["lse"][j], rtol=1e-3, atol=1e-3)
+            if sel_gpu is not None:
+                p = s.wl.L - wl.T + i
+                n = (p + 1) // wl.m
+                k_all = storage.decode(s.idx.rows(slice(0, n)))
+                sc_all = oracle_scores(quantize_query(s.inp["q_idx"][i], wl.idx_fmt), s.inp["w_idx"][i], k_all)
+                ok, msg = topk_set_ok(sel_gpu[b, i], sc_all, wl.k)
+                assert ok, (name, b, i, msg)
+                if len(s.inp["planted"]) and n > len(s.inp["planted"]):
+                    assert set(s.inp["planted"].tolist()) <= set(sel_gpu[b, i].tolist())
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_fused_step_matches_oracle(cuda_lib, name):
+    wl, lengths = CASES[name]
+    sample = None if wl.T <= 8 else [0, 1, wl.T // 2, wl.T - 2, wl.T - 1]
+    check_step(name, wl, lengths, sample)
+
+
+def test_step_twice_is_deterministic(cuda_lib):
+    wl = W.CSA_DECODE_128K.with_(B=2)
+    gb = GpuBatch(make_seqs(wl, [8192, 5000]))
+    gb.run_step()
+    o1, i1 = gb.out.clone(), gb.out_idx.clone()
+    gb.run_step()
+    assert torch.equal(gb.out, o1)
+    assert torch.equal(torch.sort(gb.out_idx, dim=-1).values, torch.sort(i1, dim=-1).values)
