@@ -280,10 +280,72 @@ __global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int sl
   if (blockIdx.x == 0 && threadIdx.x == 0) ctr[2] = th.above;
 }
 
+// Smallest index bound tau such that at least `need` of the tied candidates
+// (key == tkey) have index < tau: ties then go to the lowest indices, as in
+// a stable sort.  512 threads; returns n when every tied candidate is needed.
+__device__ uint32_t tie_bound(const uint32_t* cand, uint32_t n_cand, const float* s, uint32_t tkey,
+                              uint32_t need, uint32_t n, uint32_t* cnt) {
+  uint32_t lo = 0, hi = n;  // count(idx < hi) >= need holds for hi = n
+  while (lo < hi) {
+    const uint32_t mid = lo + (hi - lo) / 2;
+    if (threadIdx.x == 0) *cnt = 0;
+    __syncthreads();
+    uint32_t local = 0;
+    for (uint32_t c = threadIdx.x; c < n_cand; c += 512) {
+      const uint32_t g = cand[c];
+      local += (g < mid && float_key(s[g]) == tkey) ? 1u : 0u;
+    }
+    if (local) atomicAdd(cnt, local);
+    __syncthreads();
+    const uint32_t total = *cnt;
+    __syncthreads();
+    if (total >= need) hi = mid;
+    else lo = mid + 1;
+  }
+  return lo;
+}
+
+// Sort the k_eff selected (index, score) pairs by index, in shared memory
+// (bitonic network over the next power of two, <= 2048).
+__device__ void sort_selection(int32_t* out_i, float* out_s, int k_eff, int32_t* si, float* sv) {
+  int P = 1;
+  while (P < k_eff) P <<= 1;
+  for (int j = threadIdx.x; j < P; j += 512) {
+    si[j] = j < k_eff ? out_i[j] : INT32_MAX;
+    sv[j] = (j < k_eff && out_s) ? out_s[j] : 0.f;
+  }
+  __syncthreads();
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int j = threadIdx.x; j < P; j += 512) {
+        const int partner = j ^ stride;
+        if (partner > j) {
+          const bool up = (j & size) == 0;
+          const int32_t a = si[j], b = si[partner];
+          if ((a > b) == up) {
+            si[j] = b;
+            si[partner] = a;
+            const float t = sv[j];
+            sv[j] = sv[partner];
+            sv[partner] = t;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int j = threadIdx.x; j < k_eff; j += 512) {
+    out_i[j] = si[j];
+    if (out_s) out_s[j] = sv[j];
+  }
+}
+
 __global__ void __launch_bounds__(512) topk_final_kernel(IndexLaunch a) {
   __shared__ uint32_t h[kBins];
   __shared__ uint32_t scratch[512];
-  __shared__ uint32_t tie_ctr;
+  __shared__ uint32_t cnt;
+  __shared__ int32_t si[2048];
+  __shared__ float sv[2048];
   const int list = blockIdx.x;
   bool ok;
   const int64_t n = visible(a, list / a.T, list % a.T, &ok);
@@ -295,7 +357,7 @@ __global__ void __launch_bounds__(512) topk_final_kernel(IndexLaunch a) {
     out_i[j] = -1;
     if (out_s) out_s[j] = -INFINITY;
   }
-  if (n <= a.k) return;
+  if (n <= a.k) return;  // every visible entry was written in order by the collect pass
   uint32_t* ctr = a.counters + (int64_t)list * 4;
   const uint32_t above1 = ctr[2];
   const uint32_t n_cand = ctr[1];
@@ -304,7 +366,6 @@ __global__ void __launch_bounds__(512) topk_final_kernel(IndexLaunch a) {
   const float* s = a.scores + (int64_t)list * a.n_max;
   uint32_t* gh2 = a.hist + (int64_t)list * 2 * kBins + kBins;
   for (int i = threadIdx.x; i < kBins; i += 512) h[i] = gh2[i];
-  if (threadIdx.x == 0) tie_ctr = 0;
   __syncthreads();
   const Thresh t2 = find_threshold(h, need, scratch);
   for (int i = threadIdx.x; i < kBins; i += 512) h[i] = 0;
@@ -327,20 +388,37 @@ __global__ void __launch_bounds__(512) topk_final_kernel(IndexLaunch a) {
   const uint32_t need3 = need - t2.above;
   const Thresh t3 = find_threshold(h, need3, scratch);
   const uint32_t ties = need3 - t3.above;
+  const uint32_t n_tied = h[t3.bin];
+  __syncthreads();
+  // the threshold key itself: candidate digit 1 is shared; rebuild it from any tied element
+  uint32_t tau = (uint32_t)n;
+  if (n_tied > ties) {
+    // every tied element has the same full key: digit 1 | digit 2 | digit 3
+    __shared__ uint32_t tkey;
+    if (threadIdx.x == 0) tkey = 0xFFFFFFFFu;
+    __syncthreads();
+    for (uint32_t c = threadIdx.x; c < n_cand; c += 512) {
+      const uint32_t key = float_key(s[cand[c]]);
+      if (((key >> 8) & 0xFFF) == t2.bin && (key & 0xFF) == t3.bin) atomicMin(&tkey, key);
+    }
+    __syncthreads();
+    tau = tie_bound(cand, n_cand, s, tkey, ties, (uint32_t)n, &cnt);
+  }
   for (uint32_t c = threadIdx.x; c < n_cand; c += 512) {
     const uint32_t g = cand[c];
     const float v = s[g];
     const uint32_t key = float_key(v);
     if (((key >> 8) & 0xFFF) != t2.bin) continue;
     const uint32_t d3 = key & 0xFF;
-    bool take = d3 > t3.bin;
-    if (d3 == t3.bin) take = atomicAdd(&tie_ctr, 1u) < ties;
-    if (take) {
+    if (d3 > t3.bin || (d3 == t3.bin && g < tau)) {
       const uint32_t slot = atomicAdd(&ctr[0], 1u);
       out_i[slot] = (int32_t)g;
       if (out_s) out_s[slot] = v;
     }
   }
+  __threadfence_block();
+  __syncthreads();
+  sort_selection(out_i, out_s, (int)k_eff, si, sv);
 }
 
 }  // namespace

@@ -1,6 +1,8 @@
 """Per-stage parity of the CUDA library against the oracle (small shapes that
 still span several tiles and ragged tails).  Every input is seeded; every
 expected value comes from ``oracle/``."""
+import zlib
+
 import numpy as np
 import pytest
 import torch
@@ -79,7 +81,7 @@ COMPRESS_CASES = {
 @pytest.mark.parametrize("with_window", [False, True])
 def test_compress_matches_oracle(cuda_lib, case, with_window):
     fmt, tensor, m, G, dim, xdt = COMPRESS_CASES[case]
-    rng = np.random.default_rng(hash(case) % 2 ** 31)
+    rng = np.random.default_rng(zlib.crc32(case.encode()))
     B = 3
     tok_begin = 0 if m == 128 else 8 * m
     n_entries = 5 if m == 128 else 70            # > 2 CTAs of 32 entries, ragged
@@ -116,11 +118,13 @@ def test_compress_matches_oracle(cuda_lib, case, with_window):
         if fmt == "f32":
             assert rel_l2(got_v, want) <= FP32_RTOL
         else:
-            assert rel_l2(got_v, want) <= Q_RTOL
-            # codes are decided in float32 on both sides: nearly all agree
+            # stored values: the oracle stores its own pooled rows by the same rule
             st = storage.encode(fmt, want, rope)
-            same = np.mean(np.all(st.payload == got.payload, axis=1))
-            assert same > 0.9, f"only {same:.3f} of rows identical"
+            assert rel_l2(got_v, storage.decode(st)) <= Q_RTOL
+            # codes are decided in float32 on both sides: nearly all agree (a
+            # pooled value within a float32 rounding of a code boundary may flip)
+            same = np.mean(st.payload == got.payload)
+            assert same > 0.99, f"only {same:.4f} of stored bytes identical"
         # untouched rows stay zero
         assert not np.any(d[:g_lo]) and not np.any(d[g_hi:])
         if win is not None:
