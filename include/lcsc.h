@@ -185,6 +185,31 @@ int32_t lcsc_csa_index_topk(const lcsc_params* p, const void* q_idx, const float
                             void* workspace, size_t workspace_bytes, int32_t* status,
                             void* stream);
 
+/* The same indexer + top-k call for callers that cannot allocate device
+ * memory: hosts that hand every byte of device memory to their own pool up
+ * front, or callers reaching this library through a foreign-function
+ * interface with no device allocator.  (No counterpart in the paper: it is
+ * an interface of this library.)
+ *  - Arguments and results are those of lcsc_csa_index_topk, minus the
+ *    workspace; no call allocates or frees device memory.
+ *  - Scratch: one static device array of LCSC_NOALLOC_SCRATCH_BYTES (40 MiB)
+ *    inside the library, which every device that loads the library holds
+ *    until the process exits.  A request whose scratch
+ *    (lcsc_index_topk_workspace_size) exceeds it returns LCSC_ERR_WORKSPACE
+ *    and enqueues nothing (B = 16, T = 1, n_max = 262144 fits).
+ *  - The first call on a device looks up the array's device address (once
+ *    per device, with that device current); make that first call before any
+ *    stream capture.
+ *  - Every call on a device shares the array, which keeps the last call's
+ *    contents (each call clears what must start at zero): calls that overlap
+ *    on the GPU (other streams, other host threads) race and give wrong
+ *    results; serialise them. */
+#define LCSC_NOALLOC_SCRATCH_BYTES (40ll << 20)
+int32_t lcsc_csa_index_topk_noalloc(const lcsc_params* p, const void* q_idx, const float* w_idx,
+                                    const lcsc_cache* idx_keys, const int32_t* ctx_len, int64_t B,
+                                    int64_t T, int64_t n_max, int32_t* out_idx, float* out_score,
+                                    int32_t* status, void* stream);
+
 /* --------------------------------------------------------- attention (a5-a7)
  * One joint softmax per query head over a row set S (entries plus window
  * rows), with a per-head sink logit sigma[h] that only adds exp(sigma) to

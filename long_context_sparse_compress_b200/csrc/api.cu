@@ -556,3 +556,65 @@ int32_t lcsc_hca_decode(const lcsc_params* p, const lcsc_step* s, void* ws, size
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// lcsc_csa_index_topk_noalloc: the indexer + top-k call for callers that
+// cannot allocate device memory.  Its scratch is one fixed array in this
+// file's module; the caller still passes every input and output.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace lcsc {
+namespace {
+
+// Scratch of the no-allocation entry point.  Every device that loads this
+// library holds it until the process exits.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[LCSC_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  The name of the
+// array in host code is a host-side stand-in, so the address is fetched
+// once per device with cudaGetSymbolAddress (with that device current).
+int32_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return LCSC_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return LCSC_OK;
+}
+
+}  // namespace
+}  // namespace lcsc
+
+extern "C" int32_t lcsc_csa_index_topk_noalloc(const lcsc_params* p, const void* q_idx,
+                                               const float* w_idx, const lcsc_cache* idx_keys,
+                                               const int32_t* ctx_len, int64_t B, int64_t T,
+                                               int64_t n_max, int32_t* out_idx, float* out_score,
+                                               int32_t* status, void* stream) {
+  int32_t st = check_params(p);
+  if (st) return st;
+  if (B < 1 || T < 1 || n_max < 0) return LCSC_ERR_INVALID_ARG;
+  Carve need{nullptr};
+  plan_index(p, B, T, n_max, need, nullptr);
+  if (need.used > (size_t)LCSC_NOALLOC_SCRATCH_BYTES) return LCSC_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch))) return st;
+  Carve cv{reinterpret_cast<uint8_t*>(scratch)};
+  IndexLaunch L;
+  if ((st = index_setup(p, q_idx, w_idx, idx_keys, ctx_len, B, T, n_max, out_idx, out_score, cv,
+                        (size_t)LCSC_NOALLOC_SCRATCH_BYTES, status, &L)))
+    return st;
+  cudaError_t e = launch_index_topk(L, (cudaStream_t)stream);
+  return e == cudaSuccess ? LCSC_OK : cuda_fail(e);
+}

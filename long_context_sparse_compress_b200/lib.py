@@ -60,6 +60,8 @@ _SIGS = {
     "lcsc_index_topk_workspace_size": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp]),
     "lcsc_csa_index_topk": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_vp, c_vp,
                                     c_vp, c_sz, c_vp, c_vp]),
+    "lcsc_csa_index_topk_noalloc": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_vp,
+                                            c_vp, c_vp, c_vp]),
     "lcsc_attn_workspace_size": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_i32, c_vp]),
     "lcsc_csa_sparse_attn": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i64,
                                      c_i64, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
@@ -214,6 +216,20 @@ def index_topk(p, q_idx, w_idx, keys, ctx_len, n_max, out_idx, out_score=None, w
                                   ptr(ctx_len), B, T, n_max, ptr(out_idx), ptr(out_score), ptr(ws),
                                   ws.numel(), ptr(status), stream_handle(stream)))
     return ws
+
+
+NOALLOC_SCRATCH_BYTES = 40 << 20
+
+
+def index_topk_noalloc(p, q_idx, w_idx, keys, ctx_len, n_max, out_idx, out_score=None, status=None,
+                       stream=None):
+    """lcsc_csa_index_topk_noalloc: same results, no workspace argument; the
+    library's fixed scratch is used (one call at a time per device)."""
+    lib = load()
+    B, T = q_idx.shape[0], q_idx.shape[1]
+    check(lib.lcsc_csa_index_topk_noalloc(ctypes.byref(p), ptr(q_idx), ptr(w_idx), ctypes.byref(keys.c()),
+                                          ptr(ctx_len), B, T, n_max, ptr(out_idx), ptr(out_score),
+                                          ptr(status), stream_handle(stream)))
 
 
 def attn_workspace(p, B, T, n_max, dense):
