@@ -79,7 +79,7 @@ class Layer:
         self.w_ik = rn((wl.d_I, wl.d_I), 0.02).to(xdt) if csa else None
         self.b_ik = rn((wl.G, wl.d_I), 1.0) if csa else None
         self.kv = L.DeviceCache(B, n_cap, wl.kv_fmt, D, rope, device)
-        self.idx = L.DeviceCache(B, n_cap, wl.idx_fmt, wl.d_I, 0, device) if csa else None
+        self.idx = L.DeviceCache(B, L.round_capacity(n_cap, wl.idx_fmt), wl.idx_fmt, wl.d_I, 0, device) if csa else None
         self.win = L.DeviceCache(B, wl.win_cap, wl.kv_fmt, D, rope, device)
         R = synth.tail_rows(wl)
         tail_kv = rn((B, R, D), D ** -0.5).to(xdt)

@@ -55,7 +55,8 @@ extern "C" {
 
 /* Bits OR-ed into *status on the device. */
 #define LCSC_DEV_BAD_INDEX 1       /* an index outside [0, N(p)) was skipped */
-#define LCSC_DEV_BAD_LENGTH 2      /* a ctx_len smaller than T, or a window larger than the ring */
+#define LCSC_DEV_BAD_LENGTH 2      /* a ctx_len smaller than T, or past the sizes of the call */
+#define LCSC_DEV_TIMEOUT 4         /* a kernel gave up a bounded wait (no result was written) */
 
 /* Row storage formats ("DeepSeek V4 Architecture Explained", Key numbers,
  * row "KV storage precision"; "Inside DeepSeek-V4", section 1, FP4 indexer).
@@ -107,8 +108,12 @@ typedef struct lcsc_params {
 
 /* Stored rows of one tensor for B sequences (dev pointers).
  *   data:  [B][capacity][row bytes of the format]
- *   scale: [B][capacity] float32 (KV, FP8) or [B][capacity][dim/16] uint8
- *          (FP4); NULL for F32.
+ *   scale: [B][capacity] float32 (KV, FP8); NULL for F32; for FP4 uint8
+ *          block scales tiled by 128 rows, the order the tensor cores read
+ *          them: [B][ceil(capacity / 128)][dim / 64][32][4][4], the byte of
+ *          row r, 16-value block k at
+ *          [b][r / 128][k / 4][r % 32][(r % 128) / 32][k % 4].
+ *   Indexer keys in FP8 / FP4 need a capacity that is a multiple of 128.
  * Compressed entries use row g for entry g.  A window ring uses row
  * (position mod capacity). */
 typedef struct lcsc_cache {

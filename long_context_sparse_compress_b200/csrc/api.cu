@@ -32,6 +32,18 @@ struct Carve {
 
 bool valid_format(int fmt) { return fmt >= LCSC_FMT_F32 && fmt <= LCSC_FMT_FP4; }
 
+// SMs of the current device (for sizing grids that fill it); 148 when the
+// host has no device (sizes then only matter for workspace queries).
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
+
 int32_t check_params(const lcsc_params* p) {
   if (!p) return LCSC_ERR_INVALID_ARG;
   if (p->m < 1 || p->group_len < p->m || p->group_len > 2 * p->m) return LCSC_ERR_INVALID_ARG;
@@ -96,7 +108,8 @@ void plan_index(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max, Carve
   uint8_t* qdata = cv.take<uint8_t>((size_t)qrows * rb);
   void* qscale = nullptr;
   if (p->idx_format == LCSC_FMT_FP8) qscale = cv.take<float>((size_t)qrows);
-  else if (p->idx_format == LCSC_FMT_FP4) qscale = cv.take<uint8_t>((size_t)qrows * (p->idx_dim / 16));
+  else if (p->idx_format == LCSC_FMT_FP4)  // block scales tiled by 128 rows per sequence
+    qscale = cv.take<uint8_t>((size_t)B * ((T * p->idx_heads + 127) / 128) * (p->idx_dim / 64) * 512);
   float* scores = cv.take<float>((size_t)lists * n_max);
   uint32_t* hist = cv.take<uint32_t>((size_t)lists * 2 * 4096);
   uint32_t* ctr = cv.take<uint32_t>((size_t)lists * 4);
@@ -116,9 +129,14 @@ void plan_index(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max, Carve
 void plan_attn(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max, bool dense, Carve& cv,
                AttnLaunch* L) {
   const int64_t max_rows = (dense ? n_max : p->top_k) + p->window;
-  const int hpc = p->kv_format == LCSC_FMT_F32 ? 8 : 16;
   int splits, rps;
-  attention_splits(max_rows, B * T * (p->n_heads / hpc), &splits, &rps);
+  if (p->kv_format == LCSC_FMT_KV && p->head_dim == 512 && p->n_heads == 64) {
+    // tensor-core path: one CTA per (query, split) for all heads, one wave
+    attention_splits(max_rows, B * T, 128, sm_count(), &splits, &rps);
+  } else {
+    const int hpc = p->kv_format == LCSC_FMT_F32 ? 8 : 16;
+    attention_splits(max_rows, B * T * (p->n_heads / hpc), 32, 2 * sm_count(), &splits, &rps);
+  }
   float* po = cv.take<float>((size_t)B * T * splits * p->n_heads * p->v_dim);
   float* pml = cv.take<float>((size_t)B * T * splits * p->n_heads * 2);
   if (L) {
@@ -289,6 +307,7 @@ static int32_t index_setup(const lcsc_params* p, const void* q_idx, const float*
   memset(L, 0, sizeof(*L));
   if ((st = make_view(idx_keys, f, needs_scale(f.fmt), &L->keys))) return st;
   if (n_max > idx_keys->capacity) return LCSC_ERR_INVALID_ARG;
+  if (f.fmt != LCSC_FMT_F32 && idx_keys->capacity % 128 != 0) return LCSC_ERR_INVALID_ARG;
   plan_index(p, B, T, n_max, cv, L);
   if (!cv.base || !aligned16(cv.base) || ws_bytes < cv.used) return LCSC_ERR_WORKSPACE;
   L->q_idx = q_idx;

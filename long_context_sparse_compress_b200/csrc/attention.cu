@@ -272,19 +272,26 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
 
 }  // namespace
 
-void attention_splits(int64_t max_rows, int64_t n_ctas_per_split, int* splits, int* rows_per_split) {
+void attention_splits(int64_t max_rows, int64_t n_ctas_per_split, int granule, int target_ctas, int* splits,
+                      int* rows_per_split) {
   if (max_rows < 1) max_rows = 1;
-  const int64_t tiles = (max_rows + kTile - 1) / kTile;
-  int64_t s = (2 * 148 + n_ctas_per_split - 1) / n_ctas_per_split;
+  const int64_t tiles = (max_rows + granule - 1) / granule;
+  int64_t s = target_ctas / (n_ctas_per_split > 0 ? n_ctas_per_split : 1);
   if (s < 1) s = 1;
   if (s > tiles) s = tiles;
-  int64_t rps = ((max_rows + s - 1) / s + kTile - 1) / kTile * kTile;
+  int64_t rps = ((max_rows + s - 1) / s + granule - 1) / granule * granule;
   *rows_per_split = (int)rps;
   *splits = (int)((max_rows + rps - 1) / rps);
 }
 
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
   const bool sep = a.v.data != nullptr;
+  if (attn_mma_supported(a)) {
+    cudaError_t e = launch_attn_mma(a, stream);
+    if (e != cudaSuccess) return e;
+    attn_combine_kernel<512><<<dim3(a.B * a.T, a.H), 512, 0, stream>>>(a);
+    return cudaGetLastError();
+  }
   if (a.kv.f.fmt == LCSC_FMT_F32 && a.D == 128 && a.Dv == 128 && a.H % 8 == 0) {
     if (sep) return launch_attn<LCSC_FMT_F32, 128, 128, 8, true>(a, stream);
     return launch_attn<LCSC_FMT_F32, 128, 128, 8, false>(a, stream);

@@ -45,8 +45,16 @@ struct CacheView {
   __device__ __forceinline__ float* fscale(int b, int64_t r) const {
     return reinterpret_cast<float*>(scale) + (int64_t)b * capacity + r;
   }
-  __device__ __forceinline__ uint8_t* bscale(int b, int64_t r) const {
-    return reinterpret_cast<uint8_t*>(scale) + ((int64_t)b * capacity + r) * (f.dim / 16);
+  // FP4 block scales are tiled by 128 rows so that one tile's scales are one
+  // contiguous 512-byte chunk per 64 values of the row (the order the tensor
+  // cores read them in): byte of row r, block k =
+  //   [b][r / 128][k / 4][r % 32][(r % 128) / 32][k % 4].
+  __device__ __forceinline__ uint8_t* bscale_at(int b, int64_t r, int k) const {
+    const int64_t tiles = (capacity + 127) / 128;
+    const int64_t tile_bytes = (int64_t)(f.dim / 64) * 512;
+    const int m = (int)(r & 127);
+    return reinterpret_cast<uint8_t*>(scale) + ((int64_t)b * tiles + (r >> 7)) * tile_bytes + (k >> 2) * 512 +
+           (m & 31) * 16 + (m >> 5) * 4 + (k & 3);
   }
 };
 
@@ -191,7 +199,7 @@ __device__ __forceinline__ void store_row_warp(const CacheView& cv, int b, int64
 #pragma unroll
     for (int i = 0; i < VPL / 2; ++i) dst[e0 / 2 + i] = packed[i];
   }
-  if (lane % LPB == 0) cv.bscale(b, r)[e0 / 16] = sc;
+  if (lane % LPB == 0) *cv.bscale_at(b, r, e0 / 16) = sc;
 }
 
 // Dequantised value of element e of a stored row (slow path, any format).
@@ -207,7 +215,7 @@ __device__ __forceinline__ float stored_elem(const CacheView& cv, int b, int64_t
     case LCSC_FMT_FP8: return e4m3_val(row[e]) * *cv.fscale(b, r);
     case LCSC_FMT_FP4: {
       float2 v = e2m1x2_val(row[e >> 1]);
-      return ((e & 1) ? v.y : v.x) * e4m3_val(cv.bscale(b, r)[e >> 4]);
+      return ((e & 1) ? v.y : v.x) * e4m3_val(*cv.bscale_at(b, r, e >> 4));
     }
   }
   return 0.f;

@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(256) score_kernel(IndexLaunch a) {
     const int64_t qr = (int64_t)t * HI + h;
     float s = 1.f;
     if (FMT == LCSC_FMT_FP8) s = *a.q_store.fscale(b, qr);
-    else if (FMT == LCSC_FMT_FP4) s = e4m3_val(a.q_store.bscale(b, qr)[blk]);
+    else if (FMT == LCSC_FMT_FP4) s = e4m3_val(*a.q_store.bscale_at(b, qr, blk));
     sq[i] = s;
   }
   for (int i = tid; i < HI; i += 256) wq[i] = a.w_idx[(int64_t)list * HI + i];
@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(256) score_kernel(IndexLaunch a) {
           kv[2 * j] = f.x; kv[2 * j + 1] = f.y;
         }
       }
-      const float skb = FMT == LCSC_FMT_FP4 ? e4m3_val(a.keys.bscale(b, g)[blk]) : 1.f;
+      const float skb = FMT == LCSC_FMT_FP4 ? e4m3_val(*a.keys.bscale_at(b, g, blk)) : 1.f;
 #pragma unroll
       for (int i = 0; i < HPT; ++i) {
         const int h = i * HG + hg;
@@ -435,6 +435,7 @@ cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream) {
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
+  if (index_mma_supported(a)) return launch_index_mma(a, stream);
   dim3 sgrid((unsigned)((a.n_max + 63) / 64), lists);
   const int fmt = a.keys.f.fmt;
   if (fmt == LCSC_FMT_F32 && a.d_I == 32 && a.H_I == 4)

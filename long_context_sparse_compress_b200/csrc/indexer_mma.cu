@@ -1,0 +1,358 @@
+// Lightning-indexer scoring on the 5th-generation tensor cores.
+//
+// Method: "DeepSeek V4 Architecture Explained" (researchpapers.dev), "How
+// compress-then-sparsify attention works"; "Inside DeepSeek-V4"
+// (llmbytes.dev), section 1 (FP4 indexer):
+//   s[g] = sum_h w[h] * ReLU(q~[h] . k~[g])
+//
+// GEMM view: S[g][(t, h)] = K[g][:] . Q[(t, h)][:], keys on M (128 per tile),
+// the NQ queries' 64 heads on N, d_I = 128 on K.
+//  * FP4 keys and queries: tcgen05.mma kind::mxf4nvf4 with one UE4M3 scale
+//    per 16 values on both operands (the scales go smem -> TMEM with
+//    tcgen05.cp); the accumulator holds the exact dequantised dot products.
+//  * FP8 keys and queries: tcgen05.mma kind::f8f6f4 on the codes; the
+//    per-row scales are positive, so the epilogue applies them outside ReLU:
+//    s = sk[g] * sum_h (w[h] sq[h]) ReLU(acc[h]).
+// Warp roles (320 threads, one CTA per SM): warp 0 streams key tiles with TMA
+// (hardware swizzle) into a STAGES-deep ring, warp 1 issues the MMAs into
+// NACC TMEM accumulators, warps 2-9 (two groups of four taking alternate
+// tiles) drain them with tcgen05.ld, apply ReLU and the head weights, and
+// write one fp32 score per (query, key).
+#include <cudaTypedefs.h>
+
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace lcsc {
+namespace {
+
+using namespace sm100;
+
+struct MmaArgs {
+  const void* key_scale;   // FP8: float [B][cap]; FP4: tiled UE4M3 block scales
+  int64_t key_cap;         // rows per sequence (multiple of 128)
+  const uint8_t* q_scale;  // FP8: float [B][T*64]; FP4: tiled block scales (capacity T*64)
+  const float* w_idx;      // [B*T][64]
+  const int32_t* ctx_len;
+  int B, T, m;
+  int64_t n_max;
+  float* scores;           // [B*T][n_max]
+  int chunks;              // CTAs per (sequence, query group)
+  int32_t* status;
+};
+
+template <int FMT, int NQ>
+struct Cfg {
+  static constexpr int ROW = FMT == LCSC_FMT_FP4 ? 64 : 128;   // bytes per 128-value row
+  static constexpr int TILE = 128;                               // keys per tile (MMA M)
+  static constexpr int N = 64 * NQ;                              // MMA N
+  static constexpr int KSTEPS = 4 - (FMT == LCSC_FMT_FP4 ? 2 : 0);  // 32 bytes of K per MMA
+  // Ring depth: enough bytes in flight to cover DRAM latency, and more than
+  // half the shared memory so that a second CTA never shares the SM's TMEM.
+  static constexpr int STAGES = FMT == LCSC_FMT_FP4 ? 13 : (NQ == 1 ? 8 : 5);
+  // Accumulators in TMEM: the MMA runs up to NACC tiles ahead of the epilogue.
+  static constexpr int NACC = NQ == 1 ? 4 : 2;
+  static constexpr int A_BYTES = TILE * ROW;
+  static constexpr int SFA_BYTES = FMT == LCSC_FMT_FP4 ? 1024 : 0;
+  static constexpr int Q_BYTES = N * ROW;
+  static constexpr int SFB_BYTES = FMT == LCSC_FMT_FP4 ? ((N + 127) / 128) * 1024 : 0;
+  static constexpr Swizzle SW = FMT == LCSC_FMT_FP4 ? kSw64 : kSw128;
+  static constexpr int SBO = 8 * ROW;  // bytes between 8-row core-matrix groups
+  // TMEM: accumulators [0, NACC*N); FP4 also SFA (one 8-column buffer per
+  // accumulator) and SFB.
+  static constexpr int SFA_COL = NACC * N;
+  static constexpr int SFB_COL = NACC * N + 8 * NACC;
+  static constexpr int COLS_USED = NACC * N + (FMT == LCSC_FMT_FP4 ? 8 * NACC + 8 * ((N + 127) / 128) : 0);
+  static constexpr int TMEM_COLS = COLS_USED <= 32 ? 32 : COLS_USED <= 64 ? 64 : COLS_USED <= 128 ? 128
+                                   : COLS_USED <= 256 ? 256 : 512;
+  // shared memory (offsets from a 1024-aligned base)
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_Q = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_SFA = OFF_Q + Q_BYTES;
+  static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+  static constexpr int OFF_BAR = OFF_SFB + SFB_BYTES;
+  static constexpr int NBARS = 2 * STAGES + 2 * NACC + 1;
+  static constexpr int OFF_W = OFF_BAR + NBARS * 8;
+  static constexpr int OFF_TMEM = OFF_W + N * 4;
+  static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + slack to align the base
+  static_assert(COLS_USED <= 512, "TMEM budget");
+  static_assert(A_BYTES % 1024 == 0 && Q_BYTES % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+template <int FMT, int NQ>
+__global__ void __launch_bounds__(320, 1)
+    index_mma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                     const MmaArgs a) {
+  using C = Cfg<FMT, NQ>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* accf = empty + C::STAGES;  // [NACC] accumulator ready
+  uint64_t* acce = accf + C::NACC;     // [NACC] accumulator drained
+  uint64_t* qbar = acce + C::NACC;
+  float* w_s = reinterpret_cast<float*>(sm + C::OFF_W);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_TMEM);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int groups = a.T / NQ;
+  const int b = blockIdx.y / groups;
+  const int t0 = (blockIdx.y % groups) * NQ;
+  const int64_t L = a.ctx_len[b];
+  const bool ok = L >= a.T && L / a.m <= a.n_max;
+  const int64_t n_last = ok ? (L - a.T + t0 + NQ) / a.m : 0;  // N(p) of the group's last query
+  const int64_t tiles = (n_last + C::TILE - 1) / C::TILE;
+  const int64_t per = (tiles + a.chunks - 1) / a.chunks;
+  const int64_t tile_lo = (int64_t)blockIdx.x * per;
+  const int64_t tile_hi = tile_lo + per < tiles ? tile_lo + per : tiles;
+  if (tile_hi <= tile_lo) return;  // uniform over the CTA, before any barrier or TMEM use
+  const int ntile = (int)(tile_hi - tile_lo);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int j = 0; j < C::NACC; ++j) {
+      mbar_init(&accf[j], 1);
+      mbar_init(&acce[j], 4);  // the four warps of the group draining it
+    }
+    mbar_init(qbar, 1);
+    fence_barrier_init();
+  }
+  for (int i = threadIdx.x; i < C::N; i += blockDim.x) {
+    const int64_t list = (int64_t)b * a.T + t0 + i / 64;
+    float wv = a.w_idx[list * 64 + (i % 64)];
+    if (FMT == LCSC_FMT_FP8) wv *= reinterpret_cast<const float*>(a.q_scale)[list * 64 + (i % 64)];
+    w_s[i] = wv;
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_q);
+      mbar_arrive_expect_tx(qbar, C::Q_BYTES + C::SFB_BYTES);
+      tma_load_2d(sm + C::OFF_Q, &tm_q, 0, (int32_t)(((int64_t)b * a.T + t0) * 64), qbar);
+      if (FMT == LCSC_FMT_FP4) {
+        const int64_t q_tiles = ((int64_t)a.T * 64 + 127) / 128;
+        const uint8_t* src = a.q_scale + ((int64_t)b * q_tiles + (t0 * 64) / 128) * 1024;
+        bulk_load(sm + C::OFF_SFB, src, C::SFB_BYTES, qbar);
+      }
+      const int64_t key_tiles = a.key_cap / 128;
+      for (int i = 0; i < ntile; ++i) {
+        const int s = i % C::STAGES;
+        const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
+        if (!mbar_wait(&empty[s], ph ^ 1u, a.status)) break;
+        const int64_t tile = tile_lo + i;
+        mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::SFA_BYTES);
+        tma_load_2d(sm + C::OFF_A + s * C::A_BYTES, &tm_k, 0, (int32_t)((int64_t)b * a.key_cap + tile * 128),
+                    &full[s]);
+        if (FMT == LCSC_FMT_FP4) {
+          const uint8_t* src = reinterpret_cast<const uint8_t*>(a.key_scale) + ((int64_t)b * key_tiles + tile) * 1024;
+          bulk_load(sm + C::OFF_SFA + s * 1024, src, 1024, &full[s]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool live = mbar_wait(qbar, 0, a.status);
+      tc_fence_after();
+      const uint32_t q_addr = smem_u32(sm + C::OFF_Q);
+      if (live && FMT == LCSC_FMT_FP4) {
+        for (int j = 0; j < 2; ++j)
+          for (int c = 0; c < (C::N + 127) / 128; ++c)
+            tmem_cp_32x128b_x4(tmem + C::SFB_COL + 8 * c + 4 * j,
+                               smem_desc(smem_u32(sm + C::OFF_SFB + c * 1024 + j * 512), 16, 128, kSwNone));
+      }
+      const uint32_t idesc = FMT == LCSC_FMT_FP4 ? idesc_mxf4nvf4(128, C::N) : idesc_dense(0, 0, 128, C::N);
+      int issued = 0;
+      for (int i = 0; live && i < ntile; ++i) {
+        const int s = i % C::STAGES;
+        const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
+        const int ab = i % C::NACC;
+        const uint32_t au = (uint32_t)(i / C::NACC) & 1u;
+        if (!mbar_wait(&full[s], ph, a.status)) break;
+        if (!mbar_wait(&acce[ab], au ^ 1u, a.status)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(sm + C::OFF_A + s * C::A_BYTES);
+        const uint32_t d = tmem + ab * C::N;
+        if constexpr (FMT == LCSC_FMT_FP4) {
+          const uint32_t sfa = tmem + C::SFA_COL + 8 * ab;
+          for (int j = 0; j < 2; ++j)
+            tmem_cp_32x128b_x4(sfa + 4 * j, smem_desc(smem_u32(sm + C::OFF_SFA + s * 1024 + j * 512), 16, 128,
+                                                      kSwNone));
+#pragma unroll
+          for (int kk = 0; kk < C::KSTEPS; ++kk)
+            mma_mxf4nvf4(d, smem_desc(a_addr + kk * 32, 16, C::SBO, C::SW),
+                         smem_desc(q_addr + kk * 32, 16, C::SBO, C::SW), idesc, sfa + 4 * kk,
+                         tmem + C::SFB_COL + 4 * kk, kk > 0);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < C::KSTEPS; ++kk)
+            mma_ss<1>(d, smem_desc(a_addr + kk * 32, 16, C::SBO, C::SW), smem_desc(q_addr + kk * 32, 16, C::SBO, C::SW),
+                      idesc, kk > 0);
+        }
+        tc_commit(&empty[s]);
+        tc_commit(&accf[ab]);
+        ++issued;
+      }
+      if (issued > 0) {  // the accumulator of the last tile is complete before TMEM is freed
+        const int last = issued - 1;
+        mbar_wait(&accf[last % C::NACC], (uint32_t)(last / C::NACC) & 1u, a.status);
+      }
+    }
+  } else {
+    // ------------------------------------------------------ epilogue
+    // Two groups of four warps take alternate tiles; within a group warp w
+    // reads TMEM sub-partition w % 4 (rows 32 (w % 4) ..).
+    const int grp = (warp - 2) >> 2;
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const float* kscale = reinterpret_cast<const float*>(a.key_scale) + (int64_t)b * a.key_cap;
+    float wr[NQ == 1 ? 64 : 1];  // head weights in registers when one query
+    if constexpr (NQ == 1) {
+#pragma unroll
+      for (int j = 0; j < 64; ++j) wr[j] = w_s[j];
+    }
+    for (int i = grp; i < ntile; i += 2) {
+      const int ab = i % C::NACC;
+      const int64_t g = (tile_lo + i) * 128 + row;
+      const float sk = FMT == LCSC_FMT_FP8 ? kscale[g] : 1.f;
+      if (!mbar_wait(&accf[ab], (uint32_t)(i / C::NACC) & 1u, a.status)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int nq = 0; nq < NQ; ++nq) {
+        uint32_t r0[32], r1[32];
+        const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) + ab * C::N + nq * 64;
+        tmem_ld_32(taddr, r0);
+        tmem_ld_32(taddr + 32, r1);
+        tmem_ld_wait();
+        float p[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) p[j] = 0.f;
+        if constexpr (NQ == 1) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) p[j & 7] = fmaf(wr[j], fmaxf(__uint_as_float(r0[j]), 0.f), p[j & 7]);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) p[j & 7] = fmaf(wr[32 + j], fmaxf(__uint_as_float(r1[j]), 0.f), p[j & 7]);
+        } else {
+          const float* w = w_s + nq * 64;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) p[j & 7] = fmaf(w[j], fmaxf(__uint_as_float(r0[j]), 0.f), p[j & 7]);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) p[j & 7] = fmaf(w[32 + j], fmaxf(__uint_as_float(r1[j]), 0.f), p[j & 7]);
+        }
+        const float acc = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
+        const int t = t0 + nq;
+        const int64_t n_p = (L - a.T + t + 1) / a.m;
+        if (g < n_p) a.scores[((int64_t)b * a.T + t) * a.n_max + g] = acc * sk;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[ab]);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Row-major byte matrix [rows][row_bytes]; box = [box_rows][row_bytes].
+bool map_rows(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows,
+              CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)row_bytes, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int FMT, int NQ>
+cudaError_t launch_mma(const IndexLaunch& a, cudaStream_t stream) {
+  using C = Cfg<FMT, NQ>;
+  CUtensorMap tk, tq;
+  const CUtensorMapSwizzle sw = FMT == LCSC_FMT_FP4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!map_rows(&tk, a.keys.data, C::ROW, (uint64_t)a.B * a.keys.capacity, 128, sw)) return cudaErrorInvalidValue;
+  if (!map_rows(&tq, a.q_store.data, C::ROW, (uint64_t)a.B * a.T * 64, C::N, sw)) return cudaErrorInvalidValue;
+  MmaArgs m;
+  m.key_scale = a.keys.scale;
+  m.key_cap = a.keys.capacity;
+  m.q_scale = reinterpret_cast<const uint8_t*>(a.q_store.scale);
+  m.w_idx = a.w_idx;
+  m.ctx_len = a.ctx_len;
+  m.B = a.B;
+  m.T = a.T;
+  m.m = a.m;
+  m.n_max = a.n_max;
+  m.scores = a.scores;
+  m.status = a.status;
+  const int groups = a.T / NQ;
+  const int64_t ctas = (int64_t)a.B * groups;
+  m.chunks = ctas >= sm_count() ? 1 : (int)(sm_count() / ctas);
+  auto kern = index_mma_kernel<FMT, NQ>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(m.chunks, (unsigned)ctas), 320, C::SMEM, stream>>>(tk, tq, m);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool index_mma_supported(const IndexLaunch& a) {
+  const int fmt = a.keys.f.fmt;
+  if (a.d_I != 128 || a.H_I != 64) return false;
+  if (a.keys.capacity % 128 != 0) return false;
+  if (fmt == LCSC_FMT_FP8) return true;
+  if (fmt == LCSC_FMT_FP4) return a.T == 1;
+  return false;
+}
+
+cudaError_t launch_index_mma(const IndexLaunch& a, cudaStream_t stream) {
+  if (a.keys.f.fmt == LCSC_FMT_FP4) return launch_mma<LCSC_FMT_FP4, 1>(a, stream);
+  if (a.T % 4 == 0) return launch_mma<LCSC_FMT_FP8, 4>(a, stream);
+  return launch_mma<LCSC_FMT_FP8, 1>(a, stream);
+}
+
+}  // namespace lcsc

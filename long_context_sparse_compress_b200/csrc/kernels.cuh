@@ -67,6 +67,10 @@ struct IndexLaunch {
 cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream);
 cudaError_t launch_topk(const IndexLaunch& a, cudaStream_t stream);
 cudaError_t launch_index_topk(const IndexLaunch& a, cudaStream_t stream);
+// Tensor-core scoring (FP8 / FP4 keys, d_I = 128, H_I = 64, key capacity a
+// multiple of 128); index_mma_supported() tells whether it applies.
+bool index_mma_supported(const IndexLaunch& a);
+cudaError_t launch_index_mma(const IndexLaunch& a, cudaStream_t stream);
 
 struct AttnLaunch {
   const void* q;        // [B][T][H][D]
@@ -89,7 +93,14 @@ struct AttnLaunch {
 
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream);
 
-// Attention split geometry for a call (rows per split and split count).
-void attention_splits(int64_t max_rows, int64_t n_lists, int* splits, int* rows_per_split);
+// Tensor-core attention (64 heads, 512-d FP8 + BF16 rows, V = K).
+bool attn_mma_supported(const AttnLaunch& a);
+cudaError_t launch_attn_mma(const AttnLaunch& a, cudaStream_t stream);
+
+// Attention split geometry: the rows of each query are cut into `splits`
+// ranges of `rows_per_split` (a multiple of `granule`), sized so that
+// n_ctas_per_split * splits CTAs fill the GPU.
+void attention_splits(int64_t max_rows, int64_t n_ctas_per_split, int granule, int target_ctas, int* splits,
+                      int* rows_per_split);
 
 }  // namespace lcsc

@@ -133,6 +133,21 @@ def row_bytes(fmt, dim, rope=0):
     return {"f32": 4 * dim, "kv": dim + rope, "fp8": dim, "fp4": dim // 2}[fmt]
 
 
+def round_capacity(n, fmt):
+    """Rows to allocate for n rows: indexer keys in FP8 / FP4 need a multiple of 128."""
+    return (n + 127) // 128 * 128 if fmt in ("fp8", "fp4") else n
+
+
+def fp4_scale_index(capacity, dim):
+    """Position, in the tiled FP4 scale array of one sequence, of the block
+    scale (row r, block k): the layout include/lcsc.h documents.  Returns an
+    int array [capacity, dim // 16]."""
+    r = torch.arange(capacity).view(-1, 1)
+    k = torch.arange(dim // 16).view(1, -1)
+    m = r % 128
+    return ((r // 128) * (dim // 64) * 512 + (k // 4) * 512 + (m % 32) * 16 + (m // 32) * 4 + (k % 4))
+
+
 class DeviceCache:
     """Stored rows of one tensor for B sequences, in device memory."""
 
@@ -144,9 +159,34 @@ class DeviceCache:
         else:
             self.data = torch.zeros((B, capacity, row_bytes(fmt, dim, rope)), dtype=torch.uint8, device=device)
             if fmt == "fp4":
-                self.scale = torch.zeros((B, capacity, dim // 16), dtype=torch.uint8, device=device)
+                tiles = (capacity + 127) // 128
+                self.scale = torch.zeros((B, tiles * (dim // 64) * 512), dtype=torch.uint8, device=device)
             else:
                 self.scale = torch.ones((B, capacity), dtype=torch.float32, device=device)
+
+    def set_rows(self, b, payload, scale=None, row0=0):
+        """Copy stored rows (host arrays: payload [n, row], scale [n] or, for
+        FP4, [n, dim / 16] row-major block scales) into sequence b."""
+        n = payload.shape[0]
+        self.data[b, row0:row0 + n] = torch.as_tensor(payload).to(self.data.device)
+        if self.scale is None:
+            return
+        sc = torch.as_tensor(scale).to(self.scale.device)
+        if self.fmt == "fp4":
+            idx = fp4_scale_index(self.capacity, self.dim)[row0:row0 + n].to(self.scale.device)
+            self.scale[b].view(-1)[idx.reshape(-1)] = sc.reshape(-1)
+        else:
+            self.scale[b, row0:row0 + n] = sc
+
+    def get_rows(self, b):
+        """(payload, scale) of sequence b on the host, FP4 scales as [capacity, dim / 16]."""
+        d = self.data[b].cpu().numpy()
+        if self.scale is None:
+            return d, None
+        if self.fmt == "fp4":
+            idx = fp4_scale_index(self.capacity, self.dim).to(self.scale.device)
+            return d, self.scale[b][idx].cpu().numpy()
+        return d, self.scale[b].cpu().numpy()
 
     def c(self):
         return Cache(data=self.data.data_ptr(), scale=None if self.scale is None else self.scale.data_ptr(),

@@ -15,16 +15,12 @@ def dev(a, dtype=torch.float32):
 
 def upload(cache, b, st):
     """Copy oracle ``Stored`` rows into sequence b of a DeviceCache."""
-    n = st.payload.shape[0]
-    cache.data[b, :n] = torch.from_numpy(np.ascontiguousarray(st.payload)).cuda()
-    if cache.scale is not None:
-        cache.scale[b, :n] = torch.from_numpy(np.ascontiguousarray(st.scale)).cuda()
+    cache.set_rows(b, np.ascontiguousarray(st.payload),
+                   None if st.scale is None else np.ascontiguousarray(st.scale))
 
 
 def download(cache, b):
-    d = cache.data[b].cpu().numpy()
-    s = None if cache.scale is None else cache.scale[b].cpu().numpy()
-    return d, s
+    return cache.get_rows(b)
 
 
 class GpuBatch:
@@ -38,11 +34,12 @@ class GpuBatch:
         B = len(seqs)
         self.B = B
         self.n_cap = max(s.wl.L for s in seqs) // wl.m + 1
+        n_cap_idx = L.round_capacity(self.n_cap, wl.idx_fmt)
         self.n_max = max(s.wl.L for s in seqs) // wl.m
         rope = wl.rope_dim if wl.kv_fmt == "kv" else 0
         self.kv = L.DeviceCache(B, self.n_cap, wl.kv_fmt, wl.D, rope)
         self.v = L.DeviceCache(B, self.n_cap, wl.kv_fmt, wl.Dv, rope) if wl.separate_v else None
-        self.idx = L.DeviceCache(B, self.n_cap, wl.idx_fmt, wl.d_I) if wl.kind == "csa" else None
+        self.idx = L.DeviceCache(B, n_cap_idx, wl.idx_fmt, wl.d_I) if wl.kind == "csa" else None
         self.win_kv = L.DeviceCache(B, wl.win_cap, wl.kv_fmt, wl.D, rope)
         self.win_v = L.DeviceCache(B, wl.win_cap, wl.kv_fmt, wl.Dv, rope) if wl.separate_v else None
         xdt, qdt = TORCH_DT[wl.x_dtype], TORCH_DT[wl.q_dtype]

@@ -148,7 +148,7 @@ def test_index_topk_matches_oracle(cuda_lib, fmt):
     T = 3
     lengths = [4 * 5000 + 3, 4 * 37, 4 * 2100 + 1]  # one list shorter than k
     B = len(lengths)
-    n_cap = max(lengths) // m + 1
+    n_cap = L.round_capacity(max(lengths) // m + 1, fmt)
     keys_v = _rows(rng, B * n_cap, d_I).reshape(B, n_cap, d_I)
     keys_v[0, 100:110] = keys_v[0, 99]                 # a run of equal keys
     qi = (rng.standard_normal((B, T, H_I, d_I)) * d_I ** -0.5).astype(np.float32)

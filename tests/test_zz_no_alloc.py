@@ -20,13 +20,12 @@ def _inputs(fmt, lengths, T, seed):
     wl = W.PAIR_DECODE_1M_B1.layer("csa").with_(idx_fmt=fmt, k=512)
     rng = np.random.default_rng(seed)
     B = len(lengths)
-    n_cap = max(lengths) // wl.m + 1
+    n_cap = L.round_capacity(max(lengths) // wl.m + 1, fmt)
     keys = L.DeviceCache(B, n_cap, fmt, wl.d_I)
     for b in range(B):
         vals = (rng.standard_normal((n_cap, wl.d_I)) * wl.d_I ** -0.5).astype(np.float32)
         st = storage.encode(fmt, vals)
-        keys.data[b] = torch.from_numpy(st.payload).cuda()
-        keys.scale[b] = torch.from_numpy(st.scale).cuda()
+        keys.set_rows(b, st.payload, st.scale)
     qi = torch.from_numpy((rng.standard_normal((B, T, wl.H_I, wl.d_I)) * wl.d_I ** -0.5).astype(np.float32))
     wi = torch.from_numpy((np.abs(rng.standard_normal((B, T, wl.H_I))) * wl.H_I ** -0.5).astype(np.float32))
     ctx = torch.tensor(lengths, dtype=torch.int32)
