@@ -147,13 +147,18 @@ class Layer:
 
 
 def kernels_per_step(wl):
-    """Kernels of this library one step launches (memsets excluded):
-    CSA: pool + store for the KV latent and for the indexer keys (4), query
-    quantisation + scoring (2), three top-k passes (3), attention partial +
-    combine (2); HCA: pool + store (2), attention partial + combine (2)."""
+    """Kernels of this library one step launches: CSA: pool + store for the
+    KV latent and for the indexer keys (4), query quantisation + scoring (2),
+    top-k collect + final (2, plus a histogram pass when the scores come from
+    the CUDA-core scoring kernel), attention partial + combine (2); HCA: pool
+    + store (2), attention partial + combine (2)."""
+    def csa(w):
+        tensor_scored = (w.idx_fmt in ("fp8", "fp4") and w.d_I == 128 and w.H_I == 64
+                         and (w.idx_fmt == "fp8" or w.T == 1))
+        return 10 + (0 if tensor_scored else 1)
     if wl.kind == "pair":
-        return 11 + 4
-    return 11 if wl.kind == "csa" else 4
+        return csa(wl.layer("csa")) + 4
+    return csa(wl) if wl.kind == "csa" else 4
 
 
 # ------------------------------------------------------------ measurement
@@ -284,9 +289,11 @@ def run_lcsc(args):
 
     # ---- timed region: K steps, inputs resident in HBM (working set > L2)
     csa = layers[0] if layers[0].wl.kind == "csa" else None
+    hca = next((ly for ly in layers if ly.wl.kind == "hca"), None)
     n_ev = 5
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
-    for evs in events:
+    hevents = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for evs in events + hevents:
         for e in evs:
             e.record(stream)  # creates the events
     torch.cuda.synchronize()
@@ -301,6 +308,8 @@ def run_lcsc(args):
     for i in range(args.steps):
         if csa is not None:
             csa.set_events(events[i])
+        if hca is not None:
+            hca.set_events(hevents[i])
         step()
     stop.record(stream)
     torch.cuda.synchronize()
@@ -308,8 +317,13 @@ def run_lcsc(args):
     t1 = time.time()
     time.sleep(0.25)
     clocks = sampler.stop(t0, t1)
-    if csa is not None:
-        csa.clear_events()
+    for ly in (csa, hca):
+        if ly is not None:
+            ly.clear_events()
+    hca_ms = None
+    if hca is not None:
+        hca_ms = {name: round(float(np.mean([evs[a].elapsed_time(evs[b]) for evs in hevents])), 4)
+                  for name, a, b in (("compress", 0, 1), ("dense_attn", 1, 2))}
     ms_total = max_over_ranks(ws, start.elapsed_time(stop))
     ms_step = ms_total / args.steps
     queries = wl.B * wl.T * ws * args.steps
@@ -336,7 +350,7 @@ def run_lcsc(args):
                 "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                 "traffic": traffic, "algorithmic_bytes": alg_bytes, "ms_per_launch": round(score_ms, 4),
                 "peak_source": peaks["source"] + " hbm_gbs",
-                "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()}}
+                "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()}, "hca_stage_ms": hca_ms}
 
     # ---- end to end: pinned host inputs -> device, step, output -> host
     e2e = None

@@ -110,19 +110,25 @@ void plan_index(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max, Carve
   if (p->idx_format == LCSC_FMT_FP8) qscale = cv.take<float>((size_t)qrows);
   else if (p->idx_format == LCSC_FMT_FP4)  // block scales tiled by 128 rows per sequence
     qscale = cv.take<uint8_t>((size_t)B * ((T * p->idx_heads + 127) / 128) * (p->idx_dim / 64) * 512);
-  float* scores = cv.take<float>((size_t)lists * n_max);
+  const int64_t stride = (n_max + 3) / 4 * 4;
+  float* scores = cv.take<float>((size_t)lists * stride);
   uint32_t* hist = cv.take<uint32_t>((size_t)lists * 2 * 4096);
-  uint32_t* ctr = cv.take<uint32_t>((size_t)lists * 4);
-  uint32_t* cand = cv.take<uint32_t>((size_t)lists * n_max);
+  uint32_t* ctr = cv.take<uint32_t>((size_t)lists * 8);
+  uint32_t* cand = cv.take<uint32_t>((size_t)lists * stride);
+  const int64_t bit_stride = ((stride + 31) / 32 + 3) / 4 * 4;
+  uint32_t* bits = cv.take<uint32_t>((size_t)lists * bit_stride);
   if (L) {
     L->q_store.data = qdata;
     L->q_store.scale = qscale;
     L->q_store.capacity = T * p->idx_heads;
     L->q_store.f = {p->idx_format, p->idx_dim, 0, rb};
+    L->stride = stride;
     L->scores = scores;
     L->hist = hist;
     L->counters = ctr;
     L->cand = cand;
+    L->sel_bits = bits;
+    L->bit_stride = bit_stride;
   }
 }
 
@@ -132,7 +138,7 @@ void plan_attn(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max, bool d
   int splits, rps;
   if (p->kv_format == LCSC_FMT_KV && p->head_dim == 512 && p->n_heads == 64) {
     // tensor-core path: one CTA per (query, split) for all heads, one wave
-    attention_splits(max_rows, B * T, 128, sm_count(), &splits, &rps);
+    attention_splits(max_rows, B * T, 64, sm_count(), &splits, &rps);
   } else {
     const int hpc = p->kv_format == LCSC_FMT_F32 ? 8 : 16;
     attention_splits(max_rows, B * T * (p->n_heads / hpc), 32, 2 * sm_count(), &splits, &rps);

@@ -6,20 +6,23 @@
 // compressed entries plus the uncompressed window, shared-KV multi-query
 // layout; the sink enters in the combine step).
 //
-// One CTA owns (query, range of rows) and walks it in tiles of 128 rows:
-//   1. the tile's stored rows are read (gathered by index for CSA) and
-//      dequantised once into shared memory as f16, in a 128-byte-swizzled
-//      layout that is a K-major operand for Q K^T and an MN-major operand
-//      for P V (the same bytes serve as K and as V);
-//   2. S = Q K^T on tcgen05 (M = 64 heads, N = 128 rows, K = 512), into TMEM;
-//   3. one thread per head reads its S row from TMEM, applies the scale and
-//      the row mask, updates its running max (rescaling O only when the max
-//      grows by more than e^8) and writes P = exp(S - max) as f16;
-//   4. O += P V on tcgen05 (M = 64 heads, N = 2 x 256 dims, K = 128 rows).
+// One CTA owns (query, range of rows) and walks it in tiles of 64 rows with a
+// warp-specialised pipeline:
+//  * 7 loader warps resolve the tile's rows (gathered by index for CSA), read
+//    them and dequantise them once into shared memory as f16, in a
+//    128-byte-swizzled layout that is both a K-major operand for Q K^T and an
+//    MN-major operand for P V (the same bytes are K and V); two buffers, so
+//    tile t+1 is loaded while tile t is being used;
+//  * 1 MMA warp issues S = Q K^T (M = 64 heads, N = 64 rows, K = 512) for tile
+//    t+1 as soon as it is loaded, and O += P V (N = 2 x 256 dims, K = 64) for
+//    tile t once its probabilities are ready;
+//  * 4 softmax warps, one thread per head, read S from TMEM, keep a running
+//    reference max (O is rescaled only when the max grows by more than e^8),
+//    and write P = exp(S - ref) as f16.
 // Heads live on M = 64, so S and O use the half-lane TMEM layout: O at
-// lanes 0-15 of each 32-lane sub-partition (all 512 columns), S at lanes
-// 16-31 (columns 0-127).  The partial (max, sum, O) goes to the same
-// workspace the combine kernel merges.
+// lanes 0-15 of each 32-lane sub-partition (all 512 columns), S (two
+// 64-column buffers) at lanes 16-31.  The partial (ref max, sum, O) goes to
+// the workspace the combine kernel merges.
 #include "kernels.cuh"
 #include "sm100.cuh"
 
@@ -28,27 +31,37 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kH = 64;      // heads (MMA M)
-constexpr int kD = 512;     // row length (K of Q K^T, N of P V)
-constexpr int kTR = 128;    // rows per tile
-constexpr int kThr = 256;
-constexpr int kChunks = 36;  // 16-byte chunks of a 576-byte stored row
-constexpr int kLoads = kTR * kChunks / kThr;  // 18 chunks per thread per tile
+constexpr int kH = 64;       // heads (MMA M)
+constexpr int kD = 512;      // row length (K of Q K^T, N of P V)
+constexpr int kTR = 64;      // rows per tile
+constexpr int kLW = 7;       // loader warps (12 warps in all: 3 per SM sub-partition)
+constexpr int kSW = 4;       // softmax warps
+constexpr int kThr = (kSW + kLW + 1) * 32;
+constexpr int kMmaWarp = kSW + kLW;
+constexpr int kFp8Chunks = 28;  // 16-byte FP8 chunks of a stored row (448 dims)
+constexpr int kFp8Loads = kTR * kFp8Chunks / (kLW * 32);            // 8 per loader thread per tile
+constexpr int kLoads = kFp8Loads + (kTR * 8 + kLW * 32 - 1) / (kLW * 32);  // + 3 BF16 chunks
+static_assert(kTR * kFp8Chunks == kFp8Loads * kLW * 32, "FP8 units split evenly");
 constexpr float kRescale = 8.f;  // rescale O only when the max grows by more
 
 // shared memory (offsets from a 1024-aligned base)
-constexpr int OFF_Q = 0;                    // 8 K-blocks [64 heads][128 B]  = 64 KB
-constexpr int OFF_K = OFF_Q + 8 * 64 * 128;  // 8 K-blocks [128 rows][128 B] = 128 KB
-constexpr int OFF_P = OFF_K + 8 * 128 * 128;  // 2 K-blocks [64 heads][128 B] = 16 KB
-constexpr int OFF_BAR = OFF_P + 2 * 64 * 128;  // s_full, pv_done
-constexpr int OFF_ROW = OFF_BAR + 64;         // int64 [2][128]
-constexpr int OFF_SRC = OFF_ROW + 2 * kTR * 8;  // int32 [2][128]
-constexpr int OFF_SCL = OFF_SRC + 2 * kTR * 4;  // float [2][128]
-constexpr int OFF_TM = OFF_SCL + 2 * kTR * 4;
-constexpr int SMEM = OFF_TM + 16 + 1024;
+constexpr int KB_Q = kH * 128;    // one 64-dim block of Q  (8 KB)
+constexpr int KB_K = kTR * 128;   // one 64-dim block of a K tile (8 KB)
+constexpr int OFF_Q = 0;                       // 8 blocks = 64 KB
+constexpr int OFF_K = OFF_Q + 8 * KB_Q;        // 2 buffers x 8 blocks = 128 KB
+constexpr int OFF_P = OFF_K + 2 * 8 * KB_K;    // 2 buffers x [64 heads][128 B] = 16 KB
+constexpr int OFF_BAR = OFF_P + 2 * kH * 128;  // k_full[2] s_full[2] p_full[2] pv_done[2]
+constexpr int OFF_ROW = OFF_BAR + 8 * 8;       // int64 [4][64] (row info of tiles j % 4)
+constexpr int OFF_SRC = OFF_ROW + 4 * kTR * 8;  // int32 [4][64]
+constexpr int OFF_SCL = OFF_SRC + 4 * kTR * 4;  // float [4][64]
+constexpr int OFF_MASK = OFF_SCL + 4 * kTR * 4;  // uint32 [2][2] valid-row bits
+constexpr int OFF_TM = OFF_MASK + 16;
+constexpr int OFF_ABORT = OFF_TM + 4;
+constexpr int OFF_LSTOP = OFF_ABORT + 4;
+constexpr int SMEM = OFF_LSTOP + 8 + 1024;
 
 // Byte offset of (row, byte) in a [rows][128 B] block with the 128-byte swizzle
-// (16-byte chunk index XOR row % 8) that TMA and the tensor cores use.
+// (16-byte chunk index XOR row % 8) that the tensor cores read.
 __device__ __forceinline__ uint32_t swz(int row, int byte) {
   return (uint32_t)(row * 128 + ((((byte >> 4) ^ (row & 7)) << 4) | (byte & 15)));
 }
@@ -75,15 +88,30 @@ __device__ __forceinline__ Rows rows_of(const AttnLaunch& a, int b, int t) {
   return r;
 }
 
-__global__ void __launch_bounds__(kThr, 1) attn_mma_kernel(const AttnLaunch a) {
+// Bounded wait taken by a whole warp; false (for every lane) if any lane gave up.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const AttnLaunch& a,
+                                          volatile int* abort) {
+  if (*abort) return false;
+  bool ok = mbar_wait(bar, parity, a.status);
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok && (threadIdx.x & 31) == 0) *abort = 1;
+  return ok;
+}
+
+__global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* s_full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-  uint64_t* pv_done = s_full + 1;
+  uint64_t* k_full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint64_t* s_full = k_full + 2;
+  uint64_t* p_full = k_full + 4;
+  uint64_t* pv_done = k_full + 6;
   int64_t* row_s = reinterpret_cast<int64_t*>(sm + OFF_ROW);
   int32_t* src_s = reinterpret_cast<int32_t*>(sm + OFF_SRC);
   float* scl_s = reinterpret_cast<float*>(sm + OFF_SCL);
+  uint32_t* mask_s = reinterpret_cast<uint32_t*>(sm + OFF_MASK);
   uint32_t* tm_slot = reinterpret_cast<uint32_t*>(sm + OFF_TM);
+  volatile int* abort = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
+  volatile int* lstop = reinterpret_cast<volatile int*>(sm + OFF_LSTOP);  // loader-group decision
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int list = blockIdx.y;
@@ -94,263 +122,350 @@ __global__ void __launch_bounds__(kThr, 1) attn_mma_kernel(const AttnLaunch a) {
   const int64_t s_lo = (int64_t)blockIdx.x * a.rows_per_split;
   const int64_t s_hi = s_lo + a.rows_per_split < total ? s_lo + a.rows_per_split : total;
   const int ntiles = s_hi > s_lo ? (int)((s_hi - s_lo + kTR - 1) / kTR) : 0;
-  const int n_fp8 = a.kv.f.dim - a.kv.f.rope;
 
   if (tid == 0) {
-    mbar_init(s_full, 1);
-    mbar_init(pv_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], kSW);
+      mbar_init(&pv_done[i], 1);
+    }
+    *abort = 0;
+    *lstop = 0;
     fence_barrier_init();
   }
-  if (warp == 0) tmem_alloc(tm_slot, 512);
+  if (warp == kMmaWarp) tmem_alloc(tm_slot, 512);
 
-  // ---- Q (64 x 512) -> f16, K-major swizzled blocks of 64 dims
+  // ---- Q (64 x 512) -> f16, K-major swizzled blocks of 64 dims (all threads)
   for (int i = tid; i < kH * (kD / 8); i += kThr) {
     const int h = i / (kD / 8), d0 = (i % (kD / 8)) * 8;
     const int64_t base = ((int64_t)list * a.H + h) * kD + d0;
     float v[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) v[j] = load_elem(a.q, base + j, a.q_dtype);
-    uint4 u = make_uint4(pack_h2(v[0], v[1]), pack_h2(v[2], v[3]), pack_h2(v[4], v[5]), pack_h2(v[6], v[7]));
-    *reinterpret_cast<uint4*>(sm + OFF_Q + (d0 / 64) * (kH * 128) + swz(h, (d0 % 64) * 2)) = u;
+    *reinterpret_cast<uint4*>(sm + OFF_Q + (d0 / 64) * KB_Q + swz(h, (d0 % 64) * 2)) =
+        make_uint4(pack_h2(v[0], v[1]), pack_h2(v[2], v[3]), pack_h2(v[4], v[5]), pack_h2(v[6], v[7]));
   }
-
-  // ---- tile row resolution (threads 0..127) into buffer `buf`
-  auto resolve = [&](int tile, int buf) {
-    if (tid < kTR) {
-      const int64_t slot = s_lo + (int64_t)tile * kTR + tid;
-      int src = 0;
-      int64_t row = 0;
-      float sc = 1.f;
-      if (slot < s_hi) {
-        if (slot < qr.n_ent_slots) {
-          const int64_t g = a.idx ? (int64_t)a.idx[(int64_t)list * a.k + slot] : slot;
-          if (g >= 0 && g < qr.n_vis) {
-            src = 1;
-            row = g;
-            sc = *a.kv.fscale(b, g);
-          } else if (g != -1 || !a.idx) {
-            if (a.status) atomicOr(a.status, LCSC_DEV_BAD_INDEX);
-          }
-        } else {
-          src = 2;
-          row = (qr.w_lo + (slot - qr.n_ent_slots)) % a.win_kv.capacity;
-          sc = *a.win_kv.fscale(b, row);
-        }
-      }
-      row_s[buf * kTR + tid] = row;
-      src_s[buf * kTR + tid] = src;
-      scl_s[buf * kTR + tid] = sc;
-    }
-  };
-  // ---- raw 16-byte chunks of a tile into registers
-  uint4 raw[kLoads];
-  auto fetch = [&](int buf) {
-#pragma unroll
-    for (int i = 0; i < kLoads; ++i) {
-      const int idx = tid + i * kThr;
-      const int r = idx / kChunks, c = idx % kChunks;
-      const int src = src_s[buf * kTR + r];
-      raw[i] = make_uint4(0, 0, 0, 0);
-      if (src) {
-        const CacheView& cv = src == 1 ? a.kv : a.win_kv;
-        raw[i] = reinterpret_cast<const uint4*>(cv.row(b, row_s[buf * kTR + r]))[c];
-      }
-    }
-  };
-  // ---- dequantise the registers into the f16 K tile
-  auto convert = [&](int buf) {
-#pragma unroll
-    for (int i = 0; i < kLoads; ++i) {
-      const int idx = tid + i * kThr;
-      const int r = idx / kChunks, c = idx % kChunks;
-      const int byte0 = c * 16;
-      if (byte0 < n_fp8) {
-        const float s = scl_s[buf * kTR + r];
-        const uint16_t* c2 = reinterpret_cast<const uint16_t*>(&raw[i]);
-        uint32_t h[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float2 f = e4m3x2_val(c2[j]);
-          h[j] = pack_h2(f.x * s, f.y * s);
-        }
-        const int d0 = byte0;  // one byte per value
-        uint8_t* blk = sm + OFF_K + (d0 / 64) * (kTR * 128);
-        *reinterpret_cast<uint4*>(blk + swz(r, (d0 % 64) * 2)) = make_uint4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<uint4*>(blk + swz(r, (d0 % 64) * 2 + 16)) = make_uint4(h[4], h[5], h[6], h[7]);
-      } else {
-        const uint16_t* bf = reinterpret_cast<const uint16_t*>(&raw[i]);
-        uint32_t h[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) h[j] = pack_h2(bf16_val(bf[2 * j]), bf16_val(bf[2 * j + 1]));
-        const int d0 = n_fp8 + (byte0 - n_fp8) / 2;
-        uint8_t* blk = sm + OFF_K + (d0 / 64) * (kTR * 128);
-        *reinterpret_cast<uint4*>(blk + swz(r, (d0 % 64) * 2)) = make_uint4(h[0], h[1], h[2], h[3]);
-      }
-    }
-  };
-
+  fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tm_slot;
-  const uint32_t tm_s = tmem + (16u << 16);  // S: lanes 16-31 of each sub-partition
-  const bool softmax_thread = warp < 4 && lane >= 16;
-  const int head = warp * 16 + (lane & 15);  // warps 0-3: O (lane < 16) / S (lane >= 16) row
-  float m_ref = -INFINITY, l_sum = 0.f;
-  bool live = true;
 
-  if (ntiles > 0) {
-    resolve(0, 0);
-    __syncthreads();
-    fetch(0);
-  }
-  const uint32_t idesc_qk = idesc_dense(0, 0, 64, kTR);
-  const uint32_t idesc_pv = idesc_dense(0, 0, 64, 256, false, true);
-  // `live` stays uniform over the CTA: every bounded wait is folded in at a
-  // barrier, so a time-out makes all threads leave the loop together.
-  for (int j = 0; j < ntiles; ++j) {
-    const int buf = j & 1;
-    bool ok = true;
-    if (j > 0) ok = mbar_wait(pv_done, (uint32_t)(j - 1) & 1u, a.status);  // K and P smem free
-    convert(buf);
-    fence_async_smem();
-    live = __syncthreads_and(ok) != 0;
-    if (!live) break;
-    if (tid == 128) {  // ---- S = Q K^T
-      tc_fence_after();
-      const uint32_t qa = smem_u32(sm + OFF_Q), ka = smem_u32(sm + OFF_K);
+  if (warp >= kSW && warp < kMmaWarp) {
+    // =================================================== loader warps
+    // Software pipeline: the rows of tile j+1 are resolved and their bytes
+    // requested (into a second register set) before tile j is dequantised.
+    const int lt = tid - kSW * 32;  // 0 .. 223
+    // Work units of a tile, fixed per thread for the whole kernel.  Units
+    // 0-7 are 16-byte FP8 chunks (28 per row): unit u = lt + 224 i splits as
+    // q = u % 4, row-in-pair = (u / 4) % 2, then 64-dim block (7) and row pair
+    // (32), so that the 8 lanes of a 128-bit store phase cover 2 rows x 4
+    // chunks of one block: distinct 16-byte bank groups after the swizzle.
+    // Units 8-10 are 16-byte BF16 chunks (8 per row, 512 in all).  Table
+    // word: first f16 destination (16 bits) | row << 16 | chunk << 22.
+    uint32_t tab[kLoads];
+#pragma unroll
+    for (int i = 0; i < kLoads; ++i) {
+      int r, c;
+      if (i < kFp8Loads) {
+        const int u = lt + i * (kLW * 32), rest = u >> 3;
+        r = 2 * (rest / 7) + ((u >> 2) & 1);
+        c = 4 * (rest % 7) + (u & 3);
+      } else {
+        const int v = lt + (i - kFp8Loads) * (kLW * 32);
+        if (v >= kTR * 8) {
+          tab[i] = 0xFFFFFFFFu;
+          continue;
+        }
+        r = v >> 3;
+        c = kFp8Chunks + (v & 7);
+      }
+      const int dim = c < kFp8Chunks ? c * 16 : kFp8Chunks * 16 + (c - kFp8Chunks) * 8;
+      const uint32_t d0 = (dim / 64) * KB_K + swz(r, (dim % 64) * 2);
+      tab[i] = d0 | ((uint32_t)r << 16) | ((uint32_t)c << 22);
+    }
+    // Row-info threads (lt < 64, one per row of a tile) keep two global loads
+    // in flight across steps: the gather index of the row one tile ahead of
+    // the one being located, and the scale of the row just located.
+    auto slot_of = [&](int j) { return s_lo + (int64_t)j * kTR + lt; };
+    auto load_idx = [&](int j) -> int32_t {
+      const int64_t slot = slot_of(j);
+      return (a.idx && slot < s_hi && slot < qr.n_ent_slots) ? a.idx[(int64_t)list * a.k + slot] : 0;
+    };
+    // Row of tile j for this thread: pointer (null: no row) and scale address.
+    auto locate = [&](int j, int32_t gi, const float*& scp) -> const uint8_t* {
+      const int64_t slot = slot_of(j);
+      scp = nullptr;
+      if (slot >= s_hi) return nullptr;
+      if (slot < qr.n_ent_slots) {
+        const int64_t g = a.idx ? (int64_t)gi : slot;
+        if (g >= 0 && g < qr.n_vis) {
+          scp = a.kv.fscale(b, g);
+          return a.kv.row(b, g);
+        }
+        if ((g != -1 || !a.idx) && a.status) atomicOr(a.status, LCSC_DEV_BAD_INDEX);
+        return nullptr;
+      }
+      const int64_t row = (qr.w_lo + (slot - qr.n_ent_slots)) % a.win_kv.capacity;
+      scp = a.win_kv.fscale(b, row);
+      return a.win_kv.row(b, row);
+    };
+    int32_t idx_next = 0;  // gather index of tile j+1's row (in flight)
+    float sc_next = 1.f;   // scale of the row last located (in flight)
+    auto place = [&](int j, int32_t gi) {  // tile j's row info -> row buffer j % 4
+      const float* scp;
+      const uint8_t* p = locate(j, gi, scp);
+      row_s[(j & 3) * kTR + lt] = reinterpret_cast<int64_t>(p);
+      src_s[(j & 3) * kTR + lt] = p != nullptr;
+      sc_next = scp ? *scp : 1.f;
+    };
+    auto fetch = [&](int j, uint4 (&raw)[kLoads]) {
+      const int64_t* rows = row_s + (j & 3) * kTR;
+#pragma unroll
+      for (int i = 0; i < kLoads; ++i) {
+        raw[i] = make_uint4(0, 0, 0, 0);
+        if (tab[i] == 0xFFFFFFFFu) continue;
+        const uint8_t* ptr = reinterpret_cast<const uint8_t*>(rows[(tab[i] >> 16) & 63]);
+        if (ptr) raw[i] = reinterpret_cast<const uint4*>(ptr)[tab[i] >> 22];
+      }
+    };
+    auto convert = [&](int j, const uint4 (&raw)[kLoads]) {
+      const float* scl = scl_s + (j & 3) * kTR;
+      uint8_t* kt = sm + OFF_K + (j & 1) * (8 * KB_K);
+#pragma unroll
+      for (int i = 0; i < kFp8Loads; ++i) {
+        const uint32_t d0 = tab[i] & 0xFFFFu;
+        const float sc = scl[(tab[i] >> 16) & 63];
+        const uint16_t* c2 = reinterpret_cast<const uint16_t*>(&raw[i]);
+        uint32_t h[8];
+        if (sc >= 6.103515625e-05f && sc <= 65504.f) {  // a normal f16 scale: multiply in f16x2
+          const __half2 s2 = __float2half2_rn(sc);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(c2[q], __NV_E4M3);
+            const __half2 v = __hmul2(*reinterpret_cast<__half2*>(&hr), s2);
+            h[q] = *reinterpret_cast<const uint32_t*>(&v);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float2 f = e4m3x2_val(c2[q]);
+            h[q] = pack_h2(f.x * sc, f.y * sc);
+          }
+        }
+        // the second 16 bytes are the next 16-byte chunk: swizzled position ^ 1
+        *reinterpret_cast<uint4*>(kt + d0) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(kt + (d0 ^ 16u)) = make_uint4(h[4], h[5], h[6], h[7]);
+      }
+#pragma unroll
+      for (int i = kFp8Loads; i < kLoads; ++i) {
+        if (tab[i] == 0xFFFFFFFFu) continue;
+        const uint16_t* bf = reinterpret_cast<const uint16_t*>(&raw[i]);
+        uint32_t h[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) h[q] = pack_h2(bf16_val(bf[2 * q]), bf16_val(bf[2 * q + 1]));
+        *reinterpret_cast<uint4*>(kt + (tab[i] & 0xFFFFu)) = make_uint4(h[0], h[1], h[2], h[3]);
+      }
+      if (lt < kTR) {  // valid-row bits of tile j, read by the softmax after k_full
+        const uint32_t bits = __ballot_sync(0xffffffffu, src_s[(j & 3) * kTR + lt] != 0);
+        if (lane == 0) mask_s[(j & 1) * 2 + (lt >> 5)] = bits;
+      }
+    };
+    // One step: tile j+1 located and requested, tile j stored.  false: stop.
+    auto step = [&](int j, const uint4 (&cur)[kLoads], uint4 (&nxt)[kLoads]) -> bool {
+      if (lt < kTR) {
+        scl_s[(j & 3) * kTR + lt] = sc_next;  // tile j's scale, loaded one step ago
+        if (j + 1 < ntiles) {
+          place(j + 1, idx_next);
+          if (j + 2 < ntiles) idx_next = load_idx(j + 2);
+        }
+      }
+      named_sync(1, kLW * 32);
+      if (j + 1 < ntiles) fetch(j + 1, nxt);
+      // One thread decides for the group (K[j % 2] is free once the PV of
+      // tile j-2 is done); `lstop` is written only here, between group
+      // barriers, so every loader reads the same value.
+      if (lt == 0) {
+        bool ok = !*abort;
+        if (ok && j >= 2) ok = mbar_wait(&pv_done[j & 1], (uint32_t)((j - 2) >> 1) & 1u, a.status);
+        if (!ok) *abort = 1;
+        *lstop = ok ? 0 : 1;
+      }
+      named_sync(1, kLW * 32);
+      if (*lstop) return false;
+      convert(j, cur);
+      fence_async_smem();
+      named_sync(1, kLW * 32);
+      if (lt == 0) mbar_arrive(&k_full[j & 1]);
+      return true;
+    };
+    uint4 ra[kLoads], rb[kLoads];
+    if (ntiles > 0) {
+      if (lt < kTR) {
+        place(0, load_idx(0));
+        if (ntiles > 1) idx_next = load_idx(1);
+      }
+      named_sync(1, kLW * 32);
+      fetch(0, ra);
+    }
+    for (int j = 0; j < ntiles; j += 2) {
+      if (!step(j, ra, rb)) break;
+      if (j + 1 < ntiles && !step(j + 1, rb, ra)) break;
+    }
+  } else if (warp == kMmaWarp) {
+    // =================================================== MMA warp
+    const uint32_t idesc_qk = idesc_dense(0, 0, 64, kTR);
+    const uint32_t idesc_pv = idesc_dense(0, 0, 64, 256, false, true);
+    const uint32_t qa = smem_u32(sm + OFF_Q);
+    auto issue_qk = [&](int j) {
+      const int buf = j & 1;
+      const uint32_t ka = smem_u32(sm + OFF_K + buf * (8 * KB_K));
 #pragma unroll 4
       for (int kk = 0; kk < kD / 16; ++kk) {
         const uint32_t kb = kk / 4, ko = (kk % 4) * 32;
-        mma_ss<0>(tm_s, smem_desc(qa + kb * (kH * 128) + ko, 16, 1024, kSw128),
-                  smem_desc(ka + kb * (kTR * 128) + ko, 16, 1024, kSw128), idesc_qk, kk > 0);
+        mma_ss<0>(tmem + (16u << 16) + buf * kTR, smem_desc(qa + kb * KB_Q + ko, 16, 1024, kSw128),
+                  smem_desc(ka + kb * KB_K + ko, 16, 1024, kSw128), idesc_qk, kk > 0);
       }
-      tc_commit(s_full);
-    }
-    if (j + 1 < ntiles) resolve(j + 1, buf ^ 1);
-    __syncthreads();
-    if (j + 1 < ntiles) fetch(buf ^ 1);  // in flight while this tile finishes
-
-    // ---- softmax: one thread per head, S row from TMEM
-    bool need_rescale = false;
-    float alpha = 1.f;
-    bool ok2 = true;
-    if (warp < 4) {
-      ok2 = mbar_wait(s_full, (uint32_t)j & 1u, a.status);
-      tc_fence_after();
-      const int rows_here = (int)((s_hi - s_lo) - (int64_t)j * kTR < kTR ? (s_hi - s_lo) - (int64_t)j * kTR : kTR);
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < kTR; c += 32) {
-        uint32_t r[32];
-        tmem_ld_32(tmem + ((uint32_t)(warp * 32) << 16) + c, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const int col = c + q;
-          const bool valid = col < rows_here && src_s[buf * kTR + col] != 0;
-          if (valid) mx = fmaxf(mx, __uint_as_float(r[q]) * a.sm_scale);
-        }
-      }
-      if (softmax_thread) {
-        if (mx > m_ref + kRescale || (m_ref == -INFINITY && mx > -INFINITY)) {
-          const float m_new = mx;
-          if (m_ref > -INFINITY) {
-            alpha = __expf(m_ref - m_new);
-            need_rescale = true;
-            l_sum *= alpha;
-          }
-          m_ref = m_new;
-        }
-      }
-      float sum = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < kTR; c += 32) {
-        uint32_t r[32];
-        tmem_ld_32(tmem + ((uint32_t)(warp * 32) << 16) + c, r);
-        tmem_ld_wait();
-        if (softmax_thread) {
-          float p[32];
-#pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const int col = c + q;
-            const bool valid = col < rows_here && src_s[buf * kTR + col] != 0;
-            p[q] = (valid && m_ref > -INFINITY) ? __expf(__uint_as_float(r[q]) * a.sm_scale - m_ref) : 0.f;
-            sum += p[q];
-          }
-          // P row `head`, columns c..c+31: K-major [64 heads][128 rows] in two 64-row blocks
-          uint8_t* blk = sm + OFF_P + (c / 64) * (kH * 128);
-#pragma unroll
-          for (int q = 0; q < 32; q += 8)
-            *reinterpret_cast<uint4*>(blk + swz(head, ((c % 64) + q) * 2)) =
-                make_uint4(pack_h2(p[q], p[q + 1]), pack_h2(p[q + 2], p[q + 3]), pack_h2(p[q + 4], p[q + 5]),
-                           pack_h2(p[q + 6], p[q + 7]));
-        }
-      }
-      if (softmax_thread) l_sum += sum;
-      // ---- rare: rescale O rows whose max moved (O owners are lanes 0-15)
-      const float a_own = __shfl_sync(0xffffffffu, alpha, (lane & 15) + 16);
-      const bool warp_rescale = __any_sync(0xffffffffu, need_rescale);
-      if (warp_rescale && j > 0) {
-        for (int c = 0; c < kD; c += 32) {
-          uint32_t r[32];
-          tmem_ld_32(tmem + ((uint32_t)(warp * 32) << 16) + c, r);
-          tmem_ld_wait();
-          if (lane < 16) {
-#pragma unroll
-            for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * a_own);
-          }
-          tmem_st_32(tmem + ((uint32_t)(warp * 32) << 16) + c, r);
-        }
-        tmem_st_wait();
-      }
-      fence_async_smem();
-      tc_fence_before();
-    }
-    live = __syncthreads_and(ok2) != 0;
-    if (!live) break;
-    if (tid == 128) {  // ---- O += P V
-      tc_fence_after();
-      const uint32_t pa = smem_u32(sm + OFF_P), ka = smem_u32(sm + OFF_K);
+      tc_commit(&s_full[buf]);
+    };
+    auto issue_pv = [&](int j) {
+      const int buf = j & 1;
+      const uint32_t pa = smem_u32(sm + OFF_P + buf * (kH * 128));
+      const uint32_t ka = smem_u32(sm + OFF_K + buf * (8 * KB_K));
 #pragma unroll
       for (int nh = 0; nh < 2; ++nh) {
 #pragma unroll
         for (int kk = 0; kk < kTR / 16; ++kk) {
-          const uint64_t adesc = smem_desc(pa + (kk / 4) * (kH * 128) + (kk % 4) * 32, 16, 1024, kSw128);
-          const uint64_t bdesc = smem_desc(ka + nh * 4 * (kTR * 128) + kk * 2048, kTR * 128, 1024, kSw128);
+          const uint64_t adesc = smem_desc(pa + kk * 32, 16, 1024, kSw128);
+          const uint64_t bdesc = smem_desc(ka + nh * 4 * KB_K + kk * 2048, KB_K, 1024, kSw128);
           mma_ss<0>(tmem + nh * 256, adesc, bdesc, idesc_pv, j > 0 || kk > 0);
         }
       }
-      tc_commit(pv_done);
+      tc_commit(&pv_done[buf]);
+    };
+    for (int j = 0; j <= ntiles; ++j) {
+      if (j < ntiles) {
+        if (!warp_wait(&k_full[j & 1], (uint32_t)(j >> 1) & 1u, a, abort)) break;
+        tc_fence_after();
+        if (lane == 0) issue_qk(j);
+        __syncwarp();
+      }
+      if (j > 0) {
+        if (!warp_wait(&p_full[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, a, abort)) break;
+        tc_fence_after();
+        if (lane == 0) issue_pv(j - 1);
+        __syncwarp();
+      }
     }
-  }
-  // ---- partial results
-  if (ntiles > 0 && live) live = __syncthreads_and(mbar_wait(pv_done, (uint32_t)(ntiles - 1) & 1u, a.status)) != 0;
-  tc_fence_after();
-  const int64_t pidx = ((int64_t)list * a.splits + blockIdx.x) * a.H + head;
-  if (warp < 4) {
+  } else {
+    // =================================================== softmax warps
+    const bool s_lane = lane >= 16;
+    const int head = warp * 16 + (lane & 15);
+    const uint32_t row_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    float m_ref = -INFINITY, l_sum = 0.f;
+    for (int j = 0; j < ntiles; ++j) {
+      const int buf = j & 1;
+      // k_full orders the loaders' row mask before this read; s_full the TMEM S
+      if (!warp_wait(&k_full[buf], (uint32_t)(j >> 1) & 1u, a, abort)) break;
+      if (!warp_wait(&s_full[buf], (uint32_t)(j >> 1) & 1u, a, abort)) break;
+      tc_fence_after();
+      uint32_t r0[32], r1[32];
+      tmem_ld_32(row_addr + buf * kTR, r0);
+      tmem_ld_32(row_addr + buf * kTR + 32, r1);
+      tmem_ld_wait(r0, r1);
+      const uint32_t m0 = mask_s[buf * 2], m1 = mask_s[buf * 2 + 1];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        if ((m0 >> q) & 1u) mx = fmaxf(mx, __uint_as_float(r0[q]));
+        if ((m1 >> q) & 1u) mx = fmaxf(mx, __uint_as_float(r1[q]));
+      }
+      mx *= a.sm_scale;  // sm_scale > 0 keeps the order
+      // reference max: set on the first rows seen, moved only by large jumps
+      float alpha = 1.f;
+      bool moved = false;
+      if (s_lane && mx > -INFINITY && (m_ref == -INFINITY || mx > m_ref + kRescale)) {
+        if (m_ref > -INFINITY) {
+          alpha = __expf(m_ref - mx);
+          moved = true;
+          l_sum *= alpha;
+        }
+        m_ref = mx;
+      }
+      const float ref = m_ref;
+      float sum = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int q = 0; q < 32; q += 2) {
+        const float p0 = ((m0 >> q) & 1u) && ref > -INFINITY ? __expf(__uint_as_float(r0[q]) * a.sm_scale - ref) : 0.f;
+        const float p1 = ((m0 >> (q + 1)) & 1u) && ref > -INFINITY ? __expf(__uint_as_float(r0[q + 1]) * a.sm_scale - ref) : 0.f;
+        const float p2 = ((m1 >> q) & 1u) && ref > -INFINITY ? __expf(__uint_as_float(r1[q]) * a.sm_scale - ref) : 0.f;
+        const float p3 = ((m1 >> (q + 1)) & 1u) && ref > -INFINITY ? __expf(__uint_as_float(r1[q + 1]) * a.sm_scale - ref) : 0.f;
+        sum += (p0 + p1) + (p2 + p3);
+        pk[q / 2] = pack_h2(p0, p1);
+        pk[16 + q / 2] = pack_h2(p2, p3);
+      }
+      if (s_lane) l_sum += sum;
+      // O is rescaled in place (lanes 0-15) only after the previous PV is done
+      const bool warp_moved = __any_sync(0xffffffffu, moved);
+      if (warp_moved && j > 0) {
+        if (!warp_wait(&pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, a, abort)) break;
+        tc_fence_after();
+        const float a_own = __shfl_sync(0xffffffffu, alpha, (lane & 15) + 16);
+        for (int c = 0; c < kD; c += 32) {
+          uint32_t r[32];
+          tmem_ld_32(row_addr + c, r);
+          tmem_ld_wait(r);
+          if (lane < 16) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * a_own);
+          }
+          tmem_st_32(row_addr + c, r);
+        }
+        tmem_st_wait();
+      }
+      // P[buf] is free once the PV of tile j-2 is done
+      if (j >= 2 && !warp_wait(&pv_done[buf], (uint32_t)((j - 2) >> 1) & 1u, a, abort)) break;
+      if (s_lane) {
+        uint8_t* pb = sm + OFF_P + buf * (kH * 128);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<uint4*>(pb + swz(head, q * 16)) =
+              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[buf]);
+    }
+    // ---- partial results: wait for the last PV, then O (lanes 0-15) and (ref, sum)
+    bool done = ntiles > 0 && !*abort;
+    if (done) done = warp_wait(&pv_done[(ntiles - 1) & 1], (uint32_t)((ntiles - 1) >> 1) & 1u, a, abort);
+    tc_fence_after();
+    const int64_t pidx = ((int64_t)list * a.splits + blockIdx.x) * a.H + head;
     for (int c = 0; c < kD; c += 32) {
       uint32_t r[32];
-      tmem_ld_32(tmem + ((uint32_t)(warp * 32) << 16) + c, r);
-      tmem_ld_wait();
+      tmem_ld_32(row_addr + c, r);
+      tmem_ld_wait(r);
       if (lane < 16) {
         float* po = a.part_o + pidx * kD + c;
 #pragma unroll
         for (int q = 0; q < 32; q += 4)
           *reinterpret_cast<float4*>(po + q) =
-              (ntiles > 0 && live) ? make_float4(__uint_as_float(r[q]), __uint_as_float(r[q + 1]),
-                                                 __uint_as_float(r[q + 2]), __uint_as_float(r[q + 3]))
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+              done ? make_float4(__uint_as_float(r[q]), __uint_as_float(r[q + 1]), __uint_as_float(r[q + 2]),
+                                 __uint_as_float(r[q + 3]))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-    if (softmax_thread) {
-      a.part_ml[pidx * 2] = live ? m_ref : -INFINITY;
-      a.part_ml[pidx * 2 + 1] = live ? l_sum : 0.f;
+    if (s_lane) {
+      a.part_ml[pidx * 2] = done ? m_ref : -INFINITY;
+      a.part_ml[pidx * 2 + 1] = done ? l_sum : 0.f;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -360,7 +475,7 @@ __global__ void __launch_bounds__(kThr, 1) attn_mma_kernel(const AttnLaunch a) {
 
 bool attn_mma_supported(const AttnLaunch& a) {
   return a.kv.f.fmt == LCSC_FMT_KV && a.D == 512 && a.Dv == 512 && a.H == 64 && a.v.data == nullptr &&
-         a.kv.f.row_bytes == 576 && (a.kv.f.dim - a.kv.f.rope) % 16 == 0 && a.rows_per_split % kTR == 0;
+         a.kv.f.row_bytes == 576 && a.kv.f.rope == 64 && a.rows_per_split % kTR == 0;
 }
 
 cudaError_t launch_attn_mma(const AttnLaunch& a, cudaStream_t stream) {

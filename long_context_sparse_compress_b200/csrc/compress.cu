@@ -56,6 +56,18 @@ __device__ __forceinline__ SeqSpan seq_span(const Span& s, int b, int64_t win_ca
 
 // ------------------------------------------------------------ mma helpers
 
+// 16-byte global -> shared copy that completes asynchronously; `live` false
+// fills the 16 bytes with zeros (nothing is read from `src`).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool live) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src), "r"(live ? 16 : 0)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+}
+
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
   const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
@@ -80,9 +92,17 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], 
 }
 
 // ------------------------------------------------------------ pool kernel
-// grid: (ceil(n_new_max / E), dim / NC, B); block 256.
+// A CTA owns up to 128 token rows and NC output channels.  Two tilings:
+//  * by entries (bulk calls, prefill): grid (ceil(n_new_max / E), dim / NC, B),
+//    E consecutive entries of one sequence, entry e on rows e*m .. e*m+G-1
+//    (overlapping groups share rows);
+//  * packed (a step that closes at most one group per sequence): grid
+//    (ceil(B / SP), dim / NC, 1), the groups of SP = 128 / G sequences stacked,
+//    entry e = sequence b0 + e on rows e*G .. e*G+G-1.
+// Rows whose position is below 0 (or whose sequence closes no group) are
+// masked out of the softmax.
 template <bool kBf16, int DIM, int NC>
-__global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E) {
+__global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E, bool packed) {
   using Elem = typename std::conditional<kBf16, uint16_t, float>::type;
   constexpr int XS = kBf16 ? DIM + 8 : DIM + 1;   // x tile row stride (elements)
   constexpr int WS = kBf16 ? NC + 8 : NC + 1;     // W chunk row stride
@@ -91,50 +111,98 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E)
   Elem* xs = reinterpret_cast<Elem*>(smem);
   Elem* ws = reinterpret_cast<Elem*>(smem + sizeof(Elem) * kRows * XS);
   float* zs = reinterpret_cast<float*>(ws);  // reuses the W chunk after the GEMM
+  __shared__ int64_t row_src[kRows];  // element offset of the row in x, or -1 (masked)
+  __shared__ int64_t ent_out[kRows];  // pooled output row, or -1
+  __shared__ int ent_row0[kRows];     // first tile row of the entry
+  __shared__ int n_ent, rows_used;
 
-  const int b = blockIdx.z;
   const int c0 = blockIdx.y * NC;
-  const SeqSpan sp = seq_span(a.span, b, a.window.capacity, a.entries.capacity);
-  const int64_t n_e = sp.g_hi - sp.g_lo;
-  const int64_t e0 = (int64_t)blockIdx.x * E;
-  if (!sp.ok || e0 >= n_e) return;
   const int m = a.span.m, G = a.span.G;
-  const int E_cta = (int)(n_e - e0 < E ? n_e - e0 : E);
-  const int R = E_cta * m + G - m;
-  const int64_t first_pos = (sp.g_lo + e0) * m + m - G;
   const int tid = threadIdx.x;
+  if (tid == 0) { n_ent = 0; rows_used = 0; }
+  __syncthreads();
+  if (packed) {
+    const int SP = kRows / G;
+    const int e = tid;
+    const int b = blockIdx.x * SP + e;
+    if (e < SP) {
+      bool valid = false;
+      SeqSpan sp;
+      if (b < a.B) {
+        sp = seq_span(a.span, b, a.window.capacity, a.entries.capacity);
+        valid = sp.ok && sp.g_hi - sp.g_lo == 1;
+      }
+      ent_out[e] = valid ? (int64_t)b * a.n_new_max : -1;
+      ent_row0[e] = e * G;
+      for (int j = 0; j < G; ++j) {
+        const int64_t pos = valid ? sp.g_lo * m + m - G + j : -1;
+        row_src[e * G + j] = (valid && pos >= 0) ? ((int64_t)b * a.n_x + (pos - sp.x_pos0)) * DIM : -1;
+      }
+      if (b < a.B) {
+        atomicMax(&n_ent, e + 1);
+        atomicMax(&rows_used, (e + 1) * G);
+      }
+    }
+    for (int r = SP * G + tid; r < kRows; r += kThreads) row_src[r] = -1;
+  } else {
+    const int b = blockIdx.z;
+    const SeqSpan sp = seq_span(a.span, b, a.window.capacity, a.entries.capacity);
+    const int64_t n_e = sp.ok ? sp.g_hi - sp.g_lo : 0;
+    const int64_t e0 = (int64_t)blockIdx.x * E;
+    const int E_cta = e0 < n_e ? (int)(n_e - e0 < E ? n_e - e0 : E) : 0;
+    const int R = E_cta > 0 ? E_cta * m + G - m : 0;
+    const int64_t first_pos = (sp.g_lo + e0) * m + m - G;
+    for (int r = tid; r < kRows; r += kThreads) {
+      const int64_t pos = first_pos + r;
+      row_src[r] = (r < R && pos >= 0) ? ((int64_t)b * a.n_x + (pos - sp.x_pos0)) * DIM : -1;
+    }
+    for (int e = tid; e < E_cta; e += kThreads) {
+      ent_out[e] = (int64_t)b * a.n_new_max + e0 + e;
+      ent_row0[e] = e * m;
+    }
+    if (tid == 0) { n_ent = E_cta; rows_used = R; }
+  }
+  __syncthreads();
+  const int E_cta = n_ent;
+  if (E_cta == 0) return;  // uniform
 
-  // ---- x tile: rows of positions first_pos .. first_pos + R - 1 (zero past R or < 0)
-  const Elem* xb = reinterpret_cast<const Elem*>(a.x) + (int64_t)b * a.n_x * DIM;
-  constexpr int VEC = 16 / sizeof(Elem);
-  for (int i = tid; i < kRows * (DIM / VEC); i += kThreads) {
-    const int r = i / (DIM / VEC), cv = (i % (DIM / VEC)) * VEC;
-    const int64_t pos = first_pos + r;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (r < R && pos >= 0) val = *reinterpret_cast<const uint4*>(xb + (pos - sp.x_pos0) * DIM + cv);
-    Elem* d = xs + r * XS + cv;
-    if constexpr (kBf16) {
-      *reinterpret_cast<uint4*>(d) = val;  // XS*2 bytes is a multiple of 16
-    } else {
-      const float* f = reinterpret_cast<const float*>(&val);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) d[j] = f[j];
-    }
-  }
-  // ---- W chunk: columns c0 .. c0 + NC of W [DIM][DIM]
+  // ---- x tile (zero for masked rows) and the W chunk (columns c0 .. c0 + NC
+  // of W [DIM][DIM]).  bf16: asynchronous 16-byte copies, all in flight at
+  // once; fp32: converted to the padded layout through registers.
+  const Elem* xg = reinterpret_cast<const Elem*>(a.x);
   const Elem* wg = reinterpret_cast<const Elem*>(a.w);
-  for (int i = tid; i < DIM * (NC / VEC); i += kThreads) {
-    const int k = i / (NC / VEC), cv = (i % (NC / VEC)) * VEC;
-    uint4 val = *reinterpret_cast<const uint4*>(wg + (int64_t)k * DIM + c0 + cv);
-    Elem* d = ws + k * WS + cv;
-    if constexpr (kBf16) {
-      *reinterpret_cast<uint4*>(d) = val;
-    } else {
+  constexpr int VEC = 16 / sizeof(Elem);
+  const int x_rows = kBf16 ? rows_used : kRows;
+  if constexpr (kBf16) {
+    for (int i = tid; i < x_rows * (DIM / VEC); i += kThreads) {
+      const int r = i / (DIM / VEC), cv = (i % (DIM / VEC)) * VEC;
+      const bool live = row_src[r] >= 0;
+      cp_async16(xs + r * XS + cv, live ? xg + row_src[r] + cv : xg, live);
+    }
+    for (int i = tid; i < DIM * (NC / VEC); i += kThreads) {
+      const int k = i / (NC / VEC), cv = (i % (NC / VEC)) * VEC;
+      cp_async16(ws + k * WS + cv, wg + (int64_t)k * DIM + c0 + cv, true);
+    }
+    cp_async_wait_all();
+  } else {
+    for (int i = tid; i < x_rows * (DIM / VEC); i += kThreads) {
+      const int r = i / (DIM / VEC), cv = (i % (DIM / VEC)) * VEC;
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (row_src[r] >= 0) val = *reinterpret_cast<const uint4*>(xg + row_src[r] + cv);
       const float* f = reinterpret_cast<const float*>(&val);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) d[j] = f[j];
+      for (int j = 0; j < 4; ++j) xs[r * XS + cv + j] = f[j];
+    }
+    for (int i = tid; i < DIM * (NC / VEC); i += kThreads) {
+      const int k = i / (NC / VEC), cv = (i % (NC / VEC)) * VEC;
+      const uint4 val = *reinterpret_cast<const uint4*>(wg + (int64_t)k * DIM + c0 + cv);
+      const float* f = reinterpret_cast<const float*>(&val);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) ws[k * WS + cv + j] = f[j];
     }
   }
+  // rows past the used ones are zero (read by the GEMM's last row block)
+  for (int i = tid; i < (((x_rows + 15) & ~15) - x_rows) * XS; i += kThreads) xs[x_rows * XS + i] = Elem(0);
   __syncthreads();
 
   // ---- z = x W for the 128 x NC tile
@@ -143,8 +211,9 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E)
     float acc[NC / 8][4];
 #pragma unroll
     for (int j = 0; j < NC / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+    const int ks_end = warp * 16 < rows_used ? DIM / 16 : 0;  // row blocks past the used rows stay zero
 #pragma unroll 4
-    for (int ks = 0; ks < DIM / 16; ++ks) {
+    for (int ks = 0; ks < ks_end; ++ks) {
       uint32_t af[4];
       ldsm_x4(af, xs + (warp * 16 + (lane % 16)) * XS + ks * 16 + (lane / 16) * 8);
 #pragma unroll
@@ -181,6 +250,13 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E)
 #pragma unroll
     for (int i = 0; i < RPT; ++i) zs[(rg + i * RG) * ZS + c] = acc[i];
   }
+  // positional biases of the NC channels, [G][NC], behind z in the dead W area
+  float* bs = zs + kRows * ZS;
+  for (int i = tid; i < G * (NC / 4); i += kThreads) {
+    const int j = i / (NC / 4), cv = (i % (NC / 4)) * 4;
+    cp_async16(bs + j * NC + cv, a.bpos + (int64_t)j * DIM + c0 + cv, true);
+  }
+  cp_async_wait_all();
   __syncthreads();
 
   // ---- group softmax over tokens and weighted sum, per (entry, channel)
@@ -198,23 +274,24 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E)
   for (int pb = 0; pb < n_pairs; pb += pairs_per_pass) {
     const int pair = pb + tid / TP;
     const int sub = tid % TP;
-    const bool active = pair < n_pairs;
-    const int e = active ? pair / NC : 0, c = active ? pair % NC : 0;
+    const bool active = pair < n_pairs && ent_out[pair / NC] >= 0;
+    const int e = pair < n_pairs ? pair / NC : 0, c = pair % NC;
+    const int r0 = ent_row0[e];
     float mx = -INFINITY;
     if (active) {
       for (int j = sub; j < G; j += TP) {
-        const int r = e * m + j;
-        if (first_pos + r < 0) continue;
-        mx = fmaxf(mx, zs[r * ZS + c] + a.bpos[j * DIM + c0 + c]);
+        const int r = r0 + j;
+        if (row_src[r] < 0) continue;
+        mx = fmaxf(mx, zs[r * ZS + c] + bs[j * NC + c]);
       }
     }
     mx = group_max(mx, TP);
     float den = 0.f, num = 0.f;
     if (active) {
       for (int j = sub; j < G; j += TP) {
-        const int r = e * m + j;
-        if (first_pos + r < 0) continue;
-        const float p = expf(zs[r * ZS + c] + a.bpos[j * DIM + c0 + c] - mx);
+        const int r = r0 + j;
+        if (row_src[r] < 0) continue;
+        const float p = expf(zs[r * ZS + c] + bs[j * NC + c] - mx);
         float xv;
         if constexpr (kBf16) xv = bf16_val(xs[r * XS + c0 + c]);
         else xv = xs[r * XS + c0 + c];
@@ -226,8 +303,7 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E)
       den += __shfl_xor_sync(0xffffffffu, den, o);
       num += __shfl_xor_sync(0xffffffffu, num, o);
     }
-    if (active && sub == 0)
-      a.pooled[((int64_t)b * a.n_new_max + e0 + e) * DIM + c0 + c] = num / den;
+    if (active && sub == 0) a.pooled[ent_out[e] * DIM + c0 + c] = num / den;
   }
 }
 
@@ -279,18 +355,21 @@ __global__ void __launch_bounds__(256) encode_rows_kernel(const float* rows, int
 
 template <bool kBf16, int DIM, int NC>
 cudaError_t launch_pool(const CompressLaunch& a, int E, cudaStream_t stream) {
+  const bool packed = a.span.ctx_len != nullptr && a.n_new_max == 1 && a.span.G <= kRows;
   using Elem = typename std::conditional<kBf16, uint16_t, float>::type;
   constexpr int XS = kBf16 ? DIM + 8 : DIM + 1;
   constexpr int WS = kBf16 ? NC + 8 : NC + 1;
   size_t smem = sizeof(Elem) * kRows * XS;
   size_t wz = sizeof(Elem) * DIM * WS;
-  const size_t zbytes = sizeof(float) * kRows * (NC + 1);
+  const size_t zbytes = sizeof(float) * (kRows * (NC + 1) + kRows * NC);  // z, then biases of <= 128 tokens
   smem += wz > zbytes ? wz : zbytes;
   auto kern = pool_kernel<kBf16, DIM, NC>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((a.n_new_max + E - 1) / E), DIM / NC, a.B);
-  kern<<<grid, kThreads, smem, stream>>>(a, E);
+  const int SP = kRows / a.span.G;
+  dim3 grid = packed ? dim3((unsigned)((a.B + SP - 1) / SP), DIM / NC, 1)
+                     : dim3((unsigned)((a.n_new_max + E - 1) / E), DIM / NC, a.B);
+  kern<<<grid, kThreads, smem, stream>>>(a, E, packed);
   return cudaGetLastError();
 }
 

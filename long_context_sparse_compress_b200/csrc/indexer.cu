@@ -14,18 +14,22 @@
 //
 // Top-k is an exact radix select on the order-preserving integer image of
 // the float scores, three digits of 12 / 12 / 8 bits:
-//   pass 1 (all slices of a list): histogram of digit 1;
-//   pass 2 (all slices): every score above the threshold bin goes straight to
-//          the output, scores in the threshold bin become candidates and are
-//          histogrammed on digit 2;
-//   pass 3 (one CTA per list): digits 2 and 3 over the candidates; ties at
-//          the final threshold are taken in arbitrary order.
+//   digit 1: histogrammed while the scores are written (tensor-core scoring)
+//          or by a pass over them; the last CTA of a list finds the
+//          threshold bin;
+//   collect (all slices of a list): scores above the threshold bin are
+//          marked in the list's selection bitmap, those in it become
+//          candidates;
+//   final (one CTA per list): digits 2 and 3 over the candidates (held in
+//          shared memory), ties to the lowest index, the chosen ones marked,
+//          and the bitmap compacted into the output in index order.
 #include "kernels.cuh"
+#include "topk.cuh"
 
 namespace lcsc {
 namespace {
 
-constexpr int kBins = 4096;
+constexpr int kBins = kTopkBins;
 
 // Entries visible to query t of sequence b.  A context length that would
 // reach past the n_max entries the call was sized for is invalid: nothing is
@@ -42,6 +46,14 @@ __device__ __forceinline__ int64_t visible(const IndexLaunch& a, int b, int t, b
 template <int VPL>
 __global__ void __launch_bounds__(256) quantize_queries_kernel(IndexLaunch a) {
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+  {  // the top-k's digit-1 histograms and counters start at zero
+    const int64_t lists = (int64_t)a.B * a.T;
+    const int64_t n_zero = lists * (kTopkBins + 8);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_zero; i += (int64_t)gridDim.x * blockDim.x) {
+      if (i < lists * kTopkBins) a.hist[(i / kTopkBins) * 2 * kTopkBins + i % kTopkBins] = 0u;
+      else a.counters[i - lists * kTopkBins] = 0u;
+    }
+  }
   const int64_t row = (int64_t)blockIdx.x * 8 + warp;  // over B*T*H_I
   const int64_t per_b = (int64_t)a.T * a.H_I;
   if (row >= (int64_t)a.B * per_b) return;
@@ -157,15 +169,10 @@ __global__ void __launch_bounds__(256) score_kernel(IndexLaunch a) {
     sc = fmaf(wh, fmaxf(acc[i], 0.f), sc);
   }
   for (int o = HG >> 1; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
-  if (live && hg == 0) a.scores[(int64_t)list * a.n_max + g] = sc * sk_row;
+  if (live && hg == 0) a.scores[(int64_t)list * a.stride + g] = sc * sk_row;
 }
 
 // --------------------------------------------------------------- top-k
-
-struct Thresh {
-  uint32_t bin;    // threshold bin
-  uint32_t above;  // elements in bins above it
-};
 
 // Threshold bin of a 4096-bin histogram for `need` (>= 1) elements: the
 // largest bin t with sum_{d >= t} hist[d] >= need.  512 threads.
@@ -215,86 +222,96 @@ __device__ __forceinline__ ListInfo list_info(const IndexLaunch& a, int list, in
   bool ok;
   li.n = visible(a, list / a.T, list % a.T, &ok);
   li.k_eff = li.n < a.k ? li.n : a.k;
-  const int64_t per = (li.n + slices - 1) / slices;
+  const int64_t per = ((li.n + slices - 1) / slices + 31) / 32 * 32;  // whole bitmap words
   li.lo = (int64_t)blockIdx.x * per;
   li.hi = li.lo + per < li.n ? li.lo + per : li.n;
   return li;
 }
 
+// f(g, score) for every g in [lo, hi) of one score row: four 16-byte loads
+// in flight per thread (lo is a multiple of 4 and rows start 16-byte aligned).
+template <class F>
+__device__ __forceinline__ void scan_scores(const float* s, int64_t lo, int64_t hi, F&& f) {
+  const int64_t n4 = hi > lo ? (hi - lo) >> 2 : 0;
+  const float4* s4 = reinterpret_cast<const float4*>(s + lo);
+  for (int64_t base = 0; base < n4; base += 4 * 512) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = base + u * 512 + threadIdx.x;
+      v[u] = i < n4 ? s4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = base + u * 512 + threadIdx.x;
+      if (i < n4) {
+        const int64_t g = lo + 4 * i;
+        f(g, v[u].x);
+        f(g + 1, v[u].y);
+        f(g + 2, v[u].z);
+        f(g + 3, v[u].w);
+      }
+    }
+  }
+  for (int64_t g = lo + 4 * n4 + threadIdx.x; g < hi; g += 512) f(g, s[g]);
+}
+
+// Digit-1 histogram of one slice of a list (scores written by a kernel that
+// did not histogram them); the list's last CTA finds the threshold bin.
 __global__ void __launch_bounds__(512) topk_hist_kernel(IndexLaunch a, int slices) {
   __shared__ uint32_t h[kBins];
   const int list = blockIdx.y;
   const ListInfo li = list_info(a, list, slices);
-  if (li.n <= a.k) return;
   for (int i = threadIdx.x; i < kBins; i += 512) h[i] = 0;
   __syncthreads();
-  const float* s = a.scores + (int64_t)list * a.n_max;
-  for (int64_t g = li.lo + threadIdx.x; g < li.hi; g += 512) atomicAdd(&h[float_key(s[g]) >> 20], 1u);
-  __syncthreads();
-  uint32_t* gh = a.hist + (int64_t)list * 2 * kBins;
-  for (int i = threadIdx.x; i < kBins; i += 512)
-    if (h[i]) atomicAdd(&gh[i], h[i]);
+  const float* s = a.scores + (int64_t)list * a.stride;
+  if (li.n > a.k) scan_scores(s, li.lo, li.hi, [&](int64_t, float v) { atomicAdd(&h[float_key(v) >> 20], 1u); });
+  const int64_t n = li.n;
+  hist_finish(h, li.n > a.k, 1, a.hist, a.counters, list, list, gridDim.x, &n, a.k);
 }
 
+// All slices of a list: scores above the digit-1 threshold bin go to the
+// output, those in it to the candidate list.
 __global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int slices) {
-  __shared__ uint32_t h[kBins];
-  __shared__ uint32_t scratch[512];
   const int list = blockIdx.y;
   const ListInfo li = list_info(a, list, slices);
-  const float* s = a.scores + (int64_t)list * a.n_max;
+  const float* s = a.scores + (int64_t)list * a.stride;
   int32_t* out_i = a.out_idx + (int64_t)list * a.k;
   float* out_s = a.out_score ? a.out_score + (int64_t)list * a.k : nullptr;
-  if (li.n <= a.k) {  // every visible entry is kept
+  if (li.n <= a.k) {  // every visible entry is kept, in index order
     for (int64_t g = li.lo + threadIdx.x; g < li.hi; g += 512) {
       out_i[g] = (int32_t)g;
       if (out_s) out_s[g] = s[g];
     }
     return;
   }
-  uint32_t* gh = a.hist + (int64_t)list * 2 * kBins;
-  for (int i = threadIdx.x; i < kBins; i += 512) h[i] = gh[i];
+  uint32_t* ctr = a.counters + (int64_t)list * 8;
+  const uint32_t t1 = ctr[3];
+  uint32_t* bits = a.sel_bits + (int64_t)list * a.bit_stride;
+  for (int64_t w = li.lo / 32 + threadIdx.x; w < (li.hi + 31) / 32; w += 512) bits[w] = 0u;
   __syncthreads();
-  const Thresh th = find_threshold(h, (uint32_t)li.k_eff, scratch);
-  for (int i = threadIdx.x; i < kBins; i += 512) h[i] = 0;
-  __syncthreads();
-  uint32_t* ctr = a.counters + (int64_t)list * 4;
-  uint32_t* cand = a.cand + (int64_t)list * a.n_max;
-  for (int64_t g = li.lo + threadIdx.x; g < li.hi; g += 512) {
-    const float v = s[g];
-    const uint32_t key = float_key(v);
-    const uint32_t d1 = key >> 20;
-    if (d1 > th.bin) {
-      const uint32_t slot = atomicAdd(&ctr[0], 1u);
-      out_i[slot] = (int32_t)g;
-      if (out_s) out_s[slot] = v;
-    } else if (d1 == th.bin) {
-      const uint32_t c = atomicAdd(&ctr[1], 1u);
-      cand[c] = (uint32_t)g;
-      atomicAdd(&h[(key >> 8) & 0xFFF], 1u);
-    }
-  }
-  __syncthreads();
-  uint32_t* gh2 = gh + kBins;
-  for (int i = threadIdx.x; i < kBins; i += 512)
-    if (h[i]) atomicAdd(&gh2[i], h[i]);
-  if (blockIdx.x == 0 && threadIdx.x == 0) ctr[2] = th.above;
+  uint32_t* cand = a.cand + (int64_t)list * a.stride;
+  scan_scores(s, li.lo, li.hi, [&](int64_t g, float v) {
+    const uint32_t d1 = float_key(v) >> 20;
+    if (d1 > t1) atomicOr(&bits[g >> 5], 1u << (g & 31));
+    const uint32_t c = warp_append(&ctr[1], d1 == t1);
+    if (d1 == t1) cand[c] = (uint32_t)g;
+  });
 }
 
 // Smallest index bound tau such that at least `need` of the tied candidates
 // (key == tkey) have index < tau: ties then go to the lowest indices, as in
 // a stable sort.  512 threads; returns n when every tied candidate is needed.
-__device__ uint32_t tie_bound(const uint32_t* cand, uint32_t n_cand, const float* s, uint32_t tkey,
-                              uint32_t need, uint32_t n, uint32_t* cnt) {
+template <class KeyAt, class IdxAt>
+__device__ uint32_t tie_bound(uint32_t n_cand, KeyAt key_at, IdxAt idx_at, uint32_t tkey, uint32_t need,
+                              uint32_t n, uint32_t* cnt) {
   uint32_t lo = 0, hi = n;  // count(idx < hi) >= need holds for hi = n
   while (lo < hi) {
     const uint32_t mid = lo + (hi - lo) / 2;
     if (threadIdx.x == 0) *cnt = 0;
     __syncthreads();
     uint32_t local = 0;
-    for (uint32_t c = threadIdx.x; c < n_cand; c += 512) {
-      const uint32_t g = cand[c];
-      local += (g < mid && float_key(s[g]) == tkey) ? 1u : 0u;
-    }
+    for (uint32_t c = threadIdx.x; c < n_cand; c += 512) local += (idx_at(c) < mid && key_at(c) == tkey) ? 1u : 0u;
     if (local) atomicAdd(cnt, local);
     __syncthreads();
     const uint32_t total = *cnt;
@@ -305,120 +322,131 @@ __device__ uint32_t tie_bound(const uint32_t* cand, uint32_t n_cand, const float
   return lo;
 }
 
-// Sort the k_eff selected (index, score) pairs by index, in shared memory
-// (bitonic network over the next power of two, <= 2048).
-__device__ void sort_selection(int32_t* out_i, float* out_s, int k_eff, int32_t* si, float* sv) {
-  int P = 1;
-  while (P < k_eff) P <<= 1;
-  for (int j = threadIdx.x; j < P; j += 512) {
-    si[j] = j < k_eff ? out_i[j] : INT32_MAX;
-    sv[j] = (j < k_eff && out_s) ? out_s[j] : 0.f;
-  }
-  __syncthreads();
-  for (int size = 2; size <= P; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int j = threadIdx.x; j < P; j += 512) {
-        const int partner = j ^ stride;
-        if (partner > j) {
-          const bool up = (j & size) == 0;
-          const int32_t a = si[j], b = si[partner];
-          if ((a > b) == up) {
-            si[j] = b;
-            si[partner] = a;
-            const float t = sv[j];
-            sv[j] = sv[partner];
-            sv[partner] = t;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
-  for (int j = threadIdx.x; j < k_eff; j += 512) {
-    out_i[j] = si[j];
-    if (out_s) out_s[j] = sv[j];
-  }
-}
+constexpr int kCandCap = 12288;  // candidates held in shared memory (keys + indices: 96 KB)
+constexpr size_t kFinalSmem = (size_t)kCandCap * 8;
 
+// One CTA per list: digits 2 and 3 over the candidates (the scores in the
+// digit-1 threshold bin), ties to the lowest index; the chosen candidates
+// join the collect pass's marks in the bitmap, which is then compacted into
+// the output (index order).
 __global__ void __launch_bounds__(512) topk_final_kernel(IndexLaunch a) {
   __shared__ uint32_t h[kBins];
   __shared__ uint32_t scratch[512];
   __shared__ uint32_t cnt;
-  __shared__ int32_t si[2048];
-  __shared__ float sv[2048];
+  __shared__ uint32_t warp_sum[16];
+  extern __shared__ uint32_t dyn[];
+  uint32_t* ck = dyn;              // candidate keys
+  uint32_t* cg = dyn + kCandCap;   // candidate indices
   const int list = blockIdx.x;
+  const int tid = threadIdx.x;
   bool ok;
   const int64_t n = visible(a, list / a.T, list % a.T, &ok);
-  if (!ok && threadIdx.x == 0 && a.status) atomicOr(a.status, LCSC_DEV_BAD_LENGTH);
+  if (!ok && tid == 0 && a.status) atomicOr(a.status, LCSC_DEV_BAD_LENGTH);
   const int64_t k_eff = n < a.k ? n : a.k;
   int32_t* out_i = a.out_idx + (int64_t)list * a.k;
   float* out_s = a.out_score ? a.out_score + (int64_t)list * a.k : nullptr;
-  for (int64_t j = k_eff + threadIdx.x; j < a.k; j += 512) {
+  for (int64_t j = k_eff + tid; j < a.k; j += 512) {
     out_i[j] = -1;
     if (out_s) out_s[j] = -INFINITY;
   }
   if (n <= a.k) return;  // every visible entry was written in order by the collect pass
-  uint32_t* ctr = a.counters + (int64_t)list * 4;
-  const uint32_t above1 = ctr[2];
+  const uint32_t* ctr = a.counters + (int64_t)list * 8;
+  const uint32_t need2 = (uint32_t)k_eff - ctr[2];  // >= 1 by construction
+  const uint32_t t1 = ctr[3];
   const uint32_t n_cand = ctr[1];
-  const uint32_t need = (uint32_t)k_eff - above1;  // >= 1 by construction
-  const uint32_t* cand = a.cand + (int64_t)list * a.n_max;
-  const float* s = a.scores + (int64_t)list * a.n_max;
-  uint32_t* gh2 = a.hist + (int64_t)list * 2 * kBins + kBins;
-  for (int i = threadIdx.x; i < kBins; i += 512) h[i] = gh2[i];
-  __syncthreads();
-  const Thresh t2 = find_threshold(h, need, scratch);
-  for (int i = threadIdx.x; i < kBins; i += 512) h[i] = 0;
-  __syncthreads();
-  // digit 2 above the threshold: keep; at it: histogram digit 3
-  for (uint32_t c = threadIdx.x; c < n_cand; c += 512) {
-    const uint32_t g = cand[c];
-    const float v = s[g];
-    const uint32_t key = float_key(v);
-    const uint32_t d2 = (key >> 8) & 0xFFF;
-    if (d2 > t2.bin) {
-      const uint32_t slot = atomicAdd(&ctr[0], 1u);
-      out_i[slot] = (int32_t)g;
-      if (out_s) out_s[slot] = v;
-    } else if (d2 == t2.bin) {
-      atomicAdd(&h[key & 0xFF], 1u);
+  const uint32_t* cand = a.cand + (int64_t)list * a.stride;
+  const float* s = a.scores + (int64_t)list * a.stride;
+  uint32_t* bits = a.sel_bits + (int64_t)list * a.bit_stride;
+  const bool cached = n_cand <= (uint32_t)kCandCap;
+  if (cached) {
+    for (uint32_t c = tid; c < n_cand; c += 512) {
+      const uint32_t g = cand[c];
+      cg[c] = g;
+      ck[c] = float_key(s[g]);
     }
   }
+  auto key_at = [&](uint32_t c) { return cached ? ck[c] : float_key(s[cand[c]]); };
+  auto idx_at = [&](uint32_t c) { return cached ? cg[c] : cand[c]; };
+  // digit 2 (key bits 8 .. 19)
+  for (int i = tid; i < kBins; i += 512) h[i] = 0;
   __syncthreads();
-  const uint32_t need3 = need - t2.above;
+  for (uint32_t c = tid; c < n_cand; c += 512) atomicAdd(&h[(key_at(c) >> 8) & 0xFFF], 1u);
+  __syncthreads();
+  const Thresh t2 = find_threshold(h, need2, scratch);
+  const uint32_t need3 = need2 - t2.above;
+  // digit 3 (key bits 0 .. 7) inside the digit-2 threshold bin
+  for (int i = tid; i < kBins; i += 512) h[i] = 0;
+  __syncthreads();
+  for (uint32_t c = tid; c < n_cand; c += 512) {
+    const uint32_t key = key_at(c);
+    if (((key >> 8) & 0xFFF) == t2.bin) atomicAdd(&h[key & 0xFF], 1u);
+  }
+  __syncthreads();
   const Thresh t3 = find_threshold(h, need3, scratch);
   const uint32_t ties = need3 - t3.above;
   const uint32_t n_tied = h[t3.bin];
   __syncthreads();
-  // the threshold key itself: candidate digit 1 is shared; rebuild it from any tied element
-  uint32_t tau = (uint32_t)n;
-  if (n_tied > ties) {
-    // every tied element has the same full key: digit 1 | digit 2 | digit 3
-    __shared__ uint32_t tkey;
-    if (threadIdx.x == 0) tkey = 0xFFFFFFFFu;
-    __syncthreads();
-    for (uint32_t c = threadIdx.x; c < n_cand; c += 512) {
-      const uint32_t key = float_key(s[cand[c]]);
-      if (((key >> 8) & 0xFFF) == t2.bin && (key & 0xFF) == t3.bin) atomicMin(&tkey, key);
-    }
-    __syncthreads();
-    tau = tie_bound(cand, n_cand, s, tkey, ties, (uint32_t)n, &cnt);
+  const uint32_t tkey = (t1 << 20) | (t2.bin << 8) | t3.bin;
+  uint32_t tau = (uint32_t)n;  // ties go to the lowest indices
+  if (n_tied > ties) tau = tie_bound(n_cand, key_at, idx_at, tkey, ties, (uint32_t)n, &cnt);
+  for (uint32_t c = tid; c < n_cand; c += 512) {
+    const uint32_t key = key_at(c), g = idx_at(c);
+    if (key > tkey || (key == tkey && g < tau)) atomicOr(&bits[g >> 5], 1u << (g & 31));
   }
-  for (uint32_t c = threadIdx.x; c < n_cand; c += 512) {
-    const uint32_t g = cand[c];
-    const float v = s[g];
-    const uint32_t key = float_key(v);
-    if (((key >> 8) & 0xFFF) != t2.bin) continue;
-    const uint32_t d3 = key & 0xFF;
-    if (d3 > t3.bin || (d3 == t3.bin && g < tau)) {
-      const uint32_t slot = atomicAdd(&ctr[0], 1u);
-      out_i[slot] = (int32_t)g;
-      if (out_s) out_s[slot] = v;
-    }
-  }
-  __threadfence_block();
   __syncthreads();
-  sort_selection(out_i, out_s, (int)k_eff, si, sv);
+  // compaction: thread t owns bitmap words [16 t, 16 t + 16) of each 8192-word block
+  const int64_t words = (n + 31) / 32;
+  uint32_t base = 0;
+  for (int64_t w0 = 0; w0 < words; w0 += 16 * 512) {
+    const int64_t wt = w0 + 16 * tid;
+    uint32_t wv[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 v = wt + 4 * q < words ? __ldcg(reinterpret_cast<const uint4*>(bits + wt) + q) : make_uint4(0, 0, 0, 0);
+      wv[4 * q] = v.x;
+      wv[4 * q + 1] = v.y;
+      wv[4 * q + 2] = v.z;
+      wv[4 * q + 3] = v.w;
+    }
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+      if (wt + q >= words) wv[q] = 0u;  // past the list's last word (never cleared)
+    uint32_t local = 0;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) local += __popc(wv[q]);
+    // exclusive scan of `local` over the 512 threads
+    uint32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if ((tid & 31) >= o) incl += v;
+    }
+    if ((tid & 31) == 31) warp_sum[tid >> 5] = incl;
+    __syncthreads();
+    uint32_t before = 0, block_total = 0;
+    for (int w = 0; w < 16; ++w) {
+      const uint32_t ws = warp_sum[w];
+      if (w < (tid >> 5)) before += ws;
+      block_total += ws;
+    }
+    uint32_t off = base + before + incl - local;
+#pragma unroll 1
+    for (int q = 0; q < 16; ++q) {
+      uint32_t bw = wv[q];
+      while (bw) {
+        const int bit = __ffs(bw) - 1;
+        bw &= bw - 1;
+        const int64_t g = (wt + q) * 32 + bit;
+        if (off < (uint32_t)k_eff) {
+          out_i[off] = (int32_t)g;
+          if (out_s) out_s[off] = s[g];
+        }
+        ++off;
+      }
+    }
+    base += block_total;
+    __syncthreads();
+  }
 }
 
 }  // namespace
@@ -450,21 +478,22 @@ cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_topk(const IndexLaunch& a, cudaStream_t stream) {
+  // the histograms and counters were zeroed by the query quantisation of
+  // the scoring launch; tensor-core scoring also built the digit-1 histogram
   const int lists = a.B * a.T;
   cudaError_t e;
-  // histograms and counters start at zero
-  e = cudaMemsetAsync(a.hist, 0, sizeof(uint32_t) * (size_t)lists * 2 * kBins, stream);
-  if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(a.counters, 0, sizeof(uint32_t) * (size_t)lists * 4, stream);
-  if (e != cudaSuccess) return e;
   int slices = (int)((a.n_max + 16383) / 16384);
   if (slices < 1) slices = 1;
   dim3 tgrid(slices, lists);
-  topk_hist_kernel<<<tgrid, 512, 0, stream>>>(a, slices);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (!index_mma_supported(a)) {
+    topk_hist_kernel<<<tgrid, 512, 0, stream>>>(a, slices);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   topk_collect_kernel<<<tgrid, 512, 0, stream>>>(a, slices);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  topk_final_kernel<<<lists, 512, 0, stream>>>(a);
+  e = cudaFuncSetAttribute(topk_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFinalSmem);
+  if (e != cudaSuccess) return e;
+  topk_final_kernel<<<lists, 512, kFinalSmem, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -17,11 +17,13 @@
 // (hardware swizzle) into a STAGES-deep ring, warp 1 issues the MMAs into
 // NACC TMEM accumulators, warps 2-9 (two groups of four taking alternate
 // tiles) drain them with tcgen05.ld, apply ReLU and the head weights, and
-// write one fp32 score per (query, key).
+// write one fp32 score per (query, key) and count it in the list's
+// shared-memory histogram of the top-k's first digit.
 #include <cudaTypedefs.h>
 
 #include "kernels.cuh"
 #include "sm100.cuh"
+#include "topk.cuh"
 
 namespace lcsc {
 namespace {
@@ -36,8 +38,12 @@ struct MmaArgs {
   const int32_t* ctx_len;
   int B, T, m;
   int64_t n_max;
-  float* scores;           // [B*T][n_max]
+  int64_t stride;          // score row stride
+  float* scores;           // [B*T][stride]
   int chunks;              // CTAs per (sequence, query group)
+  uint32_t* hist;          // top-k digit-1 histograms [B*T][2][4096] (zeroed)
+  uint32_t* counters;      // top-k counters [B*T][8] (zeroed)
+  int64_t k;               // top-k
   int32_t* status;
 };
 
@@ -73,7 +79,8 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_SFB + SFB_BYTES;
   static constexpr int NBARS = 2 * STAGES + 2 * NACC + 1;
   static constexpr int OFF_W = OFF_BAR + NBARS * 8;
-  static constexpr int OFF_TMEM = OFF_W + N * 4;
+  static constexpr int OFF_HIST = OFF_W + N * 4;  // NQ x 4096 digit-1 counts of the scores written
+  static constexpr int OFF_TMEM = OFF_HIST + NQ * kTopkBins * 4;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + slack to align the base
   static_assert(COLS_USED <= 512, "TMEM budget");
   static_assert(A_BYTES % 1024 == 0 && Q_BYTES % 1024 == 0, "swizzle atoms need 1024-byte alignment");
@@ -104,12 +111,21 @@ __global__ void __launch_bounds__(320, 1)
   const int t0 = (blockIdx.y % groups) * NQ;
   const int64_t L = a.ctx_len[b];
   const bool ok = L >= a.T && L / a.m <= a.n_max;
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(sm + C::OFF_HIST);
+  const int64_t list0 = (int64_t)b * a.T + t0;
+  int64_t nvis[NQ];
+#pragma unroll
+  for (int l = 0; l < NQ; ++l) nvis[l] = ok ? (L - a.T + t0 + l + 1) / a.m : 0;
   const int64_t n_last = ok ? (L - a.T + t0 + NQ) / a.m : 0;  // N(p) of the group's last query
   const int64_t tiles = (n_last + C::TILE - 1) / C::TILE;
   const int64_t per = (tiles + a.chunks - 1) / a.chunks;
   const int64_t tile_lo = (int64_t)blockIdx.x * per;
   const int64_t tile_hi = tile_lo + per < tiles ? tile_lo + per : tiles;
-  if (tile_hi <= tile_lo) return;  // uniform over the CTA, before any barrier or TMEM use
+  if (tile_hi <= tile_lo) {  // uniform over the CTA, before any barrier or TMEM use
+    hist_finish(hist_s, false, NQ, a.hist, a.counters, list0, list0, gridDim.x, nvis, a.k);
+    return;
+  }
+  for (int i = threadIdx.x; i < NQ * kTopkBins; i += blockDim.x) hist_s[i] = 0u;
   const int ntile = (int)(tile_hi - tile_lo);
 
   if (threadIdx.x == 0) {
@@ -256,7 +272,11 @@ __global__ void __launch_bounds__(320, 1)
         const float acc = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
         const int t = t0 + nq;
         const int64_t n_p = (L - a.T + t + 1) / a.m;
-        if (g < n_p) a.scores[((int64_t)b * a.T + t) * a.n_max + g] = acc * sk;
+        if (g < n_p) {
+          const float v = acc * sk;
+          a.scores[((int64_t)b * a.T + t) * a.stride + g] = v;
+          atomicAdd(&hist_s[nq * kTopkBins + (float_key(v) >> 20)], 1u);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -268,6 +288,7 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+  hist_finish(hist_s, true, NQ, a.hist, a.counters, list0, list0, gridDim.x, nvis, a.k);
 }
 
 // ---------------------------------------------------------------- host side
@@ -326,7 +347,11 @@ cudaError_t launch_mma(const IndexLaunch& a, cudaStream_t stream) {
   m.T = a.T;
   m.m = a.m;
   m.n_max = a.n_max;
+  m.stride = a.stride;
   m.scores = a.scores;
+  m.hist = a.hist;
+  m.counters = a.counters;
+  m.k = a.k;
   m.status = a.status;
   const int groups = a.T / NQ;
   const int64_t ctas = (int64_t)a.B * groups;

@@ -52,11 +52,14 @@ struct IndexLaunch {
   const int32_t* ctx_len;
   int B, T, H_I, d_I, m, k;
   int64_t n_max;
-  float* scores;        // [B*T][n_max]
+  int64_t stride;       // score / candidate row stride: n_max rounded up to 4
+  float* scores;        // [B*T][stride]
   // top-k workspace
   uint32_t* hist;       // [B*T][2][4096]
-  uint32_t* counters;   // [B*T][4]
-  uint32_t* cand;       // [B*T][n_max]
+  uint32_t* counters;   // [B*T][8]
+  uint32_t* cand;       // [B*T][stride]
+  uint32_t* sel_bits;   // [B*T][bit_stride] selected-entry bitmap
+  int64_t bit_stride;   // words per bitmap row: ceil(stride / 32) rounded up to 4
   int32_t* out_idx;     // [B*T][k]
   float* out_score;     // [B*T][k] or nullptr
   int32_t* status;
