@@ -230,28 +230,47 @@ __global__ void __launch_bounds__(kThreads) attn_partial_kernel(AttnLaunch a) {
   }
 }
 
-// grid (B*T, H); block DV threads (<= 512).
+// grid (B*T, H); block DV threads (<= 512), one output dim each.  The
+// splits are read eight at a time with every load of a batch in flight.
 template <int DV>
-__global__ void attn_combine_kernel(AttnLaunch a) {
+__global__ void __launch_bounds__(DV) attn_combine_kernel(AttnLaunch a) {
+  constexpr int U = 8;
   const int list = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
   const float sigma = a.sink ? a.sink[h] : -INFINITY;
+  const float* ml = a.part_ml + ((int64_t)list * a.splits * a.H + h) * 2;  // split s at ml[s * H * 2]
+  const float* po = a.part_o + ((int64_t)list * a.splits * a.H + h) * DV + d;
+  const int64_t ml_step = (int64_t)a.H * 2, o_step = (int64_t)a.H * DV;
   float M = sigma;
-  for (int s = 0; s < a.splits; ++s)
-    M = fmaxf(M, a.part_ml[(((int64_t)list * a.splits + s) * a.H + h) * 2]);
+  for (int s0 = 0; s0 < a.splits; s0 += U) {
+    float m[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) m[u] = s0 + u < a.splits ? ml[(s0 + u) * ml_step] : -INFINITY;
+#pragma unroll
+    for (int u = 0; u < U; ++u) M = fmaxf(M, m[u]);
+  }
   float den = (M == -INFINITY) ? 0.f : expf(sigma - M);
   float acc = 0.f;
-  for (int s = 0; s < a.splits; ++s) {
-    const int64_t pidx = ((int64_t)list * a.splits + s) * a.H + h;
-    const float ms = a.part_ml[pidx * 2];
-    if (ms == -INFINITY) continue;
-    const float f = expf(ms - M);
-    den = fmaf(a.part_ml[pidx * 2 + 1], f, den);
-    acc = fmaf(a.part_o[pidx * DV + d], f, acc);
+  for (int s0 = 0; s0 < a.splits; s0 += U) {
+    float m[U], l[U], o[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const bool in = s0 + u < a.splits;
+      m[u] = in ? ml[(s0 + u) * ml_step] : -INFINITY;
+      l[u] = in ? ml[(s0 + u) * ml_step + 1] : 0.f;
+      o[u] = in ? po[(s0 + u) * o_step] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (m[u] == -INFINITY) continue;  // an empty split (its O and sum are zero)
+      const float f = expf(m[u] - M);
+      den = fmaf(l[u], f, den);
+      acc = fmaf(o[u], f, acc);
+    }
   }
-  const float o = den > 0.f ? acc / den : 0.f;
+  const float out = den > 0.f ? acc / den : 0.f;
   const int64_t oi = ((int64_t)list * a.H + h) * DV + d;
-  if (a.q_dtype == LCSC_DT_BF16) reinterpret_cast<uint16_t*>(a.out)[oi] = bf16_code(o);
-  else reinterpret_cast<float*>(a.out)[oi] = o;
+  if (a.q_dtype == LCSC_DT_BF16) reinterpret_cast<uint16_t*>(a.out)[oi] = bf16_code(out);
+  else reinterpret_cast<float*>(a.out)[oi] = out;
   if (a.lse && d == 0) a.lse[(int64_t)list * a.H + h] = (den > 0.f) ? M + logf(den) : -INFINITY;
 }
 

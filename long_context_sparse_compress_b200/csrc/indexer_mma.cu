@@ -13,11 +13,13 @@
 //  * FP8 keys and queries: tcgen05.mma kind::f8f6f4 on the codes; the
 //    per-row scales are positive, so the epilogue applies them outside ReLU:
 //    s = sk[g] * sum_h (w[h] sq[h]) ReLU(acc[h]).
-// Warp roles (320 threads, one CTA per SM): warp 0 streams key tiles with TMA
-// (hardware swizzle) into a STAGES-deep ring, warp 1 issues the MMAs into
-// NACC TMEM accumulators, warps 2-9 (two groups of four taking alternate
-// tiles) drain them with tcgen05.ld, apply ReLU and the head weights, and
-// write one fp32 score per (query, key) and count it in the list's
+// Warp roles (384 threads, one CTA per SM), every role split by tile parity
+// so that the even and odd tiles run in two independent lanes (one thread's
+// issue of TMA and tcgen05 instructions is what limits a single lane):
+// warps 0-1 stream key tiles with TMA (hardware swizzle) into a STAGES-deep
+// ring, warps 2-3 issue the MMAs into NACC TMEM accumulators, warps 4-11 (two
+// groups of four) drain them with tcgen05.ld, apply ReLU and the head
+// weights, write one fp32 score per (query, key) and count it in the list's
 // shared-memory histogram of the top-k's first digit.
 #include <cudaTypedefs.h>
 
@@ -77,7 +79,7 @@ struct Cfg {
   static constexpr int OFF_SFA = OFF_Q + Q_BYTES;
   static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
   static constexpr int OFF_BAR = OFF_SFB + SFB_BYTES;
-  static constexpr int NBARS = 2 * STAGES + 2 * NACC + 1;
+  static constexpr int NBARS = 2 * STAGES + 2 * NACC + 2;
   static constexpr int OFF_W = OFF_BAR + NBARS * 8;
   static constexpr int OFF_HIST = OFF_W + N * 4;  // NQ x 4096 digit-1 counts of the scores written
   static constexpr int OFF_TMEM = OFF_HIST + NQ * kTopkBins * 4;
@@ -90,8 +92,10 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+constexpr int kIdxThreads = 384;
+
 template <int FMT, int NQ>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(kIdxThreads, 1)
     index_mma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                      const MmaArgs a) {
   using C = Cfg<FMT, NQ>;
@@ -102,6 +106,7 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* accf = empty + C::STAGES;  // [NACC] accumulator ready
   uint64_t* acce = accf + C::NACC;     // [NACC] accumulator drained
   uint64_t* qbar = acce + C::NACC;
+  uint64_t* sfb_bar = qbar + 1;        // query scales in TMEM (FP4)
   float* w_s = reinterpret_cast<float*>(sm + C::OFF_W);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_TMEM);
 
@@ -138,6 +143,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&acce[j], 4);  // the four warps of the group draining it
     }
     mbar_init(qbar, 1);
+    mbar_init(sfb_bar, 1);
     fence_barrier_init();
   }
   for (int i = threadIdx.x; i < C::N; i += blockDim.x) {
@@ -146,15 +152,17 @@ __global__ void __launch_bounds__(320, 1)
     if (FMT == LCSC_FMT_FP8) wv *= reinterpret_cast<const float*>(a.q_scale)[list * 64 + (i % 64)];
     w_s[i] = wv;
   }
-  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  if (warp == 2) tmem_alloc(tmem_slot, C::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------ TMA producer
-    if (lane == 0) {
+  if (warp < 2) {
+    // ------------------------------------------------------ TMA producers
+    const int par = warp;
+    if (lane == 0 && par == 1) prefetch_tmap(&tm_k);
+    if (lane == 0 && par == 0) {
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_q);
       mbar_arrive_expect_tx(qbar, C::Q_BYTES + C::SFB_BYTES);
@@ -164,8 +172,10 @@ __global__ void __launch_bounds__(320, 1)
         const uint8_t* src = a.q_scale + ((int64_t)b * q_tiles + (t0 * 64) / 128) * 1024;
         bulk_load(sm + C::OFF_SFB, src, C::SFB_BYTES, qbar);
       }
+    }
+    if (lane == 0) {
       const int64_t key_tiles = a.key_cap / 128;
-      for (int i = 0; i < ntile; ++i) {
+      for (int i = par; i < ntile; i += 2) {
         const int s = i % C::STAGES;
         const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
         if (!mbar_wait(&empty[s], ph ^ 1u, a.status)) break;
@@ -179,21 +189,26 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------ MMA issuer
+  } else if (warp < 4) {
+    // ------------------------------------------------------ MMA issuers
+    const int par = warp - 2;
     if (lane == 0) {
       bool live = mbar_wait(qbar, 0, a.status);
       tc_fence_after();
       const uint32_t q_addr = smem_u32(sm + C::OFF_Q);
-      if (live && FMT == LCSC_FMT_FP4) {
+      if (live && par == 0 && FMT == LCSC_FMT_FP4) {
         for (int j = 0; j < 2; ++j)
           for (int c = 0; c < (C::N + 127) / 128; ++c)
             tmem_cp_32x128b_x4(tmem + C::SFB_COL + 8 * c + 4 * j,
                                smem_desc(smem_u32(sm + C::OFF_SFB + c * 1024 + j * 512), 16, 128, kSwNone));
       }
+      // the odd-tile issuer starts once the query scales are in TMEM
+      if (par == 0) tc_commit(sfb_bar);
+      else live = live && mbar_wait(sfb_bar, 0, a.status);
+      tc_fence_after();
       const uint32_t idesc = FMT == LCSC_FMT_FP4 ? idesc_mxf4nvf4(128, C::N) : idesc_dense(0, 0, 128, C::N);
-      int issued = 0;
-      for (int i = 0; live && i < ntile; ++i) {
+      int last = -1;
+      for (int i = par; live && i < ntile; i += 2) {
         const int s = i % C::STAGES;
         const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
         const int ab = i % C::NACC;
@@ -221,18 +236,16 @@ __global__ void __launch_bounds__(320, 1)
         }
         tc_commit(&empty[s]);
         tc_commit(&accf[ab]);
-        ++issued;
+        last = i;
       }
-      if (issued > 0) {  // the accumulator of the last tile is complete before TMEM is freed
-        const int last = issued - 1;
+      if (last >= 0)  // the accumulator of the last tile is complete before TMEM is freed
         mbar_wait(&accf[last % C::NACC], (uint32_t)(last / C::NACC) & 1u, a.status);
-      }
     }
   } else {
     // ------------------------------------------------------ epilogue
     // Two groups of four warps take alternate tiles; within a group warp w
     // reads TMEM sub-partition w % 4 (rows 32 (w % 4) ..).
-    const int grp = (warp - 2) >> 2;
+    const int grp = (warp - 4) >> 2;
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const float* kscale = reinterpret_cast<const float*>(a.key_scale) + (int64_t)b * a.key_cap;
@@ -284,7 +297,7 @@ __global__ void __launch_bounds__(320, 1)
     }
   }
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -359,7 +372,7 @@ cudaError_t launch_mma(const IndexLaunch& a, cudaStream_t stream) {
   auto kern = index_mma_kernel<FMT, NQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(m.chunks, (unsigned)ctas), 320, C::SMEM, stream>>>(tk, tq, m);
+  kern<<<dim3(m.chunks, (unsigned)ctas), kIdxThreads, C::SMEM, stream>>>(tk, tq, m);
   return cudaGetLastError();
 }
 
