@@ -114,7 +114,8 @@ void plan_index(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max, Carve
   float* scores = cv.take<float>((size_t)lists * stride);
   uint32_t* hist = cv.take<uint32_t>((size_t)lists * 2 * 4096);
   uint32_t* ctr = cv.take<uint32_t>((size_t)lists * 8);
-  uint32_t* cand = cv.take<uint32_t>((size_t)lists * stride);
+  const int64_t cand_cap = stride < 65536 ? stride : 65536;
+  uint32_t* cand = cv.take<uint32_t>((size_t)lists * 2 * cand_cap);  // (index, key) pairs
   const int64_t bit_stride = ((stride + 31) / 32 + 3) / 4 * 4;
   uint32_t* bits = cv.take<uint32_t>((size_t)lists * bit_stride);
   if (L) {
@@ -127,6 +128,7 @@ void plan_index(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max, Carve
     L->hist = hist;
     L->counters = ctr;
     L->cand = cand;
+    L->cand_cap = cand_cap;
     L->sel_bits = bits;
     L->bit_stride = bit_stride;
   }

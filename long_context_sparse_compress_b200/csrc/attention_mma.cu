@@ -136,15 +136,41 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
   }
   if (warp == kMmaWarp) tmem_alloc(tm_slot, 512);
 
-  // ---- Q (64 x 512) -> f16, K-major swizzled blocks of 64 dims (all threads)
-  for (int i = tid; i < kH * (kD / 8); i += kThr) {
+  // ---- Q (64 x 512) -> f16, K-major swizzled blocks of 64 dims (all threads;
+  // bf16 rows: every 16-byte load of a thread in flight at once)
+  constexpr int kQChunks = kH * (kD / 8), kQIter = (kQChunks + kThr - 1) / kThr;
+  auto q_store = [&](int i, const float (&v)[8]) {
     const int h = i / (kD / 8), d0 = (i % (kD / 8)) * 8;
-    const int64_t base = ((int64_t)list * a.H + h) * kD + d0;
-    float v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = load_elem(a.q, base + j, a.q_dtype);
     *reinterpret_cast<uint4*>(sm + OFF_Q + (d0 / 64) * KB_Q + swz(h, (d0 % 64) * 2)) =
         make_uint4(pack_h2(v[0], v[1]), pack_h2(v[2], v[3]), pack_h2(v[4], v[5]), pack_h2(v[6], v[7]));
+  };
+  if (a.q_dtype == LCSC_DT_BF16) {
+    const uint4* q4 = reinterpret_cast<const uint4*>(a.q) + (int64_t)list * a.H * (kD / 8);
+    uint4 raw[kQIter];
+#pragma unroll
+    for (int u = 0; u < kQIter; ++u) {
+      const int i = tid + u * kThr;
+      raw[u] = i < kQChunks ? q4[i] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kQIter; ++u) {
+      const int i = tid + u * kThr;
+      if (i >= kQChunks) continue;
+      const uint16_t* bf = reinterpret_cast<const uint16_t*>(&raw[u]);
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = bf16_val(bf[j]);
+      q_store(i, v);
+    }
+  } else {
+    for (int i = tid; i < kQChunks; i += kThr) {
+      const int h = i / (kD / 8), d0 = (i % (kD / 8)) * 8;
+      const int64_t base = ((int64_t)list * a.H + h) * kD + d0;
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = load_elem(a.q, base + j, a.q_dtype);
+      q_store(i, v);
+    }
   }
   fence_async_smem();
   tc_fence_before();
@@ -444,18 +470,24 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
     if (done) done = warp_wait(&pv_done[(ntiles - 1) & 1], (uint32_t)((ntiles - 1) >> 1) & 1u, a, abort);
     tc_fence_after();
     const int64_t pidx = ((int64_t)list * a.splits + blockIdx.x) * a.H + head;
-    for (int c = 0; c < kD; c += 32) {
-      uint32_t r[32];
-      tmem_ld_32(row_addr + c, r);
-      tmem_ld_wait(r);
+    for (int c = 0; c < kD; c += 64) {  // two TMEM loads in flight
+      uint32_t r0[32], r1[32];
+      tmem_ld_32(row_addr + c, r0);
+      tmem_ld_32(row_addr + c + 32, r1);
+      tmem_ld_wait(r0, r1);
       if (lane < 16) {
         float* po = a.part_o + pidx * kD + c;
 #pragma unroll
-        for (int q = 0; q < 32; q += 4)
+        for (int q = 0; q < 32; q += 4) {
           *reinterpret_cast<float4*>(po + q) =
-              done ? make_float4(__uint_as_float(r[q]), __uint_as_float(r[q + 1]), __uint_as_float(r[q + 2]),
-                                 __uint_as_float(r[q + 3]))
+              done ? make_float4(__uint_as_float(r0[q]), __uint_as_float(r0[q + 1]), __uint_as_float(r0[q + 2]),
+                                 __uint_as_float(r0[q + 3]))
                    : make_float4(0.f, 0.f, 0.f, 0.f);
+          *reinterpret_cast<float4*>(po + 32 + q) =
+              done ? make_float4(__uint_as_float(r1[q]), __uint_as_float(r1[q + 1]), __uint_as_float(r1[q + 2]),
+                                 __uint_as_float(r1[q + 3]))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
     }
     if (s_lane) {

@@ -174,43 +174,6 @@ __global__ void __launch_bounds__(256) score_kernel(IndexLaunch a) {
 
 // --------------------------------------------------------------- top-k
 
-// Threshold bin of a 4096-bin histogram for `need` (>= 1) elements: the
-// largest bin t with sum_{d >= t} hist[d] >= need.  512 threads.
-__device__ Thresh find_threshold(const uint32_t* hist_s, uint32_t need, uint32_t* scratch) {
-  const int tid = threadIdx.x;  // 512 threads x 8 bins, bins in descending order
-  uint32_t local = 0;
-  for (int j = 0; j < 8; ++j) local += hist_s[kBins - 1 - (tid * 8 + j)];
-  scratch[tid] = local;
-  __syncthreads();
-  // inclusive scan (Hillis-Steele) over 512 values
-  for (int off = 1; off < 512; off <<= 1) {
-    uint32_t v = tid >= off ? scratch[tid - off] : 0;
-    __syncthreads();
-    scratch[tid] += v;
-    __syncthreads();
-  }
-  __shared__ Thresh res;
-  const uint32_t incl = scratch[tid];
-  const uint32_t excl = incl - local;
-  if (excl < need && incl >= need) {
-    uint32_t run = excl;
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t bin = kBins - 1 - (tid * 8 + j);
-      const uint32_t c = hist_s[bin];
-      if (run + c >= need) {
-        res.bin = bin;
-        res.above = run;
-        break;
-      }
-      run += c;
-    }
-  }
-  __syncthreads();
-  Thresh r = res;
-  __syncthreads();
-  return r;
-}
-
 struct ListInfo {
   int64_t n;
   int64_t k_eff;
@@ -290,28 +253,29 @@ __global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int sl
   uint32_t* bits = a.sel_bits + (int64_t)list * a.bit_stride;
   for (int64_t w = li.lo / 32 + threadIdx.x; w < (li.hi + 31) / 32; w += 512) bits[w] = 0u;
   __syncthreads();
-  uint32_t* cand = a.cand + (int64_t)list * a.stride;
+  uint32_t* cand = a.cand + (int64_t)list * 2 * a.cand_cap;  // (index, key) pairs
   scan_scores(s, li.lo, li.hi, [&](int64_t g, float v) {
-    const uint32_t d1 = float_key(v) >> 20;
+    const uint32_t key = float_key(v);
+    const uint32_t d1 = key >> 20;
     if (d1 > t1) atomicOr(&bits[g >> 5], 1u << (g & 31));
     const uint32_t c = warp_append(&ctr[1], d1 == t1);
-    if (d1 == t1) cand[c] = (uint32_t)g;
+    if (d1 == t1 && c < a.cand_cap) reinterpret_cast<uint2*>(cand)[c] = make_uint2((uint32_t)g, key);
   });
 }
 
 // Smallest index bound tau such that at least `need` of the tied candidates
 // (key == tkey) have index < tau: ties then go to the lowest indices, as in
 // a stable sort.  512 threads; returns n when every tied candidate is needed.
-template <class KeyAt, class IdxAt>
-__device__ uint32_t tie_bound(uint32_t n_cand, KeyAt key_at, IdxAt idx_at, uint32_t tkey, uint32_t need,
-                              uint32_t n, uint32_t* cnt) {
+// `each(f)` calls f(index, key) for this thread's share of the candidates.
+template <class Each>
+__device__ uint32_t tie_bound(Each each, uint32_t tkey, uint32_t need, uint32_t n, uint32_t* cnt) {
   uint32_t lo = 0, hi = n;  // count(idx < hi) >= need holds for hi = n
   while (lo < hi) {
     const uint32_t mid = lo + (hi - lo) / 2;
     if (threadIdx.x == 0) *cnt = 0;
     __syncthreads();
     uint32_t local = 0;
-    for (uint32_t c = threadIdx.x; c < n_cand; c += 512) local += (idx_at(c) < mid && key_at(c) == tkey) ? 1u : 0u;
+    each([&](uint32_t g, uint32_t key) { local += (g < mid && key == tkey) ? 1u : 0u; });
     if (local) atomicAdd(cnt, local);
     __syncthreads();
     const uint32_t total = *cnt;
@@ -331,7 +295,8 @@ constexpr size_t kFinalSmem = (size_t)kCandCap * 8;
 // the output (index order).
 __global__ void __launch_bounds__(512) topk_final_kernel(IndexLaunch a) {
   __shared__ uint32_t h[kBins];
-  __shared__ uint32_t scratch[512];
+  __shared__ Thresh th;
+  __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t cnt;
   __shared__ uint32_t warp_sum[16];
   extern __shared__ uint32_t dyn[];
@@ -354,45 +319,71 @@ __global__ void __launch_bounds__(512) topk_final_kernel(IndexLaunch a) {
   const uint32_t need2 = (uint32_t)k_eff - ctr[2];  // >= 1 by construction
   const uint32_t t1 = ctr[3];
   const uint32_t n_cand = ctr[1];
-  const uint32_t* cand = a.cand + (int64_t)list * a.stride;
+  const uint2* cand = reinterpret_cast<const uint2*>(a.cand + (int64_t)list * 2 * a.cand_cap);
   const float* s = a.scores + (int64_t)list * a.stride;
   uint32_t* bits = a.sel_bits + (int64_t)list * a.bit_stride;
   const bool cached = n_cand <= (uint32_t)kCandCap;
-  if (cached) {
-    for (uint32_t c = tid; c < n_cand; c += 512) {
-      const uint32_t g = cand[c];
-      cg[c] = g;
-      ck[c] = float_key(s[g]);
+  if (cached) {  // eight pairs in flight per thread
+    for (uint32_t c0 = 0; c0 < n_cand; c0 += 8 * 512) {
+      uint2 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t c = c0 + u * 512 + tid;
+        v[u] = c < n_cand ? cand[c] : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t c = c0 + u * 512 + tid;
+        if (c < n_cand) {
+          cg[c] = v[u].x;
+          ck[c] = v[u].y;
+        }
+      }
     }
   }
-  auto key_at = [&](uint32_t c) { return cached ? ck[c] : float_key(s[cand[c]]); };
-  auto idx_at = [&](uint32_t c) { return cached ? cg[c] : cand[c]; };
+  // Candidates: in shared memory, else the workspace list, else (a list
+  // that overflowed the workspace) every score of the row in the bin again.
+  const int mode = cached ? 0 : (n_cand <= (uint32_t)a.cand_cap ? 1 : 2);
+  auto each = [&](auto&& f) {
+    if (mode == 0) {
+      for (uint32_t c = tid; c < n_cand; c += 512) f(cg[c], ck[c]);
+    } else if (mode == 1) {
+      for (uint32_t c = tid; c < n_cand; c += 512) {
+        const uint2 v = cand[c];
+        f(v.x, v.y);
+      }
+    } else {
+      for (int64_t g = tid; g < n; g += 512) {
+        const uint32_t key = float_key(s[g]);
+        if ((key >> 20) == t1) f((uint32_t)g, key);
+      }
+    }
+  };
+  auto threshold = [&](int nbins, uint32_t need) { return block_threshold(h, nbins, need, 512, warp_tot, &th); };
   // digit 2 (key bits 8 .. 19)
   for (int i = tid; i < kBins; i += 512) h[i] = 0;
   __syncthreads();
-  for (uint32_t c = tid; c < n_cand; c += 512) atomicAdd(&h[(key_at(c) >> 8) & 0xFFF], 1u);
+  each([&](uint32_t, uint32_t key) { atomicAdd(&h[(key >> 8) & 0xFFF], 1u); });
   __syncthreads();
-  const Thresh t2 = find_threshold(h, need2, scratch);
+  const Thresh t2 = threshold(kBins, need2);
   const uint32_t need3 = need2 - t2.above;
   // digit 3 (key bits 0 .. 7) inside the digit-2 threshold bin
   for (int i = tid; i < kBins; i += 512) h[i] = 0;
   __syncthreads();
-  for (uint32_t c = tid; c < n_cand; c += 512) {
-    const uint32_t key = key_at(c);
+  each([&](uint32_t, uint32_t key) {
     if (((key >> 8) & 0xFFF) == t2.bin) atomicAdd(&h[key & 0xFF], 1u);
-  }
+  });
   __syncthreads();
-  const Thresh t3 = find_threshold(h, need3, scratch);
+  const Thresh t3 = threshold(256, need3);
   const uint32_t ties = need3 - t3.above;
   const uint32_t n_tied = h[t3.bin];
   __syncthreads();
   const uint32_t tkey = (t1 << 20) | (t2.bin << 8) | t3.bin;
   uint32_t tau = (uint32_t)n;  // ties go to the lowest indices
-  if (n_tied > ties) tau = tie_bound(n_cand, key_at, idx_at, tkey, ties, (uint32_t)n, &cnt);
-  for (uint32_t c = tid; c < n_cand; c += 512) {
-    const uint32_t key = key_at(c), g = idx_at(c);
+  if (n_tied > ties) tau = tie_bound(each, tkey, ties, (uint32_t)n, &cnt);
+  each([&](uint32_t g, uint32_t key) {
     if (key > tkey || (key == tkey && g < tau)) atomicOr(&bits[g >> 5], 1u << (g & 31));
-  }
+  });
   __syncthreads();
   // compaction: thread t owns bitmap words [16 t, 16 t + 16) of each 8192-word block
   const int64_t words = (n + 31) / 32;
@@ -437,15 +428,19 @@ __global__ void __launch_bounds__(512) topk_final_kernel(IndexLaunch a) {
         const int bit = __ffs(bw) - 1;
         bw &= bw - 1;
         const int64_t g = (wt + q) * 32 + bit;
-        if (off < (uint32_t)k_eff) {
-          out_i[off] = (int32_t)g;
-          if (out_s) out_s[off] = s[g];
-        }
+        if (off < (uint32_t)k_eff) out_i[off] = (int32_t)g;
         ++off;
       }
     }
     base += block_total;
     __syncthreads();
+  }
+  if (out_s) {  // the scores, gathered once every index is out (independent loads)
+    __syncthreads();
+    for (int64_t jj = tid; jj < k_eff; jj += 512) {
+      const int32_t g = out_i[jj];
+      out_s[jj] = (g >= 0 && g < n) ? s[g] : -INFINITY;
+    }
   }
 }
 

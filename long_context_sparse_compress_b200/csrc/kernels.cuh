@@ -57,7 +57,8 @@ struct IndexLaunch {
   // top-k workspace
   uint32_t* hist;       // [B*T][2][4096]
   uint32_t* counters;   // [B*T][8]
-  uint32_t* cand;       // [B*T][stride]
+  uint32_t* cand;       // [B*T][cand_cap][2] candidate (index, key) pairs
+  int64_t cand_cap;     // min(stride, 65536)
   uint32_t* sel_bits;   // [B*T][bit_stride] selected-entry bitmap
   int64_t bit_stride;   // words per bitmap row: ceil(stride / 32) rounded up to 4
   int32_t* out_idx;     // [B*T][k]

@@ -19,41 +19,48 @@ struct Thresh {
   uint32_t above;  // elements in bins above it
 };
 
-// Threshold bin of a 4096-bin histogram in shared memory for `need` (>= 1)
-// elements: the largest bin t with sum_{d >= t} hist[d] >= need.  Called by
-// one whole warp; every lane gets the result.
-__device__ __forceinline__ Thresh warp_threshold(const uint32_t* h, uint32_t need) {
-  const int lane = threadIdx.x & 31;
-  const int top = kTopkBins - 128 * lane;  // lane l owns bins [top - 128, top): descending by lane
+// Threshold bin of an `nbins`-bin histogram in shared memory for `need`
+// (>= 1) elements: the largest bin t with sum_{d >= t} hist[d] >= need.
+// Every thread of the CTA calls it; threads tid < T (T a multiple of 32 that
+// divides nbins, <= blockDim) each sum nbins / T consecutive bins (in
+// descending order), a warp scan and a scan of the warp totals give each
+// its prefix, and the one whose range holds the need walks its bins.
+// `warp_tot` is 32 words and `res` one Thresh of shared memory.
+__device__ __forceinline__ Thresh block_threshold(const uint32_t* h, int nbins, uint32_t need, int T,
+                                                  uint32_t* warp_tot, Thresh* res) {
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int per = nbins / T;
+  const int top = nbins - 1 - tid * per;  // this thread's highest bin
   uint32_t local = 0;
-  for (int j = 0; j < 128; ++j) local += h[top - 1 - ((j + lane) & 127)];  // skewed: no bank conflicts
+  if (tid < T)
+    for (int j = 0; j < per; ++j) local += h[top - j];
   uint32_t incl = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += v;
   }
-  const uint32_t excl = incl - local;
-  const bool mine = excl < need && incl >= need;
-  Thresh r{0u, 0u};
-  if (mine) {
-    uint32_t run = excl;
-    for (int d = top - 1; d >= top - 128; --d) {
-      const uint32_t c = h[d];
-      if (run + c >= need) {
-        r.bin = (uint32_t)d;
-        r.above = run;
-        break;
+  if (tid == 0) *res = Thresh{0u, 0u};
+  if (tid < T && lane == 31) warp_tot[w] = incl;
+  __syncthreads();
+  if (tid < T) {
+    uint32_t before = 0;
+    for (int i = 0; i < w; ++i) before += warp_tot[i];
+    uint32_t run = before + incl - local;
+    if (run < need && run + local >= need) {
+      for (int j = 0; j < per; ++j) {
+        const uint32_t c = h[top - j];
+        if (run + c >= need) {
+          *res = Thresh{(uint32_t)(top - j), run};
+          break;
+        }
+        run += c;
       }
-      run += c;
     }
   }
-  const uint32_t owners = __ballot_sync(0xffffffffu, mine);
-  if (owners) {
-    const int src = __ffs(owners) - 1;
-    r.bin = __shfl_sync(0xffffffffu, r.bin, src);
-    r.above = __shfl_sync(0xffffffffu, r.above, src);
-  }
+  __syncthreads();
+  const Thresh r = *res;
+  __syncthreads();  // `res` and `warp_tot` may be reused right after
   return r;
 }
 
@@ -99,14 +106,14 @@ __device__ __forceinline__ void hist_finish(uint32_t* hist_s, bool flush, int nl
   for (int i = threadIdx.x; i < nlists * kTopkBins; i += blockDim.x)
     hist_s[i] = __ldcg(&hist_g[(list0 + i / kTopkBins) * 2 * kTopkBins + i % kTopkBins]);
   __syncthreads();
-  if (threadIdx.x < 32) {
-    for (int l = 0; l < nlists; ++l) {
-      if (n[l] <= k) continue;
-      const Thresh t = warp_threshold(hist_s + l * kTopkBins, (uint32_t)k);
-      if (threadIdx.x == 0) {
-        ctr_g[(list0 + l) * 8 + 2] = t.above;
-        ctr_g[(list0 + l) * 8 + 3] = t.bin;
-      }
+  __shared__ uint32_t warp_tot[32];
+  __shared__ Thresh res;
+  for (int l = 0; l < nlists; ++l) {
+    if (n[l] <= k) continue;  // uniform over the CTA
+    const Thresh t = block_threshold(hist_s + l * kTopkBins, kTopkBins, (uint32_t)k, 256, warp_tot, &res);
+    if (threadIdx.x == 0) {
+      ctr_g[(list0 + l) * 8 + 2] = t.above;
+      ctr_g[(list0 + l) * 8 + 3] = t.bin;
     }
   }
 }

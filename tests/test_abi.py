@@ -49,7 +49,8 @@ def test_workspace_sizes_are_host_only(lib):
     p = L.params(W.PAIR_DECODE_1M_B16.layer("csa"))
     out = ctypes.c_size_t(0)
     assert lib.lcsc_index_topk_workspace_size(ctypes.byref(p), 16, 1, 262144, ctypes.byref(out)) == 0
-    assert out.value >= 16 * 262144 * 8
+    # scores (4 B per entry) and the capped candidate (index, key) lists
+    assert out.value >= 16 * 262144 * 4 + 16 * 65536 * 8
     assert lib.lcsc_step_workspace_size(ctypes.byref(p), 1, 16, 1, 262144, ctypes.byref(out)) == 0
     assert lib.lcsc_attn_workspace_size(ctypes.byref(p), 16, 1, 8192, 1, ctypes.byref(out)) == 0
 
