@@ -562,7 +562,9 @@ static int32_t step_impl(const lcsc_params* p, const lcsc_step* s, void* ws, siz
   if (csa && (e = launch_compress(ci, strm)) != cudaSuccess) return cuda_fail(e);
   if ((e = mark()) != cudaSuccess) return cuda_fail(e);
   if (csa) {
-    if ((e = launch_index_scores(il, strm)) != cudaSuccess) return cuda_fail(e);
+    if ((e = launch_index_quantize(il, strm)) != cudaSuccess) return cuda_fail(e);
+    if ((e = mark()) != cudaSuccess) return cuda_fail(e);
+    if ((e = launch_index_score_only(il, strm)) != cudaSuccess) return cuda_fail(e);
     if ((e = mark()) != cudaSuccess) return cuda_fail(e);
     if ((e = launch_topk(il, strm)) != cudaSuccess) return cuda_fail(e);
     if ((e = mark()) != cudaSuccess) return cuda_fail(e);

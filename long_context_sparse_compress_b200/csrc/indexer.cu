@@ -446,9 +446,8 @@ __global__ void __launch_bounds__(512) topk_final_kernel(IndexLaunch a) {
 
 }  // namespace
 
-cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream) {
+cudaError_t launch_index_quantize(const IndexLaunch& a, cudaStream_t stream) {
   const int lists = a.B * a.T;
-  cudaError_t e;
   const int64_t q_rows = (int64_t)lists * a.H_I;
   const unsigned qgrid = (unsigned)((q_rows + 7) / 8);
   switch (a.d_I) {
@@ -456,8 +455,17 @@ cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream) {
     case 32: quantize_queries_kernel<1><<<qgrid, 256, 0, stream>>>(a); break;
     default: return cudaErrorInvalidValue;
   }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return cudaGetLastError();
+}
 
+cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream) {
+  cudaError_t e = launch_index_quantize(a, stream);
+  if (e != cudaSuccess) return e;
+  return launch_index_score_only(a, stream);
+}
+
+cudaError_t launch_index_score_only(const IndexLaunch& a, cudaStream_t stream) {
+  const int lists = a.B * a.T;
   if (index_mma_supported(a)) return launch_index_mma(a, stream);
   dim3 sgrid((unsigned)((a.n_max + 63) / 64), lists);
   const int fmt = a.keys.f.fmt;

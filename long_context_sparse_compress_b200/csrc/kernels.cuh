@@ -68,7 +68,9 @@ struct IndexLaunch {
 
 // Indexer scoring (query quantisation + scores) and top-k selection; the
 // stand-alone call runs both.
-cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream);
+cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream);  // quantize + score
+cudaError_t launch_index_quantize(const IndexLaunch& a, cudaStream_t stream);  // also zeroes top-k state
+cudaError_t launch_index_score_only(const IndexLaunch& a, cudaStream_t stream);
 cudaError_t launch_topk(const IndexLaunch& a, cudaStream_t stream);
 cudaError_t launch_index_topk(const IndexLaunch& a, cudaStream_t stream);
 // Tensor-core scoring (FP8 / FP4 keys, d_I = 128, H_I = 64, key capacity a
