@@ -473,6 +473,9 @@ def _cpu_model():
     return None
 
 
+REFERENCE_BUDGET_S = 120.0
+
+
 def run_reference(args):
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -481,20 +484,28 @@ def run_reference(args):
     wl = workloads.ALL[args.workload]
     layers_wl = [wl.layer("csa"), wl.layer("hca")] if wl.kind == "pair" else [wl]
     states = [oracle_sequence(lw.with_(B=1), 0, synth.SEED) for lw in layers_wl]
+    t_warm = []
     for _ in range(args.warmup):
+        tw = time.perf_counter()
         for lw, st in zip(layers_wl, states):
             oracle_step(lw.with_(B=1), *st)
+        t_warm.append(time.perf_counter() - tw)
+    # A step of the oracle takes seconds: the timed steps are capped so the
+    # run stays within a few minutes (the line reports how many ran).
+    steps = max(1, min(args.steps, int(REFERENCE_BUDGET_S / max(min(t_warm), 1e-6))))
     t0 = time.perf_counter()
-    for _ in range(args.steps):
+    for _ in range(steps):
         for lw, st in zip(layers_wl, states):
             oracle_step(lw.with_(B=1), *st)
     dt = time.perf_counter() - t0
-    value = args.steps * wl.T / dt
+    value = steps * wl.T / dt
     sample = (f"each step: 1 decode query of 1 sequence (of {wl.B}) through "
-              f"{'+'.join(x.name for x in layers_wl)} at full context")
+              f"{'+'.join(x.name for x in layers_wl)} at full context; {steps} of the {args.steps} "
+              f"requested steps timed (capped at ~{REFERENCE_BUDGET_S:.0f} s)")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "queries/s", "n_gpus": ws,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "steps": steps, "steps_requested": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded, numpy generator)",
         "config": {"workload": wl.name, "layers": [lw.name for lw in layers_wl], "context": wl.L},
