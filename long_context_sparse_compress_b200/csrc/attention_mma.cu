@@ -39,10 +39,14 @@ constexpr int kSW = 4;       // softmax warps
 constexpr int kThr = (kSW + kLW + 1) * 32;
 constexpr int kMmaWarp = kSW + kLW;
 constexpr int kFp8Chunks = 28;  // 16-byte FP8 chunks of a stored row (448 dims)
-constexpr int kFp8Loads = kTR * kFp8Chunks / (kLW * 32);            // 8 per loader thread per tile
-constexpr int kLoads = kFp8Loads + (kTR * 8 + kLW * 32 - 1) / (kLW * 32);  // + 3 BF16 chunks
-static_assert(kTR * kFp8Chunks == kFp8Loads * kLW * 32, "FP8 units split evenly");
-constexpr float kRescale = 8.f;  // rescale O only when the max grows by more
+constexpr int kLT = kLW * 32;   // loader threads
+constexpr int kFp8Units = kTR * kFp8Chunks, kBfUnits = kTR * 8;  // 16-byte chunks of a tile
+constexpr int kFp8Loads = (kFp8Units + kLT - 1) / kLT;           // FP8 chunks per loader thread
+constexpr int kLoads = kFp8Loads + (kBfUnits + kLT - 1) / kLT;   // + BF16 chunks
+// the partial last FP8 and BF16 rounds are taken by whole warps
+static_assert((kFp8Units % kLT) % 32 == 0 && (kBfUnits % kLT) % 32 == 0, "warp-uniform rounds");
+constexpr float kRescale = 8.f;
+constexpr float kLog2e = 1.4426950408889634f;  // log2(e), to work in base 2  // rescale O only when the max grows by more
 
 // shared memory (offsets from a 1024-aligned base)
 constexpr int KB_Q = kH * 128;    // one 64-dim block of Q  (8 KB)
@@ -69,6 +73,14 @@ __device__ __forceinline__ uint32_t swz(int row, int byte) {
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// 2^x on the MUFU unit (approximate, flush-to-zero), the base-2 exponential
+// the softmax works in.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 struct Rows {
@@ -182,25 +194,30 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
     // =================================================== loader warps
     // Software pipeline: the rows of tile j+1 are resolved and their bytes
     // requested (into a second register set) before tile j is dequantised.
-    const int lt = tid - kSW * 32;  // 0 .. 223
-    // Work units of a tile, fixed per thread for the whole kernel.  Units
-    // 0-7 are 16-byte FP8 chunks (28 per row): unit u = lt + 224 i splits as
-    // q = u % 4, row-in-pair = (u / 4) % 2, then 64-dim block (7) and row pair
-    // (32), so that the 8 lanes of a 128-bit store phase cover 2 rows x 4
-    // chunks of one block: distinct 16-byte bank groups after the swizzle.
-    // Units 8-10 are 16-byte BF16 chunks (8 per row, 512 in all).  Table
-    // word: first f16 destination (16 bits) | row << 16 | chunk << 22.
+    const int lt = tid - kSW * 32;  // 0 .. kLT - 1
+    // Work units of a tile, fixed per thread for the whole kernel.  The
+    // first kFp8Loads are 16-byte FP8 chunks (28 per row, 1792 in all): unit
+    // u = lt + kLT i splits as q = u % 4, row-in-pair = (u / 4) % 2, then
+    // 64-dim block (7) and row pair (32), so that the 8 lanes of a 128-bit
+    // store phase cover 2 rows x 4 chunks of one block: distinct 16-byte bank
+    // groups after the swizzle.  The rest are 16-byte BF16 chunks (8 per row,
+    // 512 in all).  Table word: first f16 destination (16 bits) | row << 16 |
+    // chunk << 22; all ones: no unit.
     uint32_t tab[kLoads];
 #pragma unroll
     for (int i = 0; i < kLoads; ++i) {
       int r, c;
       if (i < kFp8Loads) {
-        const int u = lt + i * (kLW * 32), rest = u >> 3;
+        const int u = lt + i * kLT, rest = u >> 3;
+        if (u >= kFp8Units) {
+          tab[i] = 0xFFFFFFFFu;
+          continue;
+        }
         r = 2 * (rest / 7) + ((u >> 2) & 1);
         c = 4 * (rest % 7) + (u & 3);
       } else {
-        const int v = lt + (i - kFp8Loads) * (kLW * 32);
-        if (v >= kTR * 8) {
+        const int v = lt + (i - kFp8Loads) * kLT;
+        if (v >= kBfUnits) {
           tab[i] = 0xFFFFFFFFu;
           continue;
         }
@@ -220,6 +237,9 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
       return (a.idx && slot < s_hi && slot < qr.n_ent_slots) ? a.idx[(int64_t)list * a.k + slot] : 0;
     };
     // Row of tile j for this thread: pointer (null: no row) and scale address.
+    // window ring row of window slot 0 (the ring index then only wraps once)
+    const int64_t win_cap = a.win_kv.capacity;
+    const int64_t win_base = win_cap > 0 ? qr.w_lo % win_cap : 0;  // no window: never used
     auto locate = [&](int j, int32_t gi, const float*& scp) -> const uint8_t* {
       const int64_t slot = slot_of(j);
       scp = nullptr;
@@ -233,7 +253,8 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
         if ((g != -1 || !a.idx) && a.status) atomicOr(a.status, LCSC_DEV_BAD_INDEX);
         return nullptr;
       }
-      const int64_t row = (qr.w_lo + (slot - qr.n_ent_slots)) % a.win_kv.capacity;
+      int64_t row = win_base + (slot - qr.n_ent_slots);  // < 2 * capacity: the window is <= capacity rows
+      if (row >= win_cap) row -= win_cap;
       scp = a.win_kv.fscale(b, row);
       return a.win_kv.row(b, row);
     };
@@ -246,6 +267,7 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
       src_s[(j & 3) * kTR + lt] = p != nullptr;
       sc_next = scp ? *scp : 1.f;
     };
+
     auto fetch = [&](int j, uint4 (&raw)[kLoads]) {
       const int64_t* rows = row_s + (j & 3) * kTR;
 #pragma unroll
@@ -261,6 +283,7 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
       uint8_t* kt = sm + OFF_K + (j & 1) * (8 * KB_K);
 #pragma unroll
       for (int i = 0; i < kFp8Loads; ++i) {
+        if (tab[i] == 0xFFFFFFFFu) continue;
         const uint32_t d0 = tab[i] & 0xFFFFu;
         const float sc = scl[(tab[i] >> 16) & 63];
         const uint16_t* c2 = reinterpret_cast<const uint16_t*>(&raw[i]);
@@ -370,18 +393,46 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
       }
       tc_commit(&pv_done[buf]);
     };
-    for (int j = 0; j <= ntiles; ++j) {
-      if (j < ntiles) {
-        if (!warp_wait(&k_full[j & 1], (uint32_t)(j >> 1) & 1u, a, abort)) break;
-        tc_fence_after();
-        if (lane == 0) issue_qk(j);
-        __syncwarp();
+    // Q K^T of tile q and P V of tile v are issued in whichever order their
+    // inputs become ready, so that a late tile load never holds back the P V
+    // that frees a K buffer.  Q K^T of tile q also needs S[q % 2] free: the
+    // softmax of tile q-2 has published its P (seen before P V of q-2 went out).
+    int nq = 0, nv = 0;
+    uint64_t t_last = global_timer_ns();
+    while (nv < ntiles) {
+      bool progressed = false;
+      if (nq < ntiles && nq <= nv + 1) {
+        const bool ready = __all_sync(0xffffffffu, mbar_test_wait(&k_full[nq & 1], (uint32_t)(nq >> 1) & 1u));
+        if (ready) {
+          tc_fence_after();
+          if (lane == 0) issue_qk(nq);
+          __syncwarp();
+          ++nq;
+          progressed = true;
+        }
       }
-      if (j > 0) {
-        if (!warp_wait(&p_full[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, a, abort)) break;
-        tc_fence_after();
-        if (lane == 0) issue_pv(j - 1);
-        __syncwarp();
+      if (nv < nq) {
+        const bool ready = __all_sync(0xffffffffu, mbar_test_wait(&p_full[nv & 1], (uint32_t)(nv >> 1) & 1u));
+        if (ready) {
+          tc_fence_after();
+          if (lane == 0) issue_pv(nv);
+          __syncwarp();
+          ++nv;
+          progressed = true;
+        }
+      }
+      if (progressed) {
+        t_last = global_timer_ns();
+      } else {
+        bool stop = *abort != 0;
+        if (!stop && global_timer_ns() - t_last > kWaitLimitNs) {
+          if (lane == 0 && a.status) atomicOr(a.status, LCSC_DEV_TIMEOUT);
+          stop = true;
+        }
+        if (__any_sync(0xffffffffu, stop)) {
+          if (lane == 0) *abort = 1;
+          break;
+        }
       }
     }
   } else {
@@ -401,11 +452,21 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
       tmem_ld_32(row_addr + buf * kTR + 32, r1);
       tmem_ld_wait(r0, r1);
       const uint32_t m0 = mask_s[buf * 2], m1 = mask_s[buf * 2 + 1];
+      const bool full = (m0 & m1) == 0xFFFFFFFFu;  // every row of the tile valid (the common case)
       float mx = -INFINITY;
+      if (full) {
+        float mm[8];
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        if ((m0 >> q) & 1u) mx = fmaxf(mx, __uint_as_float(r0[q]));
-        if ((m1 >> q) & 1u) mx = fmaxf(mx, __uint_as_float(r1[q]));
+        for (int q = 0; q < 8; ++q) mm[q] = fmaxf(__uint_as_float(r0[q]), __uint_as_float(r1[q]));
+#pragma unroll
+        for (int q = 8; q < 32; ++q) mm[q & 7] = fmaxf(mm[q & 7], fmaxf(__uint_as_float(r0[q]), __uint_as_float(r1[q])));
+        mx = fmaxf(fmaxf(fmaxf(mm[0], mm[1]), fmaxf(mm[2], mm[3])), fmaxf(fmaxf(mm[4], mm[5]), fmaxf(mm[6], mm[7])));
+      } else {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          if ((m0 >> q) & 1u) mx = fmaxf(mx, __uint_as_float(r0[q]));
+          if ((m1 >> q) & 1u) mx = fmaxf(mx, __uint_as_float(r1[q]));
+        }
       }
       mx *= a.sm_scale;  // sm_scale > 0 keeps the order
       // reference max: set on the first rows seen, moved only by large jumps
@@ -419,18 +480,39 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
         }
         m_ref = mx;
       }
+      // p = exp(s * sm_scale - ref) = 2^(s * c2 - ref * log2 e): one FFMA and one EX2
       const float ref = m_ref;
+      const float c2 = a.sm_scale * kLog2e, ref2 = ref * kLog2e;
       float sum = 0.f;
       uint32_t pk[32];
+      if (full && ref > -INFINITY) {
+        float sp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int q = 0; q < 32; q += 2) {
-        const float p0 = ((m0 >> q) & 1u) && ref > -INFINITY ? __expf(__uint_as_float(r0[q]) * a.sm_scale - ref) : 0.f;
-        const float p1 = ((m0 >> (q + 1)) & 1u) && ref > -INFINITY ? __expf(__uint_as_float(r0[q + 1]) * a.sm_scale - ref) : 0.f;
-        const float p2 = ((m1 >> q) & 1u) && ref > -INFINITY ? __expf(__uint_as_float(r1[q]) * a.sm_scale - ref) : 0.f;
-        const float p3 = ((m1 >> (q + 1)) & 1u) && ref > -INFINITY ? __expf(__uint_as_float(r1[q + 1]) * a.sm_scale - ref) : 0.f;
-        sum += (p0 + p1) + (p2 + p3);
-        pk[q / 2] = pack_h2(p0, p1);
-        pk[16 + q / 2] = pack_h2(p2, p3);
+        for (int q = 0; q < 32; q += 2) {
+          const float p0 = ex2(fmaf(__uint_as_float(r0[q]), c2, -ref2));
+          const float p1 = ex2(fmaf(__uint_as_float(r0[q + 1]), c2, -ref2));
+          const float p2 = ex2(fmaf(__uint_as_float(r1[q]), c2, -ref2));
+          const float p3 = ex2(fmaf(__uint_as_float(r1[q + 1]), c2, -ref2));
+          sp[0] += p0;
+          sp[1] += p1;
+          sp[2] += p2;
+          sp[3] += p3;
+          pk[q / 2] = pack_h2(p0, p1);
+          pk[16 + q / 2] = pack_h2(p2, p3);
+        }
+        sum = (sp[0] + sp[1]) + (sp[2] + sp[3]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 32; q += 2) {
+          const bool live = ref > -INFINITY;
+          const float p0 = ((m0 >> q) & 1u) && live ? ex2(fmaf(__uint_as_float(r0[q]), c2, -ref2)) : 0.f;
+          const float p1 = ((m0 >> (q + 1)) & 1u) && live ? ex2(fmaf(__uint_as_float(r0[q + 1]), c2, -ref2)) : 0.f;
+          const float p2 = ((m1 >> q) & 1u) && live ? ex2(fmaf(__uint_as_float(r1[q]), c2, -ref2)) : 0.f;
+          const float p3 = ((m1 >> (q + 1)) & 1u) && live ? ex2(fmaf(__uint_as_float(r1[q + 1]), c2, -ref2)) : 0.f;
+          sum += (p0 + p1) + (p2 + p3);
+          pk[q / 2] = pack_h2(p0, p1);
+          pk[16 + q / 2] = pack_h2(p2, p3);
+        }
       }
       if (s_lane) l_sum += sum;
       // O is rescaled in place (lanes 0-15) only after the previous PV is done
