@@ -58,7 +58,9 @@ constexpr int OFF_BAR = OFF_P + 2 * kH * 128;  // k_full[2] s_full[2] p_full[2] 
 constexpr int OFF_ROW = OFF_BAR + 8 * 8;       // int64 [4][64] (row info of tiles j % 4)
 constexpr int OFF_SRC = OFF_ROW + 4 * kTR * 8;  // int32 [4][64]
 constexpr int OFF_SCL = OFF_SRC + 4 * kTR * 4;  // float [4][64]
-constexpr int OFF_MASK = OFF_SCL + 4 * kTR * 4;  // uint32 [2][2] valid-row bits
+constexpr int OFF_SCH = OFF_SCL + 4 * kTR * 4;  // f16x2 scale [4][64]
+constexpr int OFF_NRM = OFF_SCH + 4 * kTR * 4;  // uint32 [4][2]: every scale of a tile a normal f16
+constexpr int OFF_MASK = OFF_NRM + 32;          // uint32 [2][2] valid-row bits
 constexpr int OFF_TM = OFF_MASK + 16;
 constexpr int OFF_ABORT = OFF_TM + 4;
 constexpr int OFF_LSTOP = OFF_ABORT + 4;
@@ -120,6 +122,8 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
   int64_t* row_s = reinterpret_cast<int64_t*>(sm + OFF_ROW);
   int32_t* src_s = reinterpret_cast<int32_t*>(sm + OFF_SRC);
   float* scl_s = reinterpret_cast<float*>(sm + OFF_SCL);
+  uint32_t* sch_s = reinterpret_cast<uint32_t*>(sm + OFF_SCH);
+  volatile uint32_t* nrm_s = reinterpret_cast<volatile uint32_t*>(sm + OFF_NRM);
   uint32_t* mask_s = reinterpret_cast<uint32_t*>(sm + OFF_MASK);
   uint32_t* tm_slot = reinterpret_cast<uint32_t*>(sm + OFF_TM);
   volatile int* abort = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
@@ -280,7 +284,29 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
     };
     auto convert = [&](int j, const uint4 (&raw)[kLoads]) {
       const float* scl = scl_s + (j & 3) * kTR;
+      const uint32_t* sch = sch_s + (j & 3) * kTR;
       uint8_t* kt = sm + OFF_K + (j & 1) * (8 * KB_K);
+      if (nrm_s[(j & 3) * 2] && nrm_s[(j & 3) * 2 + 1]) {
+        // every row scale a normal f16 (the usual case): no per-unit branch,
+        // so the units of a thread overlap
+#pragma unroll
+        for (int i = 0; i < kFp8Loads; ++i) {
+          if (tab[i] == 0xFFFFFFFFu) continue;
+          const uint32_t d0 = tab[i] & 0xFFFFu;
+          const uint32_t s2u = sch[(tab[i] >> 16) & 63];
+          const __half2 s2 = *reinterpret_cast<const __half2*>(&s2u);
+          const uint16_t* c2 = reinterpret_cast<const uint16_t*>(&raw[i]);
+          uint32_t h[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(c2[q], __NV_E4M3);
+            const __half2 v = __hmul2(*reinterpret_cast<__half2*>(&hr), s2);
+            h[q] = *reinterpret_cast<const uint32_t*>(&v);
+          }
+          *reinterpret_cast<uint4*>(kt + d0) = make_uint4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<uint4*>(kt + (d0 ^ 16u)) = make_uint4(h[4], h[5], h[6], h[7]);
+        }
+      } else {
 #pragma unroll
       for (int i = 0; i < kFp8Loads; ++i) {
         if (tab[i] == 0xFFFFFFFFu) continue;
@@ -307,6 +333,7 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
         *reinterpret_cast<uint4*>(kt + d0) = make_uint4(h[0], h[1], h[2], h[3]);
         *reinterpret_cast<uint4*>(kt + (d0 ^ 16u)) = make_uint4(h[4], h[5], h[6], h[7]);
       }
+      }
 #pragma unroll
       for (int i = kFp8Loads; i < kLoads; ++i) {
         if (tab[i] == 0xFFFFFFFFu) continue;
@@ -325,6 +352,11 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
     auto step = [&](int j, const uint4 (&cur)[kLoads], uint4 (&nxt)[kLoads]) -> bool {
       if (lt < kTR) {
         scl_s[(j & 3) * kTR + lt] = sc_next;  // tile j's scale, loaded one step ago
+        const bool nrm = sc_next >= 6.103515625e-05f && sc_next <= 65504.f;
+        const __half2 s2 = __float2half2_rn(nrm ? sc_next : 0.f);
+        sch_s[(j & 3) * kTR + lt] = *reinterpret_cast<const uint32_t*>(&s2);
+        const uint32_t all = __ballot_sync(0xffffffffu, nrm);
+        if (lane == 0) nrm_s[(j & 3) * 2 + (lt >> 5)] = all == 0xffffffffu;
         if (j + 1 < ntiles) {
           place(j + 1, idx_next);
           if (j + 2 < ntiles) idx_next = load_idx(j + 2);
