@@ -123,27 +123,28 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
   __syncthreads();
   if (packed) {
     const int SP = kRows / G;
-    const int e = tid;
-    const int b = blockIdx.x * SP + e;
-    if (e < SP) {
-      bool valid = false;
-      SeqSpan sp;
-      if (b < a.B) {
-        sp = seq_span(a.span, b, a.window.capacity, a.entries.capacity);
-        valid = sp.ok && sp.g_hi - sp.g_lo == 1;
+    // one thread per tile row (row r: group j = r % G of sequence r / G)
+    for (int r = tid; r < kRows; r += kThreads) {
+      const int e = r / G, j = r % G;
+      const int b = blockIdx.x * SP + e;
+      int64_t src = -1;
+      if (e < SP && b < a.B) {
+        const SeqSpan sp = seq_span(a.span, b, a.window.capacity, a.entries.capacity);
+        const bool valid = sp.ok && sp.g_hi - sp.g_lo == 1;
+        const int64_t pos = sp.g_lo * m + m - G + j;
+        if (valid && pos >= 0) src = ((int64_t)b * a.n_x + (pos - sp.x_pos0)) * DIM;
+        if (j == 0) {
+          ent_out[e] = valid ? (int64_t)b * a.n_new_max : -1;
+          ent_row0[e] = e * G;
+          atomicMax(&n_ent, e + 1);
+          atomicMax(&rows_used, (e + 1) * G);
+        }
+      } else if (e < SP && j == 0) {
+        ent_out[e] = -1;
+        ent_row0[e] = e * G;
       }
-      ent_out[e] = valid ? (int64_t)b * a.n_new_max : -1;
-      ent_row0[e] = e * G;
-      for (int j = 0; j < G; ++j) {
-        const int64_t pos = valid ? sp.g_lo * m + m - G + j : -1;
-        row_src[e * G + j] = (valid && pos >= 0) ? ((int64_t)b * a.n_x + (pos - sp.x_pos0)) * DIM : -1;
-      }
-      if (b < a.B) {
-        atomicMax(&n_ent, e + 1);
-        atomicMax(&rows_used, (e + 1) * G);
-      }
+      row_src[r] = src;
     }
-    for (int r = SP * G + tid; r < kRows; r += kThreads) row_src[r] = -1;
   } else {
     const int b = blockIdx.z;
     const SeqSpan sp = seq_span(a.span, b, a.window.capacity, a.entries.capacity);
@@ -277,26 +278,57 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
     const bool active = pair < n_pairs && ent_out[pair / NC] >= 0;
     const int e = pair < n_pairs ? pair / NC : 0, c = pair % NC;
     const int r0 = ent_row0[e];
+    // tokens j = sub, sub + TP, ...: four at a time.  When the group splits
+    // evenly no token index needs a guard, so the loads of the four overlap.
+    auto logit = [&](int j, int r) { return zs[r * ZS + c] + bs[j * NC + c]; };
+    auto xval = [&](int r) -> float {
+      if constexpr (kBf16) return bf16_val(xs[r * XS + c0 + c]);
+      else return xs[r * XS + c0 + c];
+    };
+    auto ex = [](float v) -> float {
+      if constexpr (kBf16) return __expf(v);  // storage is bf16/FP8: the fast exponential is ample
+      else return expf(v);
+    };
+    const bool even = G % (4 * TP) == 0;
     float mx = -INFINITY;
     if (active) {
-      for (int j = sub; j < G; j += TP) {
-        const int r = r0 + j;
-        if (row_src[r] < 0) continue;
-        mx = fmaxf(mx, zs[r * ZS + c] + bs[j * NC + c]);
+      for (int j0 = sub; j0 < G; j0 += 4 * TP) {
+        float z[4];
+        bool live[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = j0 + u * TP;
+          const bool in = even || j < G;
+          const int r = r0 + (in ? j : 0);
+          z[u] = logit(in ? j : 0, r);
+          live[u] = in && row_src[r] >= 0;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (live[u]) mx = fmaxf(mx, z[u]);
       }
     }
     mx = group_max(mx, TP);
     float den = 0.f, num = 0.f;
     if (active) {
-      for (int j = sub; j < G; j += TP) {
-        const int r = r0 + j;
-        if (row_src[r] < 0) continue;
-        const float p = expf(zs[r * ZS + c] + bs[j * NC + c] - mx);
-        float xv;
-        if constexpr (kBf16) xv = bf16_val(xs[r * XS + c0 + c]);
-        else xv = xs[r * XS + c0 + c];
-        den += p;
-        num = fmaf(p, xv, num);
+      for (int j0 = sub; j0 < G; j0 += 4 * TP) {
+        float z[4], xv[4];
+        bool live[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = j0 + u * TP;
+          const bool in = even || j < G;
+          const int r = r0 + (in ? j : 0);
+          z[u] = logit(in ? j : 0, r);
+          xv[u] = xval(r);
+          live[u] = in && row_src[r] >= 0;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float p = live[u] ? ex(z[u] - mx) : 0.f;
+          den += p;
+          num = fmaf(p, xv[u], num);
+        }
       }
     }
     for (int o = TP >> 1; o > 0; o >>= 1) {
