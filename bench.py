@@ -147,15 +147,17 @@ class Layer:
 
 
 def kernels_per_step(wl):
-    """Kernels of this library one step launches: CSA: pool + store for the
-    KV latent and for the indexer keys (4), query quantisation + scoring (2),
-    top-k collect + final (2, plus a histogram pass when the scores come from
-    the CUDA-core scoring kernel), attention partial + combine (2); HCA: pool
-    + store (2), attention partial + combine (2)."""
+    """Kernels of this library one step launches.  CSA: the fused pool +
+    store of the KV latent and of the indexer keys (2: each grid is one
+    cluster of channel blocks), query quantisation + scoring (2), top-k
+    collect + final (2, plus a histogram pass when the scores come from the
+    CUDA-core scoring kernel), attention partial + combine (2).  HCA: pool +
+    store (2: sixteen 8-CTA clusters do not fit at once, so the store runs as
+    its own kernel), attention partial + combine (2)."""
     def csa(w):
         tensor_scored = (w.idx_fmt in ("fp8", "fp4") and w.d_I == 128 and w.H_I == 64
                          and (w.idx_fmt == "fp8" or w.T == 1))
-        return 10 + (0 if tensor_scored else 1)
+        return 8 + (0 if tensor_scored else 1)
     if wl.kind == "pair":
         return csa(wl.layer("csa")) + 4
     return csa(wl) if wl.kind == "csa" else 4

@@ -14,6 +14,7 @@
 // softmax and the weighted sum run on the tile in shared memory, and the
 // pooled fp32 rows go to scratch.  A second kernel stores each pooled row
 // (whole row needed for the FP8 amax) and the raw window rows.
+#include <cooperative_groups.h>
 #include <type_traits>
 
 #include "kernels.cuh"
@@ -23,6 +24,22 @@ namespace {
 
 constexpr int kRows = 128;   // token rows per CTA
 constexpr int kThreads = 256;
+constexpr int kMaxEnt = 32;  // entries per CTA (their pooled rows wait in shared memory)
+
+// Dynamic shared memory of pool_kernel: x tile, then the W chunk (reused for
+// z and the biases), then the pooled rows [kMaxEnt][NC].
+template <bool kBf16, int DIM, int NC>
+__host__ __device__ constexpr size_t pool_smem_offset() {
+  constexpr size_t elem = kBf16 ? 2 : 4;
+  constexpr size_t xs = elem * kRows * (kBf16 ? DIM + 8 : DIM + 1);
+  constexpr size_t wz = elem * DIM * (kBf16 ? NC + 8 : NC + 1);
+  constexpr size_t zb = sizeof(float) * (kRows * (NC + 1) + kRows * NC);  // z, then biases of <= 128 tokens
+  return xs + (wz > zb ? wz : zb);
+}
+template <bool kBf16, int DIM, int NC>
+__host__ __device__ constexpr size_t pool_smem_bytes() {
+  return pool_smem_offset<kBf16, DIM, NC>() + sizeof(float) * kMaxEnt * NC;
+}
 
 struct SeqSpan {
   int64_t g_lo, g_hi;   // entries written
@@ -91,6 +108,80 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// ------------------------------------------------------------ fused entry store
+// Stores this CTA's NC channels of each pooled entry row in the entries'
+// cache format.  FP8 rows (and the FP8 part of KV rows) share one scale over
+// the whole row: each CTA publishes its channels' amax and reads the others'
+// from the cluster (the DIM / NC channel blocks of the same entries) through
+// distributed shared memory.  FP4 block scales (16 values) and fp32 rows need
+// nothing from other CTAs.  A warp per entry, a lane per channel pair; the
+// arithmetic is the row store's (amax / 448 with a rounded division, codes
+// of value / scale).
+template <int DIM, int NC>
+__device__ __forceinline__ void store_entries(const CompressLaunch& a, const float* pooled_s, float* pamax_s,
+                                              const int64_t* ent_out, const int* ent_b, const int64_t* ent_g,
+                                              int E_cta, int c0) {
+  namespace cg = cooperative_groups;
+  const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+  constexpr int kWarps = kThreads / kWarp;
+  const CacheView& cv = a.entries;
+  const int fmt = cv.f.fmt;
+  const int ch = 2 * lane;                 // this lane's channel pair (ch, ch + 1) of the block
+  const bool has = ch < NC;
+  if (fmt == LCSC_FMT_KV || fmt == LCSC_FMT_FP8) {
+    const int n_fp8 = cv.f.dim - (fmt == LCSC_FMT_KV ? cv.f.rope : 0);
+    const bool fp8 = has && c0 + ch < n_fp8;  // n_fp8 is even: a pair is all FP8 or all BF16
+    for (int e = warp; e < E_cta; e += kWarps) {
+      float am = 0.f;
+      if (fp8) am = fmaxf(fabsf(pooled_s[e * NC + ch]), fabsf(pooled_s[e * NC + ch + 1]));
+      am = warp_max(am);
+      if (lane == 0) pamax_s[e] = am;
+    }
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const unsigned nblk = cluster.num_blocks();
+    for (int e = warp; e < E_cta; e += kWarps) {
+      if (ent_out[e] < 0) continue;  // uniform over the warp
+      float am = 0.f;
+      for (unsigned r = 0; r < nblk; ++r) am = fmaxf(am, cluster.map_shared_rank(pamax_s, r)[e]);
+      const float sc = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
+      uint8_t* row = cv.row(ent_b[e], ent_g[e]);
+      if (fp8) {
+        const uint16_t c2 = e4m3x2_code(__fdiv_rn(pooled_s[e * NC + ch], sc), __fdiv_rn(pooled_s[e * NC + ch + 1], sc));
+        *reinterpret_cast<uint16_t*>(row + c0 + ch) = c2;
+      } else if (has) {
+        uint16_t* d = reinterpret_cast<uint16_t*>(row + n_fp8) + (c0 + ch - n_fp8);
+        d[0] = bf16_code(pooled_s[e * NC + ch]);
+        d[1] = bf16_code(pooled_s[e * NC + ch + 1]);
+      }
+      if (blockIdx.y == 0 && lane == 0) *cv.fscale(ent_b[e], ent_g[e]) = sc;
+    }
+    cluster.sync();  // no CTA leaves while another may read its amax
+  } else if (fmt == LCSC_FMT_FP4) {
+    // blocks of 16 channels = 8 lanes
+    for (int e = warp; e < E_cta; e += kWarps) {
+      if (ent_out[e] < 0) continue;
+      const float v0 = has ? pooled_s[e * NC + ch] : 0.f, v1 = has ? pooled_s[e * NC + ch + 1] : 0.f;
+      const float amax = group_max(fmaxf(fabsf(v0), fabsf(v1)), 8);
+      const uint8_t scode = (uint8_t)(e4m3x2_code(__fdiv_rn(amax, 6.f), 0.f) & 0xff);
+      const float dsc = e4m3_val(scode);
+      if (has) {
+        uint8_t* row = cv.row(ent_b[e], ent_g[e]);
+        const float y0 = dsc > 0.f ? __fdiv_rn(v0, dsc) : 0.f, y1 = dsc > 0.f ? __fdiv_rn(v1, dsc) : 0.f;
+        row[(c0 + ch) / 2] = dsc > 0.f ? e2m1x2_code(y0, y1) : (uint8_t)0;
+        if (ch % 16 == 0) *cv.bscale_at(ent_b[e], ent_g[e], (c0 + ch) / 16) = scode;
+      }
+    }
+  } else {  // fp32 rows
+    for (int e = warp; e < E_cta; e += kWarps) {
+      if (ent_out[e] < 0 || !has) continue;
+      float* row = reinterpret_cast<float*>(cv.row(ent_b[e], ent_g[e]));
+      row[c0 + ch] = pooled_s[e * NC + ch];
+      row[c0 + ch + 1] = pooled_s[e * NC + ch + 1];
+    }
+  }
+}
+
 // ------------------------------------------------------------ pool kernel
 // A CTA owns up to 128 token rows and NC output channels.  Two tilings:
 //  * by entries (bulk calls, prefill): grid (ceil(n_new_max / E), dim / NC, B),
@@ -101,7 +192,7 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], 
 //    entry e = sequence b0 + e on rows e*G .. e*G+G-1.
 // Rows whose position is below 0 (or whose sequence closes no group) are
 // masked out of the softmax.
-template <bool kBf16, int DIM, int NC>
+template <bool kBf16, int DIM, int NC, bool kFused>
 __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E, bool packed) {
   using Elem = typename std::conditional<kBf16, uint16_t, float>::type;
   constexpr int XS = kBf16 ? DIM + 8 : DIM + 1;   // x tile row stride (elements)
@@ -114,15 +205,41 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
   __shared__ int64_t row_src[kRows];  // element offset of the row in x, or -1 (masked)
   __shared__ int64_t ent_out[kRows];  // pooled output row, or -1
   __shared__ int ent_row0[kRows];     // first tile row of the entry
+  __shared__ int ent_b[kRows];        // its sequence
+  __shared__ int64_t ent_g[kRows];    // and entry index in the cache
+  __shared__ float pamax_s[kRows];    // this CTA's share of the entry's FP8 amax
   __shared__ int n_ent, rows_used;
 
   const int c0 = blockIdx.y * NC;
   const int m = a.span.m, G = a.span.G;
   const int tid = threadIdx.x;
+  constexpr int VPL = DIM / 32;
+  float* pooled_s = reinterpret_cast<float*>(smem + pool_smem_offset<kBf16, DIM, NC>());  // [entries][NC]
+
+  // ---- window rows (the raw rows of the new tokens), a warp per row, spread
+  // over the grid; independent of the pooling below
+  if (kFused && a.window.data) {
+    const int warp = tid / kWarp, lane = tid % kWarp;
+    const int64_t cta = ((int64_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+    const int64_t n_warps = (int64_t)gridDim.x * gridDim.y * gridDim.z * (kThreads / kWarp);
+    const int64_t total = (int64_t)a.B * a.n_win_max;
+    for (int64_t t = cta * (kThreads / kWarp) + warp; t < total; t += n_warps) {
+      const int b = (int)(t / a.n_win_max);
+      const int64_t i = t % a.n_win_max;
+      const SeqSpan sp = seq_span(a.span, b, a.window.capacity, a.entries.capacity);
+      if (!sp.ok || i >= sp.w_hi - sp.w_lo) continue;
+      const int64_t pos = sp.w_lo + i;
+      const int64_t base = ((int64_t)b * a.n_x + (pos - sp.x_pos0)) * DIM + lane * VPL;
+      float v[VPL];
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) v[j] = load_elem(a.x, base + j, a.x_dtype);
+      store_row_warp<VPL>(a.window, b, pos % a.window.capacity, v, lane);
+    }
+  }
   if (tid == 0) { n_ent = 0; rows_used = 0; }
   __syncthreads();
   if (packed) {
-    const int SP = kRows / G;
+    const int SP = kRows / G < kMaxEnt ? kRows / G : kMaxEnt;
     // one thread per tile row (row r: group j = r % G of sequence r / G)
     for (int r = tid; r < kRows; r += kThreads) {
       const int e = r / G, j = r % G;
@@ -134,8 +251,11 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
         const int64_t pos = sp.g_lo * m + m - G + j;
         if (valid && pos >= 0) src = ((int64_t)b * a.n_x + (pos - sp.x_pos0)) * DIM;
         if (j == 0) {
+          if (!sp.ok && blockIdx.y == 0 && a.status) atomicOr(a.status, LCSC_DEV_BAD_LENGTH);
           ent_out[e] = valid ? (int64_t)b * a.n_new_max : -1;
           ent_row0[e] = e * G;
+          ent_b[e] = b;
+          ent_g[e] = sp.g_lo;
           atomicMax(&n_ent, e + 1);
           atomicMax(&rows_used, (e + 1) * G);
         }
@@ -160,8 +280,14 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
     for (int e = tid; e < E_cta; e += kThreads) {
       ent_out[e] = (int64_t)b * a.n_new_max + e0 + e;
       ent_row0[e] = e * m;
+      ent_b[e] = b;
+      ent_g[e] = sp.g_lo + e0 + e;
     }
-    if (tid == 0) { n_ent = E_cta; rows_used = R; }
+    if (tid == 0) {
+      n_ent = E_cta;
+      rows_used = R;
+      if (!sp.ok && blockIdx.x == 0 && blockIdx.y == 0 && a.status) atomicOr(a.status, LCSC_DEV_BAD_LENGTH);
+    }
   }
   __syncthreads();
   const int E_cta = n_ent;
@@ -335,7 +461,14 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
       den += __shfl_xor_sync(0xffffffffu, den, o);
       num += __shfl_xor_sync(0xffffffffu, num, o);
     }
-    if (active && sub == 0) a.pooled[ent_out[e] * DIM + c0 + c] = num / den;
+    if (active && sub == 0) {
+      if constexpr (kFused) pooled_s[e * NC + c] = num / den;
+      else a.pooled[ent_out[e] * DIM + c0 + c] = num / den;
+    }
+  }
+  if constexpr (kFused) {
+    __syncthreads();
+    store_entries<DIM, NC>(a, pooled_s, pamax_s, ent_out, ent_b, ent_g, E_cta, c0);
   }
 }
 
@@ -385,23 +518,42 @@ __global__ void __launch_bounds__(256) encode_rows_kernel(const float* rows, int
   store_row_warp<VPL>(out, b, row0 + i, v, lane);
 }
 
+// The pooled rows are stored by the pool kernel itself when every cluster
+// of its grid (the DIM / NC channel blocks of the same entries) can be
+// resident at once; otherwise they go through scratch to the store kernel.
 template <bool kBf16, int DIM, int NC>
-cudaError_t launch_pool(const CompressLaunch& a, int E, cudaStream_t stream) {
+cudaError_t launch_pool(const CompressLaunch& a, int E, cudaStream_t stream, bool* fused) {
   const bool packed = a.span.ctx_len != nullptr && a.n_new_max == 1 && a.span.G <= kRows;
-  using Elem = typename std::conditional<kBf16, uint16_t, float>::type;
-  constexpr int XS = kBf16 ? DIM + 8 : DIM + 1;
-  constexpr int WS = kBf16 ? NC + 8 : NC + 1;
-  size_t smem = sizeof(Elem) * kRows * XS;
-  size_t wz = sizeof(Elem) * DIM * WS;
-  const size_t zbytes = sizeof(float) * (kRows * (NC + 1) + kRows * NC);  // z, then biases of <= 128 tokens
-  smem += wz > zbytes ? wz : zbytes;
-  auto kern = pool_kernel<kBf16, DIM, NC>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  constexpr size_t smem = pool_smem_bytes<kBf16, DIM, NC>();
+  const int SP = kRows / a.span.G < kMaxEnt ? kRows / a.span.G : kMaxEnt;
+  const dim3 grid = packed ? dim3((unsigned)((a.B + SP - 1) / SP), DIM / NC, 1)
+                           : dim3((unsigned)((a.n_new_max + E - 1) / E), DIM / NC, a.B);
+  auto kf = pool_kernel<kBf16, DIM, NC, true>;
+  cudaError_t e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int SP = kRows / a.span.G;
-  dim3 grid = packed ? dim3((unsigned)((a.B + SP - 1) / SP), DIM / NC, 1)
-                     : dim3((unsigned)((a.n_new_max + E - 1) / E), DIM / NC, a.B);
-  kern<<<grid, kThreads, smem, stream>>>(a, E, packed);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = DIM / NC;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int max_clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&max_clusters, kf, &cfg) != cudaSuccess) {
+    cudaGetLastError();  // clear: fall back to the unfused path
+    max_clusters = 0;
+  }
+  *fused = (int64_t)grid.x * grid.z <= max_clusters;
+  if (*fused) return cudaLaunchKernelEx(&cfg, kf, a, E, packed);
+  auto ku = pool_kernel<kBf16, DIM, NC, false>;
+  e = cudaFuncSetAttribute(ku, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  ku<<<grid, kThreads, smem, stream>>>(a, E, packed);
   return cudaGetLastError();
 }
 
@@ -409,17 +561,20 @@ cudaError_t launch_pool(const CompressLaunch& a, int E, cudaStream_t stream) {
 
 cudaError_t launch_compress(const CompressLaunch& a, cudaStream_t stream) {
   const int m = a.span.m, G = a.span.G;
-  const int E = (kRows - (G - m)) / m;
-  cudaError_t e = cudaSuccess;
+  int E = (kRows - (G - m)) / m;
+  if (E > kMaxEnt) E = kMaxEnt;
+  bool fused = false;
   if (a.n_new_max > 0) {
     const bool bf = a.x_dtype == LCSC_DT_BF16;
-    if (bf && a.dim == 512) e = launch_pool<true, 512, 64>(a, E, stream);
-    else if (bf && a.dim == 128) e = launch_pool<true, 128, 64>(a, E, stream);
-    else if (!bf && a.dim == 128) e = launch_pool<false, 128, 64>(a, E, stream);
-    else if (!bf && a.dim == 32) e = launch_pool<false, 32, 32>(a, E, stream);
+    cudaError_t e;
+    if (bf && a.dim == 512) e = launch_pool<true, 512, 64>(a, E, stream, &fused);
+    else if (bf && a.dim == 128) e = launch_pool<true, 128, 64>(a, E, stream, &fused);
+    else if (!bf && a.dim == 128) e = launch_pool<false, 128, 64>(a, E, stream, &fused);
+    else if (!bf && a.dim == 32) e = launch_pool<false, 32, 32>(a, E, stream, &fused);
     else return cudaErrorInvalidValue;
     if (e != cudaSuccess) return e;
   }
+  if (fused) return cudaSuccess;  // entries and window rows were stored
   const int rows = a.n_new_max + (a.window.data ? a.n_win_max : 0);
   if (rows == 0) return cudaSuccess;
   dim3 grid((unsigned)((rows + 7) / 8), a.B);
