@@ -277,9 +277,11 @@ typedef struct lcsc_step {
   float* out_score;             /* [B][T][k] their scores (CSA), or NULL */
   /* Optional stage timing (host array of cudaEvent_t, or NULL): event i is
    * recorded on `stream` at stage boundary i while i < n_events.
-   * CSA: 0 start, 1 after compression, 2 after indexer query
-   * quantisation, 3 after indexer scoring, 4 after top-k, 5 after
-   * attention.  HCA: 0 start, 1 after compression, 2 after attention. */
+   * CSA: 0 start, 1 after the KV latent's compression, 2 once the indexer
+   * keys' compression and the query quantisation (which run beside it on a
+   * second stream of the library's) are also done, 3 after indexer
+   * scoring, 4 after top-k, 5 after attention.  HCA: 0 start, 1 after
+   * compression, 2 after attention. */
   void* const* events;
   int32_t n_events;
 } lcsc_step;

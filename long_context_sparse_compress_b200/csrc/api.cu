@@ -2,6 +2,8 @@
 // the launch sequence of every call.  No device memory is allocated here.
 #include <string.h>
 
+#include <mutex>
+
 #include "kernels.cuh"
 
 namespace lcsc {
@@ -499,6 +501,34 @@ static int32_t step_compress(const lcsc_params* p, const lcsc_step* s, int32_t t
   return LCSC_OK;
 }
 
+// A second stream per device for the parts of a CSA step that do not depend
+// on each other (the indexer keys' compression and the query quantisation
+// run beside the KV latent's compression), with its fork / join events.
+// Enqueueing on it is serialised by a mutex; the work itself is ordered
+// only by the events.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxSideDevices = 64;
+std::mutex g_side_mu;
+SideStream g_side[kMaxSideDevices];
+
+cudaError_t side_stream(SideStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxSideDevices) return cudaErrorInvalidDevice;
+  SideStream& ss = g_side[dev];
+  if (!ss.s) {
+    if ((e = cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+  }
+  *out = &ss;
+  return cudaSuccess;
+}
+
 static int32_t step_impl(const lcsc_params* p, const lcsc_step* s, void* ws, size_t ws_bytes,
                          int32_t* status, void* stream, bool csa) {
   int32_t st = check_params(p);
@@ -557,12 +587,26 @@ static int32_t step_impl(const lcsc_params* p, const lcsc_step* s, void* ws, siz
     return cudaSuccess;
   };
   if ((e = mark()) != cudaSuccess) return cuda_fail(e);
-  if ((e = launch_compress(ck, strm)) != cudaSuccess) return cuda_fail(e);
-  if (sep && (e = launch_compress(cvv, strm)) != cudaSuccess) return cuda_fail(e);
-  if (csa && (e = launch_compress(ci, strm)) != cudaSuccess) return cuda_fail(e);
-  if ((e = mark()) != cudaSuccess) return cuda_fail(e);
   if (csa) {
-    if ((e = launch_index_quantize(il, strm)) != cudaSuccess) return cuda_fail(e);
+    // fork: indexer keys + query quantisation on the side stream
+    std::lock_guard<std::mutex> lock(g_side_mu);
+    SideStream* ss = nullptr;
+    if ((e = side_stream(&ss)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaEventRecord(ss->fork, strm)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
+    if ((e = launch_compress(ci, ss->s)) != cudaSuccess) return cuda_fail(e);
+    if ((e = launch_index_quantize(il, ss->s)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaEventRecord(ss->join, ss->s)) != cudaSuccess) return cuda_fail(e);
+    if ((e = launch_compress(ck, strm)) != cudaSuccess) return cuda_fail(e);
+    if (sep && (e = launch_compress(cvv, strm)) != cudaSuccess) return cuda_fail(e);
+    if ((e = mark()) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaStreamWaitEvent(strm, ss->join, 0)) != cudaSuccess) return cuda_fail(e);
+  } else {
+    if ((e = launch_compress(ck, strm)) != cudaSuccess) return cuda_fail(e);
+    if (sep && (e = launch_compress(cvv, strm)) != cudaSuccess) return cuda_fail(e);
+    if ((e = mark()) != cudaSuccess) return cuda_fail(e);
+  }
+  if (csa) {
     if ((e = mark()) != cudaSuccess) return cuda_fail(e);
     if ((e = launch_index_score_only(il, strm)) != cudaSuccess) return cuda_fail(e);
     if ((e = mark()) != cudaSuccess) return cuda_fail(e);

@@ -84,7 +84,7 @@ struct Cfg {
   static constexpr int OFF_HIST = OFF_W + N * 4;  // NQ x 4096 digit-1 counts of the scores written
   static constexpr int OFF_TMEM = OFF_HIST + NQ * kTopkBins * 4;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + slack to align the base
-  static_assert(COLS_USED <= 512, "TMEM budget");
+  static_assert(COLS_USED <= 512 && SFA_COL <= COLS_USED, "TMEM budget");
   static_assert(A_BYTES % 1024 == 0 && Q_BYTES % 1024 == 0, "swizzle atoms need 1024-byte alignment");
 };
 
