@@ -13,13 +13,14 @@
 //  * FP8 keys and queries: tcgen05.mma kind::f8f6f4 on the codes; the
 //    per-row scales are positive, so the epilogue applies them outside ReLU:
 //    s = sk[g] * sum_h (w[h] sq[h]) ReLU(acc[h]).
-// Warp roles (384 threads, one CTA per SM), every role split by tile parity
-// so that the even and odd tiles run in two independent lanes (one thread's
-// issue of TMA and tcgen05 instructions is what limits a single lane):
-// warps 0-1 stream key tiles with TMA (hardware swizzle) into a STAGES-deep
-// ring, warps 2-3 issue the MMAs into NACC TMEM accumulators, warps 4-11 (two
-// groups of four) drain them with tcgen05.ld, apply ReLU and the head
-// weights, write one fp32 score per (query, key) and count it in the list's
+// Warp roles (384 threads, one CTA per SM).  One thread's issue of TMA and
+// tcgen05 instructions (tens of cycles each) is what limits a single
+// pipeline, so tiles are dealt round-robin to LANES lanes (warps 0 .. LANES-1,
+// one thread each): lane r loads its tiles with TMA (hardware swizzle) into a
+// STAGES-deep ring, DIST of its tiles ahead, and issues their MMAs into NACC
+// TMEM accumulators.  Warps 4-11 (two groups of four taking alternate tiles)
+// drain the accumulators with tcgen05.ld, apply ReLU and the head weights,
+// write one fp32 score per (query, key) and count it in the list's
 // shared-memory histogram of the top-k's first digit.
 #include <cudaTypedefs.h>
 
@@ -57,9 +58,14 @@ struct Cfg {
   static constexpr int KSTEPS = 4 - (FMT == LCSC_FMT_FP4 ? 2 : 0);  // 32 bytes of K per MMA
   // Ring depth: enough bytes in flight to cover DRAM latency, and more than
   // half the shared memory so that a second CTA never shares the SM's TMEM.
-  static constexpr int STAGES = FMT == LCSC_FMT_FP4 ? 13 : (NQ == 1 ? 8 : 5);
+  static constexpr int STAGES = FMT == LCSC_FMT_FP4 ? 20 : (NQ == 1 ? 8 : 5);
   // Accumulators in TMEM: the MMA runs up to NACC tiles ahead of the epilogue.
   static constexpr int NACC = NQ == 1 ? 4 : 2;
+  // TMA + MMA lanes (warps 0 .. LANES-1) and how many of its own tiles each
+  // loads ahead; LANES * DIST < STAGES keeps every wait on an earlier tile.
+  static constexpr int LANES = FMT == LCSC_FMT_FP4 ? 4 : (NQ == 1 ? 2 : 1);
+  static constexpr int DIST = STAGES / LANES - 1;
+  static_assert(DIST >= 1 && LANES * DIST < STAGES, "lane prefetch distance");
   static constexpr int A_BYTES = TILE * ROW;
   static constexpr int SFA_BYTES = FMT == LCSC_FMT_FP4 ? 1024 : 0;
   static constexpr int Q_BYTES = N * ROW;
@@ -158,27 +164,34 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < 2) {
-    // ------------------------------------------------------ TMA producers
-    const int par = warp;
-    if (lane == 0 && par == 1) prefetch_tmap(&tm_k);
-    if (lane == 0 && par == 0) {
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_q);
-      mbar_arrive_expect_tx(qbar, C::Q_BYTES + C::SFB_BYTES);
-      tma_load_2d(sm + C::OFF_Q, &tm_q, 0, (int32_t)(((int64_t)b * a.T + t0) * 64), qbar);
-      if (FMT == LCSC_FMT_FP4) {
-        const int64_t q_tiles = ((int64_t)a.T * 64 + 127) / 128;
-        const uint8_t* src = a.q_scale + ((int64_t)b * q_tiles + (t0 * 64) / 128) * 1024;
-        bulk_load(sm + C::OFF_SFB, src, C::SFB_BYTES, qbar);
-      }
-    }
+  if (warp < C::LANES) {
+    // ------------------------------------------------------ TMA + MMA lanes
+    // Lane r (warp r, one thread) takes tiles i = r, r + LANES, ...: it loads
+    // tile i + LANES * DIST with TMA, then issues the MMAs of tile i.  Every
+    // wait of the thread handling tile i is on an earlier tile (the TMA's
+    // stage was freed by the MMAs of tile i + LANES * DIST - STAGES < i).
+    const int r = warp;
     if (lane == 0) {
       const int64_t key_tiles = a.key_cap / 128;
-      for (int i = par; i < ntile; i += 2) {
+      prefetch_tmap(&tm_k);
+      if (r == 0) {
+        prefetch_tmap(&tm_q);
+        mbar_arrive_expect_tx(qbar, C::Q_BYTES + C::SFB_BYTES);
+        tma_load_2d(sm + C::OFF_Q, &tm_q, 0, (int32_t)(((int64_t)b * a.T + t0) * 64), qbar);
+        if (FMT == LCSC_FMT_FP4) {
+          const int64_t q_tiles = ((int64_t)a.T * 64 + 127) / 128;
+          const uint8_t* src = a.q_scale + ((int64_t)b * q_tiles + (t0 * 64) / 128) * 1024;
+          bulk_load(sm + C::OFF_SFB, src, C::SFB_BYTES, qbar);
+        }
+      }
+      bool live = true;
+      auto load = [&](int i) {  // TMA of tile i into stage i % STAGES
         const int s = i % C::STAGES;
         const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u, a.status)) break;
+        if (!mbar_wait(&empty[s], ph ^ 1u, a.status)) {
+          live = false;
+          return;
+        }
         const int64_t tile = tile_lo + i;
         mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::SFA_BYTES);
         tma_load_2d(sm + C::OFF_A + s * C::A_BYTES, &tm_k, 0, (int32_t)((int64_t)b * a.key_cap + tile * 128),
@@ -187,28 +200,30 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           const uint8_t* src = reinterpret_cast<const uint8_t*>(a.key_scale) + ((int64_t)b * key_tiles + tile) * 1024;
           bulk_load(sm + C::OFF_SFA + s * 1024, src, 1024, &full[s]);
         }
-      }
-    }
-  } else if (warp < 4) {
-    // ------------------------------------------------------ MMA issuers
-    const int par = warp - 2;
-    if (lane == 0) {
-      bool live = mbar_wait(qbar, 0, a.status);
+      };
+      const int my_n = ntile > r ? (ntile - r + C::LANES - 1) / C::LANES : 0;
+      for (int t = 0; t < C::DIST && t < my_n && live; ++t) load(r + C::LANES * t);
+      live = live && mbar_wait(qbar, 0, a.status);
       tc_fence_after();
       const uint32_t q_addr = smem_u32(sm + C::OFF_Q);
-      if (live && par == 0 && FMT == LCSC_FMT_FP4) {
+      if (live && r == 0 && FMT == LCSC_FMT_FP4) {
         for (int j = 0; j < 2; ++j)
           for (int c = 0; c < (C::N + 127) / 128; ++c)
             tmem_cp_32x128b_x4(tmem + C::SFB_COL + 8 * c + 4 * j,
                                smem_desc(smem_u32(sm + C::OFF_SFB + c * 1024 + j * 512), 16, 128, kSwNone));
       }
-      // the odd-tile issuer starts once the query scales are in TMEM
-      if (par == 0) tc_commit(sfb_bar);
+      // the other lanes start once the query scales are in TMEM
+      if (r == 0) tc_commit(sfb_bar);
       else live = live && mbar_wait(sfb_bar, 0, a.status);
       tc_fence_after();
       const uint32_t idesc = FMT == LCSC_FMT_FP4 ? idesc_mxf4nvf4(128, C::N) : idesc_dense(0, 0, 128, C::N);
       int last = -1;
-      for (int i = par; live && i < ntile; i += 2) {
+      for (int t = 0; live && t < my_n; ++t) {
+        if (t + C::DIST < my_n) {
+          load(r + C::LANES * (t + C::DIST));
+          if (!live) break;
+        }
+        const int i = r + C::LANES * t;
         const int s = i % C::STAGES;
         const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
         const int ab = i % C::NACC;
@@ -241,7 +256,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       if (last >= 0)  // the accumulator of the last tile is complete before TMEM is freed
         mbar_wait(&accf[last % C::NACC], (uint32_t)(last / C::NACC) & 1u, a.status);
     }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------ epilogue
     // Two groups of four warps take alternate tiles; within a group warp w
     // reads TMEM sub-partition w % 4 (rows 32 (w % 4) ..).
