@@ -230,48 +230,69 @@ __global__ void __launch_bounds__(kThreads) attn_partial_kernel(AttnLaunch a) {
   }
 }
 
-// grid (B*T, H); block DV threads (<= 512), one output dim each.  The
-// splits are read eight at a time with every load of a batch in flight.
+// Merge of the split partials (reference max m_s, sum l_s, unnormalised
+// O_s) and the sink: one pass with a running max, every load of a batch of
+// splits in flight.  grid (B*T, H / 4); block 4 heads x DV/4 threads, four
+// dims (one float4) per thread.
 template <int DV>
 __global__ void __launch_bounds__(DV) attn_combine_kernel(AttnLaunch a) {
-  constexpr int U = 8;
-  const int list = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
+  constexpr int U = 16;         // splits per batch
+  constexpr int TPH = DV / 4;   // threads per head
+  const int list = blockIdx.x;
+  const int h = blockIdx.y * 4 + threadIdx.x / TPH;
+  const int d4 = threadIdx.x % TPH;
   const float sigma = a.sink ? a.sink[h] : -INFINITY;
   const float* ml = a.part_ml + ((int64_t)list * a.splits * a.H + h) * 2;  // split s at ml[s * H * 2]
-  const float* po = a.part_o + ((int64_t)list * a.splits * a.H + h) * DV + d;
-  const int64_t ml_step = (int64_t)a.H * 2, o_step = (int64_t)a.H * DV;
-  float M = sigma;
+  const float4* po = reinterpret_cast<const float4*>(a.part_o + ((int64_t)list * a.splits * a.H + h) * DV) + d4;
+  const int64_t ml_step = (int64_t)a.H * 2, o_step = (int64_t)a.H * DV / 4;
+  float M = sigma, den = sigma > -INFINITY ? 1.f : 0.f;  // the sink adds e^(sigma - M) to the denominator
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s0 = 0; s0 < a.splits; s0 += U) {
-    float m[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) m[u] = s0 + u < a.splits ? ml[(s0 + u) * ml_step] : -INFINITY;
-#pragma unroll
-    for (int u = 0; u < U; ++u) M = fmaxf(M, m[u]);
-  }
-  float den = (M == -INFINITY) ? 0.f : expf(sigma - M);
-  float acc = 0.f;
-  for (int s0 = 0; s0 < a.splits; s0 += U) {
-    float m[U], l[U], o[U];
+    float m[U], l[U];
+    float4 o[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const bool in = s0 + u < a.splits;
       m[u] = in ? ml[(s0 + u) * ml_step] : -INFINITY;
       l[u] = in ? ml[(s0 + u) * ml_step + 1] : 0.f;
-      o[u] = in ? po[(s0 + u) * o_step] : 0.f;
+      o[u] = in ? po[(s0 + u) * o_step] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float mb = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < U; ++u) mb = fmaxf(mb, m[u]);
+    if (mb > M) {  // rescale what has been summed to the new maximum
+      const float r = M > -INFINITY ? expf(M - mb) : 0.f;
+      den *= r;
+      acc.x *= r;
+      acc.y *= r;
+      acc.z *= r;
+      acc.w *= r;
+      M = mb;
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (m[u] == -INFINITY) continue;  // an empty split (its O and sum are zero)
       const float f = expf(m[u] - M);
       den = fmaf(l[u], f, den);
-      acc = fmaf(o[u], f, acc);
+      acc.x = fmaf(o[u].x, f, acc.x);
+      acc.y = fmaf(o[u].y, f, acc.y);
+      acc.z = fmaf(o[u].z, f, acc.z);
+      acc.w = fmaf(o[u].w, f, acc.w);
     }
   }
-  const float out = den > 0.f ? acc / den : 0.f;
-  const int64_t oi = ((int64_t)list * a.H + h) * DV + d;
-  if (a.q_dtype == LCSC_DT_BF16) reinterpret_cast<uint16_t*>(a.out)[oi] = bf16_code(out);
-  else reinterpret_cast<float*>(a.out)[oi] = out;
-  if (a.lse && d == 0) a.lse[(int64_t)list * a.H + h] = (den > 0.f) ? M + logf(den) : -INFINITY;
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  const float r[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+  const int64_t oi = ((int64_t)list * a.H + h) * DV + 4 * d4;
+  if (a.q_dtype == LCSC_DT_BF16) {
+    uint16_t* out = reinterpret_cast<uint16_t*>(a.out) + oi;
+    out[0] = bf16_code(r[0]);
+    out[1] = bf16_code(r[1]);
+    out[2] = bf16_code(r[2]);
+    out[3] = bf16_code(r[3]);
+  } else {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + oi) = make_float4(r[0], r[1], r[2], r[3]);
+  }
+  if (a.lse && d4 == 0) a.lse[(int64_t)list * a.H + h] = (den > 0.f) ? M + logf(den) : -INFINITY;
 }
 
 template <int KVFMT, int D, int DV, int HPC, bool kSepV>
@@ -285,7 +306,7 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
   dim3 grid(a.splits, a.H / HPC, a.B * a.T);
   kern<<<grid, kThreads, smem, stream>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  attn_combine_kernel<DV><<<dim3(a.B * a.T, a.H), DV, 0, stream>>>(a);
+  attn_combine_kernel<DV><<<dim3(a.B * a.T, a.H / 4), DV, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -308,7 +329,7 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
   if (attn_mma_supported(a)) {
     cudaError_t e = launch_attn_mma(a, stream);
     if (e != cudaSuccess) return e;
-    attn_combine_kernel<512><<<dim3(a.B * a.T, a.H), 512, 0, stream>>>(a);
+    attn_combine_kernel<512><<<dim3(a.B * a.T, a.H / 4), 512, 0, stream>>>(a);
     return cudaGetLastError();
   }
   if (a.kv.f.fmt == LCSC_FMT_F32 && a.D == 128 && a.Dv == 128 && a.H % 8 == 0) {
