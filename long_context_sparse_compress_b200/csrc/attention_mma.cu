@@ -49,6 +49,7 @@ constexpr float kRescale = 8.f;
 constexpr float kLog2e = 1.4426950408889634f;  // log2(e), to work in base 2  // rescale O only when the max grows by more
 
 // shared memory (offsets from a 1024-aligned base)
+constexpr int kOS = kD + 4;       // row stride (floats) of the partial O staged in shared memory
 constexpr int KB_Q = kH * 128;    // one 64-dim block of Q  (8 KB)
 constexpr int KB_K = kTR * 128;   // one 64-dim block of a K tile (8 KB)
 constexpr int OFF_Q = 0;                       // 8 blocks = 64 KB
@@ -65,6 +66,7 @@ constexpr int OFF_TM = OFF_MASK + 16;
 constexpr int OFF_ABORT = OFF_TM + 4;
 constexpr int OFF_LSTOP = OFF_ABORT + 4;
 constexpr int SMEM = OFF_LSTOP + 8 + 1024;
+static_assert(kH * kOS * 4 <= OFF_BAR - OFF_K, "the staged partial O fits in the K and P buffers");
 
 // Byte offset of (row, byte) in a [rows][128 B] block with the 128-byte swizzle
 // (16-byte chunk index XOR row % 8) that the tensor cores read.
@@ -584,13 +586,16 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
     if (done) done = warp_wait(&pv_done[(ntiles - 1) & 1], (uint32_t)((ntiles - 1) >> 1) & 1u, a, abort);
     tc_fence_after();
     const int64_t pidx = ((int64_t)list * a.splits + blockIdx.x) * a.H + head;
+    // O -> shared memory (the K tiles and P are dead: every P V is done),
+    // padded rows so the 16-byte stores of a warp's heads hit distinct banks
+    float* o_s = reinterpret_cast<float*>(sm + OFF_K);
     for (int c = 0; c < kD; c += 64) {  // two TMEM loads in flight
       uint32_t r0[32], r1[32];
       tmem_ld_32(row_addr + c, r0);
       tmem_ld_32(row_addr + c + 32, r1);
       tmem_ld_wait(r0, r1);
       if (lane < 16) {
-        float* po = a.part_o + pidx * kD + c;
+        float* po = o_s + head * kOS + c;
 #pragma unroll
         for (int q = 0; q < 32; q += 4) {
           *reinterpret_cast<float4*>(po + q) =
@@ -611,6 +616,12 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
   }
   tc_fence_before();
   __syncthreads();
+  {  // the partial O of this split, [64 heads][512] contiguous: coalesced 16-byte stores by every thread
+    const float* o_s = reinterpret_cast<const float*>(sm + OFF_K);
+    float4* dst = reinterpret_cast<float4*>(a.part_o + ((int64_t)list * a.splits + blockIdx.x) * a.H * kD);
+    for (int i = tid; i < kH * (kD / 4); i += kThr)
+      dst[i] = *reinterpret_cast<const float4*>(o_s + (i / (kD / 4)) * kOS + 4 * (i % (kD / 4)));
+  }
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
