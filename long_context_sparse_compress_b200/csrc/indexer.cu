@@ -24,6 +24,7 @@
 //          shared memory), ties to the lowest index, the chosen ones marked,
 //          and the bitmap compacted into the output in index order.
 #include "kernels.cuh"
+#include "sm100.cuh"
 #include "topk.cuh"
 
 namespace lcsc {
@@ -236,6 +237,8 @@ __global__ void __launch_bounds__(512) topk_hist_kernel(IndexLaunch a, int slice
 // All slices of a list: scores above the digit-1 threshold bin go to the
 // output, those in it to the candidate list.
 __global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int slices) {
+  extern __shared__ float4 slice_s[];  // the slice's scores, one bulk copy
+  __shared__ uint64_t bar;
   const int list = blockIdx.y;
   const ListInfo li = list_info(a, list, slices);
   const float* s = a.scores + (int64_t)list * a.stride;
@@ -248,19 +251,48 @@ __global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int sl
     }
     return;
   }
+  const int64_t n4 = li.hi > li.lo ? (li.hi - li.lo) >> 2 : 0;  // whole 16-byte groups
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && n4 > 0) {
+    sm100::mbar_arrive_expect_tx(&bar, (uint32_t)(n4 * 16));
+    sm100::bulk_load(slice_s, s + li.lo, (uint32_t)(n4 * 16), &bar);
+  }
   uint32_t* ctr = a.counters + (int64_t)list * 8;
   const uint32_t t1 = ctr[3];
   uint32_t* bits = a.sel_bits + (int64_t)list * a.bit_stride;
   for (int64_t w = li.lo / 32 + threadIdx.x; w < (li.hi + 31) / 32; w += 512) bits[w] = 0u;
   __syncthreads();
   uint32_t* cand = a.cand + (int64_t)list * 2 * a.cand_cap;  // (index, key) pairs
-  scan_scores(s, li.lo, li.hi, [&](int64_t g, float v) {
+  auto visit = [&](int64_t g, float v) {
     const uint32_t key = float_key(v);
     const uint32_t d1 = key >> 20;
     if (d1 > t1) atomicOr(&bits[g >> 5], 1u << (g & 31));
     const uint32_t c = warp_append(&ctr[1], d1 == t1);
     if (d1 == t1 && c < a.cand_cap) reinterpret_cast<uint2*>(cand)[c] = make_uint2((uint32_t)g, key);
-  });
+  };
+  if (n4 > 0 && sm100::mbar_wait(&bar, 0, a.status)) {
+    // whole warps step together; one vote per four scores, and only a warp
+    // holding a score at or above the bin takes the per-score path
+    for (int64_t i0 = 0; i0 < n4; i0 += 512) {
+      const int64_t i = i0 + threadIdx.x;
+      const bool in = i < n4;
+      const float4 v = in ? slice_s[i] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      const bool hit = in && ((float_key(v.x) >> 20) >= t1 || (float_key(v.y) >> 20) >= t1 ||
+                              (float_key(v.z) >> 20) >= t1 || (float_key(v.w) >> 20) >= t1);
+      if (__any_sync(0xffffffffu, hit) && in) {
+        const int64_t g = li.lo + 4 * i;
+        visit(g, v.x);
+        visit(g + 1, v.y);
+        visit(g + 2, v.z);
+        visit(g + 3, v.w);
+      }
+    }
+  }
+  for (int64_t g = li.lo + 4 * n4 + threadIdx.x; g < li.hi; g += 512) visit(g, s[g]);
 }
 
 // Smallest index bound tau such that at least `need` of the tied candidates
@@ -421,8 +453,8 @@ __global__ void __launch_bounds__(512) topk_final_kernel(IndexLaunch a) {
       block_total += ws;
     }
     uint32_t off = base + before + incl - local;
-#pragma unroll 1
-    for (int q = 0; q < 16; ++q) {
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {  // unrolled: wv stays in registers
       uint32_t bw = wv[q];
       while (bw) {
         const int bit = __ffs(bw) - 1;
@@ -492,7 +524,12 @@ cudaError_t launch_topk(const IndexLaunch& a, cudaStream_t stream) {
     topk_hist_kernel<<<tgrid, 512, 0, stream>>>(a, slices);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  topk_collect_kernel<<<tgrid, 512, 0, stream>>>(a, slices);
+  // the collect pass copies each slice into shared memory in one bulk copy
+  const int64_t per_max = ((a.n_max + slices - 1) / slices + 31) / 32 * 32;
+  const size_t slice_bytes = (size_t)per_max * 4;
+  e = cudaFuncSetAttribute(topk_collect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)slice_bytes);
+  if (e != cudaSuccess) return e;
+  topk_collect_kernel<<<tgrid, 512, slice_bytes, stream>>>(a, slices);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   e = cudaFuncSetAttribute(topk_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFinalSmem);
   if (e != cudaSuccess) return e;
