@@ -239,6 +239,9 @@ __global__ void __launch_bounds__(512) topk_hist_kernel(IndexLaunch a, int slice
 __global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int slices) {
   extern __shared__ float4 slice_s[];  // the slice's scores, one bulk copy
   __shared__ uint64_t bar;
+  constexpr int kLocal = 2048;          // candidates gathered in shared memory first
+  __shared__ uint2 cand_s[kLocal];
+  __shared__ uint32_t n_local, base_g;
   const int list = blockIdx.y;
   const ListInfo li = list_info(a, list, slices);
   const float* s = a.scores + (int64_t)list * a.stride;
@@ -255,6 +258,7 @@ __global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int sl
   if (threadIdx.x == 0) {
     sm100::mbar_init(&bar, 1);
     sm100::fence_barrier_init();
+    n_local = 0;
   }
   __syncthreads();
   if (threadIdx.x == 0 && n4 > 0) {
@@ -267,12 +271,21 @@ __global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int sl
   for (int64_t w = li.lo / 32 + threadIdx.x; w < (li.hi + 31) / 32; w += 512) bits[w] = 0u;
   __syncthreads();
   uint32_t* cand = a.cand + (int64_t)list * 2 * a.cand_cap;  // (index, key) pairs
+  // above the bin: a mark (no reply awaited); in it: a shared-memory slot,
+  // or past kLocal a workspace slot of its own
   auto visit = [&](int64_t g, float v) {
     const uint32_t key = float_key(v);
     const uint32_t d1 = key >> 20;
     if (d1 > t1) atomicOr(&bits[g >> 5], 1u << (g & 31));
-    const uint32_t c = warp_append(&ctr[1], d1 == t1);
-    if (d1 == t1 && c < a.cand_cap) reinterpret_cast<uint2*>(cand)[c] = make_uint2((uint32_t)g, key);
+    if (d1 == t1) {
+      const uint32_t c = atomicAdd(&n_local, 1u);
+      if (c < (uint32_t)kLocal) {
+        cand_s[c] = make_uint2((uint32_t)g, key);
+      } else {
+        const uint32_t cg = atomicAdd(&ctr[1], 1u);
+        if (cg < a.cand_cap) reinterpret_cast<uint2*>(cand)[cg] = make_uint2((uint32_t)g, key);
+      }
+    }
   };
   if (n4 > 0 && sm100::mbar_wait(&bar, 0, a.status)) {
     // whole warps step together; one vote per four scores, and only a warp
@@ -293,6 +306,13 @@ __global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int sl
     }
   }
   for (int64_t g = li.lo + 4 * n4 + threadIdx.x; g < li.hi; g += 512) visit(g, s[g]);
+  // the shared-memory candidates: one reservation for the CTA, then a copy
+  __syncthreads();
+  const uint32_t nl = n_local < (uint32_t)kLocal ? n_local : (uint32_t)kLocal;
+  if (threadIdx.x == 0) base_g = nl ? atomicAdd(&ctr[1], nl) : 0u;
+  __syncthreads();
+  for (uint32_t i = threadIdx.x; i < nl; i += 512)
+    if (base_g + i < a.cand_cap) reinterpret_cast<uint2*>(cand)[base_g + i] = cand_s[i];
 }
 
 // Smallest index bound tau such that at least `need` of the tied candidates
