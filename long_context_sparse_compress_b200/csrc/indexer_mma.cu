@@ -18,10 +18,13 @@
 // pipeline, so tiles are dealt round-robin to LANES lanes (warps 0 .. LANES-1,
 // one thread each): lane r loads its tiles with TMA (hardware swizzle) into a
 // STAGES-deep ring, DIST of its tiles ahead, and issues their MMAs into NACC
-// TMEM accumulators.  Warps 4-11 (two groups of four taking alternate tiles)
-// drain the accumulators with tcgen05.ld, apply ReLU and the head weights,
-// write one fp32 score per (query, key) and count it in the list's
-// shared-memory histogram of the top-k's first digit.
+// TMEM accumulators.  Warps 4-11 (two groups of four) drain the accumulators
+// with tcgen05.ld, apply ReLU and the head weights, write one fp32 score per
+// (query, key) and count it in the list's shared-memory histogram of the
+// top-k's first digit.  One query: the groups take alternate tiles.  Four
+// queries: both groups drain every tile (two queries each), reading TMEM in
+// the accumulator-fragment layout so that each thread's head weights stay in
+// registers; the ReLU'd products of a key row are summed within a quad.
 #include <cudaTypedefs.h>
 
 #include "kernels.cuh"
@@ -58,12 +61,12 @@ struct Cfg {
   static constexpr int KSTEPS = 4 - (FMT == LCSC_FMT_FP4 ? 2 : 0);  // 32 bytes of K per MMA
   // Ring depth: enough bytes in flight to cover DRAM latency, and more than
   // half the shared memory so that a second CTA never shares the SM's TMEM.
-  static constexpr int STAGES = FMT == LCSC_FMT_FP4 ? 20 : (NQ == 1 ? 8 : 5);
+  static constexpr int STAGES = FMT == LCSC_FMT_FP4 ? 20 : (NQ == 1 ? 8 : 6);
   // Accumulators in TMEM: the MMA runs up to NACC tiles ahead of the epilogue.
   static constexpr int NACC = NQ == 1 ? 4 : 2;
   // TMA + MMA lanes (warps 0 .. LANES-1) and how many of its own tiles each
   // loads ahead; LANES * DIST < STAGES keeps every wait on an earlier tile.
-  static constexpr int LANES = FMT == LCSC_FMT_FP4 ? 4 : (NQ == 1 ? 2 : 1);
+  static constexpr int LANES = FMT == LCSC_FMT_FP4 ? 4 : 2;
   static constexpr int DIST = STAGES / LANES - 1;
   static_assert(DIST >= 1 && LANES * DIST < STAGES, "lane prefetch distance");
   static constexpr int A_BYTES = TILE * ROW;
@@ -92,6 +95,7 @@ struct Cfg {
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + slack to align the base
   static_assert(COLS_USED <= 512 && SFA_COL <= COLS_USED, "TMEM budget");
   static_assert(A_BYTES % 1024 == 0 && Q_BYTES % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+  static_assert(OFF_W % 16 == 0, "head weights are read as float4");
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -146,7 +150,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     }
     for (int j = 0; j < C::NACC; ++j) {
       mbar_init(&accf[j], 1);
-      mbar_init(&acce[j], 4);  // the four warps of the group draining it
+      mbar_init(&acce[j], NQ == 1 ? 4 : 8);  // the warps draining it
     }
     mbar_init(qbar, 1);
     mbar_init(sfb_bar, 1);
@@ -258,57 +262,127 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------ epilogue
-    // Two groups of four warps take alternate tiles; within a group warp w
-    // reads TMEM sub-partition w % 4 (rows 32 (w % 4) ..).
+    // Warp w reads TMEM sub-partition w % 4 (key rows 32 (w % 4) ..).  One
+    // query: two groups of four warps take alternate tiles.  Several
+    // queries: both groups drain every tile, group g the queries
+    // [g NQ/2, (g + 1) NQ/2), so a tile's accumulator is free again after half
+    // the work and the other one fills meanwhile.
     const int grp = (warp - 4) >> 2;
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const float* kscale = reinterpret_cast<const float*>(a.key_scale) + (int64_t)b * a.key_cap;
-    float wr[NQ == 1 ? 64 : 1];  // head weights in registers when one query
     if constexpr (NQ == 1) {
+      float wr[64];  // head weights in registers
 #pragma unroll
       for (int j = 0; j < 64; ++j) wr[j] = w_s[j];
-    }
-    for (int i = grp; i < ntile; i += 2) {
-      const int ab = i % C::NACC;
-      const int64_t g = (tile_lo + i) * 128 + row;
-      const float sk = FMT == LCSC_FMT_FP8 ? kscale[g] : 1.f;
-      if (!mbar_wait(&accf[ab], (uint32_t)(i / C::NACC) & 1u, a.status)) break;
-      tc_fence_after();
-#pragma unroll 1
-      for (int nq = 0; nq < NQ; ++nq) {
+      for (int i = grp; i < ntile; i += 2) {
+        const int ab = i % C::NACC;
+        const int64_t g = (tile_lo + i) * 128 + row;
+        const float sk = FMT == LCSC_FMT_FP8 ? kscale[g] : 1.f;
+        if (!mbar_wait(&accf[ab], (uint32_t)(i / C::NACC) & 1u, a.status)) break;
+        tc_fence_after();
         uint32_t r0[32], r1[32];
-        const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) + ab * C::N + nq * 64;
+        const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) + ab * C::N;
         tmem_ld_32(taddr, r0);
         tmem_ld_32(taddr + 32, r1);
         tmem_ld_wait();
         float p[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) p[j] = 0.f;
-        if constexpr (NQ == 1) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) p[j & 7] = fmaf(wr[j], fmaxf(__uint_as_float(r0[j]), 0.f), p[j & 7]);
+        for (int j = 0; j < 32; ++j) p[j & 7] = fmaf(wr[j], fmaxf(__uint_as_float(r0[j]), 0.f), p[j & 7]);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) p[j & 7] = fmaf(wr[32 + j], fmaxf(__uint_as_float(r1[j]), 0.f), p[j & 7]);
-        } else {
-          const float* w = w_s + nq * 64;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) p[j & 7] = fmaf(w[j], fmaxf(__uint_as_float(r0[j]), 0.f), p[j & 7]);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) p[j & 7] = fmaf(w[32 + j], fmaxf(__uint_as_float(r1[j]), 0.f), p[j & 7]);
-        }
+        for (int j = 0; j < 32; ++j) p[j & 7] = fmaf(wr[32 + j], fmaxf(__uint_as_float(r1[j]), 0.f), p[j & 7]);
         const float acc = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
-        const int t = t0 + nq;
-        const int64_t n_p = (L - a.T + t + 1) / a.m;
+        const int64_t n_p = (L - a.T + t0 + 1) / a.m;
         if (g < n_p) {
           const float v = acc * sk;
-          a.scores[((int64_t)b * a.T + t) * a.stride + g] = v;
-          atomicAdd(&hist_s[nq * kTopkBins + (float_key(v) >> 20)], 1u);
+          a.scores[((int64_t)b * a.T + t0) * a.stride + g] = v;
+          atomicAdd(&hist_s[float_key(v) >> 20], 1u);
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acce[ab]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acce[ab]);
+    } else {
+      // TMEM is read in the mma accumulator-fragment layout (16 lanes x 64
+      // columns per load): thread t holds key rows t/4 and t/4 + 8 of a
+      // 16-row half and the 16 head columns 8c + 2 (t % 4) + {0, 1} of a
+      // query, so its head weights stay in registers for the whole kernel.
+      // The four threads of a quad share rows; a reduce-scatter over the quad
+      // leaves thread t the score of row t/4 + 8 (t % 4) of the sub-partition.
+      constexpr int QH = NQ / 2;  // queries per group
+      const int nq0 = grp * QH;
+      const int j4 = lane & 3;
+      float wq[QH][16];
+#pragma unroll
+      for (int q = 0; q < QH; ++q)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          wq[q][2 * c] = w_s[(nq0 + q) * 64 + 8 * c + 2 * j4];
+          wq[q][2 * c + 1] = w_s[(nq0 + q) * 64 + 8 * c + 2 * j4 + 1];
+        }
+      int64_t n_q[QH];  // entries visible to each of the group's queries
+#pragma unroll
+      for (int q = 0; q < QH; ++q) n_q[q] = ok ? (L - a.T + t0 + nq0 + q + 1) / a.m : 0;
+      const int my_row = q4 * 32 + (lane >> 2) + 8 * j4;
+      // partial sums of rows (t/4, t/4 + 8) of a 16-row half over this
+      // thread's columns
+      auto half_sum = [&](const uint32_t (&r)[32], const float (&w)[16], float& s0, float& s1) {
+        float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          a0 = fmaf(w[2 * c], fmaxf(__uint_as_float(r[4 * c]), 0.f), a0);
+          a1 = fmaf(w[2 * c + 1], fmaxf(__uint_as_float(r[4 * c + 1]), 0.f), a1);
+          b0 = fmaf(w[2 * c], fmaxf(__uint_as_float(r[4 * c + 2]), 0.f), b0);
+          b1 = fmaf(w[2 * c + 1], fmaxf(__uint_as_float(r[4 * c + 3]), 0.f), b1);
+        }
+        s0 = a0 + a1;
+        s1 = b0 + b1;
+      };
+      // v[j]: this thread's partial of row t/4 + 8 j; returns the quad's sum
+      // of row t/4 + 8 (t % 4)
+      auto quad_sum = [&](float v0, float v1, float v2, float v3) -> float {
+        const bool hi = j4 & 2, odd = j4 & 1;
+        float k0 = hi ? v2 : v0, k1 = hi ? v3 : v1;
+        const float s0 = hi ? v0 : v2, s1 = hi ? v1 : v3;
+        k0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+        k1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+        float k = odd ? k1 : k0;
+        const float s = odd ? k0 : k1;
+        k += __shfl_xor_sync(0xffffffffu, s, 1);
+        return k;
+      };
+      for (int i = 0; i < ntile; ++i) {
+        const int ab = i % C::NACC;
+        const int64_t g = (tile_lo + i) * 128 + my_row;
+        const float sk = FMT == LCSC_FMT_FP8 ? kscale[g] : 1.f;
+        if (!mbar_wait(&accf[ab], (uint32_t)(i / C::NACC) & 1u, a.status)) break;
+        tc_fence_after();
+        const uint32_t base = tmem + ((uint32_t)(q4 * 32) << 16) + ab * C::N + nq0 * 64;
+        uint32_t ra[32], rb[32];
+        tmem_ld_16x256b_x8(base, ra);
+        tmem_ld_wait(ra);
+#pragma unroll
+        for (int q = 0; q < QH; ++q) {
+          float v0, v1, v2, v3;
+          tmem_ld_16x256b_x8(base + (16u << 16) + 64 * q, rb);  // rows 16..31 of the sub-partition
+          half_sum(ra, wq[q], v0, v1);
+          tmem_ld_wait(rb);
+          if (q + 1 < QH) tmem_ld_16x256b_x8(base + 64 * (q + 1), ra);
+          half_sum(rb, wq[q], v2, v3);
+          const float acc = quad_sum(v0, v1, v2, v3);
+          if (g < n_q[q]) {
+            const float v = acc * sk;
+            a.scores[((int64_t)b * a.T + t0 + nq0 + q) * a.stride + g] = v;
+            atomicAdd(&hist_s[(nq0 + q) * kTopkBins + (float_key(v) >> 20)], 1u);
+          }
+          if (q + 1 < QH) tmem_ld_wait(ra);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acce[ab]);
+      }
     }
   }
   __syncthreads();
