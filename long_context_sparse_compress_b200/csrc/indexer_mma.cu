@@ -13,18 +13,19 @@
 //  * FP8 keys and queries: tcgen05.mma kind::f8f6f4 on the codes; the
 //    per-row scales are positive, so the epilogue applies them outside ReLU:
 //    s = sk[g] * sum_h (w[h] sq[h]) ReLU(acc[h]).
-// Warp roles (384 threads, one CTA per SM).  One thread's issue of TMA and
+// Warp roles (one CTA per SM).  One thread's issue of TMA and
 // tcgen05 instructions (tens of cycles each) is what limits a single
 // pipeline, so tiles are dealt round-robin to LANES lanes (warps 0 .. LANES-1,
 // one thread each): lane r loads its tiles with TMA (hardware swizzle) into a
 // STAGES-deep ring, DIST of its tiles ahead, and issues their MMAs into NACC
-// TMEM accumulators.  Warps 4-11 (two groups of four) drain the accumulators
+// TMEM accumulators.  Groups of four epilogue warps drain the accumulators
 // with tcgen05.ld, apply ReLU and the head weights, write one fp32 score per
 // (query, key) and count it in the list's shared-memory histogram of the
-// top-k's first digit.  One query: the groups take alternate tiles.  Four
-// queries: both groups drain every tile (two queries each), reading TMEM in
-// the accumulator-fragment layout so that each thread's head weights stay in
-// registers; the ReLU'd products of a key row are summed within a quad.
+// top-k's first digit.  One query (384 threads): two groups take alternate
+// tiles.  Four queries (576 threads): four groups drain every tile, one query
+// each, reading TMEM in the accumulator-fragment layout so that each
+// thread's head weights stay in registers; the ReLU'd products of a key row
+// are summed within a quad.
 #include <cudaTypedefs.h>
 
 #include "kernels.cuh"
@@ -68,6 +69,13 @@ struct Cfg {
   // loads ahead; LANES * DIST < STAGES keeps every wait on an earlier tile.
   static constexpr int LANES = FMT == LCSC_FMT_FP4 ? 4 : 2;
   static constexpr int DIST = STAGES / LANES - 1;
+  // Epilogue: GROUPS groups of four warps from warp EPI0 on (warp w reads
+  // TMEM sub-partition w % 4).  Several queries: group g drains query g of
+  // every tile.
+  static constexpr int GROUPS = NQ == 1 ? 2 : NQ;
+  static constexpr int EPI0 = NQ == 1 ? 4 : LANES;
+  static constexpr int THREADS = (EPI0 + 4 * GROUPS) * 32;
+  static_assert(NQ == 1 || GROUPS == NQ, "one query per epilogue group");
   static_assert(DIST >= 1 && LANES * DIST < STAGES, "lane prefetch distance");
   static constexpr int A_BYTES = TILE * ROW;
   static constexpr int SFA_BYTES = FMT == LCSC_FMT_FP4 ? 1024 : 0;
@@ -98,14 +106,30 @@ struct Cfg {
   static_assert(OFF_W % 16 == 0, "head weights are read as float4");
 };
 
+// Two fp32 lanes in one 64-bit register, and the packed fused multiply-add
+// of sm_100 (each lane an IEEE fma, as fmaf).
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 unpack2(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-constexpr int kIdxThreads = 384;
-
 template <int FMT, int NQ>
-__global__ void __launch_bounds__(kIdxThreads, 1)
+__global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
     index_mma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                      const MmaArgs a) {
   using C = Cfg<FMT, NQ>;
@@ -150,7 +174,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     }
     for (int j = 0; j < C::NACC; ++j) {
       mbar_init(&accf[j], 1);
-      mbar_init(&acce[j], NQ == 1 ? 4 : 8);  // the warps draining it
+      mbar_init(&acce[j], NQ == 1 ? 4 : 4 * C::GROUPS);  // the warps draining it
     }
     mbar_init(qbar, 1);
     mbar_init(sfb_bar, 1);
@@ -260,14 +284,14 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       if (last >= 0)  // the accumulator of the last tile is complete before TMEM is freed
         mbar_wait(&accf[last % C::NACC], (uint32_t)(last / C::NACC) & 1u, a.status);
     }
-  } else if (warp >= 4) {
+  } else if (warp >= C::EPI0) {
     // ------------------------------------------------------ epilogue
     // Warp w reads TMEM sub-partition w % 4 (key rows 32 (w % 4) ..).  One
     // query: two groups of four warps take alternate tiles.  Several
-    // queries: both groups drain every tile, group g the queries
-    // [g NQ/2, (g + 1) NQ/2), so a tile's accumulator is free again after half
-    // the work and the other one fills meanwhile.
-    const int grp = (warp - 4) >> 2;
+    // queries: every group drains every tile, group g query g; a warp
+    // copies its 64 columns to registers and hands the accumulator back
+    // before summing, so the MMAs of the next tiles overlap the sums.
+    const int grp = (warp - C::EPI0) >> 2;
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const float* kscale = reinterpret_cast<const float*>(a.key_scale) + (int64_t)b * a.key_cap;
@@ -311,34 +335,28 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       // query, so its head weights stay in registers for the whole kernel.
       // The four threads of a quad share rows; a reduce-scatter over the quad
       // leaves thread t the score of row t/4 + 8 (t % 4) of the sub-partition.
-      constexpr int QH = NQ / 2;  // queries per group
-      const int nq0 = grp * QH;
+      const int nq = grp;  // this group's query
       const int j4 = lane & 3;
-      float wq[QH][16];
+      uint64_t wq[8];  // (w[8c + 2 (t % 4)], w[8c + 2 (t % 4) + 1]) pairs
 #pragma unroll
-      for (int q = 0; q < QH; ++q)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          wq[q][2 * c] = w_s[(nq0 + q) * 64 + 8 * c + 2 * j4];
-          wq[q][2 * c + 1] = w_s[(nq0 + q) * 64 + 8 * c + 2 * j4 + 1];
-        }
-      int64_t n_q[QH];  // entries visible to each of the group's queries
-#pragma unroll
-      for (int q = 0; q < QH; ++q) n_q[q] = ok ? (L - a.T + t0 + nq0 + q + 1) / a.m : 0;
+      for (int c = 0; c < 8; ++c) wq[c] = pack2(w_s[nq * 64 + 8 * c + 2 * j4], w_s[nq * 64 + 8 * c + 2 * j4 + 1]);
+      const int64_t n_q = ok ? (L - a.T + t0 + nq + 1) / a.m : 0;  // entries the query sees
       const int my_row = q4 * 32 + (lane >> 2) + 8 * j4;
+      float* score_row = a.scores + ((int64_t)b * a.T + t0 + nq) * a.stride;
+      uint32_t* hist_q = hist_s + nq * kTopkBins;
       // partial sums of rows (t/4, t/4 + 8) of a 16-row half over this
-      // thread's columns
-      auto half_sum = [&](const uint32_t (&r)[32], const float (&w)[16], float& s0, float& s1) {
-        float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+      // thread's columns (the column pair of each 8-column block in one
+      // packed fma)
+      auto half_sum = [&](const uint32_t (&r)[32], float& s0, float& s1) {
+        uint64_t pa = 0, pb = 0;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          a0 = fmaf(w[2 * c], fmaxf(__uint_as_float(r[4 * c]), 0.f), a0);
-          a1 = fmaf(w[2 * c + 1], fmaxf(__uint_as_float(r[4 * c + 1]), 0.f), a1);
-          b0 = fmaf(w[2 * c], fmaxf(__uint_as_float(r[4 * c + 2]), 0.f), b0);
-          b1 = fmaf(w[2 * c + 1], fmaxf(__uint_as_float(r[4 * c + 3]), 0.f), b1);
+          pa = ffma2(wq[c], pack2(fmaxf(__uint_as_float(r[4 * c]), 0.f), fmaxf(__uint_as_float(r[4 * c + 1]), 0.f)), pa);
+          pb = ffma2(wq[c], pack2(fmaxf(__uint_as_float(r[4 * c + 2]), 0.f), fmaxf(__uint_as_float(r[4 * c + 3]), 0.f)), pb);
         }
-        s0 = a0 + a1;
-        s1 = b0 + b1;
+        const float2 a2 = unpack2(pa), b2 = unpack2(pb);
+        s0 = a2.x + a2.y;
+        s1 = b2.x + b2.y;
       };
       // v[j]: this thread's partial of row t/4 + 8 j; returns the quad's sum
       // of row t/4 + 8 (t % 4)
@@ -359,29 +377,26 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         const float sk = FMT == LCSC_FMT_FP8 ? kscale[g] : 1.f;
         if (!mbar_wait(&accf[ab], (uint32_t)(i / C::NACC) & 1u, a.status)) break;
         tc_fence_after();
-        const uint32_t base = tmem + ((uint32_t)(q4 * 32) << 16) + ab * C::N + nq0 * 64;
+        const uint32_t base = tmem + ((uint32_t)(q4 * 32) << 16) + ab * C::N + nq * 64;
+        // the query's 64 columns of this sub-partition's rows go to
+        // registers and the accumulator is handed back before the sums, so
+        // the next tile's MMAs overlap them
         uint32_t ra[32], rb[32];
         tmem_ld_16x256b_x8(base, ra);
-        tmem_ld_wait(ra);
-#pragma unroll
-        for (int q = 0; q < QH; ++q) {
-          float v0, v1, v2, v3;
-          tmem_ld_16x256b_x8(base + (16u << 16) + 64 * q, rb);  // rows 16..31 of the sub-partition
-          half_sum(ra, wq[q], v0, v1);
-          tmem_ld_wait(rb);
-          if (q + 1 < QH) tmem_ld_16x256b_x8(base + 64 * (q + 1), ra);
-          half_sum(rb, wq[q], v2, v3);
-          const float acc = quad_sum(v0, v1, v2, v3);
-          if (g < n_q[q]) {
-            const float v = acc * sk;
-            a.scores[((int64_t)b * a.T + t0 + nq0 + q) * a.stride + g] = v;
-            atomicAdd(&hist_s[(nq0 + q) * kTopkBins + (float_key(v) >> 20)], 1u);
-          }
-          if (q + 1 < QH) tmem_ld_wait(ra);
-        }
+        tmem_ld_16x256b_x8(base + (16u << 16), rb);  // rows 16..31 of the sub-partition
+        tmem_ld_wait(ra, rb);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acce[ab]);
+        float v0, v1, v2, v3;
+        half_sum(ra, v0, v1);
+        half_sum(rb, v2, v3);
+        const float acc = quad_sum(v0, v1, v2, v3);
+        if (g < n_q) {
+          const float v = acc * sk;
+          score_row[g] = v;
+          atomicAdd(&hist_q[float_key(v) >> 20], 1u);
+        }
       }
     }
   }
@@ -461,7 +476,7 @@ cudaError_t launch_mma(const IndexLaunch& a, cudaStream_t stream) {
   auto kern = index_mma_kernel<FMT, NQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(m.chunks, (unsigned)ctas), kIdxThreads, C::SMEM, stream>>>(tk, tq, m);
+  kern<<<dim3(m.chunks, (unsigned)ctas), C::THREADS, C::SMEM, stream>>>(tk, tq, m);
   return cudaGetLastError();
 }
 
