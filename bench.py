@@ -36,7 +36,9 @@ from long_context_sparse_compress_b200 import synth, workloads  # noqa: E402
 
 METRIC = "CSA/HCA decode queries/s at 128K-1M ctx; % HBM roofline; prefill % tensor peak"
 DEFAULT_WORKLOAD = workloads.PAIR_DECODE_1M_B16.name
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+# dense tensor-core rate of an operand type relative to bf16 (nominal B200 ratios)
+TENSOR_RATIO = {"fp8": 2.0, "fp4": 4.0}
 
 
 def measured_peaks():
@@ -226,15 +228,23 @@ def source_sha(*names):
     return h.hexdigest()[:16]
 
 
+def index_dtype(layer_wls):
+    """The indexer's arithmetic type, as the dtype string's first part."""
+    fmts = {lw.idx_fmt for lw in layer_wls if lw.kind == "csa"}
+    names = {"fp4": "e2m1 x e2m1 block-scaled MMA (indexer), ", "fp8": "e4m3 x e4m3 MMA (indexer), ",
+             "f32": "f32 (indexer), ", "bf16": "f32 from bf16 (indexer), "}
+    return "".join(names.get(f, f + " (indexer), ") for f in sorted(fmts))
+
+
 def recorded_traffic(kernel, workload, sha):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
     the current source of the kernel (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
-        rec = json.load(open(path))[kernel]
+        rec = json.load(open(path))[kernel][workload]
     except (OSError, ValueError, KeyError):
         return None
-    if rec.get("source_sha") != sha or rec.get("workload") != workload:
+    if rec.get("source_sha") != sha:
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -339,20 +349,36 @@ def run_lcsc(args):
                     for name, a, b in (("compress", 0, 1), ("quantize", 1, 2), ("index_score", 2, 3),
                                        ("topk", 3, 4), ("sparse_attn", 4, 5))}
         cw = csa.wl
-        key_b = L.row_bytes(cw.idx_fmt, cw.d_I) + (cw.d_I // 16 if cw.idx_fmt == "fp4" else 4)
-        n_keys = cw.B * cw.n_entries()
-        q_b = cw.B * cw.T * cw.H_I * (key_b + 4)  # quantised query rows + head weights
-        alg_bytes = n_keys * (key_b + 4) + q_b  # keys read + scores written + queries
         peaks = measured_peaks()
-        peak = float(peaks["hbm_gbs"])
-        achieved = alg_bytes / (score_ms / 1e3) / 1e9
         sha = source_sha("indexer_mma.cu", "topk.cuh", "sm100.cuh", "common.cuh", "kernels.cuh")
         traffic = recorded_traffic("index_mma_kernel", wl.name, sha)
-        roof = {"bound": "hbm", "kernel": "index_mma_kernel (tensor-core indexer scoring)", "achieved": round(achieved, 1),
-                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                "traffic": traffic, "algorithmic_bytes": alg_bytes, "ms_per_launch": round(score_ms, 4),
-                "peak_source": peaks["source"] + " hbm_gbs",
-                "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()}, "hca_stage_ms": hca_ms}
+        common = {"kernel": "index_mma_kernel (tensor-core indexer scoring)", "traffic": traffic,
+                  "ms_per_launch": round(score_ms, 4), "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+                  "hca_stage_ms": hca_ms}
+        if cw.T > 1:
+            # chunked prefill: the scoring is a contraction of T queries x 64 heads
+            # against every visible key; it is bound by the tensor pipe, whose
+            # rate for the key format is the measured sustained bf16 rate x the
+            # nominal ratio (the launch runs inside a multi-millisecond step)
+            n_vis = sum((cw.L - cw.T + t + 1) // cw.m for t in range(cw.T))
+            flops = cw.B * n_vis * 2 * cw.H_I * cw.d_I
+            ratio = TENSOR_RATIO.get(cw.idx_fmt, 1.0)
+            peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * ratio
+            achieved = flops / (score_ms / 1e3) / 1e12
+            roof = dict(bound="tensor", achieved=round(achieved, 1), peak=round(peak, 1), unit="TFLOP/s",
+                        frac=round(achieved / peak, 4), algorithmic_flops=flops,
+                        peak_source=f"{peaks['source']} bf16_tflops_sustained x {ratio:g} ({cw.idx_fmt} / bf16 nominal)",
+                        **common)
+        else:
+            key_b = L.row_bytes(cw.idx_fmt, cw.d_I) + (cw.d_I // 16 if cw.idx_fmt == "fp4" else 4)
+            n_keys = cw.B * cw.n_entries()
+            q_b = cw.B * cw.T * cw.H_I * (key_b + 4)  # quantised query rows + head weights
+            alg_bytes = n_keys * (key_b + 4) + q_b  # keys read + scores written + queries
+            peak = float(peaks["hbm_gbs"])
+            achieved = alg_bytes / (score_ms / 1e3) / 1e9
+            roof = dict(bound="hbm", achieved=round(achieved, 1), peak=peak, unit="GB/s",
+                        frac=round(achieved / peak, 4), algorithmic_bytes=alg_bytes,
+                        peak_source=peaks["source"] + " hbm_gbs", **common)
 
     # ---- end to end: pinned host inputs -> device, step, output -> host
     e2e = None
@@ -383,7 +409,7 @@ def run_lcsc(args):
         "metric": METRIC, "value": round(value, 2), "unit": "queries/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e2m1 x e2m1 block-scaled MMA (indexer), f16 MMA (attention), f32 accumulate and softmax",
+        "dtype": index_dtype(layers_wl) + "f16 MMA (attention), f32 accumulate and softmax",
         "data": "synthetic (seeded Gaussian entries with planted relevant blocks, drawn on device)",
         "config": {"workload": wl.name, "layers": [lw.name for lw in layers_wl], "batch_per_gpu": wl.B,
                    "context": wl.L, "heads": wl.H, "kv_dim": wl.D, "top_k": wl.k, "window": wl.w,

@@ -296,9 +296,11 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
     const int row = q4 * 32 + lane;
     const float* kscale = reinterpret_cast<const float*>(a.key_scale) + (int64_t)b * a.key_cap;
     if constexpr (NQ == 1) {
-      float wr[64];  // head weights in registers
+      uint64_t wr[32];  // head weight pairs (w[2j], w[2j + 1]) in registers
 #pragma unroll
-      for (int j = 0; j < 64; ++j) wr[j] = w_s[j];
+      for (int j = 0; j < 32; ++j) wr[j] = pack2(w_s[2 * j], w_s[2 * j + 1]);
+      const int64_t n_p = ok ? (L - a.T + t0 + 1) / a.m : 0;  // entries the query sees
+      float* score_row = a.scores + ((int64_t)b * a.T + t0) * a.stride;
       for (int i = grp; i < ntile; i += 2) {
         const int ab = i % C::NACC;
         const int64_t g = (tile_lo + i) * 128 + row;
@@ -310,18 +312,27 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
         tmem_ld_32(taddr, r0);
         tmem_ld_32(taddr + 32, r1);
         tmem_ld_wait();
+        // head h of the row in lane pair (h & 7) / 2 of the packed sums
+        uint64_t p2[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          p2[j & 3] = ffma2(wr[j], pack2(fmaxf(__uint_as_float(r0[2 * j]), 0.f), fmaxf(__uint_as_float(r0[2 * j + 1]), 0.f)),
+                            p2[j & 3]);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          p2[j & 3] = ffma2(wr[16 + j], pack2(fmaxf(__uint_as_float(r1[2 * j]), 0.f), fmaxf(__uint_as_float(r1[2 * j + 1]), 0.f)),
+                            p2[j & 3]);
         float p[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) p[j] = 0.f;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) p[j & 7] = fmaf(wr[j], fmaxf(__uint_as_float(r0[j]), 0.f), p[j & 7]);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) p[j & 7] = fmaf(wr[32 + j], fmaxf(__uint_as_float(r1[j]), 0.f), p[j & 7]);
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = unpack2(p2[j]);
+          p[2 * j] = f.x;
+          p[2 * j + 1] = f.y;
+        }
         const float acc = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
-        const int64_t n_p = (L - a.T + t0 + 1) / a.m;
         if (g < n_p) {
           const float v = acc * sk;
-          a.scores[((int64_t)b * a.T + t0) * a.stride + g] = v;
+          score_row[g] = v;
           atomicAdd(&hist_s[float_key(v) >> 20], 1u);
         }
         tc_fence_before();
