@@ -250,15 +250,21 @@ def recorded_traffic(kernel, workload, sha):
 
 
 def dist_setup():
+    """One process per GPU under torchrun: NCCL on GPUs (gloo on a host
+    without one, which the CPU tests use).  Returns (world size, rank, local
+    rank)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws == 1:
         return 1, 0, 0
     import datetime
     import torch.distributed as dist
     rank, local = int(os.environ["RANK"]), int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                            device_id=torch.device("cuda", local))
+    timeout = datetime.timedelta(seconds=120)
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+    else:
+        dist.init_process_group("gloo", timeout=timeout)
     return ws, rank, local
 
 
@@ -269,12 +275,26 @@ def barrier(ws):
 
 
 def max_over_ranks(ws, x):
+    """The largest x over the ranks (every rank gets it)."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def shard_seed(rank, layer):
+    """Seed of a rank's sequences for one layer: every rank owns its own
+    sequences and caches (the decode batch shards by sequence)."""
+    return synth.SEED + 1000 * rank + layer
+
+
+def job_throughput(B, T, ws, steps, ms_total):
+    """Queries per second of the whole job: the queries every rank answered
+    over the slowest rank's time."""
+    return B * T * ws * steps / (ms_total / 1e3)
 
 
 def run_lcsc(args):
@@ -284,7 +304,7 @@ def run_lcsc(args):
     L.load()
     wl = workloads.ALL[args.workload]
     layers_wl = [wl.layer("csa"), wl.layer("hca")] if wl.kind == "pair" else [wl]
-    layers = [Layer(lw, synth.SEED + 1000 * rank + i, dev) for i, lw in enumerate(layers_wl)]
+    layers = [Layer(lw, shard_seed(rank, i), dev) for i, lw in enumerate(layers_wl)]
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
@@ -338,8 +358,7 @@ def run_lcsc(args):
                   for name, a, b in (("compress", 0, 1), ("dense_attn", 1, 2))}
     ms_total = max_over_ranks(ws, start.elapsed_time(stop))
     ms_step = ms_total / args.steps
-    queries = wl.B * wl.T * ws * args.steps
-    value = queries / (ms_total / 1e3)
+    value = job_throughput(wl.B, wl.T, ws, args.steps, ms_total)
 
     # ---- dominant kernel: the CSA indexer scoring (events 2 -> 3 of each step)
     roof = None
@@ -400,7 +419,7 @@ def run_lcsc(args):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(ws, e0.elapsed_time(e1))
-        e2e = {"value": round(wl.B * wl.T * ws * args.e2e_steps / (e2e_ms / 1e3), 2), "unit": "queries/s",
+        e2e = {"value": round(job_throughput(wl.B, wl.T, ws, args.e2e_steps, e2e_ms), 2), "unit": "queries/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if rank != 0:
