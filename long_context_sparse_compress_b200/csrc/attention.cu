@@ -329,6 +329,7 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
   if (attn_mma_supported(a)) {
     cudaError_t e = launch_attn_mma(a, stream);
     if (e != cudaSuccess) return e;
+    if (a.splits == 1) return cudaSuccess;  // one split per query: the kernel wrote the output
     attn_combine_kernel<512><<<dim3(a.B * a.T, a.H / 4), 512, 0, stream>>>(a);
     return cudaGetLastError();
   }

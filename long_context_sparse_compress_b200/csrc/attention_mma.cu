@@ -586,6 +586,29 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
     if (done) done = warp_wait(&pv_done[(ntiles - 1) & 1], (uint32_t)((ntiles - 1) >> 1) & 1u, a, abort);
     tc_fence_after();
     const int64_t pidx = ((int64_t)list * a.splits + blockIdx.x) * a.H + head;
+    // One split per query: the merge with the sink happens here (the same
+    // arithmetic as the split-combine kernel) and O leaves normalised.
+    float o_scale = 1.f;
+    if (a.splits == 1) {
+      float f_own = 0.f;
+      if (s_lane) {
+        const float sigma = a.sink ? a.sink[head] : -INFINITY;
+        const float m = done ? m_ref : -INFINITY, l = done ? l_sum : 0.f;
+        float M = sigma, den = sigma > -INFINITY ? 1.f : 0.f;  // the sink's e^(sigma - M)
+        if (m > M) {
+          den *= M > -INFINITY ? expf(M - m) : 0.f;
+          M = m;
+        }
+        float f = 0.f;
+        if (m > -INFINITY) {
+          f = expf(m - M);
+          den = fmaf(l, f, den);
+        }
+        f_own = den > 0.f ? f * (1.f / den) : 0.f;
+        if (a.lse) a.lse[(int64_t)list * a.H + head] = den > 0.f ? M + logf(den) : -INFINITY;
+      }
+      o_scale = __shfl_sync(0xffffffffu, f_own, (lane & 15) + 16);
+    }
     // O -> shared memory (the K tiles and P are dead: every P V is done),
     // padded rows so the 16-byte stores of a warp's heads hit distinct banks
     float* o_s = reinterpret_cast<float*>(sm + OFF_K);
@@ -599,28 +622,41 @@ __global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
 #pragma unroll
         for (int q = 0; q < 32; q += 4) {
           *reinterpret_cast<float4*>(po + q) =
-              done ? make_float4(__uint_as_float(r0[q]), __uint_as_float(r0[q + 1]), __uint_as_float(r0[q + 2]),
-                                 __uint_as_float(r0[q + 3]))
+              done ? make_float4(__uint_as_float(r0[q]) * o_scale, __uint_as_float(r0[q + 1]) * o_scale,
+                                 __uint_as_float(r0[q + 2]) * o_scale, __uint_as_float(r0[q + 3]) * o_scale)
                    : make_float4(0.f, 0.f, 0.f, 0.f);
           *reinterpret_cast<float4*>(po + 32 + q) =
-              done ? make_float4(__uint_as_float(r1[q]), __uint_as_float(r1[q + 1]), __uint_as_float(r1[q + 2]),
-                                 __uint_as_float(r1[q + 3]))
+              done ? make_float4(__uint_as_float(r1[q]) * o_scale, __uint_as_float(r1[q + 1]) * o_scale,
+                                 __uint_as_float(r1[q + 2]) * o_scale, __uint_as_float(r1[q + 3]) * o_scale)
                    : make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
     }
-    if (s_lane) {
+    if (s_lane && a.splits > 1) {
       a.part_ml[pidx * 2] = done ? m_ref : -INFINITY;
       a.part_ml[pidx * 2 + 1] = done ? l_sum : 0.f;
     }
   }
   tc_fence_before();
   __syncthreads();
-  {  // the partial O of this split, [64 heads][512] contiguous: coalesced 16-byte stores by every thread
+  {  // O of this split, [64 heads][512] contiguous: coalesced stores by every thread, of the
+     // partial (several splits) or of the output in the query's type (one split)
     const float* o_s = reinterpret_cast<const float*>(sm + OFF_K);
-    float4* dst = reinterpret_cast<float4*>(a.part_o + ((int64_t)list * a.splits + blockIdx.x) * a.H * kD);
-    for (int i = tid; i < kH * (kD / 4); i += kThr)
-      dst[i] = *reinterpret_cast<const float4*>(o_s + (i / (kD / 4)) * kOS + 4 * (i % (kD / 4)));
+    auto row4 = [&](int i) { return *reinterpret_cast<const float4*>(o_s + (i / (kD / 4)) * kOS + 4 * (i % (kD / 4))); };
+    if (a.splits > 1) {
+      float4* dst = reinterpret_cast<float4*>(a.part_o + ((int64_t)list * a.splits + blockIdx.x) * a.H * kD);
+      for (int i = tid; i < kH * (kD / 4); i += kThr) dst[i] = row4(i);
+    } else if (a.q_dtype == LCSC_DT_BF16) {
+      uint2* dst = reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) + (int64_t)list * a.H * kD);
+      for (int i = tid; i < kH * (kD / 4); i += kThr) {
+        const float4 v = row4(i);
+        dst[i] = make_uint2((uint32_t)bf16_code(v.x) | ((uint32_t)bf16_code(v.y) << 16),
+                            (uint32_t)bf16_code(v.z) | ((uint32_t)bf16_code(v.w) << 16));
+      }
+    } else {
+      float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + (int64_t)list * a.H * kD);
+      for (int i = tid; i < kH * (kD / 4); i += kThr) dst[i] = row4(i);
+    }
   }
   if (warp == kMmaWarp) {
     tc_fence_after();
