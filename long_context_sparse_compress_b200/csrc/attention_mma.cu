@@ -34,7 +34,7 @@ using namespace sm100;
 constexpr int kH = 64;       // heads (MMA M)
 constexpr int kD = 512;      // row length (K of Q K^T, N of P V)
 constexpr int kTR = 64;      // rows per tile
-constexpr int kLW = 7;       // loader warps (12 warps in all: 3 per SM sub-partition)
+constexpr int kLW = 11;      // loader warps (16 warps in all: 4 per SM sub-partition)
 constexpr int kSW = 4;       // softmax warps
 constexpr int kThr = (kSW + kLW + 1) * 32;
 constexpr int kMmaWarp = kSW + kLW;
@@ -114,7 +114,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return ok;
 }
 
-__global__ void __maxnreg__(168) attn_mma_kernel(const AttnLaunch a) {
+__global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* k_full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
