@@ -554,16 +554,17 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
       if (warp_moved && j > 0) {
         if (!warp_wait(&pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, a, abort)) break;
         tc_fence_after();
-        const float a_own = __shfl_sync(0xffffffffu, alpha, (lane & 15) + 16);
-        for (int c = 0; c < kD; c += 32) {
+        // O's 16 lanes only (the S lanes above them may be taking the next
+        // tile's Q K^T): thread t holds heads t/4 and t/4 + 8 of the warp's 16
+        const float a_lo = __shfl_sync(0xffffffffu, alpha, 16 + (lane >> 2));
+        const float a_hi = __shfl_sync(0xffffffffu, alpha, 16 + (lane >> 2) + 8);
+        for (int c = 0; c < kD; c += 64) {
           uint32_t r[32];
-          tmem_ld_32(row_addr + c, r);
+          tmem_ld_16x256b_x8(row_addr + c, r);
           tmem_ld_wait(r);
-          if (lane < 16) {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * a_own);
-          }
-          tmem_st_32(row_addr + c, r);
+          for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * (((q >> 1) & 1) ? a_hi : a_lo));
+          tmem_st_16x256b_x8(row_addr + c, r);
         }
         tmem_st_wait();
       }

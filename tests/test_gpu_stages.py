@@ -269,6 +269,57 @@ def test_attention_matches_oracle(cuda_lib, kind, fmt_kv):
             assert np.allclose(lse_gpu[b, t], ls, rtol=1e-4, atol=1e-4)
 
 
+@pytest.mark.parametrize("T", [64, 160])  # two splits per query (combined) / one split (written directly)
+def test_attention_rescales_when_the_max_grows(cuda_lib, T):
+    """Scores that jump by more than e^8 part-way through a split: the running
+    reference max moves and the partial O accumulated so far is rescaled.
+    Keys of a few entries point along the queries' shared direction with
+    growing lengths, so every head's max jumps three times."""
+    rng = np.random.default_rng(43)
+    wl = W.CSA_DECODE_128K.with_(k=200, w=100, kind="hca", m=16, G=16, T=T)
+    m, D, H = wl.m, wl.D, wl.H
+    n_ent = 2048
+    L0 = n_ent * m  # context of the last query
+    n_cap = n_ent + 1
+    K = _rows(rng, n_cap, D)
+    u = rng.standard_normal(D)
+    u /= np.linalg.norm(u)
+    q = (u[None, None, :] * 2.0 + rng.standard_normal((1, T, H, D)) * D ** -0.5 * 0.3).astype(np.float32)
+    q = torch.from_numpy(q).to(torch.bfloat16).float().numpy()
+    base = float(np.mean(q[0] @ u))  # typical q . u
+    for first, s_target in ((180, 9.5), (700, 19.0), (1500, 28.5)):
+        for r in range(first, first + 3):
+            K[r] = (u * s_target / (wl.sm_scale * base)).astype(np.float32)
+    kv_st = storage.encode("kv", K, wl.rope_dim)
+    wk_st = storage.encode("kv", _rows(rng, wl.win_cap, D), wl.rope_dim)
+    kv = L.DeviceCache(1, n_cap, "kv", D, wl.rope_dim)
+    wk = L.DeviceCache(1, wl.win_cap, "kv", D, wl.rope_dim)
+    upload(kv, 0, kv_st)
+    upload(wk, 0, wk_st)
+    sink = rng.standard_normal(H).astype(np.float32)
+    ctx = torch.tensor([L0], dtype=torch.int32, device="cuda")
+    out = torch.zeros((1, T, H, D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((1, T, H), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.dense_attn(L.params(wl), dev(q, torch.bfloat16), kv, None, wk, None, dev(sink), ctx, n_cap, out, lse,
+                 status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    o_gpu, lse_gpu = out.float().cpu().numpy(), lse.cpu().numpy()
+    K_all, WK = storage.decode(kv_st), storage.decode(wk_st)
+    for t in list(range(0, T, 16)) + [T - 1]:
+        pp = L0 - T + t
+        n = (pp + 1) // m
+        wpos = window_positions(pp, wl.w) % wl.win_cap
+        Kr = np.concatenate([K_all[:n], WK[wpos]])
+        o, ls = joint_attention(q[0, t], Kr, Kr, sink, wl.sm_scale)
+        assert rel_l2(o_gpu[0, t], o) <= ATTN_RTOL, (t, rel_l2(o_gpu[0, t], o))
+        # the boosted rows are also the values (shared KV), so the output is
+        # far from unit scale: the absolute bound scales with it (bf16 output)
+        assert max_abs(o_gpu[0, t], o) <= ATTN_ATOL * max(1.0, float(np.abs(o).max()))
+        assert np.allclose(lse_gpu[0, t], ls, rtol=1e-4, atol=1e-4)
+
+
 def test_attention_flags_out_of_range_index(cuda_lib):
     rng = np.random.default_rng(41)
     wl = W.CSA_DECODE_4K_F32.with_(k=8, w=4)
