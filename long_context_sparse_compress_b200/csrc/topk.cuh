@@ -83,14 +83,29 @@ __device__ __forceinline__ uint32_t warp_append(uint32_t* counter, bool pred) {
 // consecutive lists (from list0) to the global ones, and the last of the
 // `total_ctas` CTAs that count on counters[done_list][6] turns the complete
 // histograms into each list's threshold bin (counters [2], [3]) for the
-// first k of its n[l] visible scores (lists with n <= k need none).
+// first k of its n[l] visible scores (lists with n <= k need none).  A CTA
+// that built its lists' histograms alone (total_ctas 1) sets the bins from
+// shared memory directly.
 // `hist_s` is nlists x 4096 words of shared memory; every thread of the CTA
 // calls this.
 __device__ __forceinline__ void hist_finish(uint32_t* hist_s, bool flush, int nlists, uint32_t* hist_g,
                                             uint32_t* ctr_g, int64_t list0, int64_t done_list,
                                             unsigned total_ctas, const int64_t* n, int64_t k) {
   __shared__ unsigned last_cta;
+  __shared__ uint32_t warp_tot[32];
+  __shared__ Thresh res;
   __syncthreads();
+  if (total_ctas == 1) {  // this CTA's histograms are the whole ones: no round trip through memory
+    for (int l = 0; l < nlists; ++l) {
+      if (n[l] <= k) continue;  // uniform over the CTA
+      const Thresh t = block_threshold(hist_s + l * kTopkBins, kTopkBins, (uint32_t)k, 256, warp_tot, &res);
+      if (threadIdx.x == 0) {
+        ctr_g[(list0 + l) * 8 + 2] = t.above;
+        ctr_g[(list0 + l) * 8 + 3] = t.bin;
+      }
+    }
+    return;
+  }
   if (flush) {
     for (int i = threadIdx.x; i < nlists * kTopkBins; i += blockDim.x) {
       const uint32_t c = hist_s[i];
@@ -106,8 +121,6 @@ __device__ __forceinline__ void hist_finish(uint32_t* hist_s, bool flush, int nl
   for (int i = threadIdx.x; i < nlists * kTopkBins; i += blockDim.x)
     hist_s[i] = __ldcg(&hist_g[(list0 + i / kTopkBins) * 2 * kTopkBins + i % kTopkBins]);
   __syncthreads();
-  __shared__ uint32_t warp_tot[32];
-  __shared__ Thresh res;
   for (int l = 0; l < nlists; ++l) {
     if (n[l] <= k) continue;  // uniform over the CTA
     const Thresh t = block_threshold(hist_s + l * kTopkBins, kTopkBins, (uint32_t)k, 256, warp_tot, &res);
