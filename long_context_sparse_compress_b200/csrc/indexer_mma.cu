@@ -96,10 +96,19 @@ struct Cfg {
   static constexpr int OFF_SFA = OFF_Q + Q_BYTES;
   static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
   static constexpr int OFF_BAR = OFF_SFB + SFB_BYTES;
-  static constexpr int NBARS = 2 * STAGES + 2 * NACC + 2;
+  // One query (decode, several CTAs per list): the lanes claim their tiles
+  // at run time, BL at a time, from a counter per list, so CTAs on faster
+  // SMs take more (static equal shares ended up to 40% apart).  A lane
+  // publishes each claim to the epilogue through a ring of RING mbarriers.
+  static constexpr bool DYN = NQ == 1;
+  static constexpr int BL = 2;
+  static constexpr int RING = 8;
+  static_assert(!DYN || RING * BL >= BL + STAGES / LANES + 2, "a claim slot is reused only after its tiles are drained");
+  static constexpr int NBARS = 2 * STAGES + 2 * NACC + 2 + (DYN ? LANES * RING : 0);
   static constexpr int OFF_W = OFF_BAR + NBARS * 8;
   static constexpr int OFF_HIST = OFF_W + N * 4;  // NQ x 4096 digit-1 counts of the scores written
-  static constexpr int OFF_TMEM = OFF_HIST + NQ * kTopkBins * 4;
+  static constexpr int OFF_CLM = OFF_HIST + NQ * kTopkBins * 4;  // int32 [LANES][RING] claimed batches
+  static constexpr int OFF_TMEM = OFF_CLM + LANES * RING * 4;
   static constexpr int SMEM = OFF_TMEM + 16 + 1024;  // + slack to align the base
   static_assert(COLS_USED <= 512 && SFA_COL <= COLS_USED, "TMEM budget");
   static_assert(A_BYTES % 1024 == 0 && Q_BYTES % 1024 == 0, "swizzle atoms need 1024-byte alignment");
@@ -141,6 +150,8 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
   uint64_t* acce = accf + C::NACC;     // [NACC] accumulator drained
   uint64_t* qbar = acce + C::NACC;
   uint64_t* sfb_bar = qbar + 1;        // query scales in TMEM (FP4)
+  uint64_t* clm_bar = sfb_bar + 1;     // [LANES][RING] claim published (DYN)
+  int32_t* clm_s = reinterpret_cast<int32_t*>(sm + C::OFF_CLM);
   float* w_s = reinterpret_cast<float*>(sm + C::OFF_W);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_TMEM);
 
@@ -158,8 +169,9 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
   const int64_t n_last = ok ? (L - a.T + t0 + NQ) / a.m : 0;  // N(p) of the group's last query
   const int64_t tiles = (n_last + C::TILE - 1) / C::TILE;
   const int64_t per = (tiles + a.chunks - 1) / a.chunks;
-  const int64_t tile_lo = (int64_t)blockIdx.x * per;
-  const int64_t tile_hi = tile_lo + per < tiles ? tile_lo + per : tiles;
+  const int64_t tile_lo = C::DYN ? 0 : (int64_t)blockIdx.x * per;
+  const int64_t tile_hi = C::DYN ? tiles : (tile_lo + per < tiles ? tile_lo + per : tiles);
+  uint32_t* tile_ctr = a.counters + list0 * 8 + 4;  // claimed batches (DYN), zeroed with the histograms
   if (tile_hi <= tile_lo) {  // uniform over the CTA, before any barrier or TMEM use
     hist_finish(hist_s, false, NQ, a.hist, a.counters, list0, list0, gridDim.x, nvis, a.k);
     return;
@@ -178,6 +190,8 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
     }
     mbar_init(qbar, 1);
     mbar_init(sfb_bar, 1);
+    if (C::DYN)
+      for (int j = 0; j < C::LANES * C::RING; ++j) mbar_init(&clm_bar[j], 1);
     fence_barrier_init();
   }
   for (int i = threadIdx.x; i < C::N; i += blockDim.x) {
@@ -213,14 +227,32 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
         }
       }
       bool live = true;
-      auto load = [&](int i) {  // TMA of tile i into stage i % STAGES
+      int32_t cur = -1;  // the batch claimed for this lane's current BL tiles (DYN)
+      // Global tile of this lane's t-th tile (local index i = r + LANES t), or
+      // -1 past the end; DYN claims a batch on the first tile of each.
+      auto tile_of = [&](int t) -> int64_t {
+        if constexpr (C::DYN) {
+          if (t % C::BL == 0) {
+            const uint32_t gb = atomicAdd(tile_ctr, 1u);
+            cur = (int64_t)gb * C::BL < tiles ? (int32_t)gb : -1;
+            const int c = t / C::BL;
+            clm_s[r * C::RING + c % C::RING] = cur;
+            mbar_arrive(&clm_bar[r * C::RING + c % C::RING]);  // release: the epilogue reads the slot after it
+          }
+          const int64_t g = (int64_t)cur * C::BL + t % C::BL;
+          return cur >= 0 && g < tiles ? g : -1;
+        } else {
+          const int i = r + C::LANES * t;
+          return i < ntile ? tile_lo + i : -1;
+        }
+      };
+      auto load = [&](int i, int64_t tile) {  // TMA of (local) tile i, global tile `tile`, into stage i % STAGES
         const int s = i % C::STAGES;
         const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
         if (!mbar_wait(&empty[s], ph ^ 1u, a.status)) {
           live = false;
           return;
         }
-        const int64_t tile = tile_lo + i;
         mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::SFA_BYTES);
         tma_load_2d(sm + C::OFF_A + s * C::A_BYTES, &tm_k, 0, (int32_t)((int64_t)b * a.key_cap + tile * 128),
                     &full[s]);
@@ -229,8 +261,18 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
           bulk_load(sm + C::OFF_SFA + s * 1024, src, 1024, &full[s]);
         }
       };
-      const int my_n = ntile > r ? (ntile - r + C::LANES - 1) / C::LANES : 0;
-      for (int t = 0; t < C::DIST && t < my_n && live; ++t) load(r + C::LANES * t);
+      int my_n = 0;       // tiles of this lane loaded so far
+      bool more = true;   // whether a next one may exist
+      auto load_next = [&]() {
+        const int64_t tile = tile_of(my_n);
+        if (tile < 0) {
+          more = false;
+          return;
+        }
+        load(r + C::LANES * my_n, tile);
+        ++my_n;
+      };
+      for (int t = 0; t < C::DIST && more && live; ++t) load_next();
       live = live && mbar_wait(qbar, 0, a.status);
       tc_fence_after();
       const uint32_t q_addr = smem_u32(sm + C::OFF_Q);
@@ -247,8 +289,8 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
       const uint32_t idesc = FMT == LCSC_FMT_FP4 ? idesc_mxf4nvf4(128, C::N) : idesc_dense(0, 0, 128, C::N);
       int last = -1;
       for (int t = 0; live && t < my_n; ++t) {
-        if (t + C::DIST < my_n) {
-          load(r + C::LANES * (t + C::DIST));
+        if (more) {  // tile t + DIST
+          load_next();
           if (!live) break;
         }
         const int i = r + C::LANES * t;
@@ -301,9 +343,54 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
       for (int j = 0; j < 32; ++j) wr[j] = pack2(w_s[2 * j], w_s[2 * j + 1]);
       const int64_t n_p = ok ? (L - a.T + t0 + 1) / a.m : 0;  // entries the query sees
       float* score_row = a.scores + ((int64_t)b * a.T + t0) * a.stride;
-      for (int i = grp; i < ntile; i += 2) {
+      // Local tile i = r + LANES t belongs to lane r = i % LANES; this group
+      // takes the lanes r = grp, grp + 2, ... (their tiles in the order i).
+      // Lane r's tiles end where its claims do (DYN) or at ntile.
+      constexpr int NL = C::LANES / 2;
+      int32_t cl[NL];  // lane grp + 2 jj's current claim
+      bool dn[NL];     // and whether its tiles have ended
+#pragma unroll
+      for (int jj = 0; jj < NL; ++jj) {
+        cl[jj] = -1;
+        dn[jj] = false;
+      }
+      int n_dn = 0;
+      for (int i = grp; n_dn < NL; i += 2) {
+        const int r = i % C::LANES, jr = r / 2, tl = i / C::LANES;
+        int64_t gtile;
+        if constexpr (C::DYN) {
+          bool d = false;
+          int32_t c = -1;
+#pragma unroll
+          for (int jj = 0; jj < NL; ++jj)
+            if (jj == jr) {
+              d = dn[jj];
+              c = cl[jj];
+            }
+          if (d) continue;
+          if (tl % C::BL == 0) {  // the lane's next claim
+            const int cb = tl / C::BL;
+            if (!mbar_wait(&clm_bar[r * C::RING + cb % C::RING], (uint32_t)(cb / C::RING) & 1u, a.status)) break;
+            c = clm_s[r * C::RING + cb % C::RING];
+          }
+          gtile = (int64_t)c * C::BL + tl % C::BL;
+          if (c < 0 || gtile >= tiles) {
+            d = true;
+            ++n_dn;
+          }
+#pragma unroll
+          for (int jj = 0; jj < NL; ++jj)
+            if (jj == jr) {
+              dn[jj] = d;
+              cl[jj] = c;
+            }
+          if (d) continue;
+        } else {
+          if (i >= ntile) break;
+          gtile = tile_lo + i;
+        }
         const int ab = i % C::NACC;
-        const int64_t g = (tile_lo + i) * 128 + row;
+        const int64_t g = gtile * 128 + row;
         const float sk = FMT == LCSC_FMT_FP8 ? kscale[g] : 1.f;
         if (!mbar_wait(&accf[ab], (uint32_t)(i / C::NACC) & 1u, a.status)) break;
         tc_fence_after();
