@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(512) topk_hist_kernel(IndexLaunch a, int slice
 
 // All slices of a list: scores above the digit-1 threshold bin go to the
 // output, those in it to the candidate list.
-__global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int slices) {
+__global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int slices, bool set_bins) {
   extern __shared__ float4 slice_s[];  // the slice's scores, one bulk copy
   __shared__ uint64_t bar;
   constexpr int kLocal = 2048;          // candidates gathered in shared memory first
@@ -266,7 +266,23 @@ __global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int sl
     sm100::bulk_load(slice_s, s + li.lo, (uint32_t)(n4 * 16), &bar);
   }
   uint32_t* ctr = a.counters + (int64_t)list * 8;
-  const uint32_t t1 = ctr[3];
+  uint32_t t1;
+  if (set_bins) {  // the list's threshold bin from its complete histogram, while the slice loads
+    __shared__ uint32_t warp_tot[32];
+    __shared__ Thresh res;
+    uint32_t* h = reinterpret_cast<uint32_t*>(cand_s);  // free until the scan
+    const uint32_t* hg = a.hist + (int64_t)list * 2 * kTopkBins;
+    for (int i = threadIdx.x; i < kTopkBins; i += 512) h[i] = __ldcg(&hg[i]);
+    __syncthreads();
+    const Thresh th = block_threshold(h, kTopkBins, (uint32_t)a.k, 256, warp_tot, &res);
+    t1 = th.bin;
+    if (threadIdx.x == 0 && blockIdx.x == 0) {
+      ctr[2] = th.above;
+      ctr[3] = th.bin;
+    }
+  } else {
+    t1 = ctr[3];
+  }
   uint32_t* bits = a.sel_bits + (int64_t)list * a.bit_stride;
   for (int64_t w = li.lo / 32 + threadIdx.x; w < (li.hi + 31) / 32; w += 512) bits[w] = 0u;
   __syncthreads();
@@ -549,7 +565,7 @@ cudaError_t launch_topk(const IndexLaunch& a, cudaStream_t stream) {
   const size_t slice_bytes = (size_t)per_max * 4;
   e = cudaFuncSetAttribute(topk_collect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)slice_bytes);
   if (e != cudaSuccess) return e;
-  topk_collect_kernel<<<tgrid, 512, slice_bytes, stream>>>(a, slices);
+  topk_collect_kernel<<<tgrid, 512, slice_bytes, stream>>>(a, slices, index_bins_in_collect(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   e = cudaFuncSetAttribute(topk_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFinalSmem);
   if (e != cudaSuccess) return e;

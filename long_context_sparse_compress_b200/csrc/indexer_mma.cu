@@ -51,6 +51,7 @@ struct MmaArgs {
   uint32_t* hist;          // top-k digit-1 histograms [B*T][2][4096] (zeroed)
   uint32_t* counters;      // top-k counters [B*T][8] (zeroed)
   int64_t k;               // top-k
+  bool bins_in_collect;    // several CTAs per list: the collect pass sets the threshold bins
   int32_t* status;
 };
 
@@ -173,7 +174,7 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
   const int64_t tile_hi = C::DYN ? tiles : (tile_lo + per < tiles ? tile_lo + per : tiles);
   uint32_t* tile_ctr = a.counters + list0 * 8 + 4;  // claimed batches (DYN), zeroed with the histograms
   if (tile_hi <= tile_lo) {  // uniform over the CTA, before any barrier or TMEM use
-    hist_finish(hist_s, false, NQ, a.hist, a.counters, list0, list0, gridDim.x, nvis, a.k);
+    hist_finish(hist_s, false, NQ, a.hist, a.counters, list0, list0, gridDim.x, nvis, a.k, !a.bins_in_collect);
     return;
   }
   for (int i = threadIdx.x; i < NQ * kTopkBins; i += blockDim.x) hist_s[i] = 0u;
@@ -503,7 +504,7 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
-  hist_finish(hist_s, true, NQ, a.hist, a.counters, list0, list0, gridDim.x, nvis, a.k);
+  hist_finish(hist_s, true, NQ, a.hist, a.counters, list0, list0, gridDim.x, nvis, a.k, !a.bins_in_collect);
 }
 
 // ---------------------------------------------------------------- host side
@@ -571,6 +572,7 @@ cudaError_t launch_mma(const IndexLaunch& a, cudaStream_t stream) {
   const int groups = a.T / NQ;
   const int64_t ctas = (int64_t)a.B * groups;
   m.chunks = ctas >= sm_count() ? 1 : (int)(sm_count() / ctas);
+  m.bins_in_collect = index_bins_in_collect(a);
   auto kern = index_mma_kernel<FMT, NQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
@@ -579,6 +581,12 @@ cudaError_t launch_mma(const IndexLaunch& a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+bool index_bins_in_collect(const IndexLaunch& a) {
+  // the one-query tensor-core configuration with several CTAs per list
+  if (!index_mma_supported(a) || (a.keys.f.fmt == LCSC_FMT_FP8 && a.T % 4 == 0)) return false;
+  return (int64_t)a.B * a.T < sm_count();
+}
 
 bool index_mma_supported(const IndexLaunch& a) {
   const int fmt = a.keys.f.fmt;

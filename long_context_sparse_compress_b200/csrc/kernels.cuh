@@ -77,6 +77,10 @@ cudaError_t launch_index_topk(const IndexLaunch& a, cudaStream_t stream);
 // multiple of 128); index_mma_supported() tells whether it applies.
 bool index_mma_supported(const IndexLaunch& a);
 cudaError_t launch_index_mma(const IndexLaunch& a, cudaStream_t stream);
+// True when the tensor-core scoring runs several CTAs per list with one query
+// each: its CTAs then only add up the digit-1 histograms, and the collect
+// pass of the top-k sets each list's threshold bin while its slice loads.
+bool index_bins_in_collect(const IndexLaunch& a);
 
 struct AttnLaunch {
   const void* q;        // [B][T][H][D]

@@ -85,12 +85,14 @@ __device__ __forceinline__ uint32_t warp_append(uint32_t* counter, bool pred) {
 // histograms into each list's threshold bin (counters [2], [3]) for the
 // first k of its n[l] visible scores (lists with n <= k need none).  A CTA
 // that built its lists' histograms alone (total_ctas 1) sets the bins from
-// shared memory directly.
+// shared memory directly; with set_bins false the CTAs only add their
+// histograms and a later kernel (the collect pass) sets the bins.
 // `hist_s` is nlists x 4096 words of shared memory; every thread of the CTA
 // calls this.
 __device__ __forceinline__ void hist_finish(uint32_t* hist_s, bool flush, int nlists, uint32_t* hist_g,
                                             uint32_t* ctr_g, int64_t list0, int64_t done_list,
-                                            unsigned total_ctas, const int64_t* n, int64_t k) {
+                                            unsigned total_ctas, const int64_t* n, int64_t k,
+                                            bool set_bins = true) {
   __shared__ unsigned last_cta;
   __shared__ uint32_t warp_tot[32];
   __shared__ Thresh res;
@@ -112,6 +114,7 @@ __device__ __forceinline__ void hist_finish(uint32_t* hist_s, bool flush, int nl
       if (c) atomicAdd(&hist_g[(list0 + i / kTopkBins) * 2 * kTopkBins + i % kTopkBins], c);
     }
   }
+  if (!set_bins) return;  // the next kernel takes the bins from the flushed histograms
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) last_cta = atomicAdd(&ctr_g[done_list * 8 + 6], 1u) == total_ctas - 1 ? 1u : 0u;
