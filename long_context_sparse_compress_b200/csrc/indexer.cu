@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int sl
   extern __shared__ float4 slice_s[];  // the slice's scores, one bulk copy
   __shared__ uint64_t bar;
   constexpr int kLocal = 2048;          // candidates gathered in shared memory first
-  __shared__ uint2 cand_s[kLocal];
+  __shared__ __align__(16) uint2 cand_s[kLocal];  // (16-byte aligned: also the histogram, read as uint4)
   __shared__ uint32_t n_local, base_g;
   const int list = blockIdx.y;
   const ListInfo li = list_info(a, list, slices);
@@ -271,8 +271,11 @@ __global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int sl
     __shared__ uint32_t warp_tot[32];
     __shared__ Thresh res;
     uint32_t* h = reinterpret_cast<uint32_t*>(cand_s);  // free until the scan
-    const uint32_t* hg = a.hist + (int64_t)list * 2 * kTopkBins;
-    for (int i = threadIdx.x; i < kTopkBins; i += 512) h[i] = __ldcg(&hg[i]);
+    const uint4* hg = reinterpret_cast<const uint4*>(a.hist + (int64_t)list * 2 * kTopkBins);
+    static_assert(kTopkBins == 2 * 4 * 512, "two 16-byte loads per thread");
+    const uint4 v0 = __ldcg(&hg[threadIdx.x]), v1 = __ldcg(&hg[threadIdx.x + 512]);
+    reinterpret_cast<uint4*>(h)[threadIdx.x] = v0;
+    reinterpret_cast<uint4*>(h)[threadIdx.x + 512] = v1;
     __syncthreads();
     const Thresh th = block_threshold(h, kTopkBins, (uint32_t)a.k, 256, warp_tot, &res);
     t1 = th.bin;
