@@ -352,6 +352,17 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
     };
     // One step: tile j+1 located and requested, tile j stored.  false: stop.
     auto step = [&](int j, const uint4 (&cur)[kLoads], uint4 (&nxt)[kLoads]) -> bool {
+      if (!a.idx && lt == 0 && j + 2 < ntiles) {
+        // dense entries are contiguous: tile j+2's rows go to L2 now, in one
+        // bulk prefetch, a step before their loads are issued (rows are
+        // 576 B from a 16-byte-aligned base, so the start is aligned)
+        const int64_t g0 = slot_of(j + 2) - lt;
+        const int64_t hi = s_hi < qr.n_ent_slots ? s_hi : qr.n_ent_slots;
+        if (g0 < hi) {
+          const int64_t cnt = hi - g0 < kTR ? hi - g0 : kTR;
+          prefetch_l2(a.kv.row(b, g0), (uint32_t)(cnt * a.kv.f.row_bytes));
+        }
+      }
       if (lt < kTR) {
         scl_s[(j & 3) * kTR + lt] = sc_next;  // tile j's scale, loaded one step ago
         const bool nrm = sc_next >= 6.103515625e-05f && sc_next <= 65504.f;
