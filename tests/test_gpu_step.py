@@ -22,6 +22,9 @@ CASES = {
     "csa_fp8_prefill": (W.CSA_PREFILL_256K.with_(B=2, T=40, n_planted=8), [4096 + 40, 2002]),
     "hca_prefill": (W.HCA_DECODE_64K.with_(B=1, T=130), [4096 + 130]),
     "csa_overlap_decode": (W.CSA_DECODE_128K.with_(B=2, G=8), [8192, 1001]),
+    # the 2,048-token window reading of the pages, without a sink
+    "csa_window2048_nosink": (W.CSA_DECODE_128K.with_(B=2, w=2048, sink=False), [12000, 1500]),
+    "hca_window2048_nosink": (W.HCA_DECODE_64K.with_(B=2, w=2048, sink=False), [16384, 2000]),
 }
 
 
