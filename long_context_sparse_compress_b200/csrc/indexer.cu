@@ -45,14 +45,15 @@ __device__ __forceinline__ int64_t visible(const IndexLaunch& a, int b, int t, b
 // ------------------------------------------------ indexer query quantisation
 // One warp per (b, t, h) row: the query row is stored in the key format.
 template <int VPL>
-__global__ void __launch_bounds__(256) quantize_queries_kernel(IndexLaunch a) {
+__global__ void __launch_bounds__(256) quantize_queries_kernel(IndexLaunch a, bool zero_hist) {
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
-  {  // the top-k's digit-1 histograms and counters start at zero
+  {  // the top-k's counters, and the digit-1 histograms when they are summed in memory, start at zero
     const int64_t lists = (int64_t)a.B * a.T;
-    const int64_t n_zero = lists * (kTopkBins + 8);
+    const int64_t nh = zero_hist ? lists * kTopkBins : 0;
+    const int64_t n_zero = nh + lists * 8;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_zero; i += (int64_t)gridDim.x * blockDim.x) {
-      if (i < lists * kTopkBins) a.hist[(i / kTopkBins) * 2 * kTopkBins + i % kTopkBins] = 0u;
-      else a.counters[i - lists * kTopkBins] = 0u;
+      if (i < nh) a.hist[(i / kTopkBins) * 2 * kTopkBins + i % kTopkBins] = 0u;
+      else a.counters[i - nh] = 0u;
     }
   }
   const int64_t row = (int64_t)blockIdx.x * 8 + warp;  // over B*T*H_I
@@ -521,9 +522,12 @@ cudaError_t launch_index_quantize(const IndexLaunch& a, cudaStream_t stream) {
   const int lists = a.B * a.T;
   const int64_t q_rows = (int64_t)lists * a.H_I;
   const unsigned qgrid = (unsigned)((q_rows + 7) / 8);
+  // tensor-core scoring with one CTA per list group keeps its histograms in
+  // shared memory: the global ones are then never read
+  const bool zero_hist = !index_mma_supported(a) || index_bins_in_collect(a) || !index_whole_lists(a);
   switch (a.d_I) {
-    case 128: quantize_queries_kernel<4><<<qgrid, 256, 0, stream>>>(a); break;
-    case 32: quantize_queries_kernel<1><<<qgrid, 256, 0, stream>>>(a); break;
+    case 128: quantize_queries_kernel<4><<<qgrid, 256, 0, stream>>>(a, zero_hist); break;
+    case 32: quantize_queries_kernel<1><<<qgrid, 256, 0, stream>>>(a, zero_hist); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -582,6 +582,12 @@ cudaError_t launch_mma(const IndexLaunch& a, cudaStream_t stream) {
 
 }  // namespace
 
+bool index_whole_lists(const IndexLaunch& a) {
+  // as launch_mma sizes the grid: one CTA per query group once the groups fill the GPU
+  const int nq = a.keys.f.fmt == LCSC_FMT_FP8 && a.T % 4 == 0 ? 4 : 1;
+  return index_mma_supported(a) && (int64_t)a.B * (a.T / nq) >= sm_count();
+}
+
 bool index_bins_in_collect(const IndexLaunch& a) {
   // the one-query tensor-core configuration with several CTAs per list
   if (!index_mma_supported(a) || (a.keys.f.fmt == LCSC_FMT_FP8 && a.T % 4 == 0)) return false;

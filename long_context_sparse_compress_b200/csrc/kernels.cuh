@@ -81,6 +81,9 @@ cudaError_t launch_index_mma(const IndexLaunch& a, cudaStream_t stream);
 // each: its CTAs then only add up the digit-1 histograms, and the collect
 // pass of the top-k sets each list's threshold bin while its slice loads.
 bool index_bins_in_collect(const IndexLaunch& a);
+// True when the tensor-core scoring runs one CTA per query group (each CTA
+// builds its lists' histograms whole, in shared memory).
+bool index_whole_lists(const IndexLaunch& a);
 
 struct AttnLaunch {
   const void* q;        // [B][T][H][D]
