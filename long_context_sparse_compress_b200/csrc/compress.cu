@@ -18,6 +18,7 @@
 #include <type_traits>
 
 #include "kernels.cuh"
+#include "sm100.cuh"
 
 namespace lcsc {
 namespace {
@@ -26,19 +27,28 @@ constexpr int kRows = 128;   // token rows per CTA
 constexpr int kThreads = 256;
 constexpr int kMaxEnt = 32;  // entries per CTA (their pooled rows wait in shared memory)
 
-// Dynamic shared memory of pool_kernel: x tile, then the W chunk (reused for
-// z and the biases), then the pooled rows [kMaxEnt][NC].
+// Dynamic shared memory of pool_kernel (from a 1024-byte-aligned base): x
+// tile, then the W chunk (reused for z and the biases), then the pooled rows
+// [kMaxEnt][NC].  bf16: x and W in the tensor cores' 128-byte-swizzled
+// layouts (x as DIM / 64 blocks of [128 rows][128 B], W as [DIM][NC = 64
+// channels = 128 B]); fp32: padded rows for the CUDA-core GEMM.
 template <bool kBf16, int DIM, int NC>
 __host__ __device__ constexpr size_t pool_smem_offset() {
   constexpr size_t elem = kBf16 ? 2 : 4;
-  constexpr size_t xs = elem * kRows * (kBf16 ? DIM + 8 : DIM + 1);
-  constexpr size_t wz = elem * DIM * (kBf16 ? NC + 8 : NC + 1);
+  constexpr size_t xs = elem * kRows * (kBf16 ? DIM : DIM + 1);
+  constexpr size_t wz = elem * DIM * (kBf16 ? NC : NC + 1);
   constexpr size_t zb = sizeof(float) * (kRows * (NC + 1) + kRows * NC);  // z, then biases of <= 128 tokens
   return xs + (wz > zb ? wz : zb);
 }
 template <bool kBf16, int DIM, int NC>
 __host__ __device__ constexpr size_t pool_smem_bytes() {
-  return pool_smem_offset<kBf16, DIM, NC>() + sizeof(float) * kMaxEnt * NC;
+  return pool_smem_offset<kBf16, DIM, NC>() + sizeof(float) * kMaxEnt * NC + 1024;  // + base alignment
+}
+
+// Byte offset of (row, byte) in a [rows][128 B] array with the 128-byte
+// swizzle (16-byte chunk index XOR row % 8) that the tensor cores read.
+__device__ __forceinline__ uint32_t swz128(int row, int byte) {
+  return (uint32_t)(row * 128 + ((((byte >> 4) ^ (row & 7)) << 4) | (byte & 15)));
 }
 
 struct SeqSpan {
@@ -195,10 +205,12 @@ __device__ __forceinline__ void store_entries(const CompressLaunch& a, const flo
 template <bool kBf16, int DIM, int NC, bool kFused>
 __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E, bool packed) {
   using Elem = typename std::conditional<kBf16, uint16_t, float>::type;
-  constexpr int XS = kBf16 ? DIM + 8 : DIM + 1;   // x tile row stride (elements)
-  constexpr int WS = kBf16 ? NC + 8 : NC + 1;     // W chunk row stride
+  constexpr int XS = kBf16 ? DIM : DIM + 1;       // x tile row stride (elements; fp32 path)
+  constexpr int WS = kBf16 ? NC : NC + 1;         // W chunk row stride (fp32 path)
   constexpr int ZS = NC + 1;                      // z tile row stride (floats)
-  extern __shared__ __align__(16) uint8_t smem[];
+  static_assert(!kBf16 || NC == 64, "bf16 W chunk rows are one 128-byte swizzle row");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Elem* xs = reinterpret_cast<Elem*>(smem);
   Elem* ws = reinterpret_cast<Elem*>(smem + sizeof(Elem) * kRows * XS);
   float* zs = reinterpret_cast<float*>(ws);  // reuses the W chunk after the GEMM
@@ -300,15 +312,17 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
   const Elem* wg = reinterpret_cast<const Elem*>(a.w);
   constexpr int VEC = 16 / sizeof(Elem);
   const int x_rows = kBf16 ? rows_used : kRows;
-  if constexpr (kBf16) {
+  uint8_t* xb = reinterpret_cast<uint8_t*>(xs);
+  uint8_t* wb = reinterpret_cast<uint8_t*>(ws);
+  if constexpr (kBf16) {  // straight into the swizzled layouts (rows past x_rows are never read back)
     for (int i = tid; i < x_rows * (DIM / VEC); i += kThreads) {
       const int r = i / (DIM / VEC), cv = (i % (DIM / VEC)) * VEC;
       const bool live = row_src[r] >= 0;
-      cp_async16(xs + r * XS + cv, live ? xg + row_src[r] + cv : xg, live);
+      cp_async16(xb + (cv / 64) * (kRows * 128) + swz128(r, (cv % 64) * 2), live ? xg + row_src[r] + cv : xg, live);
     }
     for (int i = tid; i < DIM * (NC / VEC); i += kThreads) {
       const int k = i / (NC / VEC), cv = (i % (NC / VEC)) * VEC;
-      cp_async16(ws + k * WS + cv, wg + (int64_t)k * DIM + c0 + cv, true);
+      cp_async16(wb + swz128(k, cv * 2), wg + (int64_t)k * DIM + c0 + cv, true);
     }
     cp_async_wait_all();
   } else {
@@ -328,38 +342,54 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
       for (int j = 0; j < 4; ++j) ws[k * WS + cv + j] = f[j];
     }
   }
-  // rows past the used ones are zero (read by the GEMM's last row block)
-  for (int i = tid; i < (((x_rows + 15) & ~15) - x_rows) * XS; i += kThreads) xs[x_rows * XS + i] = Elem(0);
+  // rows past the used ones are zero (fp32 path: read by the GEMM's last row block)
+  if constexpr (!kBf16)
+    for (int i = tid; i < (((x_rows + 15) & ~15) - x_rows) * XS; i += kThreads) xs[x_rows * XS + i] = Elem(0);
   __syncthreads();
 
   // ---- z = x W for the 128 x NC tile
   if constexpr (kBf16) {
+    // tcgen05: M = 128 token rows, N = 64 channels, K = DIM; x is the K-major
+    // A operand, the W chunk the MN-major B operand; z lands in 64 TMEM columns
+    __shared__ uint64_t mma_bar;
+    __shared__ uint32_t tm_slot;
     const int warp = tid / kWarp, lane = tid % kWarp;
-    float acc[NC / 8][4];
-#pragma unroll
-    for (int j = 0; j < NC / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-    const int ks_end = warp * 16 < rows_used ? DIM / 16 : 0;  // row blocks past the used rows stay zero
-#pragma unroll 4
-    for (int ks = 0; ks < ks_end; ++ks) {
-      uint32_t af[4];
-      ldsm_x4(af, xs + (warp * 16 + (lane % 16)) * XS + ks * 16 + (lane / 16) * 8);
-#pragma unroll
-      for (int j = 0; j < NC / 8; j += 2) {
-        uint32_t bf[4];
-        ldsm_x4_t(bf, ws + (ks * 16 + (lane % 8) + ((lane / 8) % 2) * 8) * WS + j * 8 + (lane / 16) * 8);
-        mma_bf16(acc[j], af, bf[0], bf[1]);
-        mma_bf16(acc[j + 1], af, bf[2], bf[3]);
-      }
+    if (tid == 0) {
+      sm100::mbar_init(&mma_bar, 1);
+      sm100::fence_barrier_init();
     }
-    __syncthreads();  // the W chunk is dead: z reuses it
-    const int g = lane / 4, t = lane % 4;
+    if (warp == 0) sm100::tmem_alloc(&tm_slot, 64);
+    sm100::fence_async_smem();  // the cp.async bytes, for the tensor cores
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tmem = tm_slot;
+    if (tid == 0) {
+      const uint32_t xa = sm100::smem_u32(xb), wa = sm100::smem_u32(wb);
+      const uint32_t idesc = sm100::idesc_dense(1, 1, 128, NC, false, true);
+#pragma unroll 4
+      for (int kk = 0; kk < DIM / 16; ++kk)
+        sm100::mma_ss<0>(tmem,
+                         sm100::smem_desc(xa + (kk / 4) * (kRows * 128) + (kk % 4) * 32, 16, 1024, sm100::kSw128),
+                         sm100::smem_desc(wa + kk * 2048, 8192, 1024, sm100::kSw128), idesc, kk > 0);
+      sm100::tc_commit(&mma_bar);
+    }
+    sm100::mbar_wait(&mma_bar, 0, a.status);
+    sm100::tc_fence_after();
+    __syncthreads();  // the MMAs are done with the W chunk: z reuses it
+    {  // warp w: rows 32 (w % 4) .., columns 32 (w / 4) ..
+      uint32_t r[32];
+      sm100::tmem_ld_32(tmem + ((uint32_t)(32 * (warp % 4)) << 16) + 32 * (warp / 4), r);
+      sm100::tmem_ld_wait(r);
+      const int row = 32 * (warp % 4) + lane;
 #pragma unroll
-    for (int j = 0; j < NC / 8; ++j) {
-      const int col = j * 8 + 2 * t;
-      zs[(warp * 16 + g) * ZS + col] = acc[j][0];
-      zs[(warp * 16 + g) * ZS + col + 1] = acc[j][1];
-      zs[(warp * 16 + g + 8) * ZS + col] = acc[j][2];
-      zs[(warp * 16 + g + 8) * ZS + col + 1] = acc[j][3];
+      for (int q = 0; q < 32; ++q) zs[row * ZS + 32 * (warp / 4) + q] = __uint_as_float(r[q]);
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+      sm100::tc_fence_after();
+      sm100::tmem_dealloc(tmem, 64);
     }
   } else {
     constexpr int RG = kThreads / NC;          // row groups
@@ -408,7 +438,10 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
     // evenly no token index needs a guard, so the loads of the four overlap.
     auto logit = [&](int j, int r) { return zs[r * ZS + c] + bs[j * NC + c]; };
     auto xval = [&](int r) -> float {
-      if constexpr (kBf16) return bf16_val(xs[r * XS + c0 + c]);
+      if constexpr (kBf16) {
+        const int d = c0 + c;
+        return bf16_val(*reinterpret_cast<const uint16_t*>(xb + (d / 64) * (kRows * 128) + swz128(r, (d % 64) * 2)));
+      }
       else return xs[r * XS + c0 + c];
     };
     auto ex = [](float v) -> float {
