@@ -278,8 +278,8 @@ typedef struct lcsc_step {
   /* Optional stage timing (host array of cudaEvent_t, or NULL): event i is
    * recorded on `stream` at stage boundary i while i < n_events.
    * CSA: 0 start, 1 after the KV latent's compression, 2 once the indexer
-   * keys' compression and the query quantisation (which run beside it on a
-   * second stream of the library's) are also done, 3 after indexer
+   * keys' compression and the query quantisation (which run beside it on two
+   * more streams of the library's) are also done, 3 after indexer
    * scoring, 4 after top-k, 5 after attention.  HCA: 0 start, 1 after
    * compression, 2 after attention. */
   void* const* events;

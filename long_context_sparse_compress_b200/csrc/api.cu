@@ -501,14 +501,14 @@ static int32_t step_compress(const lcsc_params* p, const lcsc_step* s, int32_t t
   return LCSC_OK;
 }
 
-// A second stream per device for the parts of a CSA step that do not depend
+// Two more streams per device for the parts of a CSA step that do not depend
 // on each other (the indexer keys' compression and the query quantisation
-// run beside the KV latent's compression), with its fork / join events.
+// each run beside the KV latent's compression), with fork / join events.
 // Enqueueing on it is serialised by a mutex; the work itself is ordered
 // only by the events.
 struct SideStream {
-  cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaStream_t s = nullptr, s2 = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr, join2 = nullptr;
 };
 constexpr int kMaxSideDevices = 64;
 std::mutex g_side_mu;
@@ -522,8 +522,10 @@ cudaError_t side_stream(SideStream** out) {
   SideStream& ss = g_side[dev];
   if (!ss.s) {
     if ((e = cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithFlags(&ss.s2, cudaStreamNonBlocking)) != cudaSuccess) return e;
     if ((e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
     if ((e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&ss.join2, cudaEventDisableTiming)) != cudaSuccess) return e;
   }
   *out = &ss;
   return cudaSuccess;
@@ -588,19 +590,22 @@ static int32_t step_impl(const lcsc_params* p, const lcsc_step* s, void* ws, siz
   };
   if ((e = mark()) != cudaSuccess) return cuda_fail(e);
   if (csa) {
-    // fork: indexer keys + query quantisation on the side stream
+    // fork: indexer keys and query quantisation on two side streams
     std::lock_guard<std::mutex> lock(g_side_mu);
     SideStream* ss = nullptr;
     if ((e = side_stream(&ss)) != cudaSuccess) return cuda_fail(e);
     if ((e = cudaEventRecord(ss->fork, strm)) != cudaSuccess) return cuda_fail(e);
     if ((e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaStreamWaitEvent(ss->s2, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
     if ((e = launch_compress(ci, ss->s)) != cudaSuccess) return cuda_fail(e);
-    if ((e = launch_index_quantize(il, ss->s)) != cudaSuccess) return cuda_fail(e);
     if ((e = cudaEventRecord(ss->join, ss->s)) != cudaSuccess) return cuda_fail(e);
+    if ((e = launch_index_quantize(il, ss->s2)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaEventRecord(ss->join2, ss->s2)) != cudaSuccess) return cuda_fail(e);
     if ((e = launch_compress(ck, strm)) != cudaSuccess) return cuda_fail(e);
     if (sep && (e = launch_compress(cvv, strm)) != cudaSuccess) return cuda_fail(e);
     if ((e = mark()) != cudaSuccess) return cuda_fail(e);
     if ((e = cudaStreamWaitEvent(strm, ss->join, 0)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaStreamWaitEvent(strm, ss->join2, 0)) != cudaSuccess) return cuda_fail(e);
   } else {
     if ((e = launch_compress(ck, strm)) != cudaSuccess) return cuda_fail(e);
     if (sep && (e = launch_compress(cvv, strm)) != cudaSuccess) return cuda_fail(e);
