@@ -15,10 +15,11 @@
 //    s = sk[g] * sum_h (w[h] sq[h]) ReLU(acc[h]).
 // Warp roles (one CTA per SM).  One thread's issue of TMA and
 // tcgen05 instructions (tens of cycles each) is what limits a single
-// pipeline, so tiles are dealt round-robin to LANES lanes (warps 0 .. LANES-1,
-// one thread each): lane r loads its tiles with TMA (hardware swizzle) into a
-// STAGES-deep ring, DIST of its tiles ahead, and issues their MMAs into NACC
-// TMEM accumulators.  Groups of four epilogue warps drain the accumulators
+// pipeline, so tiles go to LANES lanes (warps 0 .. LANES-1, one thread each):
+// round-robin over the CTA's share with four queries, claimed two at a time
+// from a counter per list with one (several CTAs share a list).  Lane r loads
+// its tiles with TMA (hardware swizzle) into a STAGES-deep ring, DIST of its
+// tiles ahead, and issues their MMAs into NACC TMEM accumulators.  Groups of four epilogue warps drain the accumulators
 // with tcgen05.ld, apply ReLU and the head weights, write one fp32 score per
 // (query, key) and count it in the list's shared-memory histogram of the
 // top-k's first digit.  One query (384 threads): two groups take alternate
