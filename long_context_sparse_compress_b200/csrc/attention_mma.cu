@@ -8,11 +8,12 @@
 //
 // One CTA owns (query, range of rows) and walks it in tiles of 64 rows with a
 // warp-specialised pipeline:
-//  * 7 loader warps resolve the tile's rows (gathered by index for CSA), read
-//    them and dequantise them once into shared memory as f16, in a
-//    128-byte-swizzled layout that is both a K-major operand for Q K^T and an
-//    MN-major operand for P V (the same bytes are K and V); two buffers, so
-//    tile t+1 is loaded while tile t is being used;
+//  * 11 loader warps resolve the tile's rows (gathered by index for CSA; dense
+//    tiles are also prefetched into L2 two tiles ahead), read them and
+//    dequantise them once into shared memory as f16, in a 128-byte-swizzled
+//    layout that is both a K-major operand for Q K^T and an MN-major operand
+//    for P V (the same bytes are K and V); two buffers, so tile t+1 is loaded
+//    while tile t is being used;
 //  * 1 MMA warp issues S = Q K^T (M = 64 heads, N = 64 rows, K = 512) for tile
 //    t+1 as soon as it is loaded, and O += P V (N = 2 x 256 dims, K = 64) for
 //    tile t once its probabilities are ready;
@@ -21,8 +22,9 @@
 //    and write P = exp(S - ref) as f16.
 // Heads live on M = 64, so S and O use the half-lane TMEM layout: O at
 // lanes 0-15 of each 32-lane sub-partition (all 512 columns), S (two
-// 64-column buffers) at lanes 16-31.  The partial (ref max, sum, O) goes to
-// the workspace the combine kernel merges.
+// 64-column buffers) at lanes 16-31.  With several splits per query the
+// partial (ref max, sum, O) goes to the workspace the combine kernel merges;
+// with one, the kernel merges the sink itself and writes the output.
 #include "kernels.cuh"
 #include "sm100.cuh"
 

@@ -10,10 +10,13 @@
 // Kernel design: a CTA owns up to 128 consecutive token rows (E whole groups
 // plus the G - m rows of history an overlapping group needs) and 64 output
 // channels.  The gate logits z = x W are a [128 x dim] x [dim x 64] GEMM
-// (bf16 tensor-core mma for bf16 rows, FP32 FMA for fp32 rows); the group
-// softmax and the weighted sum run on the tile in shared memory, and the
-// pooled fp32 rows go to scratch.  A second kernel stores each pooled row
-// (whole row needed for the FP8 amax) and the raw window rows.
+// (tcgen05 with the accumulator in TMEM for bf16 rows, FP32 FMA for fp32
+// rows); the group softmax and the weighted sum run on the tile in shared
+// memory.  The channel blocks of the same entries form a thread-block cluster
+// that exchanges the FP8 amax through distributed shared memory and stores
+// the entries and the raw window rows itself; when the grid's clusters cannot
+// all be resident at once, the pooled fp32 rows go to scratch and a second
+// kernel stores them (whole rows, for the amax) and the window rows.
 #include <cooperative_groups.h>
 #include <type_traits>
 

@@ -15,8 +15,9 @@
 // Top-k is an exact radix select on the order-preserving integer image of
 // the float scores, three digits of 12 / 12 / 8 bits:
 //   digit 1: histogrammed while the scores are written (tensor-core scoring)
-//          or by a pass over them; the last CTA of a list finds the
-//          threshold bin;
+//          or by a pass over them; the threshold bin is found by the CTA
+//          that scored the list alone, else by the collect pass (several
+//          tensor-core scoring CTAs per list), else by the pass's last CTA;
 //   collect (all slices of a list): scores above the threshold bin are
 //          marked in the list's selection bitmap, those in it become
 //          candidates;
