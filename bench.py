@@ -149,17 +149,24 @@ class Layer:
 
 
 def kernels_per_step(wl):
-    """Kernels of this library one step launches.  CSA: the fused pool +
-    store of the KV latent and of the indexer keys (2: each grid is one
-    cluster of channel blocks), query quantisation + scoring (2), top-k
-    collect + final (2, plus a histogram pass when the scores come from the
-    CUDA-core scoring kernel), attention partial + combine (2).  HCA: pool +
-    store (2: sixteen 8-CTA clusters do not fit at once, so the store runs as
-    its own kernel), attention partial + combine (2)."""
+    """Kernels of this library one step of a benchmark workload launches (the
+    bench reports the library's own count of the timed region and checks it
+    against this).  CSA: pooling of the indexer keys (1: one cluster of
+    channel blocks per 128 new rows stores the rows itself) and of the KV
+    latent (1 when its clusters fit on the GPU at once, as in decode; else 2,
+    pooling then a store pass, as in prefill), query quantisation + scoring
+    (2), top-k collect + final (2, plus a histogram pass when the scores come
+    from the CUDA-core scoring kernel), attention (2 with several splits per
+    query, the partials then a combine pass, as in decode; 1 with one split,
+    as in prefill, where the kernel writes the output).  HCA decode: pooling
+    + store (2: its sixteen 8-CTA clusters do not fit at once), attention +
+    combine (2)."""
     def csa(w):
         tensor_scored = (w.idx_fmt in ("fp8", "fp4") and w.d_I == 128 and w.H_I == 64
                          and (w.idx_fmt == "fp8" or w.T == 1))
-        return 8 + (0 if tensor_scored else 1)
+        pool = 2 if w.T == 1 else 3
+        attn = 2 if w.T == 1 else 1
+        return pool + 2 + 2 + (0 if tensor_scored else 1) + attn
     if wl.kind == "pair":
         return csa(wl.layer("csa")) + 4
     return csa(wl) if wl.kind == "csa" else 4
@@ -221,10 +228,39 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def strip_c_comments(src):
+    """C/C++/CUDA source with its comments removed and blank lines dropped:
+    what the compiler sees of the code, so that an edit to a comment does not
+    count as a change of the kernel."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = ("".join(out)).split("\n")
+    return "\n".join(l.rstrip() for l in lines if l.strip())
+
+
 def source_sha(*names):
+    """Hash of the named kernel sources, comments excluded."""
     h = hashlib.sha256()
     for n in names:
-        h.update(open(os.path.join(ROOT, "long_context_sparse_compress_b200", "csrc", n), "rb").read())
+        src = open(os.path.join(ROOT, "long_context_sparse_compress_b200", "csrc", n)).read()
+        h.update(strip_c_comments(src).encode())
     return h.hexdigest()[:16]
 
 
@@ -336,6 +372,7 @@ def run_lcsc(args):
     barrier(ws)
     torch.cuda.synchronize()
     t0 = time.time()
+    launches0 = L.kernel_launches()
     start.record(stream)
     for i in range(args.steps):
         if csa is not None:
@@ -344,6 +381,10 @@ def run_lcsc(args):
             hca.set_events(hevents[i])
         step()
     stop.record(stream)
+    launches = L.kernel_launches() - launches0
+    if launches != kernels_per_step(wl) * args.steps:
+        print(f"note: {launches} kernel launches in {args.steps} steps, "
+              f"{kernels_per_step(wl)} per step expected", file=sys.stderr)
     torch.cuda.synchronize()
     barrier(ws)
     t1 = time.time()
@@ -453,7 +494,7 @@ def run_lcsc(args):
                    "context": wl.L, "heads": wl.H, "kv_dim": wl.D, "top_k": wl.k, "window": wl.w,
                    "csa_entries": wl.L // wl.m, "hca_entries": wl.L // wl.m_hca if wl.kind == "pair" else None,
                    "l2": "inputs larger than L2 (working set per step > 126 MB)"},
-        "roofline": roof, "e2e": e2e, "gpu_launches": kernels_per_step(wl) * args.steps, "clocks": clocks,
+        "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
     }
     if args.cpu_baseline and ws == 1:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_queries)

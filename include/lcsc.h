@@ -128,6 +128,11 @@ int32_t lcsc_abi_version(void);
 /* cudaError_t of the last LCSC_ERR_CUDA returned on this host thread. */
 int32_t lcsc_last_cuda_error(void);
 const char* lcsc_status_string(int32_t status);
+/* Kernels this library has enqueued since it was loaded, over all host
+ * threads and streams.  A kernel counts when its launch is enqueued, not when
+ * it runs; read the count before and after a region to learn how many
+ * launches that region issued. */
+uint64_t lcsc_kernel_launches(void);
 /* Bytes of one stored row for a format and dimension (0 if invalid). */
 int64_t lcsc_row_bytes(int32_t format, int32_t dim, int32_t rope_dim);
 

@@ -2,11 +2,18 @@
 // the launch sequence of every call.  No device memory is allocated here.
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "kernels.cuh"
+#include "launches.h"
 
 namespace lcsc {
+
+std::atomic<uint64_t> g_kernel_launches{0};
+
+void note_launch() { g_kernel_launches.fetch_add(1, std::memory_order_relaxed); }
+
 namespace {
 
 thread_local int32_t g_last_cuda_error = 0;
@@ -176,6 +183,8 @@ extern "C" {
 int32_t lcsc_abi_version(void) { return LCSC_ABI_VERSION; }
 
 int32_t lcsc_last_cuda_error(void) { return g_last_cuda_error; }
+
+uint64_t lcsc_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }
 
 const char* lcsc_status_string(int32_t s) {
   switch (s) {

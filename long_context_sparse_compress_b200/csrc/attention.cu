@@ -15,6 +15,7 @@
 // softmax over 32-row tiles; a combine kernel merges the ranges' (max, sum,
 // unnormalised output) and adds the sink to the denominator.
 #include "kernels.cuh"
+#include "launches.h"
 
 namespace lcsc {
 namespace {
@@ -305,9 +306,9 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   dim3 grid(a.splits, a.H / HPC, a.B * a.T);
   kern<<<grid, kThreads, smem, stream>>>(a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = counted(cudaGetLastError())) != cudaSuccess) return e;
   attn_combine_kernel<DV><<<dim3(a.B * a.T, a.H / 4), DV, 0, stream>>>(a);
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 }  // namespace
@@ -331,7 +332,7 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     if (a.splits == 1) return cudaSuccess;  // one split per query: the kernel wrote the output
     attn_combine_kernel<512><<<dim3(a.B * a.T, a.H / 4), 512, 0, stream>>>(a);
-    return cudaGetLastError();
+    return counted(cudaGetLastError());
   }
   if (a.kv.f.fmt == LCSC_FMT_F32 && a.D == 128 && a.Dv == 128 && a.H % 8 == 0) {
     if (sep) return launch_attn<LCSC_FMT_F32, 128, 128, 8, true>(a, stream);

@@ -26,6 +26,7 @@
 // partial (ref max, sum, O) goes to the workspace the combine kernel merges;
 // with one, the kernel merges the sink itself and writes the output.
 #include "kernels.cuh"
+#include "launches.h"
 #include "sm100.cuh"
 
 namespace lcsc {
@@ -689,7 +690,7 @@ cudaError_t launch_attn_mma(const AttnLaunch& a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(attn_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
   attn_mma_kernel<<<dim3(a.splits, a.B * a.T), kThr, SMEM, stream>>>(a);
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 }  // namespace lcsc

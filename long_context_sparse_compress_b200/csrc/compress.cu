@@ -21,6 +21,7 @@
 #include <type_traits>
 
 #include "kernels.cuh"
+#include "launches.h"
 #include "sm100.cuh"
 
 namespace lcsc {
@@ -585,12 +586,12 @@ cudaError_t launch_pool(const CompressLaunch& a, int E, cudaStream_t stream, boo
     max_clusters = 0;
   }
   *fused = (int64_t)grid.x * grid.z <= max_clusters;
-  if (*fused) return cudaLaunchKernelEx(&cfg, kf, a, E, packed);
+  if (*fused) return counted(cudaLaunchKernelEx(&cfg, kf, a, E, packed));
   auto ku = pool_kernel<kBf16, DIM, NC, false>;
   e = cudaFuncSetAttribute(ku, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ku<<<grid, kThreads, smem, stream>>>(a, E, packed);
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 }  // namespace
@@ -620,7 +621,7 @@ cudaError_t launch_compress(const CompressLaunch& a, cudaStream_t stream) {
     case 32: store_kernel<1><<<grid, 256, 0, stream>>>(a); break;
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 cudaError_t launch_encode_rows(const float* rows, int B, int64_t n, int64_t row0,
@@ -633,7 +634,7 @@ cudaError_t launch_encode_rows(const float* rows, int B, int64_t n, int64_t row0
     case 32: encode_rows_kernel<1><<<grid, 256, 0, stream>>>(rows, n, row0, out); break;
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 }  // namespace lcsc

@@ -25,6 +25,7 @@
 //          shared memory), ties to the lowest index, the chosen ones marked,
 //          and the bitmap compacted into the output in index order.
 #include "kernels.cuh"
+#include "launches.h"
 #include "sm100.cuh"
 #include "topk.cuh"
 
@@ -531,7 +532,7 @@ cudaError_t launch_index_quantize(const IndexLaunch& a, cudaStream_t stream) {
     case 32: quantize_queries_kernel<1><<<qgrid, 256, 0, stream>>>(a, zero_hist); break;
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream) {
@@ -542,7 +543,7 @@ cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream) {
 
 cudaError_t launch_index_score_only(const IndexLaunch& a, cudaStream_t stream) {
   const int lists = a.B * a.T;
-  if (index_mma_supported(a)) return launch_index_mma(a, stream);
+  if (index_mma_supported(a)) return counted(launch_index_mma(a, stream));
   dim3 sgrid((unsigned)((a.n_max + 63) / 64), lists);
   const int fmt = a.keys.f.fmt;
   if (fmt == LCSC_FMT_F32 && a.d_I == 32 && a.H_I == 4)
@@ -553,7 +554,7 @@ cudaError_t launch_index_score_only(const IndexLaunch& a, cudaStream_t stream) {
     score_kernel<LCSC_FMT_FP4, 128, 64><<<sgrid, 256, 0, stream>>>(a);
   else
     return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 cudaError_t launch_topk(const IndexLaunch& a, cudaStream_t stream) {
@@ -566,7 +567,7 @@ cudaError_t launch_topk(const IndexLaunch& a, cudaStream_t stream) {
   dim3 tgrid(slices, lists);
   if (!index_mma_supported(a)) {
     topk_hist_kernel<<<tgrid, 512, 0, stream>>>(a, slices);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = counted(cudaGetLastError())) != cudaSuccess) return e;
   }
   // the collect pass copies each slice into shared memory in one bulk copy
   const int64_t per_max = ((a.n_max + slices - 1) / slices + 31) / 32 * 32;
@@ -574,11 +575,11 @@ cudaError_t launch_topk(const IndexLaunch& a, cudaStream_t stream) {
   e = cudaFuncSetAttribute(topk_collect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)slice_bytes);
   if (e != cudaSuccess) return e;
   topk_collect_kernel<<<tgrid, 512, slice_bytes, stream>>>(a, slices, index_bins_in_collect(a));
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = counted(cudaGetLastError())) != cudaSuccess) return e;
   e = cudaFuncSetAttribute(topk_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFinalSmem);
   if (e != cudaSuccess) return e;
   topk_final_kernel<<<lists, 512, kFinalSmem, stream>>>(a);
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 cudaError_t launch_index_topk(const IndexLaunch& a, cudaStream_t stream) {

@@ -50,6 +50,7 @@ _SIGS = {
     "lcsc_abi_version": (c_i32, []),
     "lcsc_last_cuda_error": (c_i32, []),
     "lcsc_status_string": (ctypes.c_char_p, [c_i32]),
+    "lcsc_kernel_launches": (ctypes.c_uint64, []),
     "lcsc_row_bytes": (c_i64, [c_i32, c_i32, c_i32]),
     "lcsc_compress_workspace_size": (c_i32, [c_vp, c_i64, c_i64, c_vp]),
     "lcsc_csa_compress": (c_i32, [c_vp, c_i32, c_vp, c_i64, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp,
@@ -96,6 +97,11 @@ def load(path=LIB_PATH):
         raise LcscError("liblcsc.so ABI version mismatch: rebuild it")
     _lib = lib
     return lib
+
+
+def kernel_launches():
+    """Kernels the library has enqueued since it was loaded (host-side count)."""
+    return int(load().lcsc_kernel_launches())
 
 
 def check(status):

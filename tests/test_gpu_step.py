@@ -91,3 +91,25 @@ def test_step_twice_is_deterministic(cuda_lib):
     for b in range(2):
         v = sel[b, 0][sel[b, 0] >= 0]
         assert np.all(np.diff(v) > 0)
+
+
+@pytest.mark.parametrize("name,expected", [
+    # every sequence completes a group this step (16384 and 6000 are multiples
+    # of 4): pooling of the indexer keys and of the KV latent, one cluster per
+    # sequence, each storing its rows (2); query quantisation + tensor-core
+    # scoring (2); top-k collect + final (2); attention with several splits
+    # per query + the combine pass (2)
+    ("csa_fp4_decode", 8),
+    # 4096 and 1152 complete a 128-token group: one pooling launch that stores
+    # the entries and window rows itself (three clusters fit), attention +
+    # combine
+    ("hca_decode", 3),
+])
+def test_library_counts_its_launches(cuda_lib, name, expected):
+    from long_context_sparse_compress_b200 import lib as L
+    wl, lengths = CASES[name]
+    gb = GpuBatch(make_seqs(wl, lengths))
+    n0 = L.kernel_launches()
+    gb.run_step()
+    assert L.kernel_launches() - n0 == expected
+    assert gb.status.item() == 0
