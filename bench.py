@@ -148,30 +148,6 @@ class Layer:
         return self.out, torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
 
 
-def kernels_per_step(wl):
-    """Kernels of this library one step of a benchmark workload launches (the
-    bench reports the library's own count of the timed region and checks it
-    against this).  CSA: pooling of the indexer keys (1: one cluster of
-    channel blocks per 128 new rows stores the rows itself) and of the KV
-    latent (1 when its clusters fit on the GPU at once, as in decode; else 2,
-    pooling then a store pass, as in prefill), query quantisation + scoring
-    (2), top-k collect + final (2, plus a histogram pass when the scores come
-    from the CUDA-core scoring kernel), attention (2 with several splits per
-    query, the partials then a combine pass, as in decode; 1 with one split,
-    as in prefill, where the kernel writes the output).  HCA decode: pooling
-    + store (2: its sixteen 8-CTA clusters do not fit at once), attention +
-    combine (2)."""
-    def csa(w):
-        tensor_scored = (w.idx_fmt in ("fp8", "fp4") and w.d_I == 128 and w.H_I == 64
-                         and (w.idx_fmt == "fp8" or w.T == 1))
-        pool = 2 if w.T == 1 else 3
-        attn = 2 if w.T == 1 else 1
-        return pool + 2 + 2 + (0 if tensor_scored else 1) + attn
-    if wl.kind == "pair":
-        return csa(wl.layer("csa")) + 4
-    return csa(wl) if wl.kind == "csa" else 4
-
-
 # ------------------------------------------------------------ measurement
 
 class ClockSampler:
@@ -382,9 +358,6 @@ def run_lcsc(args):
         step()
     stop.record(stream)
     launches = L.kernel_launches() - launches0
-    if launches != kernels_per_step(wl) * args.steps:
-        print(f"note: {launches} kernel launches in {args.steps} steps, "
-              f"{kernels_per_step(wl)} per step expected", file=sys.stderr)
     torch.cuda.synchronize()
     barrier(ws)
     t1 = time.time()

@@ -316,10 +316,21 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
 void attention_splits(int64_t max_rows, int64_t n_ctas_per_split, int granule, int target_ctas, int* splits,
                       int* rows_per_split) {
   if (max_rows < 1) max_rows = 1;
+  if (n_ctas_per_split < 1) n_ctas_per_split = 1;
+  if (target_ctas < 1) target_ctas = 1;
   const int64_t tiles = (max_rows + granule - 1) / granule;
-  int64_t s = target_ctas / (n_ctas_per_split > 0 ? n_ctas_per_split : 1);
-  if (s < 1) s = 1;
-  if (s > tiles) s = tiles;
+  // Time of s splits, in tiles of one CTA: the waves of n * s CTAs that
+  // target_ctas resident ones take, times a split's tiles plus about three
+  // tiles of fixed work (queries in, the first gathers, partials out), plus
+  // about two for the combine pass when s > 1.  The fewest splits within 5%
+  // of the best (fewer partials to write and combine).
+  auto cost = [&](int64_t s) {
+    return ((n_ctas_per_split * s + target_ctas - 1) / target_ctas) * ((tiles + s - 1) / s + 3) + (s > 1 ? 2 : 0);
+  };
+  int64_t best = cost(1);
+  for (int64_t c = 2; c <= tiles; ++c) best = cost(c) < best ? cost(c) : best;
+  int64_t s = 1;
+  while (s < tiles && cost(s) * 20 > best * 21) ++s;
   int64_t rps = ((max_rows + s - 1) / s + granule - 1) / granule * granule;
   *rows_per_split = (int)rps;
   *splits = (int)((max_rows + rps - 1) / rps);

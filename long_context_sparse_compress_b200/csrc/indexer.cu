@@ -7,8 +7,9 @@
 //   s[g] = sum_h w[h] * ReLU(q~[h] . k~[g]),  g < N(p) = floor((p + 1) / m)
 // with q~ the indexer query stored in the key format.
 //
-// Scoring keeps the stored codes unscaled in the dot products and applies
-// the scales afterwards: FP8 rows have one scale per row, so
+// FP8 and FP4 keys are scored on the tensor cores (indexer_mma.cu), fp32 keys
+// here.  Scoring keeps the stored codes unscaled in the dot products and
+// applies the scales afterwards: FP8 rows have one scale per row, so
 // q~[h].k~[g] = sq[h] * sk[g] * (codes . codes); FP4 rows have one scale per
 // 16-block, applied per block.  ReLU commutes with the positive scales.
 //
@@ -70,16 +71,15 @@ __global__ void __launch_bounds__(256) quantize_queries_kernel(IndexLaunch a, bo
 }
 
 // --------------------------------------------------------------- scoring
-// grid (ceil(n_max / 64), B*T); block 256 = 64 keys x 4 head groups.
-template <int FMT, int DI, int HI>
+// CUDA-core scoring of fp32 keys (FP8 and FP4 keys are scored on the tensor
+// cores).  grid (ceil(n_max / 64), B*T); block 256 = 64 keys x 4 head groups.
+template <int DI, int HI>
 __global__ void __launch_bounds__(256) score_kernel(IndexLaunch a) {
   constexpr int KEYS = 64;
   constexpr int HG = HI < 4 ? HI : 4;
   constexpr int HPT = HI / HG;
   constexpr int QS = DI + 1;
-  constexpr int NB = DI / 16;
   __shared__ float qs[HI * QS];
-  __shared__ float sq[HI * NB];
   __shared__ float wq[HI];
 
   const int list = blockIdx.y;
@@ -90,27 +90,9 @@ __global__ void __launch_bounds__(256) score_kernel(IndexLaunch a) {
   if (g0 >= n) return;
   const int tid = threadIdx.x;
 
-  // stored query rows (codes, unscaled) and their scales
   for (int i = tid; i < HI * DI; i += 256) {
     const int h = i / DI, c = i % DI;
-    const int64_t qr = (int64_t)t * HI + h;
-    const uint8_t* row = a.q_store.row(b, qr);
-    float v;
-    if (FMT == LCSC_FMT_F32) v = reinterpret_cast<const float*>(row)[c];
-    else if (FMT == LCSC_FMT_FP8) v = e4m3_val(row[c]);
-    else {
-      const float2 p = e2m1x2_val(row[c >> 1]);
-      v = (c & 1) ? p.y : p.x;
-    }
-    qs[h * QS + c] = v;
-  }
-  for (int i = tid; i < HI * NB; i += 256) {
-    const int h = i / NB, blk = i % NB;
-    const int64_t qr = (int64_t)t * HI + h;
-    float s = 1.f;
-    if (FMT == LCSC_FMT_FP8) s = *a.q_store.fscale(b, qr);
-    else if (FMT == LCSC_FMT_FP4) s = e4m3_val(*a.q_store.bscale_at(b, qr, blk));
-    sq[i] = s;
+    qs[h * QS + c] = reinterpret_cast<const float*>(a.q_store.row(b, (int64_t)t * HI + h))[c];
   }
   for (int i = tid; i < HI; i += 256) wq[i] = a.w_idx[(int64_t)list * HI + i];
   __syncthreads();
@@ -121,59 +103,31 @@ __global__ void __launch_bounds__(256) score_kernel(IndexLaunch a) {
   float acc[HPT];
 #pragma unroll
   for (int i = 0; i < HPT; ++i) acc[i] = 0.f;
-  float sk_row = 1.f;
   if (live) {
-    const uint8_t* krow = a.keys.row(b, g);
-    if (FMT == LCSC_FMT_FP8) sk_row = *a.keys.fscale(b, g);
+    const float4* krow = reinterpret_cast<const float4*>(a.keys.row(b, g));
 #pragma unroll 1
-    for (int blk = 0; blk < NB; ++blk) {
+    for (int blk = 0; blk < DI / 16; ++blk) {
       float kv[16];
-      if (FMT == LCSC_FMT_F32) {
-        const float4* p = reinterpret_cast<const float4*>(krow) + blk * 4;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float4 f = p[j];
-          kv[4 * j] = f.x; kv[4 * j + 1] = f.y; kv[4 * j + 2] = f.z; kv[4 * j + 3] = f.w;
-        }
-      } else if (FMT == LCSC_FMT_FP8) {
-        const uint4 u = reinterpret_cast<const uint4*>(krow)[blk];
-        const uint16_t* c2 = reinterpret_cast<const uint16_t*>(&u);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float2 f = e4m3x2_val(c2[j]);
-          kv[2 * j] = f.x; kv[2 * j + 1] = f.y;
-        }
-      } else {
-        const uint2 u = reinterpret_cast<const uint2*>(krow)[blk];
-        const uint8_t* c2 = reinterpret_cast<const uint8_t*>(&u);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float2 f = e2m1x2_val(c2[j]);
-          kv[2 * j] = f.x; kv[2 * j + 1] = f.y;
-        }
+      for (int j = 0; j < 4; ++j) {
+        const float4 f = krow[blk * 4 + j];
+        kv[4 * j] = f.x; kv[4 * j + 1] = f.y; kv[4 * j + 2] = f.z; kv[4 * j + 3] = f.w;
       }
-      const float skb = FMT == LCSC_FMT_FP4 ? e4m3_val(*a.keys.bscale_at(b, g, blk)) : 1.f;
 #pragma unroll
       for (int i = 0; i < HPT; ++i) {
-        const int h = i * HG + hg;
-        const float* qrow = qs + h * QS + blk * 16;
+        const float* qrow = qs + (i * HG + hg) * QS + blk * 16;
         float part = 0.f;
 #pragma unroll
         for (int j = 0; j < 16; ++j) part = fmaf(qrow[j], kv[j], part);
-        if (FMT == LCSC_FMT_FP4) acc[i] = fmaf(sq[h * NB + blk] * skb, part, acc[i]);
-        else acc[i] += part;
+        acc[i] += part;
       }
     }
   }
   float sc = 0.f;
 #pragma unroll
-  for (int i = 0; i < HPT; ++i) {
-    const int h = i * HG + hg;
-    const float wh = FMT == LCSC_FMT_FP8 ? wq[h] * sq[h * NB] : wq[h];
-    sc = fmaf(wh, fmaxf(acc[i], 0.f), sc);
-  }
+  for (int i = 0; i < HPT; ++i) sc = fmaf(wq[i * HG + hg], fmaxf(acc[i], 0.f), sc);
   for (int o = HG >> 1; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
-  if (live && hg == 0) a.scores[(int64_t)list * a.stride + g] = sc * sk_row;
+  if (live && hg == 0) a.scores[(int64_t)list * a.stride + g] = sc;
 }
 
 // --------------------------------------------------------------- top-k
@@ -545,13 +499,8 @@ cudaError_t launch_index_score_only(const IndexLaunch& a, cudaStream_t stream) {
   const int lists = a.B * a.T;
   if (index_mma_supported(a)) return counted(launch_index_mma(a, stream));
   dim3 sgrid((unsigned)((a.n_max + 63) / 64), lists);
-  const int fmt = a.keys.f.fmt;
-  if (fmt == LCSC_FMT_F32 && a.d_I == 32 && a.H_I == 4)
-    score_kernel<LCSC_FMT_F32, 32, 4><<<sgrid, 256, 0, stream>>>(a);
-  else if (fmt == LCSC_FMT_FP8 && a.d_I == 128 && a.H_I == 64)
-    score_kernel<LCSC_FMT_FP8, 128, 64><<<sgrid, 256, 0, stream>>>(a);
-  else if (fmt == LCSC_FMT_FP4 && a.d_I == 128 && a.H_I == 64)
-    score_kernel<LCSC_FMT_FP4, 128, 64><<<sgrid, 256, 0, stream>>>(a);
+  if (a.keys.f.fmt == LCSC_FMT_F32 && a.d_I == 32 && a.H_I == 4)
+    score_kernel<32, 4><<<sgrid, 256, 0, stream>>>(a);
   else
     return cudaErrorInvalidValue;
   return counted(cudaGetLastError());

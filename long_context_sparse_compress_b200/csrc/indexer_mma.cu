@@ -10,6 +10,9 @@
 //  * FP4 keys and queries: tcgen05.mma kind::mxf4nvf4 with one UE4M3 scale
 //    per 16 values on both operands (the scales go smem -> TMEM with
 //    tcgen05.cp); the accumulator holds the exact dequantised dot products.
+//    The query scales are tiled by 128 rows, two queries to a tile: the
+//    CTA of an odd query moves its rows' scales to the tile's first half
+//    before the copy to TMEM.
 //  * FP8 keys and queries: tcgen05.mma kind::f8f6f4 on the codes; the
 //    per-row scales are positive, so the epilogue applies them outside ReLU:
 //    s = sk[g] * sum_h (w[h] sq[h]) ReLU(acc[h]).
@@ -279,6 +282,15 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
       tc_fence_after();
       const uint32_t q_addr = smem_u32(sm + C::OFF_Q);
       if (live && r == 0 && FMT == LCSC_FMT_FP4) {
+        if (NQ == 1 && (t0 & 1)) {
+          // an odd query's 64 rows are rows 64-127 of its 128-row scale
+          // tile, whose bytes hold rows 64-95 and 96-127 at chunks 2 and 3
+          // of each 16-byte lane entry: move them to chunks 0 and 1, where
+          // an N = 64 MMA reads its B scales
+          uint2* sfb = reinterpret_cast<uint2*>(sm + C::OFF_SFB);
+          for (int e = 0; e < 64; ++e) sfb[2 * e] = sfb[2 * e + 1];
+          fence_async_smem();
+        }
         for (int j = 0; j < 2; ++j)
           for (int c = 0; c < (C::N + 127) / 128; ++c)
             tmem_cp_32x128b_x4(tmem + C::SFB_COL + 8 * c + 4 * j,
@@ -547,6 +559,22 @@ int sm_count() {
   return n;
 }
 
+// Queries per CTA (the MMA's N = 64 per query): four FP8 queries when T
+// allows it, else one.
+int queries_per_cta(const IndexLaunch& a) { return a.keys.f.fmt == LCSC_FMT_FP8 && a.T % 4 == 0 ? 4 : 1; }
+
+// CTAs per query group: as many as fit beside the other groups' on the SMs
+// (one CTA per SM), at least one.  One query per CTA claims its tiles at run
+// time, so it takes two as soon as the groups leave SMs idle: where both
+// fit they share the list; a CTA that waits for an SM joins its list late
+// and takes what is left.
+int chunks_per_group(const IndexLaunch& a) {
+  const int64_t ctas = (int64_t)a.B * (a.T / queries_per_cta(a));
+  if (ctas >= sm_count()) return 1;
+  const int fit = (int)(sm_count() / ctas);
+  return queries_per_cta(a) == 1 && fit < 2 ? 2 : fit;
+}
+
 template <int FMT, int NQ>
 cudaError_t launch_mma(const IndexLaunch& a, cudaStream_t stream) {
   using C = Cfg<FMT, NQ>;
@@ -572,7 +600,7 @@ cudaError_t launch_mma(const IndexLaunch& a, cudaStream_t stream) {
   m.status = a.status;
   const int groups = a.T / NQ;
   const int64_t ctas = (int64_t)a.B * groups;
-  m.chunks = ctas >= sm_count() ? 1 : (int)(sm_count() / ctas);
+  m.chunks = chunks_per_group(a);
   m.bins_in_collect = index_bins_in_collect(a);
   auto kern = index_mma_kernel<FMT, NQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -584,15 +612,13 @@ cudaError_t launch_mma(const IndexLaunch& a, cudaStream_t stream) {
 }  // namespace
 
 bool index_whole_lists(const IndexLaunch& a) {
-  // as launch_mma sizes the grid: one CTA per query group once the groups fill the GPU
-  const int nq = a.keys.f.fmt == LCSC_FMT_FP8 && a.T % 4 == 0 ? 4 : 1;
-  return index_mma_supported(a) && (int64_t)a.B * (a.T / nq) >= sm_count();
+  // one CTA per query group: its histograms never leave shared memory
+  return index_mma_supported(a) && chunks_per_group(a) == 1;
 }
 
 bool index_bins_in_collect(const IndexLaunch& a) {
-  // the one-query tensor-core configuration with several CTAs per list
-  if (!index_mma_supported(a) || (a.keys.f.fmt == LCSC_FMT_FP8 && a.T % 4 == 0)) return false;
-  return (int64_t)a.B * a.T < sm_count();
+  // the one-query configuration with several CTAs per list
+  return index_mma_supported(a) && queries_per_cta(a) == 1 && chunks_per_group(a) > 1;
 }
 
 bool index_mma_supported(const IndexLaunch& a) {
@@ -600,13 +626,13 @@ bool index_mma_supported(const IndexLaunch& a) {
   if (a.d_I != 128 || a.H_I != 64) return false;
   if (a.keys.capacity % 128 != 0) return false;
   if (fmt == LCSC_FMT_FP8) return true;
-  if (fmt == LCSC_FMT_FP4) return a.T == 1;
+  if (fmt == LCSC_FMT_FP4) return true;
   return false;
 }
 
 cudaError_t launch_index_mma(const IndexLaunch& a, cudaStream_t stream) {
   if (a.keys.f.fmt == LCSC_FMT_FP4) return launch_mma<LCSC_FMT_FP4, 1>(a, stream);
-  if (a.T % 4 == 0) return launch_mma<LCSC_FMT_FP8, 4>(a, stream);
+  if (queries_per_cta(a) == 4) return launch_mma<LCSC_FMT_FP8, 4>(a, stream);
   return launch_mma<LCSC_FMT_FP8, 1>(a, stream);
 }
 

@@ -111,8 +111,9 @@ bool attn_mma_supported(const AttnLaunch& a);
 cudaError_t launch_attn_mma(const AttnLaunch& a, cudaStream_t stream);
 
 // Attention split geometry: the rows of each query are cut into `splits`
-// ranges of `rows_per_split` (a multiple of `granule`), sized so that
-// n_ctas_per_split * splits CTAs fill the GPU.
+// ranges of `rows_per_split` (a multiple of `granule`); n_ctas_per_split *
+// splits CTAs run, target_ctas of them at a time, and the split count is
+// the one that finishes them soonest.
 void attention_splits(int64_t max_rows, int64_t n_ctas_per_split, int granule, int target_ctas, int* splits,
                       int* rows_per_split);
 

@@ -21,13 +21,15 @@ struct Thresh {
 
 // Threshold bin of an `nbins`-bin histogram in shared memory for `need`
 // (>= 1) elements: the largest bin t with sum_{d >= t} hist[d] >= need.
-// Every thread of the CTA calls it; threads tid < T (T a multiple of 32 that
-// divides nbins, <= blockDim) each sum nbins / T consecutive bins (in
-// descending order), a warp scan and a scan of the warp totals give each
-// its prefix, and the one whose range holds the need walks its bins.
-// `warp_tot` is 32 words and `res` one Thresh of shared memory.
+// Every thread of the CTA calls it; threads tid < T (T, or nbins when that
+// is smaller: a multiple of 32 that divides nbins, <= blockDim) each sum
+// nbins / T consecutive bins (in descending order), a warp scan and a scan
+// of the warp totals give each its prefix, and the one whose range holds the
+// need walks its bins.  `warp_tot` is 32 words and `res` one Thresh of
+// shared memory.
 __device__ __forceinline__ Thresh block_threshold(const uint32_t* h, int nbins, uint32_t need, int T,
                                                   uint32_t* warp_tot, Thresh* res) {
+  if (T > nbins) T = nbins;  // at least one bin per summing thread
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int per = nbins / T;
   const int top = nbins - 1 - tid * per;  // this thread's highest bin

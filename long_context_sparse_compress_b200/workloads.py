@@ -87,11 +87,15 @@ PAIR_DECODE_1M_B16 = Workload(
 
 PAIR_DECODE_1M_B1 = PAIR_DECODE_1M_B16.with_(name="csa_hca_pair_decode_1m_b1", B=1)
 
+# Multi-token decode: five new tokens per sequence (a draft to verify) on the
+# 1M pair, each its own query.
+PAIR_DECODE_1M_B16_T5 = PAIR_DECODE_1M_B16.with_(name="csa_hca_pair_decode_1m_b16_t5", T=5)
+
 # Single-layer halves of the 1M pair at B = 8, for kernel profiles (inputs
 # still larger than L2, a smaller device footprint).
 CSA_DECODE_1M_B8 = PAIR_DECODE_1M_B16.layer("csa").with_(name="csa_decode_1m_b8_fp4", B=8)
 HCA_DECODE_1M_B8 = PAIR_DECODE_1M_B16.layer("hca").with_(name="hca_decode_1m_b8", B=8)
 
 ALL = {w.name: w for w in (CSA_DECODE_4K_F32, HCA_DECODE_64K, CSA_DECODE_128K,
-                           CSA_PREFILL_256K, PAIR_DECODE_1M_B16, PAIR_DECODE_1M_B1,
+                           CSA_PREFILL_256K, PAIR_DECODE_1M_B16, PAIR_DECODE_1M_B1, PAIR_DECODE_1M_B16_T5,
                            CSA_DECODE_1M_B8, HCA_DECODE_1M_B8)}

@@ -139,14 +139,64 @@ def test_compress_matches_oracle(cuda_lib, case, with_window):
 
 @pytest.mark.parametrize("fmt", ["f32", "fp8", "fp4"])
 def test_index_topk_matches_oracle(cuda_lib, fmt):
-    rng = np.random.default_rng(21)
+    # three lists per sequence (an odd query index among them); tensor-core
+    # scoring runs several CTAs per list here
+    lengths = [4 * 5000 + 3, 4 * 37, 4 * 2100 + 1]  # one list shorter than k
+    check_index_topk(fmt, lengths, T=3, seed=21)
+
+
+# 150 lists: one tensor-core scoring CTA per query, whose own histogram gives
+# the threshold bins; 78 and 80 lists: two CTAs per query (some wait for an
+# SM and join late).  T = 5: five draft-token queries per sequence.
+@pytest.mark.parametrize("fmt,B,T", [("fp8", 50, 3), ("fp4", 30, 5), ("fp8", 26, 3), ("fp4", 16, 5)])
+def test_index_topk_many_lists(cuda_lib, fmt, B, T):
+    rng = np.random.default_rng(5)
+    lengths = [int(v) for v in rng.integers(4 * 300, 4 * 2500, size=B)]
+    check_index_topk(fmt, lengths, T=T, seed=22)
+
+
+def test_topk_resolves_the_last_digit(cuda_lib):
+    """Forty keys whose scores are s0 (1 + 4e-6 j), about seven to a bin of
+    the first 24 key bits: the 17th largest falls inside such a bin, so the
+    last 8 bits decide which of its scores are kept.  fp32 keys (no
+    quantisation) keep the spacing; the band of uncertainty is 1e-6, well
+    under it."""
+    rng = np.random.default_rng(9)
+    wl = W.CSA_DECODE_4K_F32.with_(k=17)
+    H_I, d_I, m = wl.H_I, wl.d_I, wl.m
+    L_ctx = 4096
+    n = L_ctx // m
+    qi = (rng.standard_normal((1, 1, H_I, d_I)) * d_I ** -0.5).astype(np.float32)
+    wi = np.full((1, 1, H_I), 0.5, dtype=np.float32)
+    k0 = qi[0, 0].sum(axis=0)  # positive against every head's query (checked below)
+    assert np.all(qi[0, 0] @ k0 > 0)
+    keys_v = _rows(rng, n, d_I, scale=1e-3 * d_I ** -0.5)
+    pos = rng.choice(n, size=40, replace=False)
+    for j, g in enumerate(pos):
+        keys_v[g] = (k0 * (1.0 + 4e-6 * j)).astype(np.float32)
+    p = L.params(wl)
+    keys = L.DeviceCache(1, n, "f32", d_I)
+    st = storage.encode("f32", keys_v)
+    upload(keys, 0, st)
+    ctx = torch.tensor([L_ctx], dtype=torch.int32, device="cuda")
+    out_idx = torch.full((1, 1, wl.k), -5, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.index_topk(p, dev(qi), dev(wi), keys, ctx, n, out_idx, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    sc = oracle_scores(quantize_query(qi[0, 0], "f32"), wi[0, 0], storage.decode(st))
+    ok, msg = topk_set_ok(out_idx.cpu().numpy()[0, 0], sc, wl.k, band=1e-6)
+    assert ok, msg
+    assert set(out_idx.cpu().numpy()[0, 0].tolist()) == set(pos[23:].tolist())
+
+
+def check_index_topk(fmt, lengths, T, seed):
+    rng = np.random.default_rng(seed)
     if fmt == "f32":
         wl = W.CSA_DECODE_4K_F32.with_(k=64)
     else:
         wl = W.CSA_DECODE_128K.with_(idx_fmt=fmt, k=300)
     H_I, d_I, m = wl.H_I, wl.d_I, wl.m
-    T = 3
-    lengths = [4 * 5000 + 3, 4 * 37, 4 * 2100 + 1]  # one list shorter than k
     B = len(lengths)
     n_cap = L.round_capacity(max(lengths) // m + 1, fmt)
     keys_v = _rows(rng, B * n_cap, d_I).reshape(B, n_cap, d_I)
@@ -269,7 +319,8 @@ def test_attention_matches_oracle(cuda_lib, kind, fmt_kv):
             assert np.allclose(lse_gpu[b, t], ls, rtol=1e-4, atol=1e-4)
 
 
-@pytest.mark.parametrize("T", [64, 160])  # two splits per query (combined) / one split (written directly)
+# two splits per query (combined) / one split with 148 SMs (written directly)
+@pytest.mark.parametrize("T", [64, 148])
 def test_attention_rescales_when_the_max_grows(cuda_lib, T):
     """Scores that jump by more than e^8 part-way through a split: the running
     reference max moves and the partial O accumulated so far is rescaled.

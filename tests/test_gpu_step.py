@@ -18,6 +18,9 @@ CASES = {
     "csa_f32_decode": (W.CSA_DECODE_4K_F32.with_(B=3), [4096, 1000, 101]),
     "csa_fp8_decode": (W.CSA_DECODE_128K.with_(B=3), [8192, 4100, 300]),
     "csa_fp4_decode": (W.PAIR_DECODE_1M_B1.layer("csa").with_(B=2, n_planted=16), [16384, 6000]),
+    # five draft tokens per sequence
+    "csa_fp4_multitoken": (W.PAIR_DECODE_1M_B16_T5.layer("csa").with_(B=2, n_planted=16), [16384, 6003]),
+    "hca_multitoken": (W.PAIR_DECODE_1M_B16_T5.layer("hca").with_(B=2), [16384 + 2, 5000]),
     "hca_decode": (W.HCA_DECODE_64K.with_(B=3), [4096, 1024 + 128, 100]),
     "csa_fp8_prefill": (W.CSA_PREFILL_256K.with_(B=2, T=40, n_planted=8), [4096 + 40, 2002]),
     "hca_prefill": (W.HCA_DECODE_64K.with_(B=1, T=130), [4096 + 130]),
@@ -101,9 +104,10 @@ def test_step_twice_is_deterministic(cuda_lib):
     # per query + the combine pass (2)
     ("csa_fp4_decode", 8),
     # 4096 and 1152 complete a 128-token group: one pooling launch that stores
-    # the entries and window rows itself (three clusters fit), attention +
-    # combine
-    ("hca_decode", 3),
+    # the entries and window rows itself (three clusters fit); attention over
+    # at most 32 entries + 128 window rows runs one split per query, which
+    # writes the output itself
+    ("hca_decode", 2),
 ])
 def test_library_counts_its_launches(cuda_lib, name, expected):
     from long_context_sparse_compress_b200 import lib as L
