@@ -524,7 +524,7 @@ def oracle_step(wl_layer, P, inp, kv, idx, ring):
                       ring_kv=ring, ring_v=None, x_kv=tail(inp["x_kv"]), x_v=None,
                       x_idx=tail(inp.get("x_idx")), W_kv=P["W_kv"], B_kv=P["B_kv"], W_v=None, B_v=None,
                       W_idx=P.get("W_idx"), B_idx=P.get("B_idx"), q=inp["q"], q_idx=inp.get("q_idx"),
-                      w_idx=inp.get("w_idx"), sink=P["sink"])
+                      w_idx=inp.get("w_idx"), sink=P["sink"], out_rope_base=w.out_rope_base)
 
 
 def blas_threads():

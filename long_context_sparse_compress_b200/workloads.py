@@ -37,6 +37,7 @@ class Workload:
     q_dtype: str = "bf16"  # queries and the output
     n_planted: int = 0   # planted relevant entries per sequence
     sink: bool = True
+    out_rope_base: float = 0.0  # > 0: the output's rope dims rotated back by the query position
 
     @property
     def sm_scale(self):
@@ -88,8 +89,9 @@ PAIR_DECODE_1M_B16 = Workload(
 PAIR_DECODE_1M_B1 = PAIR_DECODE_1M_B16.with_(name="csa_hca_pair_decode_1m_b1", B=1)
 
 # Multi-token decode: five new tokens per sequence (a draft to verify) on the
-# 1M pair, each its own query.
-PAIR_DECODE_1M_B16_T5 = PAIR_DECODE_1M_B16.with_(name="csa_hca_pair_decode_1m_b16_t5", T=5)
+# 1M pair, each its own query, outputs rotated back by their positions.
+PAIR_DECODE_1M_B16_T5 = PAIR_DECODE_1M_B16.with_(name="csa_hca_pair_decode_1m_b16_t5", T=5,
+                                                 out_rope_base=10000.0)
 
 # Single-layer halves of the 1M pair at B = 8, for kernel profiles (inputs
 # still larger than L2, a smaller device footprint).

@@ -61,6 +61,32 @@ def attention_weights(q, K, sink, sm_scale):
     return e / Z[:, None]
 
 
+def inverse_rope(o, p, rope_dim, base):
+    """The output rotated back by its query's position ("How DeepSeek V4
+    Handles 1M Token Context", Component 1: keys and values are one shared
+    vector, and inverse RoPE restores the positional information).
+
+    Reading (the page gives no formula): the last ``rope_dim`` dims of o,
+    which carry the keys' rotary components through V = K, are turned back
+    by the query position p, so that the output holds the keys' positions
+    relative to the query.  Pairs (2j, 2j + 1) of those dims, the common
+    interleaved convention, turn by the angle -p * base^(-2j / rope_dim):
+        (x, y) -> (x cos a - y sin a, x sin a + y cos a),  a = -p theta_j.
+    ``base`` <= 0 leaves o as it is."""
+    o = np.array(o, dtype=np.float64, copy=True)
+    if base <= 0 or rope_dim <= 0:
+        return o
+    j = np.arange(rope_dim // 2, dtype=np.float64)
+    a = -float(p) * np.power(float(base), -2.0 * j / rope_dim)
+    c, s = np.cos(a), np.sin(a)
+    lo = o.shape[-1] - rope_dim
+    x = o[..., lo::2].copy()
+    y = o[..., lo + 1::2].copy()
+    o[..., lo::2] = x * c - y * s
+    o[..., lo + 1::2] = x * s + y * c
+    return o
+
+
 def window_positions(p, w):
     """Raw positions in the sliding window of a query at position p."""
     return np.arange(max(0, p - w + 1), p + 1)

@@ -21,7 +21,7 @@ L - (T + G - 1) .. L - 1 (rows at negative positions are never read).
 import numpy as np
 
 from . import storage
-from .attention import joint_attention, window_positions
+from .attention import inverse_rope, joint_attention, window_positions
 from .compress import compress_entries, n_visible
 from .indexer import quantize_query, scores, topk
 
@@ -36,7 +36,7 @@ def _store_rows(cache, rows_idx, values, fmt, rope_dim):
 def layer_step(kind, *, m, G, w, k, sm_scale, kv_fmt, rope_dim, idx_fmt, L, T,
                kv, v, idx, ring_kv, ring_v, x_kv, x_v, x_idx,
                W_kv, B_kv, W_v, B_v, W_idx, B_idx,
-               q, q_idx, w_idx, sink, queries=None):
+               q, q_idx, w_idx, sink, queries=None, out_rope_base=0.0):
     """Run one step for ONE sequence.
 
     kind: "csa" or "hca".  kv / v / idx / ring_kv / ring_v are
@@ -45,6 +45,8 @@ def layer_step(kind, *, m, G, w, k, sm_scale, kv_fmt, rope_dim, idx_fmt, L, T,
     None when V is the shared latent (V = K).  q [T, H, D]; q_idx
     [T, H_I, d_I] and w_idx [T, H_I] (CSA only); sink [H].
     ``queries``: optional subset of query indices i to evaluate.
+    ``out_rope_base`` > 0: each output is rotated back by its query's
+    position (``inverse_rope`` over the last ``rope_dim`` dims).
 
     Returns dict with o [nq, H, Dv], lse [nq, H], and for CSA sel (list of
     index arrays) and sel_scores (list of score arrays), plus new_entries
@@ -97,6 +99,7 @@ def layer_step(kind, *, m, G, w, k, sm_scale, kv_fmt, rope_dim, idx_fmt, L, T,
             V_rows = np.concatenate([storage.decode(v.rows(ent)),
                                      storage.decode(ring_v.rows(wpos % win_cap))], axis=0)
         o, lse = joint_attention(q[i], K_rows, V_rows, sink, sm_scale)
+        o = inverse_rope(o, p, rope_dim, out_rope_base)
         o_all.append(o)
         lse_all.append(lse)
     out = dict(o=np.stack(o_all), lse=np.stack(lse_all), new_entries=(g_lo, g_hi))

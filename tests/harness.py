@@ -77,7 +77,7 @@ class OracleSequence:
             idx=self.idx, ring_kv=self.ring_kv, ring_v=self.ring_v, x_kv=t("x_kv"), x_v=t("x_v"),
             x_idx=t("x_idx"), W_kv=P["W_kv"], B_kv=P["B_kv"], W_v=P.get("W_v"), B_v=P.get("B_v"),
             W_idx=P.get("W_idx"), B_idx=P.get("B_idx"), q=inp["q"], q_idx=inp.get("q_idx"),
-            w_idx=inp.get("w_idx"), sink=P["sink"], queries=queries)
+            w_idx=inp.get("w_idx"), sink=P["sink"], queries=queries, out_rope_base=wl.out_rope_base)
 
 
 # ---------------------------------------------------------------- comparisons

@@ -7,7 +7,7 @@ import torch
 import torch.nn.functional as Fn
 
 from oracle import storage
-from oracle.attention import attention_weights, joint_attention, window_positions
+from oracle.attention import attention_weights, inverse_rope, joint_attention, window_positions
 from oracle.step import layer_step
 
 
@@ -187,3 +187,75 @@ def test_step_compresses_only_closing_groups():
         q = rng.standard_normal((T, H, D))
         out = _run("hca", x, q, m=4, G=4, w=2, k=0, L=L, T=T, sink=np.zeros(H))
         assert out["new_entries"] == want
+
+
+# ------------------------------------------------------- output inverse RoPE
+
+def _rotate_complex(v, p, base, sign):
+    """Pairs (2j, 2j + 1) as complex numbers x + iy times exp(sign i p theta_j),
+    theta_j = base^(-2j / d): an independent statement of the rotation."""
+    d = v.shape[-1]
+    z = v[..., 0::2] + 1j * v[..., 1::2]
+    theta = base ** (-2.0 * np.arange(d // 2) / d)
+    z = z * np.exp(sign * 1j * p * theta)
+    out = np.empty_like(v, dtype=np.float64)
+    out[..., 0::2], out[..., 1::2] = z.real, z.imag
+    return out
+
+
+def test_inverse_rope_closed_forms():
+    # one pair, theta_0 = 1: (1, 0) turned by -1 radian
+    o = np.array([[7.0, 1.0, 0.0]])
+    got = inverse_rope(o, 1, 2, 10000.0)
+    assert got[0, 0] == 7.0
+    assert np.allclose(got[0, 1:], [np.cos(1.0), -np.sin(1.0)], rtol=0, atol=1e-15)
+    # second pair of four dims with base 100: theta_1 = 0.1, p = 5 -> -0.5 rad
+    o = np.array([0.0, 0.0, 0.0, 2.0])
+    got = inverse_rope(o, 5, 4, 100.0)
+    assert np.allclose(got[2:], [-2.0 * np.sin(-0.5), 2.0 * np.cos(-0.5)], rtol=0, atol=1e-15)
+    # position 0 and a zero base leave the output unchanged
+    rng = np.random.default_rng(1)
+    o = rng.standard_normal((3, 16))
+    assert np.array_equal(inverse_rope(o, 0, 8, 10000.0), o)
+    assert np.array_equal(inverse_rope(o, 123, 8, 0.0), o)
+
+
+def test_inverse_rope_matches_complex_rotation_and_undoes_rope():
+    rng = np.random.default_rng(2)
+    H, D, R = 4, 24, 8
+    o = rng.standard_normal((H, D))
+    p = 1_000_003
+    got = inverse_rope(o, p, R, 10000.0)
+    assert np.array_equal(got[:, :D - R], o[:, :D - R])            # the other dims untouched
+    assert np.allclose(got[:, D - R:], _rotate_complex(o[:, D - R:], p, 10000.0, -1), rtol=1e-9, atol=1e-12)
+    pair_norm = lambda v: np.hypot(v[..., 0::2], v[..., 1::2])
+    assert np.allclose(pair_norm(got[:, D - R:]), pair_norm(o[:, D - R:]), rtol=1e-12)
+    forward = o.copy()
+    forward[:, D - R:] = _rotate_complex(o[:, D - R:], p, 10000.0, +1)
+    assert np.allclose(inverse_rope(forward, p, R, 10000.0), o, rtol=1e-9, atol=1e-12)
+
+
+def test_inverse_rope_leaves_relative_positions():
+    """Values whose rope dims are a vector turned by their key positions: after
+    the inverse rotation by the query position the output depends only on
+    the key positions relative to the query (a common shift changes nothing).
+    The query's rope dims are zero, so the weights do not move either."""
+    rng = np.random.default_rng(3)
+    S, D, R, H = 6, 16, 8, 2
+    base_rows = rng.standard_normal((S, D))
+    q = rng.standard_normal((H, D))
+    q[:, D - R:] = 0.0
+    key_pos = rng.integers(0, 500, size=S)
+    p_q = 700
+
+    def out(shift):
+        K = base_rows.copy()
+        for j in range(S):
+            K[j, D - R:] = _rotate_complex(base_rows[j, D - R:], key_pos[j] + shift, 10000.0, +1)
+        o, _ = joint_attention(q, K, K, np.full(H, -np.inf), 0.3)
+        return inverse_rope(o, p_q + shift, R, 10000.0)
+
+    assert np.allclose(out(0), out(12345), rtol=1e-9, atol=1e-12)
+    # turning the other way (a sign slip) would not be shift-invariant
+    o0 = joint_attention(q, base_rows, base_rows, np.full(H, -np.inf), 0.3)[0]
+    assert not np.allclose(inverse_rope(o0, 1, R, 10000.0), inverse_rope(o0, -1, R, 10000.0))
