@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define LCSC_ABI_VERSION 1
+#define LCSC_ABI_VERSION 2
 
 /* Return codes. */
 #define LCSC_OK 0
@@ -104,6 +104,15 @@ typedef struct lcsc_params {
   int32_t idx_format;  /* LCSC_FMT_F32, LCSC_FMT_FP8 or LCSC_FMT_FP4 */
   int32_t x_dtype;     /* LCSC_DT_*: raw token rows and gate weights W */
   int32_t q_dtype;     /* LCSC_DT_*: queries, indexer queries and the output */
+  /* Inverse RoPE of the output ("How DeepSeek V4 Handles 1M Token Context",
+   * Component 1: K and V are one shared vector and inverse RoPE restores the
+   * positional information).  out_rope_base > 0: the last out_rope_dim dims
+   * of every output row, in pairs (2j, 2j+1), are turned by the angle
+   * -p * out_rope_base^(-2j / out_rope_dim), p the query's position, so the
+   * output carries the key positions relative to the query.  0: off.
+   * out_rope_dim: a multiple of 4, <= v_dim, when on. */
+  int32_t out_rope_dim;
+  float out_rope_base;
 } lcsc_params;
 
 /* Stored rows of one tensor for B sequences (dev pointers).

@@ -65,6 +65,10 @@ int32_t check_params(const lcsc_params* p) {
   if (p->x_dtype != LCSC_DT_F32 && p->x_dtype != LCSC_DT_BF16) return LCSC_ERR_INVALID_ARG;
   if (p->q_dtype != LCSC_DT_F32 && p->q_dtype != LCSC_DT_BF16) return LCSC_ERR_INVALID_ARG;
   if (!(p->sm_scale == p->sm_scale)) return LCSC_ERR_INVALID_ARG;
+  if (!(p->out_rope_base >= 0.f) || p->out_rope_base == INFINITY) return LCSC_ERR_INVALID_ARG;
+  if (p->out_rope_base > 0.f &&
+      (p->out_rope_dim < 4 || p->out_rope_dim % 4 != 0 || p->out_rope_dim > p->v_dim))
+    return LCSC_ERR_INVALID_ARG;
   return LCSC_OK;
 }
 
@@ -420,6 +424,8 @@ static int32_t attn_setup(const lcsc_params* p, const void* q, const lcsc_cache*
   L->k = p->top_k;
   L->n_max = n_max;
   L->sm_scale = p->sm_scale;
+  L->out_rope_dim = p->out_rope_base > 0.f ? p->out_rope_dim : 0;
+  L->out_rope_base = p->out_rope_base;
   L->out = out;
   L->lse = lse;
   L->status = status;

@@ -16,6 +16,7 @@
 // unnormalised output) and adds the sink to the denominator.
 #include "kernels.cuh"
 #include "launches.h"
+#include "rope.cuh"
 
 namespace lcsc {
 namespace {
@@ -282,7 +283,11 @@ __global__ void __launch_bounds__(DV) attn_combine_kernel(AttnLaunch a) {
     }
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  const float r[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+  float4 o4 = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  RopePair2 rot;
+  const int64_t pos = (int64_t)a.ctx_len[list / a.T] - a.T + list % a.T;
+  if (inverse_rope_angles(4 * d4, DV, a.out_rope_dim, a.out_rope_base, pos, &rot)) o4 = rotate2(o4, rot);
+  const float r[4] = {o4.x, o4.y, o4.z, o4.w};
   const int64_t oi = ((int64_t)list * a.H + h) * DV + 4 * d4;
   if (a.q_dtype == LCSC_DT_BF16) {
     uint16_t* out = reinterpret_cast<uint16_t*>(a.out) + oi;

@@ -27,6 +27,7 @@
 // with one, the kernel merges the sink itself and writes the output.
 #include "kernels.cuh"
 #include "launches.h"
+#include "rope.cuh"
 #include "sm100.cuh"
 
 namespace lcsc {
@@ -658,19 +659,28 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
      // partial (several splits) or of the output in the query's type (one split)
     const float* o_s = reinterpret_cast<const float*>(sm + OFF_K);
     auto row4 = [&](int i) { return *reinterpret_cast<const float4*>(o_s + (i / (kD / 4)) * kOS + 4 * (i % (kD / 4))); };
+    // one split: the output itself, rotated back by the query position where
+    // asked (a thread's dims are the same in every row: kThr is a multiple
+    // of kD / 4)
+    static_assert(kThr % (kD / 4) == 0, "fixed dims per thread");
+    RopePair2 rot;
+    const bool turn = a.splits == 1 &&
+                      inverse_rope_angles(4 * (tid % (kD / 4)), kD, a.out_rope_dim, a.out_rope_base,
+                                          (int64_t)a.ctx_len[list / a.T] - a.T + list % a.T, &rot);
+    auto out4 = [&](int i) { return turn ? rotate2(row4(i), rot) : row4(i); };
     if (a.splits > 1) {
       float4* dst = reinterpret_cast<float4*>(a.part_o + ((int64_t)list * a.splits + blockIdx.x) * a.H * kD);
       for (int i = tid; i < kH * (kD / 4); i += kThr) dst[i] = row4(i);
     } else if (a.q_dtype == LCSC_DT_BF16) {
       uint2* dst = reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) + (int64_t)list * a.H * kD);
       for (int i = tid; i < kH * (kD / 4); i += kThr) {
-        const float4 v = row4(i);
+        const float4 v = out4(i);
         dst[i] = make_uint2((uint32_t)bf16_code(v.x) | ((uint32_t)bf16_code(v.y) << 16),
                             (uint32_t)bf16_code(v.z) | ((uint32_t)bf16_code(v.w) << 16));
       }
     } else {
       float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + (int64_t)list * a.H * kD);
-      for (int i = tid; i < kH * (kD / 4); i += kThr) dst[i] = row4(i);
+      for (int i = tid; i < kH * (kD / 4); i += kThr) dst[i] = out4(i);
     }
   }
   if (warp == kMmaWarp) {

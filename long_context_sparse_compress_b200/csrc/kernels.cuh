@@ -95,6 +95,8 @@ struct AttnLaunch {
   int B, T, H, D, Dv, m, w, k;
   int64_t n_max;
   float sm_scale;
+  int out_rope_dim;     // > 0: the output's last dims rotated back by the query position
+  float out_rope_base;
   int splits;           // row splits per query
   int rows_per_split;
   float* part_o;        // [B*T][splits][H][Dv]

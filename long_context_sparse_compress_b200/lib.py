@@ -13,7 +13,7 @@ from . import workloads
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblcsc.so")
-ABI_VERSION = 1
+ABI_VERSION = 2
 
 FMT = {"f32": 0, "kv": 1, "fp8": 2, "fp4": 3}
 DT = {"f32": 0, "bf16": 1}
@@ -28,7 +28,8 @@ class Params(ctypes.Structure):
     _fields_ = [("m", c_i32), ("group_len", c_i32), ("window", c_i32), ("top_k", c_i32),
                 ("sm_scale", c_f32), ("n_heads", c_i32), ("head_dim", c_i32), ("rope_dim", c_i32),
                 ("v_dim", c_i32), ("idx_heads", c_i32), ("idx_dim", c_i32), ("kv_format", c_i32),
-                ("idx_format", c_i32), ("x_dtype", c_i32), ("q_dtype", c_i32)]
+                ("idx_format", c_i32), ("x_dtype", c_i32), ("q_dtype", c_i32),
+                ("out_rope_dim", c_i32), ("out_rope_base", c_f32)]
 
 
 class Cache(ctypes.Structure):
@@ -132,7 +133,8 @@ def params(wl):
                   sm_scale=wl.sm_scale, n_heads=wl.H, head_dim=wl.D,
                   rope_dim=wl.rope_dim if wl.kv_fmt == "kv" else 0, v_dim=wl.Dv, idx_heads=wl.H_I,
                   idx_dim=wl.d_I, kv_format=FMT[wl.kv_fmt], idx_format=FMT[wl.idx_fmt],
-                  x_dtype=DT[wl.x_dtype], q_dtype=DT[wl.q_dtype])
+                  x_dtype=DT[wl.x_dtype], q_dtype=DT[wl.q_dtype],
+                  out_rope_dim=wl.rope_dim if wl.out_rope_base > 0 else 0, out_rope_base=wl.out_rope_base)
 
 
 def row_bytes(fmt, dim, rope=0):

@@ -69,6 +69,16 @@ def test_bad_arguments_are_rejected_before_launch(lib):
     # group length beyond 2m
     bad = L.params(W.CSA_DECODE_128K.with_(G=12))
     assert lib.lcsc_index_topk_workspace_size(ctypes.byref(bad), 1, 1, 10, ctypes.byref(out)) == 1
+    # the output's inverse RoPE: a base that is negative, not a number or
+    # infinite, and rotated dims that are not a multiple of 4 or exceed Dv
+    rope_on = L.params(W.CSA_DECODE_128K.with_(out_rope_base=10000.0))
+    assert lib.lcsc_attn_workspace_size(ctypes.byref(rope_on), 1, 1, 10, 0, ctypes.byref(out)) == 0
+    for field, value in (("out_rope_base", -1.0), ("out_rope_base", float("nan")),
+                         ("out_rope_base", float("inf")), ("out_rope_dim", 6), ("out_rope_dim", 0),
+                         ("out_rope_dim", 516)):
+        bad = L.params(W.CSA_DECODE_128K.with_(out_rope_base=10000.0))
+        setattr(bad, field, value)
+        assert lib.lcsc_attn_workspace_size(ctypes.byref(bad), 1, 1, 10, 0, ctypes.byref(out)) == 1, field
     # a dimension the kernels are not built for
     odd = L.params(W.CSA_DECODE_128K.with_(d_I=96))
     s = L.Step(B=1, T=1, n_max=10, ctx_len=16)

@@ -21,6 +21,11 @@ CASES = {
     # five draft tokens per sequence
     "csa_fp4_multitoken": (W.PAIR_DECODE_1M_B16_T5.layer("csa").with_(B=2, n_planted=16), [16384, 6003]),
     "hca_multitoken": (W.PAIR_DECODE_1M_B16_T5.layer("hca").with_(B=2), [16384 + 2, 5000]),
+    # the output's inverse RoPE where the attention writes the output itself
+    # (one split: prefill) and through the CUDA-core fp32 path
+    "csa_prefill_inverse_rope": (W.CSA_PREFILL_256K.with_(B=2, T=40, n_planted=8, out_rope_base=10000.0),
+                                 [4096 + 40, 2002]),
+    "csa_f32_inverse_rope": (W.CSA_DECODE_4K_F32.with_(B=3, out_rope_base=500.0), [4096, 1000, 101]),
     "hca_decode": (W.HCA_DECODE_64K.with_(B=3), [4096, 1024 + 128, 100]),
     "csa_fp8_prefill": (W.CSA_PREFILL_256K.with_(B=2, T=40, n_planted=8), [4096 + 40, 2002]),
     "hca_prefill": (W.HCA_DECODE_64K.with_(B=1, T=130), [4096 + 130]),
