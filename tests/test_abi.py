@@ -86,3 +86,32 @@ def test_bad_arguments_are_rejected_before_launch(lib):
     assert lib.lcsc_csa_decode(ctypes.byref(odd), ctypes.byref(s), ws, 64, null, null) == 2
     # misaligned pointer in encode_rows
     assert lib.lcsc_encode_rows(ctypes.byref(p), 0, 3, 1, 1, 0, null, null) == 1
+
+
+def _attn_splits(lib, wl, B, T, n_max, dense):
+    """The attention's split count, read back from its workspace size: one
+    [B*T][splits][H][Dv] fp32 partial O and one [B*T][splits][H][2] fp32
+    (max, sum) array, each rounded up to 256 bytes."""
+    p = L.params(wl)
+    out = ctypes.c_size_t(0)
+    assert lib.lcsc_attn_workspace_size(ctypes.byref(p), B, T, n_max, int(dense), ctypes.byref(out)) == 0
+    up = lambda x: (x + 255) // 256 * 256
+    for s in range(1, 4096):
+        if up(B * T * s * wl.H * wl.Dv * 4) + up(B * T * s * wl.H * 2 * 4) == out.value:
+            return s
+    raise AssertionError(f"no split count gives {out.value} bytes")
+
+
+def test_attention_split_counts(lib):
+    """The split cost model on this host (no GPU: 148 SMs assumed): one wave
+    of several splits for the decode pair, fewer for five queries per
+    sequence, one for chunked prefill (the kernel then writes the output
+    itself)."""
+    pair = W.PAIR_DECODE_1M_B16
+    csa, hca = pair.layer("csa"), pair.layer("hca")
+    assert _attn_splits(lib, hca, 16, 1, 8192, True) == 9       # 8,320 rows: 144 CTAs
+    assert _attn_splits(lib, csa, 16, 1, 262144, False) == 9    # 1,152 rows: 144 CTAs
+    assert _attn_splits(lib, hca, 16, 5, 8192, True) == 5       # 80 queries: 400 CTAs
+    assert _attn_splits(lib, csa, 16, 5, 262144, False) == 1    # 80 queries, 18 tiles each
+    assert _attn_splits(lib, W.CSA_PREFILL_256K, 1, 4096, 66560, False) == 1
+    assert _attn_splits(lib, W.CSA_DECODE_128K, 8, 1, 32768, False) == 18  # a 64-row tile per split
