@@ -260,7 +260,8 @@ int32_t lcsc_hca_dense_attn(const lcsc_params* p, const void* q, const lcsc_cach
                             size_t workspace_bytes, int32_t* status, void* stream);
 
 /* ------------------------------------------------------------ fused steps
- * One decode (T = 1) or chunked-prefill (T > 1) step of a layer: pool every
+ * One step of a layer over T new tokens per sequence (T = 1 decode, a few
+ * draft tokens, or a chunked-prefill block), each its own query: pool every
  * group that closes inside the T new tokens (entries
  * [floor((L - T) / m), floor(L / m))), store the T new raw rows in the
  * window rings, then (CSA) score + select + attend, or (HCA) attend densely.
