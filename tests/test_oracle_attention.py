@@ -82,7 +82,8 @@ def _f32(a):
     return np.asarray(a, dtype=np.float32).astype(np.float64)
 
 
-def _run(kind, x, q, *, m, G, w, k, L, T, sink, qi=None, wi=None, xi=None, cap=None):
+def _run(kind, x, q, *, m, G, w, k, L, T, sink, qi=None, wi=None, xi=None, cap=None, rope_dim=0,
+         out_rope_base=0.0):
     """A step over raw f32 tokens x [L, D] (float32-exact values, as the f32
     format stores them) whose cache already holds every entry before the
     step's tokens (pooled with zero gates)."""
@@ -109,12 +110,12 @@ def _run(kind, x, q, *, m, G, w, k, L, T, sink, qi=None, wi=None, xi=None, cap=N
     xit = None
     if kind == "csa":
         xit = np.concatenate([np.zeros((max(0, -lo), xi.shape[1])), xi[max(lo, 0):L]])
-    return layer_step(kind, m=m, G=G, w=w, k=k, sm_scale=1 / np.sqrt(D), kv_fmt="f32", rope_dim=0,
+    return layer_step(kind, m=m, G=G, w=w, k=k, sm_scale=1 / np.sqrt(D), kv_fmt="f32", rope_dim=rope_dim,
                       idx_fmt="f32", L=L, T=T, kv=kv, v=None, idx=idx, ring_kv=ring, ring_v=None,
                       x_kv=xt, x_v=None, x_idx=xit, W_kv=W0, B_kv=B0, W_v=None, B_v=None,
                       W_idx=None if kind != "csa" else np.zeros((xi.shape[1],) * 2),
                       B_idx=None if kind != "csa" else np.zeros((G, xi.shape[1])),
-                      q=q, q_idx=qi, w_idx=wi, sink=sink)
+                      q=q, q_idx=qi, w_idx=wi, sink=sink, out_rope_base=out_rope_base)
 
 
 def _causal_sdpa(x, q, L, T):
@@ -259,3 +260,30 @@ def test_inverse_rope_leaves_relative_positions():
     # turning the other way (a sign slip) would not be shift-invariant
     o0 = joint_attention(q, base_rows, base_rows, np.full(H, -np.inf), 0.3)[0]
     assert not np.allclose(inverse_rope(o0, 1, R, 10000.0), inverse_rope(o0, -1, R, 10000.0))
+
+
+@pytest.mark.parametrize("kind", ["csa", "hca"])
+def test_t_token_step_equals_t_decode_steps(kind):
+    """Five new tokens in one step (draft-token decode) answer each query as
+    five successive one-token steps would: same visible entries (groups
+    closing inside the chunk included), same window, same selection, same
+    output after the inverse rotation by each query's own position."""
+    rng = np.random.default_rng(11)
+    L, D, H, T, R = 61, 8, 2, 5, 4
+    m, G, w, k = 4, 8, 5, 6
+    x = _f32(rng.standard_normal((L, D)))
+    q = rng.standard_normal((T, H, D))
+    sink = rng.standard_normal(H)
+    kw = dict(m=m, G=G, w=w, k=k if kind == "csa" else 0, sink=sink, rope_dim=R, out_rope_base=100.0)
+    if kind == "csa":
+        xi = _f32(rng.standard_normal((L, 4)))
+        qi, wi = rng.standard_normal((T, 2, 4)), np.abs(rng.standard_normal((T, 2)))
+    whole = _run(kind, x, q, L=L, T=T, **kw, **({"qi": qi, "wi": wi, "xi": xi} if kind == "csa" else {}))
+    for t in range(T):
+        Lt = L - T + t + 1
+        one = _run(kind, x[:Lt], q[t:t + 1], L=Lt, T=1, cap=T + w - 1, **kw,
+                   **({"qi": qi[t:t + 1], "wi": wi[t:t + 1], "xi": xi[:Lt]} if kind == "csa" else {}))
+        assert np.allclose(whole["o"][t], one["o"][0], rtol=1e-12, atol=1e-13)
+        assert np.allclose(whole["lse"][t], one["lse"][0], rtol=1e-12)
+        if kind == "csa":
+            assert np.array_equal(np.sort(whole["sel"][t]), np.sort(one["sel"][0]))
