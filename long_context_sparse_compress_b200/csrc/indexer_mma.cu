@@ -20,9 +20,10 @@
 // tcgen05 instructions (tens of cycles each) is what limits a single
 // pipeline, so tiles go to LANES lanes (warps 0 .. LANES-1, one thread each):
 // round-robin over the CTA's share with four queries, claimed two at a time
-// from a counter per list with one (several CTAs share a list).  Lane r loads
-// its tiles with TMA (hardware swizzle) into a STAGES-deep ring, DIST of its
-// tiles ahead, and issues their MMAs into NACC TMEM accumulators.  Groups of four epilogue warps drain the accumulators
+// from a counter per list with one (the list's CTAs share its tiles).  Lane
+// r loads its tiles with TMA (hardware swizzle) into a STAGES-deep ring,
+// DIST of its tiles ahead, and issues their MMAs into NACC TMEM
+// accumulators.  Groups of four epilogue warps drain the accumulators
 // with tcgen05.ld, apply ReLU and the head weights, write one fp32 score per
 // (query, key) and count it in the list's shared-memory histogram of the
 // top-k's first digit.  One query (384 threads): two groups take alternate
@@ -101,9 +102,10 @@ struct Cfg {
   static constexpr int OFF_SFA = OFF_Q + Q_BYTES;
   static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
   static constexpr int OFF_BAR = OFF_SFB + SFB_BYTES;
-  // One query (decode, several CTAs per list): the lanes claim their tiles
-  // at run time, BL at a time, from a counter per list, so CTAs on faster
-  // SMs take more (static equal shares ended up to 40% apart).  A lane
+  // One query per CTA (decode, draft tokens): the lanes claim their tiles
+  // at run time, BL at a time, from a counter per list, so the CTAs of a
+  // list on faster SMs take more (static equal shares ended up to 40%
+  // apart).  A lane
   // publishes each claim to the epilogue through a ring of RING mbarriers.
   static constexpr bool DYN = NQ == 1;
   static constexpr int BL = 2;
