@@ -5,8 +5,8 @@
 // Method: "DeepSeek V4 Architecture Explained" (researchpapers.dev), "How
 // compress-then-sparsify attention works": exact attention over the
 // selected compressed entries, a sliding-window branch of uncompressed recent
-// tokens and an attention-sink term that lets a head's scores sum to less
-// than one; HCA is the same without selection, with the shared-KV
+// tokens and a sink term that keeps part of each head's probability mass off
+// every row; HCA is the same without selection, with the shared-KV
 // multi-query layout.  One softmax spans both branches:
 //   o[h] = sum_j e^{l_j - M} V_j / (e^{sigma_h - M} + sum_j e^{l_j - M}).
 //

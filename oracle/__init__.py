@@ -20,7 +20,8 @@ What it computes (each module cites the passage it restates):
                    Component 3).
 * ``attention`` -- one joint softmax over the selected (CSA) or all (HCA)
                    compressed entries, the uncompressed sliding window and a
-                   per-head attention sink.
+                   per-head attention sink (a learned logit, or the raw row
+                   of position 0 in the sink-token reading, see ``step``).
 * ``step``      -- one decode / chunked-prefill step of a CSA or HCA layer.
 
 All arithmetic is float64 except the decisions that produce stored codes

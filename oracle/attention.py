@@ -4,9 +4,9 @@ Test infrastructure only (see ``oracle/__init__.py``).
 
 Sources: "DeepSeek V4 Architecture Explained", "How compress-then-sparsify
 attention works" (exact attention over the selected compressed entries, a
-small sliding-window branch of uncompressed recent tokens, and an
-attention-sink term that lets a head's weights sum to less than one; HCA is
-the same with larger groups and no selection, with the shared-KV
+small sliding-window branch of uncompressed recent tokens, and a sink term
+that leaves part of each head's probability mass unassigned to any row; HCA
+is the same with larger groups and no selection, with the shared-KV
 multi-query layout); "Inside DeepSeek-V4", sections 1-2 (window w = 128);
 "How DeepSeek V4 Handles 1M Token Context", Component 3 (scaled dot-product
 attention over the gathered entries, plus the 128-token window).

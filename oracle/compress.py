@@ -20,6 +20,13 @@ separately the gate logit of token j is
 the weights are alpha_j[c] = softmax over the group's tokens of z_j[c], and
 the entry is  e_g[c] = sum_j alpha_j[c] * x_j[c].  Each compressed tensor
 (the shared KV latent, a separate V, the indexer keys) has its own W, Bpos.
+
+Caller-given gate logits (a second reading, since the pages do not say
+what the trainable compression weights act on): a per-token logit row u_j
+takes the place of x_j W, and the positional bias of the token's place in
+the group is still added, z_j[c] = u_j[c] + Bpos[j - (g*m + m - G), c].  A
+token shared by two overlapping groups keeps its u_j and gets the bias of
+its place in each group.
 """
 import numpy as np
 
@@ -29,27 +36,32 @@ def group_span(g, m, G):
     return g * m + m - G, g * m + m
 
 
-def pool_group(x_tok, W, bpos_rows):
+def pool_group(x_tok, W, bpos_rows, u_tok=None):
     """One entry from its tokens.
 
     x_tok: [J, D] token rows (float64) of the group, oldest first.
     W: [D, D] gate projection (input channel d, output channel c).
     bpos_rows: [J, D] the positional-bias rows of those tokens.
+    u_tok: optional [J, D] caller-given gate logits of those tokens, used in
+    place of x_tok @ W (W is then not read).
     Returns the pooled row [D] and the gate weights alpha [J, D].
     """
     x_tok = np.asarray(x_tok, dtype=np.float64)
-    z = x_tok @ np.asarray(W, dtype=np.float64) + np.asarray(bpos_rows, dtype=np.float64)
+    gate = (x_tok @ np.asarray(W, dtype=np.float64)) if u_tok is None else np.asarray(u_tok, dtype=np.float64)
+    z = gate + np.asarray(bpos_rows, dtype=np.float64)
     z = z - z.max(axis=0, keepdims=True)
     a = np.exp(z)
     alpha = a / a.sum(axis=0, keepdims=True)
     return (alpha * x_tok).sum(axis=0), alpha
 
 
-def compress_entries(x, x_pos0, W, Bpos, m, G, entries):
+def compress_entries(x, x_pos0, W, Bpos, m, G, entries, U=None):
     """Pool entries ``entries`` (iterable of g) from raw rows.
 
     x: [n, D] raw token rows for positions x_pos0 .. x_pos0 + n - 1; every
     non-negative position an entry needs must be present.
+    U: optional [n, D] caller-given gate logits of the same positions (in
+    place of x W).
     Returns float64 [len(entries), D].
     """
     x = np.asarray(x, dtype=np.float64)
@@ -61,7 +73,8 @@ def compress_entries(x, x_pos0, W, Bpos, m, G, entries):
             raise ValueError(f"entry {g} needs positions [{first}, {stop}) not all in x")
         rows = x[first - x_pos0: stop - x_pos0]
         brows = np.asarray(Bpos)[first - start: stop - start]
-        e, _ = pool_group(rows, W, brows)
+        urows = None if U is None else np.asarray(U)[first - x_pos0: stop - x_pos0]
+        e, _ = pool_group(rows, W, brows, urows)
         out.append(e)
     return np.stack(out) if out else np.zeros((0, x.shape[1]))
 

@@ -17,6 +17,13 @@ sit at positions p = L - T + i.  Before attending, the step
 
 Raw rows reach the step as ``x_*`` arrays covering positions
 L - (T + G - 1) .. L - 1 (rows at negative positions are never read).
+
+Sink token (``sink_mode="token"``), the other reading of the pages' sink
+("DeepSeek V4 Architecture Explained", "How compress-then-sparsify attention
+works"): instead of a learned logit, the raw row of position 0 is a member
+of every query's row set.  It enters once: when the window already holds
+position 0 nothing is added.  The step that receives position 0 stores its
+raw row (in the KV format) in a one-row array, which later steps read.
 """
 import numpy as np
 
@@ -36,7 +43,8 @@ def _store_rows(cache, rows_idx, values, fmt, rope_dim):
 def layer_step(kind, *, m, G, w, k, sm_scale, kv_fmt, rope_dim, idx_fmt, L, T,
                kv, v, idx, ring_kv, ring_v, x_kv, x_v, x_idx,
                W_kv, B_kv, W_v, B_v, W_idx, B_idx,
-               q, q_idx, w_idx, sink, queries=None, out_rope_base=0.0):
+               q, q_idx, w_idx, sink, queries=None, out_rope_base=0.0,
+               U_kv=None, U_v=None, U_idx=None, sink_mode="logit", tok_kv=None, tok_v=None):
     """Run one step for ONE sequence.
 
     kind: "csa" or "hca".  kv / v / idx / ring_kv / ring_v are
@@ -47,6 +55,11 @@ def layer_step(kind, *, m, G, w, k, sm_scale, kv_fmt, rope_dim, idx_fmt, L, T,
     ``queries``: optional subset of query indices i to evaluate.
     ``out_rope_base`` > 0: each output is rotated back by its query's
     position (``inverse_rope`` over the last ``rope_dim`` dims).
+    ``U_*``: caller-given gate logits aligned with ``x_*`` (None: x W).
+    ``sink_mode``: "logit" (``sink`` holds sigma per head) or "token" (the
+    raw row of position 0 joins every row set; ``sink`` is not used);
+    ``tok_kv`` / ``tok_v`` are that row's one-row ``Stored`` arrays (updated
+    in place by the step that receives position 0).
 
     Returns dict with o [nq, H, Dv], lse [nq, H], and for CSA sel (list of
     index arrays) and sel_scores (list of score arrays), plus new_entries
@@ -56,14 +69,23 @@ def layer_step(kind, *, m, G, w, k, sm_scale, kv_fmt, rope_dim, idx_fmt, L, T,
     g_lo, g_hi = (L - T) // m, L // m
     new_g = range(g_lo, g_hi)
     if len(new_g):
-        e_kv = compress_entries(x_kv, x_pos0, W_kv, B_kv, m, G, new_g)
+        e_kv = compress_entries(x_kv, x_pos0, W_kv, B_kv, m, G, new_g, U_kv)
         _store_rows(kv, np.arange(g_lo, g_hi), e_kv, kv_fmt, rope_dim)
         if v is not None:
-            e_v = compress_entries(x_v, x_pos0, W_v, B_v, m, G, new_g)
+            e_v = compress_entries(x_v, x_pos0, W_v, B_v, m, G, new_g, U_v)
             _store_rows(v, np.arange(g_lo, g_hi), e_v, kv_fmt, rope_dim)
         if kind == "csa":
-            e_i = compress_entries(x_idx, x_pos0, W_idx, B_idx, m, G, new_g)
+            e_i = compress_entries(x_idx, x_pos0, W_idx, B_idx, m, G, new_g, U_idx)
             _store_rows(idx, np.arange(g_lo, g_hi), e_i, idx_fmt, 0)
+    token = sink_mode == "token"
+    if sink_mode not in ("logit", "token"):
+        raise ValueError(sink_mode)
+    if token:
+        sink = np.full(q.shape[1], -np.inf)  # no learned logit in this reading
+        if L - T <= 0:  # position 0 is one of the new tokens: keep its raw row
+            _store_rows(tok_kv, [0], np.asarray(x_kv)[-x_pos0][None], kv_fmt, rope_dim)
+            if tok_v is not None:
+                _store_rows(tok_v, [0], np.asarray(x_v)[-x_pos0][None], kv_fmt, rope_dim)
 
     win_cap = ring_kv.payload.shape[0]
     new_pos = np.arange(L - T, L)
@@ -91,13 +113,15 @@ def layer_step(kind, *, m, G, w, k, sm_scale, kv_fmt, rope_dim, idx_fmt, L, T,
         else:
             ent = np.arange(n)
         wpos = window_positions(p, w)
-        K_rows = np.concatenate([storage.decode(kv.rows(ent)),
-                                 storage.decode(ring_kv.rows(wpos % win_cap))], axis=0)
-        if v is None:
-            V_rows = K_rows
-        else:
-            V_rows = np.concatenate([storage.decode(v.rows(ent)),
-                                     storage.decode(ring_v.rows(wpos % win_cap))], axis=0)
+        parts_k = [storage.decode(kv.rows(ent)), storage.decode(ring_kv.rows(wpos % win_cap))]
+        parts_v = None if v is None else [storage.decode(v.rows(ent)),
+                                          storage.decode(ring_v.rows(wpos % win_cap))]
+        if token and not (len(wpos) and wpos[0] == 0):  # position 0 not in the window yet
+            parts_k.append(storage.decode(tok_kv.rows([0])))
+            if parts_v is not None:
+                parts_v.append(storage.decode(tok_v.rows([0])))
+        K_rows = np.concatenate(parts_k, axis=0)
+        V_rows = K_rows if v is None else np.concatenate(parts_v, axis=0)
         o, lse = joint_attention(q[i], K_rows, V_rows, sink, sm_scale)
         o = inverse_rope(o, p, rope_dim, out_rope_base)
         o_all.append(o)
