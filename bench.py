@@ -248,6 +248,102 @@ def index_dtype(layer_wls):
     return "".join(names.get(f, f + " (indexer), ") for f in sorted(fmts))
 
 
+# ------------------------------------------------- algorithmic work of a step
+# What one step of a layer must move and compute at least once, from the
+# shapes alone (the per-unit figures of the kernels' rooflines): every stored
+# row it reads once, every row it writes once, the queries and outputs once.
+
+def _kv_row_bytes(lw):
+    """Stored KV row with its scale."""
+    rope = lw.rope_dim if lw.kv_fmt == "kv" else 0
+    return L.row_bytes(lw.kv_fmt, lw.D, rope) + (4 if lw.kv_fmt != "f32" else 0)
+
+
+def _idx_row_bytes(lw):
+    """Stored indexer key with its scales (FP4: one byte per 16 values)."""
+    extra = {"fp4": lw.d_I // 16, "fp8": 4, "f32": 0}[lw.idx_fmt]
+    return L.row_bytes(lw.idx_fmt, lw.d_I) + extra
+
+
+def layer_step_bytes(lw):
+    """Algorithmic bytes of one step of a single layer over its B sequences."""
+    x_b = 2 if lw.x_dtype == "bf16" else 4
+    q_b = 2 if lw.q_dtype == "bf16" else 4
+    nv = 2 if lw.separate_v else 1            # K and V tensors
+    kv_row = _kv_row_bytes(lw)
+    T, m, G = lw.T, lw.m, lw.G
+    n_new = lw.L // m - (lw.L - T) // m       # entries the step pools
+    seq = T * lw.H * (lw.D + lw.Dv) * q_b     # queries in, outputs out
+    seq += (T + G - 1) * lw.D * x_b * nv      # raw rows of the closing groups and new tokens
+    seq += (n_new + T) * kv_row * nv          # new entries and window rows written
+    seq += min(T + lw.w - 1, lw.L) * kv_row * nv  # window rows read (distinct positions)
+    if lw.kind == "csa":
+        ik = _idx_row_bytes(lw)
+        seq += (lw.L // m) * ik                           # every visible indexer key, once
+        seq += (T + G - 1) * lw.d_I * x_b + n_new * ik    # its raw rows and new keys
+        seq += T * lw.H_I * (lw.d_I * q_b + 4)            # indexer queries and head weights
+        n_ent = lw.L // m
+        seq += min(T * min(lw.k, n_ent), n_ent) * kv_row * nv  # gathered entries (each stored row once)
+        seq += T * min(lw.k, n_ent) * 4                      # selection written
+    else:
+        seq += (lw.L // m) * kv_row * nv                  # every visible entry, once
+    layer = nv * (lw.D * lw.D * x_b + G * lw.D * 4) + lw.H * 4  # gates, biases, sink
+    if lw.kind == "csa":
+        layer += lw.d_I * lw.d_I * x_b + G * lw.d_I * 4
+    return lw.B * seq + layer
+
+
+def layer_step_flops(lw):
+    """Algorithmic flops of one step of a layer, by the operand type of the
+    contraction that carries them: {"fp4" / "fp8" / "f32": indexer scoring,
+    "bf16": attention (f16 MMA, the same tensor rate) and the gate GEMM}."""
+    out = {}
+    T, m = lw.T, lw.m
+    pos = [lw.L - T + t for t in range(T)]
+    vis = [(p + 1) // m for p in pos]
+    if lw.kind == "csa":
+        out[lw.idx_fmt] = lw.B * sum(vis) * 2 * lw.H_I * lw.d_I
+        rows = [min(lw.k, n) + min(lw.w, p + 1) for n, p in zip(vis, pos)]
+    else:
+        rows = [n + min(lw.w, p + 1) for n, p in zip(vis, pos)]
+    attn = lw.B * sum(rows) * 2 * lw.H * (lw.D + lw.Dv)
+    n_new = lw.L // m - (lw.L - T) // m
+    gate = lw.B * n_new * lw.G * 2 * (lw.D * lw.D * (2 if lw.separate_v else 1) +
+                                      (lw.d_I * lw.d_I if lw.kind == "csa" else 0))
+    out["bf16"] = out.get("bf16", 0) + attn + gate
+    return out
+
+
+def step_work(wl):
+    """(bytes, flops by type) of one step of a workload (both layers of a pair)."""
+    layers_wl = [wl.layer("csa"), wl.layer("hca")] if wl.kind == "pair" else [wl]
+    fl = {}
+    for lw in layers_wl:
+        for k, v in layer_step_flops(lw).items():
+            fl[k] = fl.get(k, 0) + v
+    return sum(layer_step_bytes(lw) for lw in layers_wl), fl
+
+
+def step_roofline(wl, ms_step, peaks):
+    """The whole step against its bound: decode steps against HBM (bytes /
+    time / measured copy bandwidth), chunked prefill against the tensor pipe
+    (sum of flops_i / peak_i over the contractions, divided by the time, with
+    the burst bf16 peak times the nominal ratio of each operand type: the
+    step lasts milliseconds, not seconds)."""
+    nbytes, fl = step_work(wl)
+    if wl.T >= 64:
+        bf = float(peaks["bf16_tflops"])
+        ideal_s = sum(v / (bf * TENSOR_RATIO.get(k, 1.0) * 1e12) for k, v in fl.items())
+        return {"bound": "tensor", "frac": round(ideal_s / (ms_step / 1e3), 4),
+                "ideal_ms": round(ideal_s * 1e3, 4), "ms_per_step": round(ms_step, 5),
+                "flops_by_type": fl, "peak": f"{peaks['source']} bf16_tflops {bf} x nominal ratio per type",
+                "algorithmic_bytes": nbytes}
+    gbs = nbytes / (ms_step / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": round(gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+            "frac": round(gbs / float(peaks["hbm_gbs"]), 4), "algorithmic_bytes": nbytes,
+            "ms_per_step": round(ms_step, 5), "peak_source": peaks["source"] + " hbm_gbs"}
+
+
 def recorded_traffic(kernel, workload, sha):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
     the current source of the kernel (else None)."""
@@ -307,6 +403,107 @@ def job_throughput(B, T, ws, steps, ms_total):
     """Queries per second of the whole job: the queries every rank answered
     over the slowest rank's time."""
     return B * T * ws * steps / (ms_total / 1e3)
+
+
+L2_BYTES = 126 * 2 ** 20
+SUB_WORKLOADS = (workloads.PAIR_DECODE_1M_B1.name, workloads.CSA_DECODE_128K.name,
+                 workloads.CSA_PREFILL_256K.name)
+
+
+def measure_sub(name, dev, peaks, warmup, target_s=0.4, max_steps=5000):
+    """One more workload timed in the same run: its own layers, warm-up,
+    clocks and timed steps (as many as fill about ``target_s``).  A step
+    whose working set fits in L2 is timed alone, with L2 flushed before it
+    (a 256 MiB buffer written, then a second one read, outside the step's
+    events); larger ones run back to back."""
+    wl = workloads.ALL[name]
+    layers_wl = [wl.layer("csa"), wl.layer("hca")] if wl.kind == "pair" else [wl]
+    layers = [Layer(lw, shard_seed(0, i), dev) for i, lw in enumerate(layers_wl)]
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for ly in layers:
+            ly.run(stream)
+
+    nbytes, _ = step_work(wl)
+    flush = nbytes < 2 * L2_BYTES
+    if flush:
+        fw = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        fr = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        fw.fill_(1)
+        fr.sum()
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    for ly in layers:
+        if int(ly.status.item()) != 0:
+            raise RuntimeError(f"device status {int(ly.status.item())} in {ly.wl.name}")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    est_ms = max(e0.elapsed_time(e1), 1e-3)
+    steps = int(min(max_steps, max(20, target_s * 1e3 / est_ms)))
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    n0 = L.kernel_launches()
+    if flush:
+        for i in range(steps):
+            flush_l2()
+            starts[i].record(stream)
+            step()
+            stops[i].record(stream)
+    else:
+        starts[0].record(stream)
+        for i in range(steps):
+            step()
+        stops[0].record(stream)
+    launches = L.kernel_launches() - n0
+    torch.cuda.synchronize()
+    t1 = time.time()
+    time.sleep(0.25)
+    clocks = sampler.stop(t0, t1)
+    if flush:
+        ms = float(np.mean([a.elapsed_time(b) for a, b in zip(starts, stops)]))
+    else:
+        ms = starts[0].elapsed_time(stops[0]) / steps
+    for ly in layers:
+        if int(ly.status.item()) != 0:
+            raise RuntimeError(f"device status {int(ly.status.item())} in {ly.wl.name}")
+    unit = "tokens/s" if wl.T >= 64 else "queries/s"
+    rec = {"workload": wl.name, "layers": [lw.name for lw in layers_wl], "batch": wl.B, "context": wl.L,
+           "new_tokens": wl.T, "steps": steps, "warmup": warmup, "ms_per_step": round(ms, 5),
+           "value": round(wl.B * wl.T / (ms / 1e3), 2), "unit": unit,
+           "step_roofline": step_roofline(wl, ms, peaks), "gpu_launches_per_step": launches / steps,
+           "clocks": clocks,
+           "l2": ("flushed before every step (256 MiB written, 256 MiB read; outside the step's events); "
+                  "the step's own events, mean over steps") if flush else
+                 "inputs larger than L2; steps back to back"}
+    del layers
+    if flush:
+        del fw, fr
+    torch.cuda.empty_cache()
+    return rec
+
+
+def workload_config(wl):
+    """The ``config`` object of a bench line (both arms)."""
+    layers_wl = [wl.layer("csa"), wl.layer("hca")] if wl.kind == "pair" else [wl]
+    nbytes, _ = step_work(wl)
+    return {"workload": wl.name, "layers": [lw.name for lw in layers_wl], "batch_per_gpu": wl.B,
+            "context": wl.L, "new_tokens": wl.T, "heads": wl.H, "kv_dim": wl.D, "top_k": wl.k, "window": wl.w,
+            "csa_entries": wl.L // wl.m, "hca_entries": wl.L // wl.m_hca if wl.kind == "pair" else None,
+            "l2": ("inputs larger than L2 (working set per step > 126 MB)" if nbytes > 2 * L2_BYTES
+                   else "working set fits in L2")}
 
 
 def run_lcsc(args):
@@ -391,16 +588,16 @@ def run_lcsc(args):
         if cw.T > 1:
             # chunked prefill: the scoring is a contraction of T queries x 64 heads
             # against every visible key; it is bound by the tensor pipe, whose
-            # rate for the key format is the measured sustained bf16 rate x the
-            # nominal ratio (the launch runs inside a multi-millisecond step)
+            # rate for the key format is the measured burst bf16 rate x the
+            # nominal ratio (the launch lasts milliseconds, not seconds)
             n_vis = sum((cw.L - cw.T + t + 1) // cw.m for t in range(cw.T))
             flops = cw.B * n_vis * 2 * cw.H_I * cw.d_I
             ratio = TENSOR_RATIO.get(cw.idx_fmt, 1.0)
-            peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * ratio
+            peak = float(peaks["bf16_tflops"]) * ratio
             achieved = flops / (score_ms / 1e3) / 1e12
             roof = dict(bound="tensor", achieved=round(achieved, 1), peak=round(peak, 1), unit="TFLOP/s",
                         frac=round(achieved / peak, 4), algorithmic_flops=flops,
-                        peak_source=f"{peaks['source']} bf16_tflops_sustained x {ratio:g} ({cw.idx_fmt} / bf16 nominal)",
+                        peak_source=f"{peaks['source']} bf16_tflops (burst) x {ratio:g} ({cw.idx_fmt} / bf16 nominal)",
                         **common)
         else:
             key_b = L.row_bytes(cw.idx_fmt, cw.d_I) + (cw.d_I // 16 if cw.idx_fmt == "fp4" else 4)
@@ -471,12 +668,12 @@ def run_lcsc(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": index_dtype(layers_wl) + "f16 MMA (attention), f32 accumulate and softmax",
         "data": "synthetic (seeded Gaussian entries with planted relevant blocks, drawn on device)",
-        "config": {"workload": wl.name, "layers": [lw.name for lw in layers_wl], "batch_per_gpu": wl.B,
-                   "context": wl.L, "heads": wl.H, "kv_dim": wl.D, "top_k": wl.k, "window": wl.w,
-                   "csa_entries": wl.L // wl.m, "hca_entries": wl.L // wl.m_hca if wl.kind == "pair" else None,
-                   "l2": "inputs larger than L2 (working set per step > 126 MB)"},
+        "config": workload_config(wl),
         "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
     }
+    line["step_roofline"] = step_roofline(wl, ms_step, measured_peaks())
+    if args.sub_records and ws == 1 and wl.name == DEFAULT_WORKLOAD:
+        line["sub_records"] = [measure_sub(n, dev, measured_peaks(), args.warmup) for n in SUB_WORKLOADS]
     if args.cpu_baseline and ws == 1:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_queries)
     return line
@@ -596,7 +793,7 @@ def run_reference(args):
         "ms_per_step": round(dt / steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded, numpy generator)",
-        "config": {"workload": wl.name, "layers": [lw.name for lw in layers_wl], "context": wl.L},
+        "config": workload_config(wl),
         "cpu_baseline": {"value": round(value, 5), "unit": "queries/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 5), "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -612,6 +809,8 @@ def main():
     ap.add_argument("--impl", default="lcsc", choices=["lcsc", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-sub-records", dest="sub_records", action="store_false",
+                    help="skip the 1M pair at B = 1, the 128K decode and the prefill step timed after the main line")
     ap.add_argument("--cpu-queries", type=int, default=2)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps

@@ -15,8 +15,19 @@
  *
  * Conventions for every call
  *  - Pointers marked (dev) are device pointers owned by the caller; the
- *    library never allocates device memory and keeps no state between
- *    calls.  Pointers marked (host) are read before the call returns.
+ *    library never allocates device memory.  Pointers marked (host) are
+ *    read before the call returns.
+ *  - State the library keeps for the life of the process: a count of the
+ *    kernels it has enqueued (lcsc_kernel_launches) and, per device, two
+ *    streams and three events of its own, created by the first fused CSA
+ *    step on that device (lcsc_csa_decode runs the indexer keys' pooling
+ *    and the query quantisation on them, joined back to the caller's
+ *    stream before the scoring).  Fused CSA steps on one device share
+ *    them, so steps issued on independent caller streams are ordered
+ *    against each other's side work; issue independent layers' CSA steps
+ *    on one stream, or accept that ordering.  Make the first fused CSA
+ *    call on a device before any stream capture.  The no-allocation call
+ *    below also keeps a fixed array per device.
  *  - Every call enqueues its kernels on `stream` (a cudaStream_t) and
  *    returns without synchronising.
  *  - On a non-zero return nothing has been enqueued.
@@ -44,7 +55,7 @@
 extern "C" {
 #endif
 
-#define LCSC_ABI_VERSION 2
+#define LCSC_ABI_VERSION 3
 
 /* Return codes. */
 #define LCSC_OK 0
@@ -57,6 +68,31 @@ extern "C" {
 #define LCSC_DEV_BAD_INDEX 1       /* an index outside [0, N(p)) was skipped */
 #define LCSC_DEV_BAD_LENGTH 2      /* a ctx_len smaller than T, or past the sizes of the call */
 #define LCSC_DEV_TIMEOUT 4         /* a kernel gave up a bounded wait (no result was written) */
+#define LCSC_DEV_RANGE 8           /* a stored KV row outside the tensor-core attention's range (below) */
+
+/* What the sink of a layer is (lcsc_params.sink_mode); "DeepSeek V4
+ * Architecture Explained", "How compress-then-sparsify attention works": a
+ * sink term lets each head leave part of its weight on no row.
+ *  LCSC_SINK_LOGIT: a learned logit sigma[h] per head whose value vector is
+ *                   zero: exp(sigma[h]) joins the softmax denominator only
+ *                   (the `sink` argument; NULL: no sink).
+ *  LCSC_SINK_TOKEN: the raw row of position 0 is one more member of every
+ *                   query's row set, once (nothing is added while the window
+ *                   already holds position 0).  The row lives in a one-row
+ *                   cache per sequence (`sink_kv`, and `sink_v` when V is
+ *                   separate) that a fused step fills when position 0 is
+ *                   one of its new tokens; `sink` must be NULL. */
+#define LCSC_SINK_LOGIT 0
+#define LCSC_SINK_TOKEN 1
+
+/* Where the compression gate's logits come from (lcsc_params.gate_src).
+ *  LCSC_GATE_PROJ:   z_j = x_j W + Bpos[place of j] with W [dim][dim].
+ *  LCSC_GATE_LOGITS: z_j = u_j + Bpos[place of j], u_j a float32 logit row
+ *                    per token given by the caller in place of x_j W (a
+ *                    token of two overlapping groups gets the bias of its
+ *                    place in each). */
+#define LCSC_GATE_PROJ 0
+#define LCSC_GATE_LOGITS 1
 
 /* Row storage formats ("DeepSeek V4 Architecture Explained", Key numbers,
  * row "KV storage precision"; "Inside DeepSeek-V4", section 1, FP4 indexer).
@@ -113,6 +149,8 @@ typedef struct lcsc_params {
    * out_rope_dim: a multiple of 4, <= v_dim, when on. */
   int32_t out_rope_dim;
   float out_rope_base;
+  int32_t sink_mode;   /* LCSC_SINK_LOGIT or LCSC_SINK_TOKEN */
+  int32_t gate_src;    /* LCSC_GATE_PROJ or LCSC_GATE_LOGITS */
 } lcsc_params;
 
 /* Stored rows of one tensor for B sequences (dev pointers).
@@ -160,7 +198,9 @@ int64_t lcsc_row_bytes(int32_t format, int32_t dim, int32_t rope_dim);
  *             tok_begin - (G - m) .. tok_end - 1, n_x = tok_end - tok_begin + G - m
  *             (rows at negative positions are never read).
  *   tok_begin % m == 0; every group that ends before tok_end is written.
- *   w_gate (dev): [dim][dim] x_dtype.  b_pos (dev): [G][dim] float32.
+ *   w_gate (dev): LCSC_GATE_PROJ: W [dim][dim] x_dtype; LCSC_GATE_LOGITS:
+ *             the logit rows u [B][n_x][dim] float32 of the same positions
+ *             as x.  b_pos (dev): [G][dim] float32.
  *   entries: written rows; window (nullable): the window ring, which also
  *   receives the raw rows of positions max(tok_begin, tok_end - capacity) ..
  *   tok_end - 1 (KV / V only).
@@ -231,17 +271,30 @@ int32_t lcsc_csa_index_topk_noalloc(const lcsc_params* p, const void* q_idx, con
 
 /* --------------------------------------------------------- attention (a5-a7)
  * One joint softmax per query head over a row set S (entries plus window
- * rows), with a per-head sink logit sigma[h] that only adds exp(sigma) to
- * the denominator ("an attention-sink term that lets a head's attention
- * scores sum to less than one"):
- *     l_j = sm_scale * q[h] . K_j
+ * rows, plus the position-0 row with LCSC_SINK_TOKEN), with a per-head sink
+ * logit sigma[h] (LCSC_SINK_LOGIT) that only adds exp(sigma) to the
+ * denominator ("DeepSeek V4 Architecture Explained", "How
+ * compress-then-sparsify attention works"):
+ *     l_j = sm_scale * q[h] . K_j          (sm_scale > 0)
  *     o[h] = sum_j e^{l_j - M} V_j / (e^{sigma[h] - M} + sum_j e^{l_j - M})
  * K_j, V_j are dequantised stored rows; V = K unless `v` is given.
  *   q (dev): [B][T][H][D] q_dtype.   out (dev): [B][T][H][Dv] q_dtype.
  *   lse (dev, nullable): [B][T][H] float32 = M + log(denominator).
- *   sink (dev, nullable): [H] float32; NULL means no sink.
+ *   sink (dev, nullable): [H] float32 sigma; NULL means no sink (must be
+ *   NULL with LCSC_SINK_TOKEN).
+ *   sink_kv, sink_v (LCSC_SINK_TOKEN only, else nullable and unread): the
+ *   stored row of position 0 of each sequence, capacity 1 ([B][1] rows);
+ *   sink_v only when V is separate.
  *   kv, v (v nullable): stored entries; win_kv, win_v (win_v nullable): the
  *   window rings, which must hold positions max(0, p - w + 1) .. p.
+ * Range of the 512-dim FP8 + BF16 path (64 heads; its products run on the
+ * tensor cores in f16 with float32 sums): every query is used at any
+ * finite bf16 magnitude (each head is scaled by a power of two into the
+ * f16 range, and the scale is undone on its logits); a dequantised KV value
+ * (E4M3 code x row scale, or a BF16 RoPE dim) is held as f16, so a row
+ * whose scale exceeds 65504 / 448 or whose BF16 dims exceed 65504 in
+ * magnitude sets LCSC_DEV_RANGE (its result is then not defined), and
+ * values below 2^-14 keep f16 subnormal precision.
  * lcsc_csa_sparse_attn: S = {idx[b][t][j] >= 0} U window (idx (dev):
  *   [B][T][k] int32, e.g. from lcsc_csa_index_topk).
  * lcsc_hca_dense_attn: S = {all g < N(p)} U window. */
@@ -250,12 +303,14 @@ int32_t lcsc_attn_workspace_size(const lcsc_params* p, int64_t B, int64_t T, int
 int32_t lcsc_csa_sparse_attn(const lcsc_params* p, const void* q, const lcsc_cache* kv,
                              const lcsc_cache* v, const lcsc_cache* win_kv,
                              const lcsc_cache* win_v, const int32_t* idx, const float* sink,
+                             const lcsc_cache* sink_kv, const lcsc_cache* sink_v,
                              const int32_t* ctx_len, int64_t B, int64_t T, void* out, float* lse,
                              void* workspace, size_t workspace_bytes, int32_t* status,
                              void* stream);
 int32_t lcsc_hca_dense_attn(const lcsc_params* p, const void* q, const lcsc_cache* kv,
                             const lcsc_cache* v, const lcsc_cache* win_kv, const lcsc_cache* win_v,
-                            const float* sink, const int32_t* ctx_len, int64_t B, int64_t T,
+                            const float* sink, const lcsc_cache* sink_kv, const lcsc_cache* sink_v,
+                            const int32_t* ctx_len, int64_t B, int64_t T,
                             int64_t n_max, void* out, float* lse, void* workspace,
                             size_t workspace_bytes, int32_t* status, void* stream);
 
@@ -269,7 +324,11 @@ int32_t lcsc_hca_dense_attn(const lcsc_params* p, const void* q, const lcsc_cach
  * [B][T + G - 1][dim] x_dtype for positions L - (T + G - 1) .. L - 1.
  * The caches must already hold every entry below floor((L - T) / m) and the
  * rings the rows of positions L - T - w + 1 .. L - T - 1; the rings need at
- * least T + w - 1 rows. */
+ * least T + w - 1 rows.  With LCSC_SINK_TOKEN, sink_kv (and sink_v) must
+ * hold the row of position 0 unless L - T <= 0, in which case the step
+ * stores it there.  With LCSC_GATE_LOGITS, w_kv / w_v / w_idx are the
+ * float32 gate logit rows [B][T + G - 1][dim] of the same positions as the
+ * raw rows. */
 typedef struct lcsc_step {
   int64_t B, T;
   int64_t n_max;                /* >= floor(L / m) for every sequence */
@@ -277,7 +336,7 @@ typedef struct lcsc_step {
   const void* x_kv;             /* raw rows of the KV latent (or K) */
   const void* x_v;              /* raw rows of a separate V, or NULL */
   const void* x_idx;            /* raw rows of the indexer keys (CSA) */
-  const void* w_kv;  const float* b_kv;    /* gates of each tensor: W [dim][dim], Bpos [G][dim] */
+  const void* w_kv;  const float* b_kv;    /* gates of each tensor: W [dim][dim] (or logits), Bpos [G][dim] */
   const void* w_v;   const float* b_v;
   const void* w_idx; const float* b_idx;
   lcsc_cache kv, v, idx_keys;   /* entries (v.data NULL when V = K) */
@@ -299,6 +358,7 @@ typedef struct lcsc_step {
    * compression, 2 after attention. */
   void* const* events;
   int32_t n_events;
+  lcsc_cache sink_kv, sink_v;   /* LCSC_SINK_TOKEN: the position-0 rows ([B][1]); else unread */
 } lcsc_step;
 
 int32_t lcsc_step_workspace_size(const lcsc_params* p, int32_t csa, int64_t B, int64_t T,

@@ -64,7 +64,9 @@ int32_t check_params(const lcsc_params* p) {
   if (p->idx_format == LCSC_FMT_KV) return LCSC_ERR_INVALID_ARG;
   if (p->x_dtype != LCSC_DT_F32 && p->x_dtype != LCSC_DT_BF16) return LCSC_ERR_INVALID_ARG;
   if (p->q_dtype != LCSC_DT_F32 && p->q_dtype != LCSC_DT_BF16) return LCSC_ERR_INVALID_ARG;
-  if (!(p->sm_scale == p->sm_scale)) return LCSC_ERR_INVALID_ARG;
+  if (!(p->sm_scale > 0.f) || p->sm_scale == INFINITY) return LCSC_ERR_INVALID_ARG;
+  if (p->sink_mode != LCSC_SINK_LOGIT && p->sink_mode != LCSC_SINK_TOKEN) return LCSC_ERR_INVALID_ARG;
+  if (p->gate_src != LCSC_GATE_PROJ && p->gate_src != LCSC_GATE_LOGITS) return LCSC_ERR_INVALID_ARG;
   if (!(p->out_rope_base >= 0.f) || p->out_rope_base == INFINITY) return LCSC_ERR_INVALID_ARG;
   if (p->out_rope_base > 0.f &&
       (p->out_rope_dim < 4 || p->out_rope_dim % 4 != 0 || p->out_rope_dim > p->v_dim))
@@ -149,7 +151,7 @@ void plan_index(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max, Carve
 
 void plan_attn(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max, bool dense, Carve& cv,
                AttnLaunch* L) {
-  const int64_t max_rows = (dense ? n_max : p->top_k) + p->window;
+  const int64_t max_rows = (dense ? n_max : p->top_k) + p->window + (p->sink_mode == LCSC_SINK_TOKEN ? 1 : 0);
   int splits, rps;
   if (p->kv_format == LCSC_FMT_KV && p->head_dim == 512 && p->n_heads == 64) {
     // tensor-core path: one CTA per (query, split) for all heads, one wave
@@ -255,6 +257,7 @@ static int32_t compress_impl(const lcsc_params* p, int32_t tensor, const void* x
   L.x_dtype = p->x_dtype;
   L.n_x = tok_end - tok_begin + p->group_len - p->m;
   L.w = w_gate;
+  L.gate_logits = p->gate_src == LCSC_GATE_LOGITS;
   L.bpos = b_pos;
   L.dim = f.dim;
   L.B = (int)B;
@@ -307,7 +310,8 @@ int32_t lcsc_index_topk_workspace_size(const lcsc_params* p, int64_t B, int64_t 
                                        size_t* bytes) {
   int32_t st = check_params(p);
   if (st) return st;
-  if (!bytes || B < 1 || T < 1 || n_max < 0) return LCSC_ERR_INVALID_ARG;
+  if (!bytes || B < 1 || T < 1 || T > 65535 || B > 65535 / T || n_max < 0 || n_max > ((int64_t)1 << 40))
+    return LCSC_ERR_INVALID_ARG;
   Carve cv{nullptr};
   plan_index(p, B, T, n_max, cv, nullptr);
   *bytes = cv.used;
@@ -323,7 +327,7 @@ static int32_t index_setup(const lcsc_params* p, const void* q_idx, const float*
   if (!q_idx || !w_idx || !ctx_len || !out_idx) return LCSC_ERR_INVALID_ARG;
   if (!aligned16(q_idx) || !aligned16(w_idx) || !aligned16(out_idx)) return LCSC_ERR_INVALID_ARG;
   if (out_score && !aligned16(out_score)) return LCSC_ERR_INVALID_ARG;
-  if (B < 1 || T < 1 || B * T > 65535 || n_max < 0) return LCSC_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || T > 65535 || B > 65535 / T || n_max < 0) return LCSC_ERR_INVALID_ARG;
   RowFmt f;
   int32_t st;
   if ((st = tensor_fmt(p, LCSC_TENSOR_IDX, &f))) return st;
@@ -371,7 +375,8 @@ int32_t lcsc_attn_workspace_size(const lcsc_params* p, int64_t B, int64_t T, int
                                  int32_t dense, size_t* bytes) {
   int32_t st = check_params(p);
   if (st) return st;
-  if (!bytes || B < 1 || T < 1 || n_max < 0) return LCSC_ERR_INVALID_ARG;
+  if (!bytes || B < 1 || T < 1 || T > 65535 || B > 65535 / T || n_max < 0 || n_max > ((int64_t)1 << 40))
+    return LCSC_ERR_INVALID_ARG;
   Carve cv{nullptr};
   plan_attn(p, B, T, n_max, dense != 0, cv, nullptr);
   *bytes = cv.used;
@@ -380,14 +385,15 @@ int32_t lcsc_attn_workspace_size(const lcsc_params* p, int64_t B, int64_t T, int
 
 static int32_t attn_setup(const lcsc_params* p, const void* q, const lcsc_cache* kv,
                           const lcsc_cache* v, const lcsc_cache* win_kv, const lcsc_cache* win_v,
-                          const int32_t* idx, const float* sink, const int32_t* ctx_len, int64_t B,
+                          const int32_t* idx, const float* sink, const lcsc_cache* sink_kv,
+                          const lcsc_cache* sink_v, const int32_t* ctx_len, int64_t B,
                           int64_t T, int64_t n_max, void* out, float* lse, Carve& cv,
                           size_t ws_bytes, int32_t* status, AttnLaunch* L) {
   if (!kv_supported(p)) return LCSC_ERR_UNSUPPORTED;
   if (!q || !ctx_len || !out || !aligned16(q) || !aligned16(out)) return LCSC_ERR_INVALID_ARG;
   if (lse && !aligned16(lse)) return LCSC_ERR_INVALID_ARG;
   if (sink && ((uintptr_t)sink & 3u)) return LCSC_ERR_INVALID_ARG;
-  if (B < 1 || T < 1 || B * T > 65535 || n_max < 0) return LCSC_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || T > 65535 || B > 65535 / T || n_max < 0) return LCSC_ERR_INVALID_ARG;
   const bool sep = v && v->data;
   if (sep != (win_v && win_v->data)) return LCSC_ERR_INVALID_ARG;
   if (sep && p->kv_format != LCSC_FMT_F32) return LCSC_ERR_UNSUPPORTED;
@@ -407,6 +413,12 @@ static int32_t attn_setup(const lcsc_params* p, const void* q, const lcsc_cache*
   }
   if (n_max > kv->capacity) return LCSC_ERR_INVALID_ARG;
   if (p->window > 0 && win_kv->capacity < T + p->window - 1) return LCSC_ERR_INVALID_ARG;
+  if (p->sink_mode == LCSC_SINK_TOKEN) {  // the stored position-0 row replaces the sink logit
+    if (sink) return LCSC_ERR_INVALID_ARG;
+    if ((st = make_view(sink_kv, fk, ns, &L->tok_kv))) return st;
+    if (sep && (st = make_view(sink_v, fv, ns, &L->tok_v))) return st;
+    L->sink_token = 1;
+  }
   plan_attn(p, B, T, n_max, idx == nullptr, cv, L);
   if (!cv.base || !aligned16(cv.base) || ws_bytes < cv.used) return LCSC_ERR_WORKSPACE;
   L->q = q;
@@ -435,6 +447,7 @@ static int32_t attn_setup(const lcsc_params* p, const void* q, const lcsc_cache*
 int32_t lcsc_csa_sparse_attn(const lcsc_params* p, const void* q, const lcsc_cache* kv,
                              const lcsc_cache* v, const lcsc_cache* win_kv,
                              const lcsc_cache* win_v, const int32_t* idx, const float* sink,
+                             const lcsc_cache* sink_kv, const lcsc_cache* sink_v,
                              const int32_t* ctx_len, int64_t B, int64_t T, void* out, float* lse,
                              void* ws, size_t ws_bytes, int32_t* status, void* stream) {
   int32_t st = check_params(p);
@@ -442,8 +455,8 @@ int32_t lcsc_csa_sparse_attn(const lcsc_params* p, const void* q, const lcsc_cac
   if (!idx || !aligned16(idx) || p->top_k < 1) return LCSC_ERR_INVALID_ARG;
   Carve cv{reinterpret_cast<uint8_t*>(ws)};
   AttnLaunch L;
-  if ((st = attn_setup(p, q, kv, v, win_kv, win_v, idx, sink, ctx_len, B, T, kv ? kv->capacity : 0,
-                       out, lse, cv, ws_bytes, status, &L)))
+  if ((st = attn_setup(p, q, kv, v, win_kv, win_v, idx, sink, sink_kv, sink_v, ctx_len, B, T,
+                       kv ? kv->capacity : 0, out, lse, cv, ws_bytes, status, &L)))
     return st;
   cudaError_t e = launch_attention(L, (cudaStream_t)stream);
   return e == cudaSuccess ? LCSC_OK : cuda_fail(e);
@@ -451,15 +464,15 @@ int32_t lcsc_csa_sparse_attn(const lcsc_params* p, const void* q, const lcsc_cac
 
 int32_t lcsc_hca_dense_attn(const lcsc_params* p, const void* q, const lcsc_cache* kv,
                             const lcsc_cache* v, const lcsc_cache* win_kv, const lcsc_cache* win_v,
-                            const float* sink, const int32_t* ctx_len, int64_t B, int64_t T,
-                            int64_t n_max, void* out, float* lse, void* ws, size_t ws_bytes,
-                            int32_t* status, void* stream) {
+                            const float* sink, const lcsc_cache* sink_kv, const lcsc_cache* sink_v,
+                            const int32_t* ctx_len, int64_t B, int64_t T, int64_t n_max, void* out,
+                            float* lse, void* ws, size_t ws_bytes, int32_t* status, void* stream) {
   int32_t st = check_params(p);
   if (st) return st;
   Carve cv{reinterpret_cast<uint8_t*>(ws)};
   AttnLaunch L;
-  if ((st = attn_setup(p, q, kv, v, win_kv, win_v, nullptr, sink, ctx_len, B, T, n_max, out, lse,
-                       cv, ws_bytes, status, &L)))
+  if ((st = attn_setup(p, q, kv, v, win_kv, win_v, nullptr, sink, sink_kv, sink_v, ctx_len, B, T, n_max,
+                       out, lse, cv, ws_bytes, status, &L)))
     return st;
   cudaError_t e = launch_attention(L, (cudaStream_t)stream);
   return e == cudaSuccess ? LCSC_OK : cuda_fail(e);
@@ -471,7 +484,8 @@ int32_t lcsc_step_workspace_size(const lcsc_params* p, int32_t csa, int64_t B, i
                                  int64_t n_max, size_t* bytes) {
   int32_t st = check_params(p);
   if (st) return st;
-  if (!bytes || B < 1 || T < 1 || n_max < 0) return LCSC_ERR_INVALID_ARG;
+  if (!bytes || B < 1 || T < 1 || T > 65535 || B > 65535 / T || n_max < 0 || n_max > ((int64_t)1 << 40))
+    return LCSC_ERR_INVALID_ARG;
   Carve cv{nullptr};
   const int64_t n_new = new_entries_max(T, p->m);
   plan_compress(p, B, n_new, p->head_dim, cv, nullptr);
@@ -488,8 +502,8 @@ int32_t lcsc_step_workspace_size(const lcsc_params* p, int32_t csa, int64_t B, i
 
 static int32_t step_compress(const lcsc_params* p, const lcsc_step* s, int32_t tensor,
                              const void* x, const void* w, const float* bpos,
-                             const lcsc_cache* ent, const lcsc_cache* win, Carve& cv,
-                             int32_t* status, CompressLaunch* L) {
+                             const lcsc_cache* ent, const lcsc_cache* win, const lcsc_cache* tok,
+                             Carve& cv, int32_t* status, CompressLaunch* L) {
   RowFmt f;
   int32_t st;
   if ((st = tensor_fmt(p, tensor, &f))) return st;
@@ -499,6 +513,7 @@ static int32_t step_compress(const lcsc_params* p, const lcsc_step* s, int32_t t
   memset(L, 0, sizeof(*L));
   if ((st = make_view(ent, f, needs_scale(f.fmt), &L->entries))) return st;
   if (win && (st = make_view(win, f, needs_scale(f.fmt), &L->window))) return st;
+  if (tok && (st = make_view(tok, f, needs_scale(f.fmt), &L->sink_tok))) return st;
   if (s->n_max > ent->capacity) return LCSC_ERR_INVALID_ARG;
   const int64_t n_new = new_entries_max(s->T, p->m);
   plan_compress(p, s->B, n_new, f.dim, cv, &L->pooled);
@@ -506,6 +521,7 @@ static int32_t step_compress(const lcsc_params* p, const lcsc_step* s, int32_t t
   L->x_dtype = p->x_dtype;
   L->n_x = s->T + p->group_len - 1;
   L->w = w;
+  L->gate_logits = p->gate_src == LCSC_GATE_LOGITS;
   L->bpos = bpos;
   L->dim = f.dim;
   L->B = (int)s->B;
@@ -550,7 +566,7 @@ static int32_t step_impl(const lcsc_params* p, const lcsc_step* s, void* ws, siz
                          int32_t* status, void* stream, bool csa) {
   int32_t st = check_params(p);
   if (st) return st;
-  if (!s || s->B < 1 || s->T < 1 || s->B * s->T > 65535 || s->n_max < 0 || !s->ctx_len)
+  if (!s || s->B < 1 || s->T < 1 || s->T > 65535 || s->B > 65535 / s->T || s->n_max < 0 || !s->ctx_len)
     return LCSC_ERR_INVALID_ARG;
   if (p->group_len > 128) return LCSC_ERR_UNSUPPORTED;
   if (csa && (!idx_supported(p) || p->top_k < 1)) return csa && p->top_k < 1 ? LCSC_ERR_INVALID_ARG : LCSC_ERR_UNSUPPORTED;
@@ -562,12 +578,13 @@ static int32_t step_impl(const lcsc_params* p, const lcsc_step* s, void* ws, siz
 
   Carve cv{reinterpret_cast<uint8_t*>(ws)};
   CompressLaunch ck, cvv, ci;
-  if ((st = step_compress(p, s, LCSC_TENSOR_KV, s->x_kv, s->w_kv, s->b_kv, &s->kv, &s->win_kv, cv,
-                          status, &ck)))
+  const bool tok = p->sink_mode == LCSC_SINK_TOKEN;
+  if ((st = step_compress(p, s, LCSC_TENSOR_KV, s->x_kv, s->w_kv, s->b_kv, &s->kv, &s->win_kv,
+                          tok ? &s->sink_kv : nullptr, cv, status, &ck)))
     return st;
   if (sep) {
-    if ((st = step_compress(p, s, LCSC_TENSOR_V, s->x_v, s->w_v, s->b_v, &s->v, &s->win_v, cv, status,
-                            &cvv)))
+    if ((st = step_compress(p, s, LCSC_TENSOR_V, s->x_v, s->w_v, s->b_v, &s->v, &s->win_v,
+                            tok ? &s->sink_v : nullptr, cv, status, &cvv)))
       return st;
   } else {
     plan_compress(p, s->B, new_entries_max(s->T, p->m), p->v_dim, cv, nullptr);
@@ -576,7 +593,7 @@ static int32_t step_impl(const lcsc_params* p, const lcsc_step* s, void* ws, siz
   int32_t* sel = nullptr;
   if (csa) {
     if ((st = step_compress(p, s, LCSC_TENSOR_IDX, s->x_idx, s->w_idx, s->b_idx, &s->idx_keys,
-                            nullptr, cv, status, &ci)))
+                            nullptr, nullptr, cv, status, &ci)))
       return st;
     // the selection buffer: the caller's out_idx, else workspace (planned either way)
     int32_t* sel_ws = cv.take<int32_t>((size_t)s->B * s->T * p->top_k);
@@ -588,8 +605,8 @@ static int32_t step_impl(const lcsc_params* p, const lcsc_step* s, void* ws, siz
   }
   AttnLaunch al;
   if ((st = attn_setup(p, s->q, &s->kv, sep ? &s->v : nullptr, &s->win_kv, sep ? &s->win_v : nullptr,
-                       sel, s->sink, s->ctx_len, s->B, s->T, s->n_max, s->out, s->lse, cv,
-                       (size_t)-1, status, &al)))
+                       sel, s->sink, &s->sink_kv, sep ? &s->sink_v : nullptr, s->ctx_len, s->B, s->T,
+                       s->n_max, s->out, s->lse, cv, (size_t)-1, status, &al)))
     return st;
   if (ws_bytes < cv.used) return LCSC_ERR_WORKSPACE;
 
@@ -697,7 +714,11 @@ extern "C" int32_t lcsc_csa_index_topk_noalloc(const lcsc_params* p, const void*
                                                int32_t* status, void* stream) {
   int32_t st = check_params(p);
   if (st) return st;
-  if (B < 1 || T < 1 || n_max < 0) return LCSC_ERR_INVALID_ARG;
+  // the limits index_setup applies, checked before the plan's size products
+  // (division: B * T itself cannot overflow), so that the total compared
+  // with the fixed scratch size is exact
+  if (B < 1 || T < 1 || n_max < 0 || T > 65535 || B > 65535 / T || n_max > ((int64_t)1 << 40))
+    return LCSC_ERR_INVALID_ARG;
   Carve need{nullptr};
   plan_index(p, B, T, n_max, need, nullptr);
   if (need.used > (size_t)LCSC_NOALLOC_SCRATCH_BYTES) return LCSC_ERR_WORKSPACE;

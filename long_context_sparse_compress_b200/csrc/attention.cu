@@ -28,6 +28,7 @@ struct QueryRows {
   int64_t p, n_vis;      // position, visible entries
   int64_t n_ent_slots;   // entry slots (k for CSA, n_vis for HCA)
   int64_t w_lo, n_win;   // window positions w_lo .. w_lo + n_win - 1
+  int64_t n_tok;         // 1: the stored position-0 row follows the window
   bool ok;
 };
 
@@ -42,6 +43,8 @@ __device__ __forceinline__ QueryRows query_rows(const AttnLaunch& a, int b, int 
   r.w_lo = r.p - a.w + 1 > 0 ? r.p - a.w + 1 : 0;
   r.n_win = r.ok ? r.p - r.w_lo + 1 : 0;
   if (a.w == 0) r.n_win = 0;
+  // sink token: position 0 joins once, unless the window already holds it
+  r.n_tok = (r.ok && a.sink_token && !(r.n_win > 0 && r.w_lo == 0)) ? 1 : 0;
   return r;
 }
 
@@ -97,7 +100,7 @@ __global__ void __launch_bounds__(kThreads) attn_partial_kernel(AttnLaunch a) {
   float* ls = ms + HPC;                    // running sum [HPC]
   float* al = ls + HPC;                    // rescale factor [HPC]
   __shared__ int64_t rows_s[kTile];
-  __shared__ int8_t src_s[kTile];          // 0 invalid, 1 entry, 2 window
+  __shared__ int8_t src_s[kTile];          // 0 invalid, 1 entry, 2 window, 3 position-0 row
 
   const int list = blockIdx.z;
   const int b = list / a.T, t = list % a.T;
@@ -106,7 +109,7 @@ __global__ void __launch_bounds__(kThreads) attn_partial_kernel(AttnLaunch a) {
   const QueryRows qr = query_rows(a, b, t);
   if (!qr.ok && tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 && a.status)
     atomicOr(a.status, LCSC_DEV_BAD_LENGTH);
-  const int64_t total = qr.ok ? qr.n_ent_slots + qr.n_win : 0;
+  const int64_t total = qr.ok ? qr.n_ent_slots + qr.n_win + qr.n_tok : 0;
   const int64_t s_lo = (int64_t)blockIdx.x * a.rows_per_split;
   int64_t s_hi = s_lo + a.rows_per_split;
   if (s_hi > total) s_hi = total;
@@ -141,9 +144,12 @@ __global__ void __launch_bounds__(kThreads) attn_partial_kernel(AttnLaunch a) {
           } else if (g != -1 || !a.idx) {
             if (a.status) atomicOr(a.status, LCSC_DEV_BAD_INDEX);
           }
-        } else {
+        } else if (slot < qr.n_ent_slots + qr.n_win) {
           src = 2;
           row = (qr.w_lo + (slot - qr.n_ent_slots)) % a.win_kv.capacity;
+        } else {
+          src = 3;
+          row = 0;
         }
       }
       rows_s[tid] = row;
@@ -160,6 +166,9 @@ __global__ void __launch_bounds__(kThreads) attn_partial_kernel(AttnLaunch a) {
       } else if (src == 2) {
         load_row<KVFMT, D>(a.win_kv, b, rows_s[j], ks + j * KS, lt, 8);
         if (kSepV) load_row<KVFMT, DV>(a.win_v, b, rows_s[j], vs + j * VS, lt, 8);
+      } else if (src == 3) {
+        load_row<KVFMT, D>(a.tok_kv, b, 0, ks + j * KS, lt, 8);
+        if (kSepV) load_row<KVFMT, DV>(a.tok_v, b, 0, vs + j * VS, lt, 8);
       }
     }
     __syncthreads();

@@ -69,7 +69,10 @@ constexpr int OFF_MASK = OFF_NRM + 32;          // uint32 [2][2] valid-row bits
 constexpr int OFF_TM = OFF_MASK + 16;
 constexpr int OFF_ABORT = OFF_TM + 4;
 constexpr int OFF_LSTOP = OFF_ABORT + 4;
-constexpr int SMEM = OFF_LSTOP + 8 + 1024;
+constexpr int OFF_QSC = OFF_LSTOP + 4;          // float [64]: per-head amax of q, then its power-of-two scale
+constexpr int SMEM = OFF_QSC + kH * 4 + 1024;
+// Largest row scale whose E4M3 codes (|code| <= 448) stay finite as f16.
+constexpr float kMaxRowScale = 65504.f / 448.f;
 static_assert(kH * kOS * 4 <= OFF_BAR - OFF_K, "the staged partial O fits in the K and P buffers");
 
 // Byte offset of (row, byte) in a [rows][128 B] block with the 128-byte swizzle
@@ -93,6 +96,7 @@ __device__ __forceinline__ float ex2(float x) {
 
 struct Rows {
   int64_t n_vis, n_ent_slots, w_lo, n_win;
+  int64_t n_tok;  // 1: the stored position-0 row (sink token) follows the window
   bool ok;
 };
 
@@ -105,6 +109,7 @@ __device__ __forceinline__ Rows rows_of(const AttnLaunch& a, int b, int t) {
   r.n_ent_slots = a.idx ? a.k : r.n_vis;
   r.w_lo = p - a.w + 1 > 0 ? p - a.w + 1 : 0;
   r.n_win = (r.ok && a.w > 0) ? p - r.w_lo + 1 : 0;
+  r.n_tok = (r.ok && a.sink_token && !(r.n_win > 0 && r.w_lo == 0)) ? 1 : 0;
   return r;
 }
 
@@ -134,17 +139,19 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
   uint32_t* tm_slot = reinterpret_cast<uint32_t*>(sm + OFF_TM);
   volatile int* abort = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
   volatile int* lstop = reinterpret_cast<volatile int*>(sm + OFF_LSTOP);  // loader-group decision
+  float* qsc_s = reinterpret_cast<float*>(sm + OFF_QSC);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int list = blockIdx.y;
   const int b = list / a.T, t = list % a.T;
   const Rows qr = rows_of(a, b, t);
   if (!qr.ok && tid == 0 && blockIdx.x == 0 && a.status) atomicOr(a.status, LCSC_DEV_BAD_LENGTH);
-  const int64_t total = qr.ok ? qr.n_ent_slots + qr.n_win : 0;
+  const int64_t total = qr.ok ? qr.n_ent_slots + qr.n_win + qr.n_tok : 0;
   const int64_t s_lo = (int64_t)blockIdx.x * a.rows_per_split;
   const int64_t s_hi = s_lo + a.rows_per_split < total ? s_lo + a.rows_per_split : total;
   const int ntiles = s_hi > s_lo ? (int)((s_hi - s_lo + kTR - 1) / kTR) : 0;
 
+  if (tid < kH) qsc_s[tid] = 0.f;  // per-head amax of q (non-negative: compared as integers)
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&k_full[i], 1);
@@ -159,41 +166,82 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
   if (warp == kMmaWarp) tmem_alloc(tm_slot, 512);
 
   // ---- Q (64 x 512) -> f16, K-major swizzled blocks of 64 dims (all threads;
-  // bf16 rows: every 16-byte load of a thread in flight at once)
+  // bf16 rows: every 16-byte load of a thread in flight at once).  Each head
+  // is multiplied by a power of two that puts its largest |q| in
+  // [2^14, 2^15), so that any finite query keeps f16 precision; the softmax
+  // multiplies that head's logits back (qsc_s holds 2^e per head).
   constexpr int kQChunks = kH * (kD / 8), kQIter = (kQChunks + kThr - 1) / kThr;
-  auto q_store = [&](int i, const float (&v)[8]) {
-    const int h = i / (kD / 8), d0 = (i % (kD / 8)) * 8;
-    *reinterpret_cast<uint4*>(sm + OFF_Q + (d0 / 64) * KB_Q + swz(h, (d0 % 64) * 2)) =
-        make_uint4(pack_h2(v[0], v[1]), pack_h2(v[2], v[3]), pack_h2(v[4], v[5]), pack_h2(v[6], v[7]));
+  static_assert(kThr % 64 == 0 && (kD / 8) == 64 && kQChunks % kThr == 0,
+                "the lanes of a warp share one head per chunk round; every thread has kQIter chunks");
+  // the multiplier 2^-e of head h from its amax (0: 1)
+  auto q_mult = [&](int h) -> float {
+    const int bits = __float_as_int(qsc_s[h]);
+    if (bits == 0) return 1.f;
+    int ex = ((bits >> 23) & 0xff) - 127 - 14;  // amax in [2^(ex+14), 2^(ex+15)) (normal amax)
+    ex = ex < -126 ? -126 : (ex > 126 ? 126 : ex);
+    return __int_as_float((127 - ex) << 23);
   };
-  if (a.q_dtype == LCSC_DT_BF16) {
-    const uint4* q4 = reinterpret_cast<const uint4*>(a.q) + (int64_t)list * a.H * (kD / 8);
+  // Pass 1: each chunk's bf16 bits go to their final place in shared memory
+  // (f16 and bf16 chunks have the same size) and its amax to the head's slot;
+  // pass 2 converts every chunk in place once the head's scale is known.
+  // fp32 rows are read from memory in both passes.
+  const bool q_bf = a.q_dtype == LCSC_DT_BF16;
+  auto q_addr = [&](int i) {
+    const int h = i / (kD / 8), d0 = (i % (kD / 8)) * 8;
+    return reinterpret_cast<uint4*>(sm + OFF_Q + (d0 / 64) * KB_Q + swz(h, (d0 % 64) * 2));
+  };
+  auto f32_chunk = [&](int i, float (&v)[8]) {
+    const int64_t base = ((int64_t)list * a.H + i / (kD / 8)) * kD + (i % (kD / 8)) * 8;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = load_elem(a.q, base + j, a.q_dtype);
+  };
+  __syncthreads();  // the amax slots are zero
+  if (q_bf) {
     uint4 raw[kQIter];
 #pragma unroll
-    for (int u = 0; u < kQIter; ++u) {
-      const int i = tid + u * kThr;
-      raw[u] = i < kQChunks ? q4[i] : make_uint4(0, 0, 0, 0);
-    }
+    for (int u = 0; u < kQIter; ++u)
+      raw[u] = reinterpret_cast<const uint4*>(a.q)[(int64_t)list * a.H * (kD / 8) + tid + u * kThr];
 #pragma unroll
     for (int u = 0; u < kQIter; ++u) {
       const int i = tid + u * kThr;
-      if (i >= kQChunks) continue;
-      const uint16_t* bf = reinterpret_cast<const uint16_t*>(&raw[u]);
-      float v[8];
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(&raw[u]);
+      uint32_t mb = 0;  // largest |bf16| bit pattern: the order of the magnitudes
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = bf16_val(bf[j]);
-      q_store(i, v);
+      for (int j = 0; j < 4; ++j) mb = max(mb, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+      const float mx = warp_max(__uint_as_float(mb << 16));  // one head per warp and round
+      if (lane == 0) atomicMax(reinterpret_cast<int*>(qsc_s) + i / (kD / 8), __float_as_int(mx));
+      *q_addr(i) = raw[u];
     }
   } else {
-    for (int i = tid; i < kQChunks; i += kThr) {
-      const int h = i / (kD / 8), d0 = (i % (kD / 8)) * 8;
-      const int64_t base = ((int64_t)list * a.H + h) * kD + d0;
-      float v[8];
+    for (int u = 0; u < kQIter; ++u) {
+      const int i = tid + u * kThr;
+      float v[8], mx = 0.f;
+      f32_chunk(i, v);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = load_elem(a.q, base + j, a.q_dtype);
-      q_store(i, v);
+      for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(v[j]));
+      mx = warp_max(mx);
+      if (lane == 0) atomicMax(reinterpret_cast<int*>(qsc_s) + i / (kD / 8), __float_as_int(mx));
     }
   }
+  __syncthreads();
+  for (int u = 0; u < kQIter; ++u) {
+    const int i = tid + u * kThr;
+    const float f = q_mult(i / (kD / 8));
+    float v[8];
+    if (q_bf) {
+      const uint4 r = *q_addr(i);
+      const uint16_t* bf = reinterpret_cast<const uint16_t*>(&r);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = bf16_val(bf[j]) * f;
+    } else {
+      f32_chunk(i, v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] *= f;
+    }
+    *q_addr(i) = make_uint4(pack_h2(v[0], v[1]), pack_h2(v[2], v[3]), pack_h2(v[4], v[5]), pack_h2(v[6], v[7]));
+  }
+  __syncthreads();  // every multiplier was read: the slots now take 2^e
+  if (tid < kH) qsc_s[tid] = 1.f / q_mult(tid);
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -262,6 +310,10 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
         }
         if ((g != -1 || !a.idx) && a.status) atomicOr(a.status, LCSC_DEV_BAD_INDEX);
         return nullptr;
+      }
+      if (slot >= qr.n_ent_slots + qr.n_win) {  // the sink token: position 0's stored row
+        scp = a.tok_kv.fscale(b, 0);
+        return a.tok_kv.row(b, 0);
       }
       int64_t row = win_base + (slot - qr.n_ent_slots);  // < 2 * capacity: the window is <= capacity rows
       if (row >= win_cap) row -= win_cap;
@@ -345,8 +397,14 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
         if (tab[i] == 0xFFFFFFFFu) continue;
         const uint16_t* bf = reinterpret_cast<const uint16_t*>(&raw[i]);
         uint32_t h[4];
+        float big = 0.f;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) h[q] = pack_h2(bf16_val(bf[2 * q]), bf16_val(bf[2 * q + 1]));
+        for (int q = 0; q < 4; ++q) {
+          const float x0 = bf16_val(bf[2 * q]), x1 = bf16_val(bf[2 * q + 1]);
+          big = fmaxf(big, fmaxf(fabsf(x0), fabsf(x1)));
+          h[q] = pack_h2(x0, x1);
+        }
+        if (big > 65504.f && a.status) atomicOr(a.status, LCSC_DEV_RANGE);
         *reinterpret_cast<uint4*>(kt + (tab[i] & 0xFFFFu)) = make_uint4(h[0], h[1], h[2], h[3]);
       }
       if (lt < kTR) {  // valid-row bits of tile j, read by the softmax after k_full
@@ -369,6 +427,7 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
       }
       if (lt < kTR) {
         scl_s[(j & 3) * kTR + lt] = sc_next;  // tile j's scale, loaded one step ago
+        if (!(sc_next <= kMaxRowScale) && a.status) atomicOr(a.status, LCSC_DEV_RANGE);
         const bool nrm = sc_next >= 6.103515625e-05f && sc_next <= 65504.f;
         const __half2 s2 = __float2half2_rn(nrm ? sc_next : 0.f);
         sch_s[(j & 3) * kTR + lt] = *reinterpret_cast<const uint32_t*>(&s2);
@@ -489,6 +548,8 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
     const bool s_lane = lane >= 16;
     const int head = warp * 16 + (lane & 15);
     const uint32_t row_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    // this head's logit scale: sm_scale times the power of two q was divided by
+    const float sm_h = a.sm_scale * qsc_s[head];
     float m_ref = -INFINITY, l_sum = 0.f;
     for (int j = 0; j < ntiles; ++j) {
       const int buf = j & 1;
@@ -517,7 +578,7 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
           if ((m1 >> q) & 1u) mx = fmaxf(mx, __uint_as_float(r1[q]));
         }
       }
-      mx *= a.sm_scale;  // sm_scale > 0 keeps the order
+      mx *= sm_h;  // sm_scale > 0 keeps the order
       // reference max: set on the first rows seen, moved only by large jumps
       float alpha = 1.f;
       bool moved = false;
@@ -531,7 +592,7 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
       }
       // p = exp(s * sm_scale - ref) = 2^(s * c2 - ref * log2 e): one FFMA and one EX2
       const float ref = m_ref;
-      const float c2 = a.sm_scale * kLog2e, ref2 = ref * kLog2e;
+      const float c2 = sm_h * kLog2e, ref2 = ref * kLog2e;
       float sum = 0.f;
       uint32_t pk[32];
       if (full && ref > -INFINITY) {

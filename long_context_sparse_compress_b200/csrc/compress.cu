@@ -227,6 +227,7 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
 #pragma unroll
       for (int j = 0; j < VPL; ++j) v[j] = load_elem(a.x, base + j, a.x_dtype);
       store_row_warp<VPL>(a.window, b, pos % a.window.capacity, v, lane);
+      if (pos == 0 && a.sink_tok.data) store_row_warp<VPL>(a.sink_tok, b, 0, v, lane);
     }
   }
   if (tid == 0) { n_ent = 0; rows_used = 0; }
@@ -301,10 +302,11 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
       const bool live = row_src[r] >= 0;
       cp_async16(xb + (cv / 64) * (kRows * 128) + swz128(r, (cv % 64) * 2), live ? xg + row_src[r] + cv : xg, live);
     }
-    for (int i = tid; i < DIM * (NC / VEC); i += kThreads) {
-      const int k = i / (NC / VEC), cv = (i % (NC / VEC)) * VEC;
-      cp_async16(wb + swz128(k, cv * 2), wg + (int64_t)k * DIM + c0 + cv, true);
-    }
+    if (!a.gate_logits)
+      for (int i = tid; i < DIM * (NC / VEC); i += kThreads) {
+        const int k = i / (NC / VEC), cv = (i % (NC / VEC)) * VEC;
+        cp_async16(wb + swz128(k, cv * 2), wg + (int64_t)k * DIM + c0 + cv, true);
+      }
     cp_async_wait_all();
   } else {
     for (int i = tid; i < x_rows * (DIM / VEC); i += kThreads) {
@@ -315,21 +317,35 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
 #pragma unroll
       for (int j = 0; j < 4; ++j) xs[r * XS + cv + j] = f[j];
     }
-    for (int i = tid; i < DIM * (NC / VEC); i += kThreads) {
-      const int k = i / (NC / VEC), cv = (i % (NC / VEC)) * VEC;
-      const uint4 val = *reinterpret_cast<const uint4*>(wg + (int64_t)k * DIM + c0 + cv);
-      const float* f = reinterpret_cast<const float*>(&val);
+    if (!a.gate_logits)
+      for (int i = tid; i < DIM * (NC / VEC); i += kThreads) {
+        const int k = i / (NC / VEC), cv = (i % (NC / VEC)) * VEC;
+        const uint4 val = *reinterpret_cast<const uint4*>(wg + (int64_t)k * DIM + c0 + cv);
+        const float* f = reinterpret_cast<const float*>(&val);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) ws[k * WS + cv + j] = f[j];
-    }
+        for (int j = 0; j < 4; ++j) ws[k * WS + cv + j] = f[j];
+      }
   }
   // rows past the used ones are zero (fp32 path: read by the GEMM's last row block)
   if constexpr (!kBf16)
     for (int i = tid; i < (((x_rows + 15) & ~15) - x_rows) * XS; i += kThreads) xs[x_rows * XS + i] = Elem(0);
   __syncthreads();
 
-  // ---- z = x W for the 128 x NC tile
-  if constexpr (kBf16) {
+  // ---- z = x W for the 128 x NC tile, or the caller's logit rows
+  if (a.gate_logits) {
+    // u has the rows of x (same element offsets), in float32; masked rows are
+    // never read by the softmax below
+    const float* ug = reinterpret_cast<const float*>(a.w);
+    for (int i = tid; i < x_rows * (NC / 4); i += kThreads) {
+      const int r = i / (NC / 4), cv = (i % (NC / 4)) * 4;
+      float4 u4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (row_src[r] >= 0) u4 = *reinterpret_cast<const float4*>(ug + row_src[r] + c0 + cv);
+      zs[r * ZS + cv] = u4.x;
+      zs[r * ZS + cv + 1] = u4.y;
+      zs[r * ZS + cv + 2] = u4.z;
+      zs[r * ZS + cv + 3] = u4.w;
+    }
+  } else if constexpr (kBf16) {
     // tcgen05: M = 128 token rows, N = 64 channels, K = DIM; x is the K-major
     // A operand, the W chunk the MN-major B operand; z lands in 64 TMEM columns
     __shared__ uint64_t mma_bar;
@@ -514,6 +530,7 @@ __global__ void __launch_bounds__(256) store_kernel(CompressLaunch a) {
 #pragma unroll
     for (int j = 0; j < VPL; ++j) v[j] = load_elem(a.x, base + j, a.x_dtype);
     store_row_warp<VPL>(a.window, b, pos % a.window.capacity, v, lane);
+    if (pos == 0 && a.sink_tok.data) store_row_warp<VPL>(a.sink_tok, b, 0, v, lane);
   }
 }
 

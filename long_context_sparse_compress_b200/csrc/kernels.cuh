@@ -25,7 +25,8 @@ struct CompressLaunch {
   const void* x;        // [B][n_x][dim] raw rows
   int x_dtype;
   int64_t n_x;
-  const void* w;        // [dim][dim]
+  const void* w;        // [dim][dim] x_dtype, or (gate_logits) float32 [B][n_x][dim] logit rows
+  int gate_logits;      // the gate logits are given (w) instead of computed as x W
   const float* bpos;    // [G][dim]
   int dim;
   int B;
@@ -35,6 +36,7 @@ struct CompressLaunch {
   CacheView entries;
   CacheView window;     // data == nullptr: no window write
   int n_win_max;        // max window rows per sequence
+  CacheView sink_tok;   // data != nullptr: the raw row of position 0 is also stored here (row 0)
   int32_t* status;
 };
 
@@ -91,6 +93,8 @@ struct AttnLaunch {
   CacheView kv, v, win_kv, win_v;  // v / win_v data == nullptr: V = K
   const int32_t* idx;   // [B][T][k] or nullptr (dense)
   const float* sink;    // [H] or nullptr
+  int sink_token;       // the stored row of position 0 (tok_kv / tok_v, row 0) joins every row set
+  CacheView tok_kv, tok_v;
   const int32_t* ctx_len;
   int B, T, H, D, Dv, m, w, k;
   int64_t n_max;

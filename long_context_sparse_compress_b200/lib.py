@@ -13,13 +13,17 @@ from . import workloads
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblcsc.so")
-ABI_VERSION = 2
+ABI_VERSION = 3
 
 FMT = {"f32": 0, "kv": 1, "fp8": 2, "fp4": 3}
 DT = {"f32": 0, "bf16": 1}
 TENSOR = {"kv": 0, "v": 1, "idx": 2}
+SINK = {"logit": 0, "token": 1}
+GATE = {"proj": 0, "logits": 1}
 DEV_BAD_INDEX = 1
 DEV_BAD_LENGTH = 2
+DEV_TIMEOUT = 4
+DEV_RANGE = 8
 
 c_i32, c_i64, c_f32, c_vp, c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
@@ -29,7 +33,8 @@ class Params(ctypes.Structure):
                 ("sm_scale", c_f32), ("n_heads", c_i32), ("head_dim", c_i32), ("rope_dim", c_i32),
                 ("v_dim", c_i32), ("idx_heads", c_i32), ("idx_dim", c_i32), ("kv_format", c_i32),
                 ("idx_format", c_i32), ("x_dtype", c_i32), ("q_dtype", c_i32),
-                ("out_rope_dim", c_i32), ("out_rope_base", c_f32)]
+                ("out_rope_dim", c_i32), ("out_rope_base", c_f32), ("sink_mode", c_i32),
+                ("gate_src", c_i32)]
 
 
 class Cache(ctypes.Structure):
@@ -44,7 +49,8 @@ class Step(ctypes.Structure):
                 ("kv", Cache), ("v", Cache), ("idx_keys", Cache), ("win_kv", Cache), ("win_v", Cache),
                 ("q", c_vp), ("q_idx", c_vp), ("w_heads", c_vp), ("sink", c_vp),
                 ("out", c_vp), ("lse", c_vp), ("out_idx", c_vp), ("out_score", c_vp),
-                ("events", ctypes.POINTER(c_vp)), ("n_events", c_i32)]
+                ("events", ctypes.POINTER(c_vp)), ("n_events", c_i32), ("sink_kv", Cache),
+                ("sink_v", Cache)]
 
 
 _SIGS = {
@@ -65,10 +71,10 @@ _SIGS = {
     "lcsc_csa_index_topk_noalloc": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_vp,
                                             c_vp, c_vp, c_vp]),
     "lcsc_attn_workspace_size": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_i32, c_vp]),
-    "lcsc_csa_sparse_attn": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i64,
-                                     c_i64, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
-    "lcsc_hca_dense_attn": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64,
-                                    c_i64, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
+    "lcsc_csa_sparse_attn": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                     c_i64, c_i64, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
+    "lcsc_hca_dense_attn": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i64,
+                                    c_i64, c_i64, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
     "lcsc_step_workspace_size": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, c_vp]),
     "lcsc_csa_decode": (c_i32, [c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
     "lcsc_hca_decode": (c_i32, [c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
@@ -134,7 +140,8 @@ def params(wl):
                   rope_dim=wl.rope_dim if wl.kv_fmt == "kv" else 0, v_dim=wl.Dv, idx_heads=wl.H_I,
                   idx_dim=wl.d_I, kv_format=FMT[wl.kv_fmt], idx_format=FMT[wl.idx_fmt],
                   x_dtype=DT[wl.x_dtype], q_dtype=DT[wl.q_dtype],
-                  out_rope_dim=wl.rope_dim if wl.out_rope_base > 0 else 0, out_rope_base=wl.out_rope_base)
+                  out_rope_dim=wl.rope_dim if wl.out_rope_base > 0 else 0, out_rope_base=wl.out_rope_base,
+                  sink_mode=SINK[wl.sink_mode], gate_src=GATE[wl.gate_src])
 
 
 def row_bytes(fmt, dim, rope=0):
@@ -284,29 +291,33 @@ def attn_workspace(p, B, T, n_max, dense):
     return _ws_size(load().lcsc_attn_workspace_size, ctypes.byref(p), B, T, n_max, int(dense))
 
 
+def _cref(c):
+    return ref(c.c() if c is not None else None)
+
+
 def sparse_attn(p, q, kv, v, win_kv, win_v, idx, sink, ctx_len, out, lse=None, ws=None, status=None,
-                stream=None):
+                stream=None, sink_kv=None, sink_v=None):
     lib = load()
     B, T = q.shape[0], q.shape[1]
     if ws is None:
         ws = workspace(attn_workspace(p, B, T, kv.capacity, False), q.device)
     check(lib.lcsc_csa_sparse_attn(
-        ctypes.byref(p), ptr(q), ctypes.byref(kv.c()), ref(v.c() if v else None),
-        ctypes.byref(win_kv.c()), ref(win_v.c() if win_v else None), ptr(idx), ptr(sink), ptr(ctx_len),
-        B, T, ptr(out), ptr(lse), ptr(ws), ws.numel(), ptr(status), stream_handle(stream)))
+        ctypes.byref(p), ptr(q), ctypes.byref(kv.c()), _cref(v), ctypes.byref(win_kv.c()), _cref(win_v),
+        ptr(idx), ptr(sink), _cref(sink_kv), _cref(sink_v), ptr(ctx_len), B, T, ptr(out), ptr(lse), ptr(ws),
+        ws.numel(), ptr(status), stream_handle(stream)))
     return ws
 
 
 def dense_attn(p, q, kv, v, win_kv, win_v, sink, ctx_len, n_max, out, lse=None, ws=None, status=None,
-               stream=None):
+               stream=None, sink_kv=None, sink_v=None):
     lib = load()
     B, T = q.shape[0], q.shape[1]
     if ws is None:
         ws = workspace(attn_workspace(p, B, T, n_max, True), q.device)
     check(lib.lcsc_hca_dense_attn(
-        ctypes.byref(p), ptr(q), ctypes.byref(kv.c()), ref(v.c() if v else None),
-        ctypes.byref(win_kv.c()), ref(win_v.c() if win_v else None), ptr(sink), ptr(ctx_len), B, T, n_max,
-        ptr(out), ptr(lse), ptr(ws), ws.numel(), ptr(status), stream_handle(stream)))
+        ctypes.byref(p), ptr(q), ctypes.byref(kv.c()), _cref(v), ctypes.byref(win_kv.c()), _cref(win_v),
+        ptr(sink), _cref(sink_kv), _cref(sink_v), ptr(ctx_len), B, T, n_max, ptr(out), ptr(lse), ptr(ws),
+        ws.numel(), ptr(status), stream_handle(stream)))
     return ws
 
 
@@ -315,8 +326,12 @@ def step_workspace(p, csa, B, T, n_max):
 
 
 def make_step(B, T, n_max, ctx_len, x_kv, x_v, x_idx, w_kv, b_kv, w_v, b_v, w_idx, b_idx, kv, v, idx_keys,
-              win_kv, win_v, q, q_idx, w_heads, sink, out, lse=None, out_idx=None, out_score=None):
-    """An lcsc_step struct over device tensors / caches (None -> NULL)."""
+              win_kv, win_v, q, q_idx, w_heads, sink, out, lse=None, out_idx=None, out_score=None,
+              sink_kv=None, sink_v=None):
+    """An lcsc_step struct over device tensors / caches (None -> NULL).
+    With gate logits (gate_src "logits") w_kv / w_v / w_idx are the float32
+    logit rows; with a sink token, sink_kv / sink_v are the one-row caches of
+    position 0."""
     cc = lambda c: c.c() if c is not None else null_cache()
     s = Step(B=B, T=T, n_max=n_max)
     for name, t in dict(ctx_len=ctx_len, x_kv=x_kv, x_v=x_v, x_idx=x_idx, w_kv=w_kv, b_kv=b_kv, w_v=w_v,
@@ -324,6 +339,7 @@ def make_step(B, T, n_max, ctx_len, x_kv, x_v, x_idx, w_kv, b_kv, w_v, b_v, w_id
                         out=out, lse=lse, out_idx=out_idx, out_score=out_score).items():
         setattr(s, name, None if t is None else t.data_ptr())
     s.kv, s.v, s.idx_keys, s.win_kv, s.win_v = cc(kv), cc(v), cc(idx_keys), cc(win_kv), cc(win_v)
+    s.sink_kv, s.sink_v = cc(sink_kv), cc(sink_v)
     return s
 
 

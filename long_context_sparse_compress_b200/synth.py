@@ -14,6 +14,13 @@ alone.  Values follow the benchmark recipe:
   the mean query head, the indexer key along sum_h w[h] q_idx[h] (averaged
   over the step's queries).  This makes the top-k non-degenerate.
 
+Layers with caller-given gate logits get per-token logit rows U ~ N(0, 1)
+aligned with the raw rows.  Layers whose sink is the position-0 token get
+that token's raw row as a sink would look: gamma times the unit mean query
+head (plus N(0, 0.01/d) noise), gamma = 4 sqrt(D H), so that its logit is a
+few units above the others' and it draws a large share of every head's
+weight; when the tail reaches position 0, that tail row is the same row.
+
 Rows that the layer stores as bf16 (raw rows, gate weights, queries) are
 rounded to bf16 here with torch's own cast; everything else is float32.
 The existing cache is described by its *pre-storage* float32 entry values;
@@ -27,7 +34,7 @@ SEED = 20261202
 _LAYER = {"csa": 0, "hca": 1}
 _TENSOR = {name: i + 1 for i, name in enumerate(
     ["x_kv", "x_v", "x_idx", "W_kv", "B_kv", "W_v", "B_v", "W_idx", "B_idx", "q", "q_idx",
-     "w_idx", "sink", "e_kv", "e_v", "e_idx", "planted"])}
+     "w_idx", "sink", "e_kv", "e_v", "e_idx", "planted", "x0_kv", "x0_v", "U_kv", "U_v", "U_idx"])}
 
 
 def stream(seed, layer, tensor, b=0):
@@ -102,6 +109,23 @@ def sequence_inputs(wl, b, seed=SEED, entries=True):
                                                    (wl.T, wl.H_I, wl.d_I), wl.d_I ** -0.5))
         w = np.abs(normal(stream(seed, lay, "w_idx", b), (wl.T, wl.H_I), 1.0)) * np.float32(wl.H_I ** -0.5)
         out["w_idx"] = w.astype(np.float32)
+    if wl.gate_src == "logits":
+        out["U_kv"] = normal(stream(seed, lay, "U_kv", b), (R, wl.D), 1.0)
+        if wl.separate_v:
+            out["U_v"] = normal(stream(seed, lay, "U_v", b), (R, wl.Dv), 1.0)
+        if wl.kind == "csa":
+            out["U_idx"] = normal(stream(seed, lay, "U_idx", b), (R, wl.d_I), 1.0)
+    if wl.sink_mode == "token":
+        u_q = _unit(out["q"].astype(np.float64).mean(axis=(0, 1)))
+        gamma = 4.0 * np.sqrt(wl.D * wl.H)
+        x0 = gamma * u_q + normal(stream(seed, lay, "x0_kv", b), (wl.D,), 0.1 * wl.D ** -0.5)
+        out["x0_kv"] = as_dtype(wl.x_dtype, x0.astype(np.float32))
+        if wl.separate_v:
+            out["x0_v"] = as_dtype(wl.x_dtype, normal(stream(seed, lay, "x0_v", b), (wl.Dv,), wl.Dv ** -0.5))
+        if wl.L - R <= 0:  # the tail reaches position 0: it holds the same row
+            out["x_kv"][R - wl.L] = out["x0_kv"]
+            if wl.separate_v:
+                out["x_v"][R - wl.L] = out["x0_v"]
     if not entries:
         return out
     n_old = (wl.L - wl.T) // wl.m

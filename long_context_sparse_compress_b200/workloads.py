@@ -36,8 +36,10 @@ class Workload:
     x_dtype: str = "bf16"  # raw rows and gate weights
     q_dtype: str = "bf16"  # queries and the output
     n_planted: int = 0   # planted relevant entries per sequence
-    sink: bool = True
+    sink: bool = True    # a sink is present (sink_mode "logit": a learned logit per head)
     out_rope_base: float = 0.0  # > 0: the output's rope dims rotated back by the query position
+    sink_mode: str = "logit"    # "logit" or "token" (the raw row of position 0 joins every row set)
+    gate_src: str = "proj"      # "proj" (z = x W) or "logits" (per-token gate logits given)
 
     @property
     def sm_scale(self):

@@ -42,6 +42,9 @@ class GpuBatch:
         self.idx = L.DeviceCache(B, n_cap_idx, wl.idx_fmt, wl.d_I) if wl.kind == "csa" else None
         self.win_kv = L.DeviceCache(B, wl.win_cap, wl.kv_fmt, wl.D, rope)
         self.win_v = L.DeviceCache(B, wl.win_cap, wl.kv_fmt, wl.Dv, rope) if wl.separate_v else None
+        tok = wl.sink_mode == "token"
+        self.tok_kv = L.DeviceCache(B, 1, wl.kv_fmt, wl.D, rope) if tok else None
+        self.tok_v = L.DeviceCache(B, 1, wl.kv_fmt, wl.Dv, rope) if tok and wl.separate_v else None
         xdt, qdt = TORCH_DT[wl.x_dtype], TORCH_DT[wl.q_dtype]
         for b, s in enumerate(seqs):
             snap = s.snapshot()
@@ -53,18 +56,26 @@ class GpuBatch:
             upload(self.win_kv, b, snap["ring_kv"])
             if self.win_v is not None:
                 upload(self.win_v, b, snap["ring_v"])
+            if self.tok_kv is not None:
+                upload(self.tok_kv, b, snap["tok_kv"])
+            if self.tok_v is not None:
+                upload(self.tok_v, b, snap["tok_v"])
         stack = lambda key, dt: dev(np.stack([s.inp[key] for s in seqs]), dt)
         stack_tail = lambda key: dev(np.stack([step_tail(s.wl, s.inp[key]) for s in seqs]), xdt)
         self.x_kv = stack_tail("x_kv")
         self.x_v = stack_tail("x_v") if wl.separate_v else None
         self.x_idx = stack_tail("x_idx") if wl.kind == "csa" else None
         P = seqs[0].P
-        self.w_kv, self.b_kv = dev(P["W_kv"], xdt), dev(P["B_kv"])
-        self.w_v = dev(P["W_v"], xdt) if wl.separate_v else None
+        # gates: W, or with caller-given logits the float32 logit rows of the step's positions
+        logits = wl.gate_src == "logits"
+        gate = lambda key, Wkey: (dev(np.stack([step_tail(s.wl, s.inp[key]) for s in seqs]))
+                                  if logits else dev(P[Wkey], xdt))
+        self.w_kv, self.b_kv = gate("U_kv", "W_kv"), dev(P["B_kv"])
+        self.w_v = gate("U_v", "W_v") if wl.separate_v else None
         self.b_v = dev(P["B_v"]) if wl.separate_v else None
-        self.w_idx = dev(P["W_idx"], xdt) if wl.kind == "csa" else None
+        self.w_idx = gate("U_idx", "W_idx") if wl.kind == "csa" else None
         self.b_idx = dev(P["B_idx"]) if wl.kind == "csa" else None
-        self.sink = dev(P["sink"]) if wl.sink else None
+        self.sink = dev(P["sink"]) if wl.sink and not tok else None
         self.q = stack("q", qdt)
         self.q_idx = stack("q_idx", qdt) if wl.kind == "csa" else None
         self.w_heads = stack("w_idx", torch.float32) if wl.kind == "csa" else None
@@ -82,7 +93,8 @@ class GpuBatch:
         return L.make_step(self.B, self.wl.T, self.n_max, self.ctx_len, self.x_kv, self.x_v, self.x_idx,
                            self.w_kv, self.b_kv, self.w_v, self.b_v, self.w_idx, self.b_idx, self.kv,
                            self.v, self.idx, self.win_kv, self.win_v, self.q, self.q_idx, self.w_heads,
-                           self.sink, self.out, self.lse, self.out_idx, self.out_score)
+                           self.sink, self.out, self.lse, self.out_idx, self.out_score, self.tok_kv,
+                           self.tok_v)
 
     def run_step(self):
         csa = self.wl.kind == "csa"

@@ -58,6 +58,14 @@ class OracleSequence:
         self.idx = stored_entries(wl, self.inp, "idx") if wl.kind == "csa" else None
         self.ring_kv = stored_ring(wl, self.inp["x_kv"], wl.D)
         self.ring_v = stored_ring(wl, self.inp["x_v"], wl.Dv) if wl.separate_v else None
+        # sink token: the stored row of position 0, present once a step before this one received it
+        self.tok_kv = self._tok_row("kv", wl.D) if wl.sink_mode == "token" else None
+        self.tok_v = self._tok_row("v", wl.Dv) if wl.sink_mode == "token" and wl.separate_v else None
+
+    def _tok_row(self, key, dim):
+        rope = self.wl.rope_dim if self.wl.kv_fmt == "kv" else 0
+        row = self.inp["x0_" + key] if self.wl.L - self.wl.T > 0 else np.zeros(dim, np.float32)
+        return storage.encode(self.wl.kv_fmt, np.asarray(row, np.float32)[None], rope)
 
     def snapshot(self):
         """Copies of the stored arrays (the GPU side gets these bytes)."""
@@ -66,7 +74,7 @@ class OracleSequence:
                 return None
             return storage.Stored(st.fmt, st.payload.copy(), None if st.scale is None else st.scale.copy(),
                                   st.dim, st.rope_dim)
-        return {k: cp(getattr(self, k)) for k in ("kv", "v", "idx", "ring_kv", "ring_v")}
+        return {k: cp(getattr(self, k)) for k in ("kv", "v", "idx", "ring_kv", "ring_v", "tok_kv", "tok_v")}
 
     def step(self, queries=None):
         wl, P, inp = self.wl, self.P, self.inp
@@ -77,7 +85,10 @@ class OracleSequence:
             idx=self.idx, ring_kv=self.ring_kv, ring_v=self.ring_v, x_kv=t("x_kv"), x_v=t("x_v"),
             x_idx=t("x_idx"), W_kv=P["W_kv"], B_kv=P["B_kv"], W_v=P.get("W_v"), B_v=P.get("B_v"),
             W_idx=P.get("W_idx"), B_idx=P.get("B_idx"), q=inp["q"], q_idx=inp.get("q_idx"),
-            w_idx=inp.get("w_idx"), sink=P["sink"], queries=queries, out_rope_base=wl.out_rope_base)
+            w_idx=inp.get("w_idx"), sink=P["sink"] if wl.sink else np.full(wl.H, -np.inf), queries=queries,
+            out_rope_base=wl.out_rope_base,
+            U_kv=t("U_kv"), U_v=t("U_v"), U_idx=t("U_idx"), sink_mode=wl.sink_mode, tok_kv=self.tok_kv,
+            tok_v=self.tok_v)
 
 
 # ---------------------------------------------------------------- comparisons

@@ -39,6 +39,7 @@ def test_abi_version_and_strings(lib):
     assert lib.lcsc_abi_version() == L.ABI_VERSION
     for code in range(5):
         assert lib.lcsc_status_string(code)
+    assert L.Params.sink_mode.offset == 68 and L.Params.gate_src.offset == 72
     assert lib.lcsc_row_bytes(L.FMT["kv"], 512, 64) == 576
     assert lib.lcsc_row_bytes(L.FMT["fp8"], 128, 0) == 128
     assert lib.lcsc_row_bytes(L.FMT["fp4"], 128, 0) == 64
@@ -79,6 +80,24 @@ def test_bad_arguments_are_rejected_before_launch(lib):
         bad = L.params(W.CSA_DECODE_128K.with_(out_rope_base=10000.0))
         setattr(bad, field, value)
         assert lib.lcsc_attn_workspace_size(ctypes.byref(bad), 1, 1, 10, 0, ctypes.byref(out)) == 1, field
+    # the sink and gate readings take only their two values; the softmax
+    # scale must be a positive number
+    for field, value in (("sink_mode", 2), ("sink_mode", -1), ("gate_src", 2), ("sm_scale", 0.0),
+                         ("sm_scale", -0.1), ("sm_scale", float("nan")), ("sm_scale", float("inf"))):
+        bad = L.params(W.CSA_DECODE_128K)
+        setattr(bad, field, value)
+        assert lib.lcsc_attn_workspace_size(ctypes.byref(bad), 1, 1, 10, 0, ctypes.byref(out)) == 1, field
+    # with a sink token the sink logit pointer must be NULL and the position-0
+    # rows given (checked before any pointer is dereferenced on the device)
+    tok = L.params(W.HCA_DECODE_64K.with_(sink_mode="token"))
+    c = L.Cache(data=16, scale=16, capacity=1000)  # room for the window: only the sink arguments are wrong
+    q_ptr = ctypes.c_void_p(16)
+    assert lib.lcsc_hca_dense_attn(ctypes.byref(tok), q_ptr, ctypes.byref(c), null, ctypes.byref(c), null,
+                                   ctypes.c_void_p(16), ctypes.byref(c), null, ctypes.c_void_p(16), 1, 1, 4,
+                                   q_ptr, null, ctypes.c_void_p(256), 1 << 20, null, null) == 1
+    assert lib.lcsc_hca_dense_attn(ctypes.byref(tok), q_ptr, ctypes.byref(c), null, ctypes.byref(c), null,
+                                   null, null, null, ctypes.c_void_p(16), 1, 1, 4, q_ptr, null,
+                                   ctypes.c_void_p(256), 1 << 20, null, null) == 1
     # a dimension the kernels are not built for
     odd = L.params(W.CSA_DECODE_128K.with_(d_I=96))
     s = L.Step(B=1, T=1, n_max=10, ctx_len=16)

@@ -398,3 +398,93 @@ def test_attention_flags_out_of_range_index(cuda_lib):
     o, _ = joint_attention(q[0, 0].cpu().double().numpy(), np.concatenate([Kn[ent], Wk[wpos]]),
                            np.concatenate([Vn[ent], Wv[wpos]]), np.full(H, -np.inf), wl.sm_scale)
     assert rel_l2(out[0, 0].cpu().numpy(), o) < 1e-5
+
+
+def _dense_kv_case(rng, wl, n_cap, rope_scale=1.0):
+    """One sequence of stored KV entries and window rows for the 512-dim
+    FP8 + BF16 path; the BF16 RoPE dims multiplied by ``rope_scale``."""
+    D, R = wl.D, wl.rope_dim
+    K = _rows(rng, n_cap, D)
+    K[:, D - R:] *= rope_scale
+    Wr = _rows(rng, wl.win_cap, D)
+    Wr[:, D - R:] *= rope_scale
+    kv_st, wk_st = storage.encode("kv", K, R), storage.encode("kv", Wr, R)
+    kv = L.DeviceCache(1, n_cap, "kv", D, R)
+    wk = L.DeviceCache(1, wl.win_cap, "kv", D, R)
+    upload(kv, 0, kv_st)
+    upload(wk, 0, wk_st)
+    return kv, wk, storage.decode(kv_st), storage.decode(wk_st)
+
+
+@pytest.mark.parametrize("q_scale", [2.0 ** 20, 2.0 ** -20, 2.0 ** 60, 2.0 ** -60])
+def test_attention_query_magnitude_outside_f16(cuda_lib, q_scale):
+    """Queries far outside the f16 range (bf16 holds them) with the softmax
+    scale divided by the same factor, so the logits stay as they were: the
+    tensor-core path scales each head into range and gives the oracle's
+    answer (before that scaling, 2^20 overflowed f16 and 2^-20 lost the
+    queries to f16 subnormals)."""
+    rng = np.random.default_rng(51)
+    wl = W.CSA_DECODE_128K.with_(k=200, w=100, kind="hca", m=16, G=16, T=2)
+    n_cap = 600
+    L0 = (n_cap - 1) * wl.m
+    kv, wk, K_all, WK = _dense_kv_case(rng, wl, n_cap)
+    q = (rng.standard_normal((1, 2, wl.H, wl.D)) * wl.D ** -0.5 * 8 * q_scale)
+    q = torch.from_numpy(q.astype(np.float32)).to(torch.bfloat16)
+    p = L.params(wl)
+    p.sm_scale = wl.sm_scale / q_scale
+    sink = rng.standard_normal(wl.H).astype(np.float32)
+    ctx = torch.tensor([L0], dtype=torch.int32, device="cuda")
+    out = torch.zeros((1, 2, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((1, 2, wl.H), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.dense_attn(p, q.cuda(), kv, None, wk, None, dev(sink), ctx, n_cap, out, lse, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    qf = q.float().numpy().astype(np.float64)
+    for t in range(2):
+        pp = L0 - 2 + t
+        wpos = window_positions(pp, wl.w) % wl.win_cap
+        Kr = np.concatenate([K_all[:(pp + 1) // wl.m], WK[wpos]])
+        o, ls = joint_attention(qf[0, t], Kr, Kr, sink, float(np.float32(p.sm_scale)))
+        got = out[0, t].float().cpu().numpy()
+        assert np.all(np.isfinite(got))
+        assert rel_l2(got, o) <= ATTN_RTOL, (q_scale, t, rel_l2(got, o))
+        assert max_abs(got, o) <= ATTN_ATOL
+        assert np.allclose(lse[0, t].cpu().numpy(), ls, rtol=1e-4, atol=1e-4)
+
+
+def test_attention_kv_range(cuda_lib):
+    """Stored KV rows: tiny BF16 RoPE dims (f16 subnormals) still give the
+    oracle's answer; RoPE dims above the f16 range, or an FP8 row scale whose
+    codes would overflow f16, set LCSC_DEV_RANGE."""
+    rng = np.random.default_rng(52)
+    wl = W.CSA_DECODE_128K.with_(k=200, w=100, kind="hca", m=16, G=16, T=1)
+    n_cap = 300
+    L0 = (n_cap - 1) * wl.m
+    q = torch.from_numpy((rng.standard_normal((1, 1, wl.H, wl.D)) * wl.D ** -0.5 * 8).astype(np.float32))
+    q = q.to(torch.bfloat16)
+    sink = dev(rng.standard_normal(wl.H).astype(np.float32))
+    ctx = torch.tensor([L0], dtype=torch.int32, device="cuda")
+
+    def run(kv, wk):
+        out = torch.zeros((1, 1, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        L.dense_attn(L.params(wl), q.cuda(), kv, None, wk, None, sink, ctx, n_cap, out, None, status=status)
+        torch.cuda.synchronize()
+        return out, int(status.item())
+
+    kv, wk, K_all, WK = _dense_kv_case(rng, wl, n_cap, rope_scale=1e-6)
+    out, st = run(kv, wk)
+    assert st == 0
+    wpos = window_positions(L0 - 1, wl.w) % wl.win_cap
+    Kr = np.concatenate([K_all[:L0 // wl.m], WK[wpos]])
+    o, _ = joint_attention(q.float().numpy()[0, 0].astype(np.float64), Kr, Kr, sink.cpu().numpy(), wl.sm_scale)
+    got = out[0, 0].float().cpu().numpy()
+    assert rel_l2(got, o) <= ATTN_RTOL and max_abs(got, o) <= ATTN_ATOL
+    kv, wk, _, _ = _dense_kv_case(rng, wl, n_cap, rope_scale=1e6)  # RoPE dims ~ 4e4 .. 2e5
+    _, st = run(kv, wk)
+    assert st & L.DEV_RANGE
+    kv, wk, _, _ = _dense_kv_case(rng, wl, n_cap)
+    kv.scale[0, 7] = 200.0  # one entry's E4M3 codes times 200 pass 65504
+    _, st = run(kv, wk)
+    assert st & L.DEV_RANGE

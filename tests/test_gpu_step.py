@@ -33,6 +33,23 @@ CASES = {
     # the 2,048-token window reading of the pages, without a sink
     "csa_window2048_nosink": (W.CSA_DECODE_128K.with_(B=2, w=2048, sink=False), [12000, 1500]),
     "hca_window2048_nosink": (W.HCA_DECODE_64K.with_(B=2, w=2048, sink=False), [16384, 2000]),
+    # the sink-token reading: the raw row of position 0 in every row set
+    # (L = 100 keeps position 0 inside the window: it enters once)
+    "csa_fp8_sink_token": (W.CSA_DECODE_128K.with_(B=3, sink_mode="token"), [8192, 4100, 100]),
+    "hca_sink_token": (W.HCA_DECODE_64K.with_(B=3, sink_mode="token"), [4096, 1152, 100]),
+    "csa_f32_sink_token": (W.CSA_DECODE_4K_F32.with_(B=3, sink_mode="token"), [4096, 1000, 101]),
+    # a chunk that starts at position 0 stores the position-0 row itself, and
+    # its later queries (past the 4-token window) attend to it
+    "hca_sink_token_from_zero": (W.HCA_DECODE_64K.with_(B=2, T=16, w=4, sink_mode="token"), [16, 4096 + 16]),
+    "csa_fp8_sink_token_from_zero": (W.CSA_PREFILL_256K.with_(B=2, T=40, w=8, n_planted=0, sink_mode="token"),
+                                     [40, 2002]),
+    # caller-given gate logits, with and without overlapping groups
+    "csa_fp4_gate_logits": (W.PAIR_DECODE_1M_B1.layer("csa").with_(B=2, n_planted=16, gate_src="logits"),
+                            [16384, 6000]),
+    "csa_overlap_gate_logits": (W.CSA_DECODE_128K.with_(B=2, G=8, gate_src="logits"), [8192, 1001]),
+    "hca_gate_logits": (W.HCA_DECODE_64K.with_(B=3, gate_src="logits"), [4096, 1024 + 128, 100]),
+    "csa_f32_gate_logits_sink_token": (W.CSA_DECODE_4K_F32.with_(B=2, gate_src="logits", sink_mode="token"),
+                                       [4096, 1000]),
 }
 
 
@@ -55,6 +72,11 @@ def check_step(name, wl, lengths, query_sample=None):
                                                 s.kv.dim, s.kv.rope_dim))
             want = storage.decode(s.kv.rows(slice(g_lo, g_hi)))
             assert rel_l2(got, want) <= (1e-5 if s.kv.fmt == "f32" else 1e-2)
+        if gb.tok_kv is not None:  # the position-0 row, stored by the oracle's rule
+            td, tsc = download(gb.tok_kv, b)
+            assert np.array_equal(td[0], s.tok_kv.payload[0]), "position-0 row"
+            if tsc is not None:
+                assert tsc[0] == s.tok_kv.scale[0]
         wd, _ = download(gb.win_kv, b)
         for pos in range(s.wl.L - wl.T, s.wl.L):
             r = pos % wl.win_cap

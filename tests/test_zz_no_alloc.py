@@ -42,6 +42,14 @@ def test_noalloc_equals_workspace_call_twice(cuda_lib, fmt):
     ref_sc = torch.zeros((B, T, k), dtype=torch.float32, device="cuda")
     L.index_topk(p, qi, wi, keys, ctx, n_max, ref_idx, ref_sc)
     torch.cuda.synchronize()
+    # a larger request first (more lists, longer lists, the other key format),
+    # so that the calls compared below start on scratch it left behind
+    other = "fp8" if fmt == "fp4" else "fp4"
+    wl2, keys2, qi2, wi2, ctx2, n_max2 = _inputs(other, [4 * 200000] * 4, T=3, seed=6)
+    p2 = L.params(wl2)
+    big_idx = torch.empty((4, 3, wl2.k), dtype=torch.int32, device="cuda")
+    L.index_topk_noalloc(p2, qi2, wi2, keys2, ctx2, n_max2, big_idx, None)
+    torch.cuda.synchronize()
     for call in range(2):
         out_idx = torch.full((B, T, k), -9, dtype=torch.int32, device="cuda")
         out_sc = torch.zeros((B, T, k), dtype=torch.float32, device="cuda")
@@ -66,5 +74,10 @@ def test_noalloc_rejects_requests_beyond_its_scratch():
     rc = lib.lcsc_csa_index_topk_noalloc(ctypes.byref(p), None, None, None, None, 64, 1, 1 << 20, None, None,
                                          None, None)
     assert rc == 4
+    # sizes whose products would overflow are refused before any size is formed
+    for B, T, n in ((1 << 40, 1 << 40, 10), (70000, 1, 10), (1, 1, 1 << 62)):
+        rc = lib.lcsc_csa_index_topk_noalloc(ctypes.byref(p), None, None, None, None, B, T, n, None, None,
+                                             None, None)
+        assert rc == 1, (B, T, n)
     need = L.index_topk_workspace(p, 16, 1, 262144)
     assert need <= L.NOALLOC_SCRATCH_BYTES
