@@ -148,6 +148,38 @@ class Layer:
         return self.out, torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
 
 
+class StepRunner:
+    """Issues one step of a workload's layers.  The two layers of a pair take
+    independent inputs (queries and caches of their own), so the HCA layer
+    runs on a second stream beside the CSA layer: every step forks it from the
+    caller's stream and joins it back, so a step still ends when both layers
+    have.  ``hca_first``: which layer is enqueued first."""
+
+    def __init__(self, layers, stream, hca_first=True):
+        self.layers, self.stream, self.hca_first = layers, stream, hca_first
+        self.streams = [stream] + [torch.cuda.Stream(device=stream.device) for _ in layers[1:]]
+        self.fork = torch.cuda.Event()
+        self.joins = [torch.cuda.Event() for _ in layers]
+
+    def run(self, before=None):
+        """One step; ``before(i, s)`` runs on layer i's stream before it (the
+        end-to-end loop waits there for the layer's uploads)."""
+        if len(self.layers) > 1:
+            self.fork.record(self.stream)
+            for s in self.streams[1:]:
+                s.wait_event(self.fork)
+        order = list(range(len(self.layers)))
+        if self.hca_first:
+            order.reverse()
+        for i in order:
+            if before is not None:
+                before(i, self.streams[i])
+            self.layers[i].run(self.streams[i])
+        for i in range(1, len(self.layers)):
+            self.joins[i].record(self.streams[i])
+            self.stream.wait_event(self.joins[i])
+
+
 # ------------------------------------------------------------ measurement
 
 class ClockSampler:
@@ -420,10 +452,7 @@ def measure_sub(name, dev, peaks, warmup, target_s=0.4, max_steps=5000):
     layers_wl = [wl.layer("csa"), wl.layer("hca")] if wl.kind == "pair" else [wl]
     layers = [Layer(lw, shard_seed(0, i), dev) for i, lw in enumerate(layers_wl)]
     stream = torch.cuda.current_stream()
-
-    def step():
-        for ly in layers:
-            ly.run(stream)
+    step = StepRunner(layers, stream).run
 
     nbytes, _ = step_work(wl)
     flush = nbytes < 2 * L2_BYTES
@@ -450,21 +479,35 @@ def measure_sub(name, dev, peaks, warmup, target_s=0.4, max_steps=5000):
     steps = int(min(max_steps, max(20, target_s * 1e3 / est_ms)))
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     stops = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    # stage boundaries of every layer's step (the library records them)
+    n_ev = {"csa": 6, "hca": 3}
+    stage_ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(n_ev[ly.wl.kind])] for ly in layers]
+                for _ in range(steps)]
+    for evs in stage_ev:
+        for le in evs:
+            for e in le:
+                e.record(stream)  # creates the events
     sampler = ClockSampler(dev.index)
     sampler.start()
     time.sleep(0.3)
     torch.cuda.synchronize()
     t0 = time.time()
     n0 = L.kernel_launches()
+    def with_events(i):
+        for ly, le in zip(layers, stage_ev[i]):
+            ly.set_events(le)
+
     if flush:
         for i in range(steps):
             flush_l2()
+            with_events(i)
             starts[i].record(stream)
             step()
             stops[i].record(stream)
     else:
         starts[0].record(stream)
         for i in range(steps):
+            with_events(i)
             step()
         stops[0].record(stream)
     launches = L.kernel_launches() - n0
@@ -477,13 +520,22 @@ def measure_sub(name, dev, peaks, warmup, target_s=0.4, max_steps=5000):
     else:
         ms = starts[0].elapsed_time(stops[0]) / steps
     for ly in layers:
+        ly.clear_events()
         if int(ly.status.item()) != 0:
             raise RuntimeError(f"device status {int(ly.status.item())} in {ly.wl.name}")
+    names = {"csa": ("idx_compress", "quantize_join", "index_score", "topk", "kv_join_sparse_attn"),
+             "hca": ("compress", "dense_attn")}
+    stage_ms = {}
+    for j, ly in enumerate(layers):
+        for k, nm in enumerate(names[ly.wl.kind]):
+            stage_ms[ly.wl.kind + "." + nm] = round(float(np.mean(
+                [stage_ev[i][j][k].elapsed_time(stage_ev[i][j][k + 1]) for i in range(steps)])), 4)
     unit = "tokens/s" if wl.T >= 64 else "queries/s"
     rec = {"workload": wl.name, "layers": [lw.name for lw in layers_wl], "batch": wl.B, "context": wl.L,
            "new_tokens": wl.T, "steps": steps, "warmup": warmup, "ms_per_step": round(ms, 5),
            "value": round(wl.B * wl.T / (ms / 1e3), 2), "unit": unit,
            "step_roofline": step_roofline(wl, ms, peaks), "gpu_launches_per_step": launches / steps,
+           "stage_ms": stage_ms,
            "clocks": clocks,
            "l2": ("flushed before every step (256 MiB written, 256 MiB read; outside the step's events); "
                   "the step's own events, mean over steps") if flush else
@@ -516,10 +568,8 @@ def run_lcsc(args):
     layers = [Layer(lw, shard_seed(rank, i), dev) for i, lw in enumerate(layers_wl)]
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
-
-    def step():
-        for ly in layers:
-            ly.run(stream)
+    runner = StepRunner(layers, stream)
+    step = runner.run
 
     for _ in range(args.warmup):
         step()
@@ -576,8 +626,8 @@ def run_lcsc(args):
     if csa is not None:
         score_ms = float(np.mean([evs[2].elapsed_time(evs[3]) for evs in events]))
         stage_ms = {name: float(np.mean([evs[a].elapsed_time(evs[b]) for evs in events]))
-                    for name, a, b in (("compress", 0, 1), ("quantize", 1, 2), ("index_score", 2, 3),
-                                       ("topk", 3, 4), ("sparse_attn", 4, 5))}
+                    for name, a, b in (("idx_compress", 0, 1), ("quantize_join", 1, 2), ("index_score", 2, 3),
+                                       ("topk", 3, 4), ("kv_join_sparse_attn", 4, 5))}
         cw = csa.wl
         peaks = measured_peaks()
         sha = source_sha("indexer_mma.cu", "topk.cuh", "sm100.cuh", "common.cuh", "kernels.cuh")
@@ -612,9 +662,10 @@ def run_lcsc(args):
 
     # ---- end to end: pinned host inputs -> device, step, output -> host.
     # Every step copies all of its inputs in and its outputs out.  The copies
-    # run on a second stream: a layer's inputs go up while the layer before
-    # it computes, and its output comes down while the next one computes
-    # (with one layer, the copies and the compute run one after the other).
+    # run on a stream of their own: a layer's inputs go up while the layer
+    # enqueued before it starts, and each output comes down once its layer
+    # is done (with one layer, the copies and the compute run one after the
+    # other).
     e2e = None
     if args.e2e_steps > 0:
         ins = [ly.host_inputs() for ly in layers]
@@ -626,16 +677,17 @@ def run_lcsc(args):
         done_ev = [torch.cuda.Event() for _ in layers]
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
+        order = list(range(len(layers)))[::-1] if runner.hca_first else list(range(len(layers)))
+
         def e2e_step():
             with torch.cuda.stream(copy):  # in the copy stream's order: after last step's downloads
-                for i in range(len(layers)):
+                for i in order:
                     for d, h in ins[i]:
                         d.copy_(h, non_blocking=True)
                     in_ev[i].record(copy)
-            for i, ly in enumerate(layers):
-                stream.wait_event(in_ev[i])
-                ly.run(stream)
-                done_ev[i].record(stream)
+            runner.run(before=lambda i, s: s.wait_event(in_ev[i]))
+            for i in order:
+                done_ev[i].record(runner.streams[i])
                 copy.wait_event(done_ev[i])
                 with torch.cuda.stream(copy):
                     outs[i][1].copy_(outs[i][0], non_blocking=True)
@@ -656,9 +708,9 @@ def run_lcsc(args):
         e2e_ms = max_over_ranks(ws, e0.elapsed_time(e1))
         e2e = {"value": round(job_throughput(wl.B, wl.T, ws, args.e2e_steps, e2e_ms), 2), "unit": "queries/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "copies": "pinned host buffers on a second stream: a layer's inputs upload while the layer "
-                         "before it computes and its output downloads while the next one computes; every "
-                         "copy of a step stays inside that step"}
+               "copies": "pinned host buffers on a stream of their own: a layer's inputs upload while the "
+                         "layer enqueued before it starts, each output downloads once its layer is done; "
+                         "every copy of a step stays inside that step"}
 
     if rank != 0:
         return None

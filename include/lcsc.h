@@ -20,9 +20,9 @@
  *  - State the library keeps for the life of the process: a count of the
  *    kernels it has enqueued (lcsc_kernel_launches) and, per device, two
  *    streams and three events of its own, created by the first fused CSA
- *    step on that device (lcsc_csa_decode runs the indexer keys' pooling
- *    and the query quantisation on them, joined back to the caller's
- *    stream before the scoring).  Fused CSA steps on one device share
+ *    step on that device (lcsc_csa_decode runs the KV latent's pooling and
+ *    the query quantisation on them, joined back to the caller's stream
+ *    before the attention and the scoring).  Fused CSA steps on one device share
  *    them, so steps issued on independent caller streams are ordered
  *    against each other's side work; issue independent layers' CSA steps
  *    on one stream, or accept that ordering.  Make the first fused CSA
@@ -162,11 +162,23 @@ typedef struct lcsc_params {
  *          [b][r / 128][k / 4][r % 32][(r % 128) / 32][k % 4].
  *   Indexer keys in FP8 / FP4 need a capacity that is a multiple of 128.
  * Compressed entries use row g for entry g.  A window ring uses row
- * (position mod capacity). */
+ * (position mod capacity).
+ * Entry shards (rows > 0; compressed entries only): the cache holds the
+ *   entries [row0, row0 + rows) of each sequence, entry g in row g - row0
+ *   (rows <= capacity), the way one GPU of several holds its range of a
+ *   long sequence.  Entries outside the range belong to other shards:
+ *   pooling does not write them, the indexer neither scores nor selects
+ *   them (its out_idx still holds global entry numbers), the attention
+ *   skips them without a status bit (an index outside [0, N(p)) still sets
+ *   LCSC_DEV_BAD_INDEX).  The fused steps take unsharded caches only
+ *   (rows = 0, row0 = 0: entry g in row g); lcsc_topk_merge and
+ *   lcsc_attn_merge below combine the shards' results. */
 typedef struct lcsc_cache {
   void* data;
   void* scale;
   int64_t capacity;
+  int64_t row0;   /* first entry held (shards; else 0) */
+  int64_t rows;   /* entries held from row0 (shards); 0: unsharded */
 } lcsc_cache;
 
 /* ---------------------------------------------------------------- misc */
@@ -351,10 +363,11 @@ typedef struct lcsc_step {
   float* out_score;             /* [B][T][k] their scores (CSA), or NULL */
   /* Optional stage timing (host array of cudaEvent_t, or NULL): event i is
    * recorded on `stream` at stage boundary i while i < n_events.
-   * CSA: 0 start, 1 after the KV latent's compression, 2 once the indexer
-   * keys' compression and the query quantisation (which run beside it on two
-   * more streams of the library's) are also done, 3 after indexer
-   * scoring, 4 after top-k, 5 after attention.  HCA: 0 start, 1 after
+   * CSA: 0 start, 1 after the indexer keys' compression, 2 once the query
+   * quantisation (on a stream of the library's) is also done, 3 after
+   * indexer scoring, 4 after top-k, 5 after attention (the KV latent's
+   * compression and window rows run on a second stream of the library's
+   * from 0 and are joined before the attention).  HCA: 0 start, 1 after
    * compression, 2 after attention. */
   void* const* events;
   int32_t n_events;
@@ -367,6 +380,45 @@ int32_t lcsc_csa_decode(const lcsc_params* p, const lcsc_step* s, void* workspac
                         size_t workspace_bytes, int32_t* status, void* stream);
 int32_t lcsc_hca_decode(const lcsc_params* p, const lcsc_step* s, void* workspace,
                         size_t workspace_bytes, int32_t* status, void* stream);
+
+/* ------------------------------------------------------ entry-shard merges
+ * One long sequence split by entry range over G GPUs ("Inside DeepSeek-V4",
+ * section 1: top-1,024 over the ~262K entries of a 1M-token context): GPU r
+ * holds the entries [row0_r, row0_r + rows_r) in caches with those fields
+ * set (lcsc_cache), and per step
+ *   1. lcsc_csa_index_topk on its keys gives its own top-k (global entry
+ *      numbers, with scores);
+ *   2. the G lists are gathered (a collective of the caller's) and
+ *      lcsc_topk_merge gives the top-k over all entries, the same list on
+ *      every GPU;
+ *   3. lcsc_csa_sparse_attn with that list, no sink and no output rotation
+ *      (sink NULL, out_rope_base 0) attends to the listed entries this GPU
+ *      holds; one GPU also takes the window rows (window w, the others 0);
+ *      each writes its normalised output and lse (an empty share: lse -inf);
+ *   4. the G (out, lse) pairs are gathered and lcsc_attn_merge folds them
+ *      into the output a single GPU would give, with the sink and the
+ *      inverse RoPE.
+ * Both merges are pure functions of their inputs (dev pointers, caller
+ * owned); parts are concatenated along the first dimension.
+ *
+ * lcsc_topk_merge: part_idx, part_score [n_parts][B*T][k] (k = top_k; pads
+ *   -1); out_idx [B*T][k] (and out_score, nullable): the min(k, candidates)
+ *   largest scores, ties to the lower entry, in the order of the parts
+ *   (index order for parts given in range order), padded with -1.
+ *   n_parts * k <= LCSC_MERGE_MAX_CANDIDATES.
+ * lcsc_attn_merge: part_out [n_parts][B*T][H][Dv] q_dtype, part_lse
+ *   [n_parts][B*T][H] float32; with M = max(sigma[h], lse_r) the output is
+ *   sum_r e^{lse_r - M} out_r / (e^{sigma[h] - M} + sum_r e^{lse_r - M}),
+ *   rotated back by the query position when out_rope_base > 0; lse
+ *   (nullable) [B*T][H].  sink NULL: no sink (NULL with LCSC_SINK_TOKEN:
+ *   the position-0 row is then one of the parts' rows). */
+#define LCSC_MERGE_MAX_CANDIDATES 16384
+int32_t lcsc_topk_merge(const lcsc_params* p, int32_t n_parts, const int32_t* part_idx,
+                        const float* part_score, int64_t B, int64_t T, int32_t* out_idx,
+                        float* out_score, void* stream);
+int32_t lcsc_attn_merge(const lcsc_params* p, int32_t n_parts, const void* part_out, const float* part_lse,
+                        const float* sink, const int32_t* ctx_len, int64_t B, int64_t T, void* out,
+                        float* lse, void* stream);
 
 #ifdef __cplusplus
 }

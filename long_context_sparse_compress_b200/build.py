@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "liblcsc.so")
 
-SOURCES = ["api.cu", "compress.cu", "indexer.cu", "indexer_mma.cu", "attention.cu", "attention_mma.cu"]
+SOURCES = ["api.cu", "compress.cu", "indexer.cu", "indexer_mma.cu", "attention.cu", "attention_mma.cu", "shard.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

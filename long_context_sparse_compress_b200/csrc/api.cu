@@ -101,15 +101,24 @@ int32_t tensor_fmt(const lcsc_params* p, int32_t tensor, RowFmt* f) {
   return LCSC_OK;
 }
 
-int32_t make_view(const lcsc_cache* c, const RowFmt& f, bool need_scale, CacheView* v) {
+// `shard_ok`: the cache may be an entry shard (rows > 0); every other cache
+// must have row0 = rows = 0.
+int32_t make_view(const lcsc_cache* c, const RowFmt& f, bool need_scale, CacheView* v, bool shard_ok = false) {
   if (!c || !c->data || c->capacity < 1 || !aligned16(c->data)) return LCSC_ERR_INVALID_ARG;
   if (need_scale && (!c->scale || ((uintptr_t)c->scale & 3u))) return LCSC_ERR_INVALID_ARG;
+  if (c->rows < 0 || c->row0 < 0 || (c->rows == 0 && c->row0 != 0)) return LCSC_ERR_INVALID_ARG;
+  if (c->rows > 0 && (!shard_ok || c->rows > c->capacity || c->row0 > ((int64_t)1 << 40)))
+    return LCSC_ERR_INVALID_ARG;
   v->data = reinterpret_cast<uint8_t*>(c->data);
   v->scale = c->scale;
   v->capacity = c->capacity;
   v->f = f;
+  v->row0 = c->row0;
+  v->rows = c->rows;
   return LCSC_OK;
 }
+
+bool same_shard(const lcsc_cache* a, const lcsc_cache* b) { return a->row0 == b->row0 && a->rows == b->rows; }
 
 bool needs_scale(int fmt) { return fmt != LCSC_FMT_F32; }
 
@@ -241,13 +250,13 @@ static int32_t compress_impl(const lcsc_params* p, int32_t tensor, const void* x
   if (tok_begin < 0 || tok_end < tok_begin || tok_begin % p->m) return LCSC_ERR_INVALID_ARG;
   CompressLaunch L;
   memset(&L, 0, sizeof(L));
-  if ((st = make_view(entries, f, needs_scale(f.fmt), &L.entries))) return st;
+  if ((st = make_view(entries, f, needs_scale(f.fmt), &L.entries, true))) return st;
   if (window) {
     if (tensor == LCSC_TENSOR_IDX) return LCSC_ERR_INVALID_ARG;
     if ((st = make_view(window, f, needs_scale(f.fmt), &L.window))) return st;
   }
   const int64_t g_lo = tok_begin / p->m, g_hi = tok_end / p->m;
-  if (g_hi > entries->capacity) return LCSC_ERR_INVALID_ARG;
+  if (entries->rows == 0 && g_hi > entries->capacity) return LCSC_ERR_INVALID_ARG;
   const int64_t n_new = g_hi - g_lo;
   Carve cv{reinterpret_cast<uint8_t*>(ws)};
   plan_compress(p, B, n_new, f.dim, cv, &L.pooled);
@@ -298,7 +307,7 @@ int32_t lcsc_encode_rows(const lcsc_params* p, int32_t tensor, const float* rows
   if ((st = tensor_fmt(p, tensor, &f))) return st;
   if (!rows || !aligned16(rows) || B < 1 || B > 65535 || n < 0 || row0 < 0) return LCSC_ERR_INVALID_ARG;
   CacheView v;
-  if ((st = make_view(out, f, needs_scale(f.fmt), &v))) return st;
+  if ((st = make_view(out, f, needs_scale(f.fmt), &v, true))) return st;  // a shard: its local rows
   if (row0 + n > out->capacity) return LCSC_ERR_INVALID_ARG;
   cudaError_t e = launch_encode_rows(rows, (int)B, n, row0, v, (cudaStream_t)stream);
   return e == cudaSuccess ? LCSC_OK : cuda_fail(e);
@@ -332,7 +341,7 @@ static int32_t index_setup(const lcsc_params* p, const void* q_idx, const float*
   int32_t st;
   if ((st = tensor_fmt(p, LCSC_TENSOR_IDX, &f))) return st;
   memset(L, 0, sizeof(*L));
-  if ((st = make_view(idx_keys, f, needs_scale(f.fmt), &L->keys))) return st;
+  if ((st = make_view(idx_keys, f, needs_scale(f.fmt), &L->keys, true))) return st;
   if (n_max > idx_keys->capacity) return LCSC_ERR_INVALID_ARG;
   if (f.fmt != LCSC_FMT_F32 && idx_keys->capacity % 128 != 0) return LCSC_ERR_INVALID_ARG;
   plan_index(p, B, T, n_max, cv, L);
@@ -404,10 +413,11 @@ static int32_t attn_setup(const lcsc_params* p, const void* q, const lcsc_cache*
   if ((st = tensor_fmt(p, LCSC_TENSOR_V, &fv))) return st;
   memset(L, 0, sizeof(*L));
   const bool ns = needs_scale(fk.fmt);
-  if ((st = make_view(kv, fk, ns, &L->kv))) return st;
+  if ((st = make_view(kv, fk, ns, &L->kv, true))) return st;
   if ((st = make_view(win_kv, fk, ns, &L->win_kv))) return st;
   if (sep) {
-    if ((st = make_view(v, fv, ns, &L->v))) return st;
+    if ((st = make_view(v, fv, ns, &L->v, true))) return st;
+    if (!same_shard(kv, v)) return LCSC_ERR_INVALID_ARG;
     if ((st = make_view(win_v, fv, ns, &L->win_v))) return st;
     if (win_v->capacity != win_kv->capacity) return LCSC_ERR_INVALID_ARG;
   }
@@ -533,8 +543,9 @@ static int32_t step_compress(const lcsc_params* p, const lcsc_step* s, int32_t t
 }
 
 // Two more streams per device for the parts of a CSA step that do not depend
-// on each other (the indexer keys' compression and the query quantisation
-// each run beside the KV latent's compression), with fork / join events.
+// on each other (the KV latent's compression runs beside the indexer keys'
+// compression, scoring and top-k; the query quantisation beside the indexer
+// keys' compression), with fork / join events.
 // Enqueueing on it is serialised by a mutex; the work itself is ordered
 // only by the events.
 struct SideStream {
@@ -575,6 +586,9 @@ static int32_t step_impl(const lcsc_params* p, const lcsc_step* s, void* ws, siz
   const bool sep = s->v.data != nullptr;
   if (sep != (s->win_v.data != nullptr) || sep != (s->x_v != nullptr)) return LCSC_ERR_INVALID_ARG;
   if (p->window > 0 && s->win_kv.capacity < s->T + p->window - 1) return LCSC_ERR_INVALID_ARG;
+  // the fused steps select over every entry: entry shards go through the
+  // separate calls and the merges
+  if (s->kv.rows || s->v.rows || s->idx_keys.rows) return LCSC_ERR_INVALID_ARG;
 
   Carve cv{reinterpret_cast<uint8_t*>(ws)};
   CompressLaunch ck, cvv, ci;
@@ -622,37 +636,96 @@ static int32_t step_impl(const lcsc_params* p, const lcsc_step* s, void* ws, siz
   };
   if ((e = mark()) != cudaSuccess) return cuda_fail(e);
   if (csa) {
-    // fork: indexer keys and query quantisation on two side streams
+    // Fork: the KV latent's pooling (and window rows) on one side stream,
+    // joined only before the attention, which alone reads them; the query
+    // quantisation on the other, joined before the scoring.  The indexer
+    // keys' pooling stays on the caller's stream: the scoring reads it.
+    // The lock covers every record of the shared events up to its wait.
     std::lock_guard<std::mutex> lock(g_side_mu);
     SideStream* ss = nullptr;
     if ((e = side_stream(&ss)) != cudaSuccess) return cuda_fail(e);
     if ((e = cudaEventRecord(ss->fork, strm)) != cudaSuccess) return cuda_fail(e);
     if ((e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
     if ((e = cudaStreamWaitEvent(ss->s2, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
-    if ((e = launch_compress(ci, ss->s)) != cudaSuccess) return cuda_fail(e);
+    if ((e = launch_compress(ck, ss->s)) != cudaSuccess) return cuda_fail(e);
+    if (sep && (e = launch_compress(cvv, ss->s)) != cudaSuccess) return cuda_fail(e);
     if ((e = cudaEventRecord(ss->join, ss->s)) != cudaSuccess) return cuda_fail(e);
     if ((e = launch_index_quantize(il, ss->s2)) != cudaSuccess) return cuda_fail(e);
     if ((e = cudaEventRecord(ss->join2, ss->s2)) != cudaSuccess) return cuda_fail(e);
-    if ((e = launch_compress(ck, strm)) != cudaSuccess) return cuda_fail(e);
-    if (sep && (e = launch_compress(cvv, strm)) != cudaSuccess) return cuda_fail(e);
+    if ((e = launch_compress(ci, strm)) != cudaSuccess) return cuda_fail(e);
     if ((e = mark()) != cudaSuccess) return cuda_fail(e);
-    if ((e = cudaStreamWaitEvent(strm, ss->join, 0)) != cudaSuccess) return cuda_fail(e);
     if ((e = cudaStreamWaitEvent(strm, ss->join2, 0)) != cudaSuccess) return cuda_fail(e);
-  } else {
-    if ((e = launch_compress(ck, strm)) != cudaSuccess) return cuda_fail(e);
-    if (sep && (e = launch_compress(cvv, strm)) != cudaSuccess) return cuda_fail(e);
-    if ((e = mark()) != cudaSuccess) return cuda_fail(e);
-  }
-  if (csa) {
     if ((e = mark()) != cudaSuccess) return cuda_fail(e);
     if ((e = launch_index_score_only(il, strm)) != cudaSuccess) return cuda_fail(e);
     if ((e = mark()) != cudaSuccess) return cuda_fail(e);
     if ((e = launch_topk(il, strm)) != cudaSuccess) return cuda_fail(e);
     if ((e = mark()) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaStreamWaitEvent(strm, ss->join, 0)) != cudaSuccess) return cuda_fail(e);
+  } else {
+    if ((e = launch_compress(ck, strm)) != cudaSuccess) return cuda_fail(e);
+    if (sep && (e = launch_compress(cvv, strm)) != cudaSuccess) return cuda_fail(e);
+    if ((e = mark()) != cudaSuccess) return cuda_fail(e);
   }
   if ((e = launch_attention(al, strm)) != cudaSuccess) return cuda_fail(e);
   if ((e = mark()) != cudaSuccess) return cuda_fail(e);
   return LCSC_OK;
+}
+
+// ------------------------------------------------------------ shard merges
+
+int32_t lcsc_topk_merge(const lcsc_params* p, int32_t n_parts, const int32_t* part_idx,
+                        const float* part_score, int64_t B, int64_t T, int32_t* out_idx,
+                        float* out_score, void* stream) {
+  int32_t st = check_params(p);
+  if (st) return st;
+  if (p->top_k < 1 || n_parts < 1 || (int64_t)n_parts * p->top_k > LCSC_MERGE_MAX_CANDIDATES)
+    return LCSC_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || T > 65535 || B > 65535 / T) return LCSC_ERR_INVALID_ARG;
+  if (!part_idx || !part_score || !out_idx) return LCSC_ERR_INVALID_ARG;
+  if (!aligned16(part_idx) || !aligned16(part_score) || !aligned16(out_idx)) return LCSC_ERR_INVALID_ARG;
+  if (out_score && !aligned16(out_score)) return LCSC_ERR_INVALID_ARG;
+  TopkMergeLaunch L;
+  L.n_parts = n_parts;
+  L.lists = B * T;
+  L.k = p->top_k;
+  L.part_idx = part_idx;
+  L.part_score = part_score;
+  L.out_idx = out_idx;
+  L.out_score = out_score;
+  cudaError_t e = launch_topk_merge(L, (cudaStream_t)stream);
+  return e == cudaSuccess ? LCSC_OK : cuda_fail(e);
+}
+
+int32_t lcsc_attn_merge(const lcsc_params* p, int32_t n_parts, const void* part_out, const float* part_lse,
+                        const float* sink, const int32_t* ctx_len, int64_t B, int64_t T, void* out,
+                        float* lse, void* stream) {
+  int32_t st = check_params(p);
+  if (st) return st;
+  if (n_parts < 1 || n_parts > 4096) return LCSC_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || T > 65535 || B > 65535 / T) return LCSC_ERR_INVALID_ARG;
+  if (p->v_dim != 512 && p->v_dim != 128) return LCSC_ERR_UNSUPPORTED;
+  if (p->n_heads % 4 != 0) return LCSC_ERR_UNSUPPORTED;
+  if (p->sink_mode == LCSC_SINK_TOKEN && sink) return LCSC_ERR_INVALID_ARG;
+  if (!part_out || !part_lse || !ctx_len || !out) return LCSC_ERR_INVALID_ARG;
+  if (!aligned16(part_out) || !aligned16(part_lse) || !aligned16(out)) return LCSC_ERR_INVALID_ARG;
+  if ((lse && !aligned16(lse)) || (sink && ((uintptr_t)sink & 3u))) return LCSC_ERR_INVALID_ARG;
+  AttnMergeLaunch L;
+  L.n_parts = n_parts;
+  L.lists = B * T;
+  L.T = (int)T;
+  L.H = p->n_heads;
+  L.Dv = p->v_dim;
+  L.dtype = p->q_dtype;
+  L.part_out = part_out;
+  L.part_lse = part_lse;
+  L.sink = sink;
+  L.ctx_len = ctx_len;
+  L.out_rope_dim = p->out_rope_base > 0.f ? p->out_rope_dim : 0;
+  L.out_rope_base = p->out_rope_base;
+  L.out = out;
+  L.lse = lse;
+  cudaError_t e = launch_attn_merge(L, (cudaStream_t)stream);
+  return e == cudaSuccess ? LCSC_OK : cuda_fail(e);
 }
 
 int32_t lcsc_csa_decode(const lcsc_params* p, const lcsc_step* s, void* ws, size_t ws_bytes,

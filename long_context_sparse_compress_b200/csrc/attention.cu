@@ -36,10 +36,11 @@ __device__ __forceinline__ QueryRows query_rows(const AttnLaunch& a, int b, int 
   QueryRows r;
   const int64_t L = a.ctx_len[b];
   // a context whose entries would pass the caches' n_max rows is invalid
-  r.ok = L >= a.T && L / a.m <= a.n_max;
+  // (an entry shard holds a range of them: no limit)
+  r.ok = L >= a.T && (a.kv.rows > 0 || L / a.m <= a.n_max);
   r.p = L - a.T + t;
   r.n_vis = r.ok ? (r.p + 1) / a.m : 0;
-  r.n_ent_slots = a.idx ? a.k : r.n_vis;
+  r.n_ent_slots = a.idx ? a.k : a.kv.local_count(r.n_vis);
   r.w_lo = r.p - a.w + 1 > 0 ? r.p - a.w + 1 : 0;
   r.n_win = r.ok ? r.p - r.w_lo + 1 : 0;
   if (a.w == 0) r.n_win = 0;
@@ -137,10 +138,11 @@ __global__ void __launch_bounds__(kThreads) attn_partial_kernel(AttnLaunch a) {
       int64_t row = 0;
       if (slot < s_hi) {
         if (slot < qr.n_ent_slots) {
-          const int64_t g = a.idx ? (int64_t)a.idx[(int64_t)list * a.k + slot] : slot;
+          const int64_t g = a.idx ? (int64_t)a.idx[(int64_t)list * a.k + slot] : slot + a.kv.row0;
           if (g >= 0 && g < qr.n_vis) {
-            src = 1;
-            row = g;
+            row = a.kv.local(g);  // -1: another shard holds it
+            src = row >= 0 ? 1 : 0;
+            if (row < 0) row = 0;
           } else if (g != -1 || !a.idx) {
             if (a.status) atomicOr(a.status, LCSC_DEV_BAD_INDEX);
           }

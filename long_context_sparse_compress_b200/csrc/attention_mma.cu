@@ -103,10 +103,10 @@ struct Rows {
 __device__ __forceinline__ Rows rows_of(const AttnLaunch& a, int b, int t) {
   Rows r;
   const int64_t L = a.ctx_len[b];
-  r.ok = L >= a.T && L / a.m <= a.n_max;
+  r.ok = L >= a.T && (a.kv.rows > 0 || L / a.m <= a.n_max);  // a shard holds a range: no limit
   const int64_t p = L - a.T + t;
   r.n_vis = r.ok ? (p + 1) / a.m : 0;
-  r.n_ent_slots = a.idx ? a.k : r.n_vis;
+  r.n_ent_slots = a.idx ? a.k : a.kv.local_count(r.n_vis);
   r.w_lo = p - a.w + 1 > 0 ? p - a.w + 1 : 0;
   r.n_win = (r.ok && a.w > 0) ? p - r.w_lo + 1 : 0;
   r.n_tok = (r.ok && a.sink_token && !(r.n_win > 0 && r.w_lo == 0)) ? 1 : 0;
@@ -303,10 +303,12 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
       scp = nullptr;
       if (slot >= s_hi) return nullptr;
       if (slot < qr.n_ent_slots) {
-        const int64_t g = a.idx ? (int64_t)gi : slot;
+        const int64_t g = a.idx ? (int64_t)gi : slot + a.kv.row0;
         if (g >= 0 && g < qr.n_vis) {
-          scp = a.kv.fscale(b, g);
-          return a.kv.row(b, g);
+          const int64_t r = a.kv.local(g);
+          if (r < 0) return nullptr;  // another shard holds it
+          scp = a.kv.fscale(b, r);
+          return a.kv.row(b, r);
         }
         if ((g != -1 || !a.idx) && a.status) atomicOr(a.status, LCSC_DEV_BAD_INDEX);
         return nullptr;

@@ -39,6 +39,21 @@ struct CacheView {
   void* scale;
   int64_t capacity;
   RowFmt f;
+  int64_t row0;  // an entry shard holds the entries [row0, row0 + rows) in rows 0 ..
+  int64_t rows;  // 0: unsharded (entry g in row g)
+  // Local row of global entry g in this view, or -1 when another shard holds it.
+  __host__ __device__ __forceinline__ int64_t local(int64_t g) const {
+    if (rows <= 0) return g;
+    const int64_t r = g - row0;
+    return (r >= 0 && r < rows) ? r : -1;
+  }
+  // Visible entries of this view among the first n global ones: the count of
+  // local rows 0 .. that hold entries below n.
+  __host__ __device__ __forceinline__ int64_t local_count(int64_t n) const {
+    if (rows <= 0) return n;
+    const int64_t c = n - row0;
+    return c <= 0 ? 0 : (c < rows ? c : rows);
+  }
   __device__ __forceinline__ uint8_t* row(int b, int64_t r) const {
     return data + ((int64_t)b * capacity + r) * f.row_bytes;
   }

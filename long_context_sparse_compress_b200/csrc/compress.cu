@@ -64,11 +64,12 @@ struct SeqSpan {
 
 // `cap` is the entries' capacity: a context length whose entries would not
 // fit makes the sequence invalid (nothing is written; the status flags it).
+// An entry shard holds a range of the entries (cap < 0: no limit).
 __device__ __forceinline__ SeqSpan seq_span(const Span& s, int b, int64_t win_cap, int64_t cap) {
   SeqSpan r;
   if (s.ctx_len) {
     const int64_t L = s.ctx_len[b];
-    r.ok = L >= s.T && L / s.m <= cap;
+    r.ok = L >= s.T && (cap < 0 || L / s.m <= cap);
     r.g_lo = r.ok ? (L - s.T) / s.m : 0;
     r.g_hi = r.ok ? L / s.m : 0;
     r.x_pos0 = L - (s.T + s.G - 1);
@@ -83,6 +84,11 @@ __device__ __forceinline__ SeqSpan seq_span(const Span& s, int b, int64_t win_ca
     r.w_hi = s.tok_end;
   }
   return r;
+}
+
+// Capacity bound of seq_span: none for an entry shard.
+__device__ __forceinline__ int64_t ent_cap(const CompressLaunch& a) {
+  return a.entries.rows > 0 ? -1 : a.entries.capacity;
 }
 
 // ------------------------------------------------------------ mma helpers
@@ -219,7 +225,7 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
     for (int64_t t = cta * (kThreads / kWarp) + warp; t < total; t += n_warps) {
       const int b = (int)(t / a.n_win_max);
       const int64_t i = t % a.n_win_max;
-      const SeqSpan sp = seq_span(a.span, b, a.window.capacity, a.entries.capacity);
+      const SeqSpan sp = seq_span(a.span, b, a.window.capacity, ent_cap(a));
       if (!sp.ok || i >= sp.w_hi - sp.w_lo) continue;
       const int64_t pos = sp.w_lo + i;
       const int64_t base = ((int64_t)b * a.n_x + (pos - sp.x_pos0)) * DIM + lane * VPL;
@@ -240,8 +246,9 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
       const int b = blockIdx.x * SP + e;
       int64_t src = -1;
       if (e < SP && b < a.B) {
-        const SeqSpan sp = seq_span(a.span, b, a.window.capacity, a.entries.capacity);
-        const bool valid = sp.ok && sp.g_hi - sp.g_lo == 1;
+        const SeqSpan sp = seq_span(a.span, b, a.window.capacity, ent_cap(a));
+        const int64_t row = a.entries.local(sp.g_lo);  // -1: another shard's entry
+        const bool valid = sp.ok && sp.g_hi - sp.g_lo == 1 && row >= 0;
         const int64_t pos = sp.g_lo * m + m - G + j;
         if (valid && pos >= 0) src = ((int64_t)b * a.n_x + (pos - sp.x_pos0)) * DIM;
         if (j == 0) {
@@ -249,7 +256,7 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
           ent_out[e] = valid ? (int64_t)b * a.n_new_max : -1;
           ent_row0[e] = e * G;
           ent_b[e] = b;
-          ent_g[e] = sp.g_lo;
+          ent_g[e] = row;
           atomicMax(&n_ent, e + 1);
           atomicMax(&rows_used, (e + 1) * G);
         }
@@ -261,7 +268,7 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
     }
   } else {
     const int b = blockIdx.z;
-    const SeqSpan sp = seq_span(a.span, b, a.window.capacity, a.entries.capacity);
+    const SeqSpan sp = seq_span(a.span, b, a.window.capacity, ent_cap(a));
     const int64_t n_e = sp.ok ? sp.g_hi - sp.g_lo : 0;
     const int64_t e0 = (int64_t)blockIdx.x * E;
     const int E_cta = e0 < n_e ? (int)(n_e - e0 < E ? n_e - e0 : E) : 0;
@@ -272,10 +279,11 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
       row_src[r] = (r < R && pos >= 0) ? ((int64_t)b * a.n_x + (pos - sp.x_pos0)) * DIM : -1;
     }
     for (int e = tid; e < E_cta; e += kThreads) {
-      ent_out[e] = (int64_t)b * a.n_new_max + e0 + e;
+      const int64_t row = a.entries.local(sp.g_lo + e0 + e);  // -1: another shard's entry
+      ent_out[e] = row >= 0 ? (int64_t)b * a.n_new_max + e0 + e : -1;
       ent_row0[e] = e * m;
       ent_b[e] = b;
-      ent_g[e] = sp.g_lo + e0 + e;
+      ent_g[e] = row;
     }
     if (tid == 0) {
       n_ent = E_cta;
@@ -509,7 +517,7 @@ __global__ void __launch_bounds__(256) store_kernel(CompressLaunch a) {
   const int b = blockIdx.y;
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
   const int64_t i = (int64_t)blockIdx.x * 8 + warp;
-  const SeqSpan sp = seq_span(a.span, b, a.window.capacity, a.entries.capacity);
+  const SeqSpan sp = seq_span(a.span, b, a.window.capacity, ent_cap(a));
   if (!sp.ok) {
     if (i == 0 && lane == 0 && a.status) atomicOr(a.status, LCSC_DEV_BAD_LENGTH);
     return;
@@ -519,10 +527,12 @@ __global__ void __launch_bounds__(256) store_kernel(CompressLaunch a) {
   constexpr int DIM = VPL * 32;
   float v[VPL];
   if (i < n_e) {
+    const int64_t row = a.entries.local(sp.g_lo + i);
+    if (row < 0) return;  // another shard's entry
     const float* src = a.pooled + ((int64_t)b * a.n_new_max + i) * DIM + lane * VPL;
 #pragma unroll
     for (int j = 0; j < VPL; ++j) v[j] = src[j];
-    store_row_warp<VPL>(a.entries, b, sp.g_lo + i, v, lane);
+    store_row_warp<VPL>(a.entries, b, row, v, lane);
   } else if (i < n_e + n_w) {
     const int64_t pos = sp.w_lo + (i - n_e);
     const int64_t xr = pos - sp.x_pos0;

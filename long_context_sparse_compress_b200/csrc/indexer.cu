@@ -35,14 +35,19 @@ namespace {
 
 constexpr int kBins = kTopkBins;
 
-// Entries visible to query t of sequence b.  A context length that would
-// reach past the n_max entries the call was sized for is invalid: nothing is
-// scored or selected for it, and the status flags it.
+// Key rows query t of sequence b scores: its N(p) visible entries, or for an
+// entry shard those of them the shard holds (at most n_max).  An unsharded
+// context length that would reach past the n_max entries the call was sized
+// for is invalid: nothing is scored or selected for it, and the status flags
+// it.
 __device__ __forceinline__ int64_t visible(const IndexLaunch& a, int b, int t, bool* ok) {
   const int64_t L = a.ctx_len[b];
   const int64_t p = L - a.T + t;
-  *ok = L >= a.T && L / a.m <= a.n_max;
-  return *ok ? (p + 1) / a.m : 0;
+  const bool shard = a.keys.rows > 0;
+  *ok = L >= a.T && (shard || L / a.m <= a.n_max);
+  if (!*ok) return 0;
+  const int64_t n = a.keys.local_count((p + 1) / a.m);
+  return shard && n > a.n_max ? a.n_max : n;
 }
 
 // ------------------------------------------------ indexer query quantisation
@@ -206,7 +211,7 @@ __global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int sl
   float* out_s = a.out_score ? a.out_score + (int64_t)list * a.k : nullptr;
   if (li.n <= a.k) {  // every visible entry is kept, in index order
     for (int64_t g = li.lo + threadIdx.x; g < li.hi; g += 512) {
-      out_i[g] = (int32_t)g;
+      out_i[g] = (int32_t)(g + a.keys.row0);  // global entry number
       if (out_s) out_s[g] = s[g];
     }
     return;
@@ -456,7 +461,7 @@ __global__ void __launch_bounds__(512) topk_final_kernel(IndexLaunch a) {
         const int bit = __ffs(bw) - 1;
         bw &= bw - 1;
         const int64_t g = (wt + q) * 32 + bit;
-        if (off < (uint32_t)k_eff) out_i[off] = (int32_t)g;
+        if (off < (uint32_t)k_eff) out_i[off] = (int32_t)(g + a.keys.row0);
         ++off;
       }
     }
@@ -466,8 +471,8 @@ __global__ void __launch_bounds__(512) topk_final_kernel(IndexLaunch a) {
   if (out_s) {  // the scores, gathered once every index is out (independent loads)
     __syncthreads();
     for (int64_t jj = tid; jj < k_eff; jj += 512) {
-      const int32_t g = out_i[jj];
-      out_s[jj] = (g >= 0 && g < n) ? s[g] : -INFINITY;
+      const int64_t g = (int64_t)out_i[jj] - a.keys.row0;
+      out_s[jj] = (out_i[jj] >= 0 && g >= 0 && g < n) ? s[g] : -INFINITY;
     }
   }
 }

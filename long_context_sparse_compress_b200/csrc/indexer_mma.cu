@@ -57,8 +57,26 @@ struct MmaArgs {
   uint32_t* counters;      // top-k counters [B*T][8] (zeroed)
   int64_t k;               // top-k
   bool bins_in_collect;    // several CTAs per list: the collect pass sets the threshold bins
+  int64_t shard_row0, shard_rows;  // keys of an entry shard: entries [row0, row0 + rows) in rows 0 ..
   int32_t* status;
 };
+
+// A context length the call can serve (an unsharded call must have been sized
+// for every entry the sequence has).
+__device__ __forceinline__ bool length_ok(const MmaArgs& a, int64_t L) {
+  return L >= a.T && (a.shard_rows > 0 || L / a.m <= a.n_max);
+}
+
+// Key rows the query at position p scores: its N(p) = floor((p + 1) / m)
+// visible entries, or for a shard those of them it holds (at most n_max).
+__device__ __forceinline__ int64_t rows_seen(const MmaArgs& a, int64_t p) {
+  const int64_t n = (p + 1) / a.m;
+  if (a.shard_rows <= 0) return n;
+  int64_t c = n - a.shard_row0;
+  c = c < a.shard_rows ? c : a.shard_rows;
+  c = c < a.n_max ? c : a.n_max;
+  return c > 0 ? c : 0;
+}
 
 template <int FMT, int NQ>
 struct Cfg {
@@ -167,13 +185,13 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
   const int b = blockIdx.y / groups;
   const int t0 = (blockIdx.y % groups) * NQ;
   const int64_t L = a.ctx_len[b];
-  const bool ok = L >= a.T && L / a.m <= a.n_max;
+  const bool ok = length_ok(a, L);
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(sm + C::OFF_HIST);
   const int64_t list0 = (int64_t)b * a.T + t0;
   int64_t nvis[NQ];
 #pragma unroll
-  for (int l = 0; l < NQ; ++l) nvis[l] = ok ? (L - a.T + t0 + l + 1) / a.m : 0;
-  const int64_t n_last = ok ? (L - a.T + t0 + NQ) / a.m : 0;  // N(p) of the group's last query
+  for (int l = 0; l < NQ; ++l) nvis[l] = ok ? rows_seen(a, L - a.T + t0 + l) : 0;
+  const int64_t n_last = ok ? rows_seen(a, L - a.T + t0 + NQ - 1) : 0;  // rows the group's last query sees
   const int64_t tiles = (n_last + C::TILE - 1) / C::TILE;
   const int64_t per = (tiles + a.chunks - 1) / a.chunks;
   const int64_t tile_lo = C::DYN ? 0 : (int64_t)blockIdx.x * per;
@@ -357,7 +375,7 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
       uint64_t wr[32];  // head weight pairs (w[2j], w[2j + 1]) in registers
 #pragma unroll
       for (int j = 0; j < 32; ++j) wr[j] = pack2(w_s[2 * j], w_s[2 * j + 1]);
-      const int64_t n_p = ok ? (L - a.T + t0 + 1) / a.m : 0;  // entries the query sees
+      const int64_t n_p = ok ? rows_seen(a, L - a.T + t0) : 0;  // entries the query sees
       float* score_row = a.scores + ((int64_t)b * a.T + t0) * a.stride;
       // Local tile i = r + LANES t belongs to lane r = i % LANES; this group
       // takes the lanes r = grp, grp + 2, ... (their tiles in the order i).
@@ -454,7 +472,7 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
       uint64_t wq[8];  // (w[8c + 2 (t % 4)], w[8c + 2 (t % 4) + 1]) pairs
 #pragma unroll
       for (int c = 0; c < 8; ++c) wq[c] = pack2(w_s[nq * 64 + 8 * c + 2 * j4], w_s[nq * 64 + 8 * c + 2 * j4 + 1]);
-      const int64_t n_q = ok ? (L - a.T + t0 + nq + 1) / a.m : 0;  // entries the query sees
+      const int64_t n_q = ok ? rows_seen(a, L - a.T + t0 + nq) : 0;  // entries the query sees
       const int my_row = q4 * 32 + (lane >> 2) + 8 * j4;
       float* score_row = a.scores + ((int64_t)b * a.T + t0 + nq) * a.stride;
       uint32_t* hist_q = hist_s + nq * kTopkBins;
@@ -599,6 +617,8 @@ cudaError_t launch_mma(const IndexLaunch& a, cudaStream_t stream) {
   m.hist = a.hist;
   m.counters = a.counters;
   m.k = a.k;
+  m.shard_row0 = a.keys.row0;
+  m.shard_rows = a.keys.rows;
   m.status = a.status;
   const int groups = a.T / NQ;
   const int64_t ctas = (int64_t)a.B * groups;

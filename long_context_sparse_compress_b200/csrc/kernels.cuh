@@ -116,6 +116,32 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream);
 bool attn_mma_supported(const AttnLaunch& a);
 cudaError_t launch_attn_mma(const AttnLaunch& a, cudaStream_t stream);
 
+// Merges of entry shards' results (shard.cu).
+struct TopkMergeLaunch {
+  int n_parts;
+  int64_t lists, k;            // lists = B * T
+  const int32_t* part_idx;     // [n_parts][lists][k] global entries, -1 pads
+  const float* part_score;     // [n_parts][lists][k]
+  int32_t* out_idx;            // [lists][k]
+  float* out_score;            // [lists][k] or nullptr
+};
+cudaError_t launch_topk_merge(const TopkMergeLaunch& a, cudaStream_t stream);
+
+struct AttnMergeLaunch {
+  int n_parts;
+  int64_t lists;               // B * T
+  int T, H, Dv, dtype;
+  const void* part_out;        // [n_parts][lists][H][Dv] dtype
+  const float* part_lse;       // [n_parts][lists][H]
+  const float* sink;           // [H] or nullptr
+  const int32_t* ctx_len;      // [B]
+  int out_rope_dim;
+  float out_rope_base;
+  void* out;                   // [lists][H][Dv] dtype
+  float* lse;                  // [lists][H] or nullptr
+};
+cudaError_t launch_attn_merge(const AttnMergeLaunch& a, cudaStream_t stream);
+
 // Attention split geometry: the rows of each query are cut into `splits`
 // ranges of `rows_per_split` (a multiple of `granule`); n_ctas_per_split *
 // splits CTAs run, target_ctas of them at a time, and the split count is

@@ -38,7 +38,7 @@ class Params(ctypes.Structure):
 
 
 class Cache(ctypes.Structure):
-    _fields_ = [("data", c_vp), ("scale", c_vp), ("capacity", c_i64)]
+    _fields_ = [("data", c_vp), ("scale", c_vp), ("capacity", c_i64), ("row0", c_i64), ("rows", c_i64)]
 
 
 class Step(ctypes.Structure):
@@ -78,6 +78,8 @@ _SIGS = {
     "lcsc_step_workspace_size": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_i64, c_vp]),
     "lcsc_csa_decode": (c_i32, [c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
     "lcsc_hca_decode": (c_i32, [c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
+    "lcsc_topk_merge": (c_i32, [c_vp, c_i32, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_vp]),
+    "lcsc_attn_merge": (c_i32, [c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_vp]),
 }
 
 EXPORTS = tuple(_SIGS)
@@ -164,10 +166,13 @@ def fp4_scale_index(capacity, dim):
 
 
 class DeviceCache:
-    """Stored rows of one tensor for B sequences, in device memory."""
+    """Stored rows of one tensor for B sequences, in device memory.  An entry
+    shard (``rows`` > 0) holds the entries row0 .. row0 + rows - 1 in its
+    rows 0 .. rows - 1."""
 
-    def __init__(self, B, capacity, fmt, dim, rope=0, device="cuda"):
+    def __init__(self, B, capacity, fmt, dim, rope=0, device="cuda", row0=0, rows=0):
         self.B, self.capacity, self.fmt, self.dim, self.rope = B, capacity, fmt, dim, rope
+        self.row0, self.rows = row0, rows
         if fmt == "f32":
             self.data = torch.zeros((B, capacity, dim), dtype=torch.float32, device=device)
             self.scale = None
@@ -205,7 +210,7 @@ class DeviceCache:
 
     def c(self):
         return Cache(data=self.data.data_ptr(), scale=None if self.scale is None else self.scale.data_ptr(),
-                     capacity=self.capacity)
+                     capacity=self.capacity, row0=self.row0, rows=self.rows)
 
     def seq(self, b):
         """A one-sequence view (sequence b) usable wherever a cache is."""
@@ -219,7 +224,8 @@ class _SeqView:
     def c(self):
         c = self.cache
         return Cache(data=c.data[self.b].data_ptr(),
-                     scale=None if c.scale is None else c.scale[self.b].data_ptr(), capacity=c.capacity)
+                     scale=None if c.scale is None else c.scale[self.b].data_ptr(), capacity=c.capacity,
+                     row0=c.row0, rows=c.rows)
 
 
 def null_cache():
@@ -356,6 +362,20 @@ def decode_step(p, step, csa, ws, status=None, stream=None):
     lib = load()
     fn = lib.lcsc_csa_decode if csa else lib.lcsc_hca_decode
     check(fn(ctypes.byref(p), ctypes.byref(step), ptr(ws), ws.numel(), ptr(status), stream_handle(stream)))
+
+
+def topk_merge(p, part_idx, part_score, out_idx, out_score=None, stream=None):
+    """lcsc_topk_merge: parts [n][B][T][k] -> the top-k over all of them."""
+    n, B, T = part_idx.shape[0], part_idx.shape[1], part_idx.shape[2]
+    check(load().lcsc_topk_merge(ctypes.byref(p), n, ptr(part_idx), ptr(part_score), B, T, ptr(out_idx),
+                                 ptr(out_score), stream_handle(stream)))
+
+
+def attn_merge(p, part_out, part_lse, sink, ctx_len, out, lse=None, stream=None):
+    """lcsc_attn_merge: parts [n][B][T][H][Dv] (+ lse [n][B][T][H]) -> one output."""
+    n, B, T = part_out.shape[0], part_out.shape[1], part_out.shape[2]
+    check(load().lcsc_attn_merge(ctypes.byref(p), n, ptr(part_out), ptr(part_lse), ptr(sink), ptr(ctx_len), B, T,
+                                 ptr(out), ptr(lse), stream_handle(stream)))
 
 
 __all__ = ["load", "params", "DeviceCache", "compress", "encode_rows", "index_topk", "sparse_attn",
