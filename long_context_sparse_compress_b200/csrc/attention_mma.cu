@@ -59,8 +59,8 @@ constexpr int KB_K = kTR * 128;   // one 64-dim block of a K tile (8 KB)
 constexpr int OFF_Q = 0;                       // 8 blocks = 64 KB
 constexpr int OFF_K = OFF_Q + 8 * KB_Q;        // 2 buffers x 8 blocks = 128 KB
 constexpr int OFF_P = OFF_K + 2 * 8 * KB_K;    // 2 buffers x [64 heads][128 B] = 16 KB
-constexpr int OFF_BAR = OFF_P + 2 * kH * 128;  // k_full[2] s_full[2] p_full[2] pv_done[2]
-constexpr int OFF_ROW = OFF_BAR + 8 * 8;       // int64 [4][64] (row info of tiles j % 4)
+constexpr int OFF_BAR = OFF_P + 2 * kH * 128;  // k_full[2] s_full[2] p_full[2] pv_done[2] drain
+constexpr int OFF_ROW = OFF_BAR + 9 * 8;       // int64 [4][64] (row info of tiles j % 4)
 constexpr int OFF_SRC = OFF_ROW + 4 * kTR * 8;  // int32 [4][64]
 constexpr int OFF_SCL = OFF_SRC + 4 * kTR * 4;  // float [4][64]
 constexpr int OFF_SCH = OFF_SCL + 4 * kTR * 4;  // f16x2 scale [4][64]
@@ -130,6 +130,7 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
   uint64_t* s_full = k_full + 2;
   uint64_t* p_full = k_full + 4;
   uint64_t* pv_done = k_full + 6;
+  uint64_t* drain = k_full + 8;  // every MMA issued has completed (before TMEM is freed)
   int64_t* row_s = reinterpret_cast<int64_t*>(sm + OFF_ROW);
   int32_t* src_s = reinterpret_cast<int32_t*>(sm + OFF_SRC);
   float* scl_s = reinterpret_cast<float*>(sm + OFF_SCL);
@@ -159,6 +160,7 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
       mbar_init(&p_full[i], kSW);
       mbar_init(&pv_done[i], 1);
     }
+    mbar_init(drain, 1);
     *abort = 0;
     *lstop = 0;
     fence_barrier_init();
@@ -545,6 +547,13 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
         }
       }
     }
+    // whether the loop ended or gave up, the MMAs it issued finish before the
+    // CTA frees TMEM (bounded: a commit that never arrives is left behind)
+    if (lane == 0) {
+      tc_commit(drain);
+      mbar_wait(drain, 0, a.status, kDrainLimitNs);
+    }
+    __syncwarp();
   } else {
     // =================================================== softmax warps
     const bool s_lane = lane >= 16;

@@ -271,6 +271,7 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
           return i < ntile ? tile_lo + i : -1;
         }
       };
+      int my_n = 0;       // tiles of this lane whose copies were issued
       auto load = [&](int i, int64_t tile) {  // TMA of (local) tile i, global tile `tile`, into stage i % STAGES
         const int s = i % C::STAGES;
         const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
@@ -278,6 +279,7 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
           live = false;
           return;
         }
+        ++my_n;
         mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::SFA_BYTES);
         tma_load_2d(sm + C::OFF_A + s * C::A_BYTES, &tm_k, 0, (int32_t)((int64_t)b * a.key_cap + tile * 128),
                     &full[s]);
@@ -286,7 +288,6 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
           bulk_load(sm + C::OFF_SFA + s * 1024, src, 1024, &full[s]);
         }
       };
-      int my_n = 0;       // tiles of this lane loaded so far
       bool more = true;   // whether a next one may exist
       auto load_next = [&]() {
         const int64_t tile = tile_of(my_n);
@@ -295,7 +296,6 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
           return;
         }
         load(r + C::LANES * my_n, tile);
-        ++my_n;
       };
       for (int t = 0; t < C::DIST && more && live; ++t) load_next();
       live = live && mbar_wait(qbar, 0, a.status);
@@ -322,7 +322,8 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
       tc_fence_after();
       const uint32_t idesc = FMT == LCSC_FMT_FP4 ? idesc_mxf4nvf4(128, C::N) : idesc_dense(0, 0, 128, C::N);
       int last = -1;
-      for (int t = 0; live && t < my_n; ++t) {
+      int t = 0;  // this lane's first tile whose copies were not yet consumed
+      for (; live && t < my_n; ++t) {
         if (more) {  // tile t + DIST
           load_next();
           if (!live) break;
@@ -359,6 +360,14 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
       }
       if (last >= 0)  // the accumulator of the last tile is complete before TMEM is freed
         mbar_wait(&accf[last % C::NACC], (uint32_t)(last / C::NACC) & 1u, a.status);
+      // After a wait gave up: the copies this lane issued and did not consume
+      // (and the query's, on lane 0) land before the CTA's shared memory is
+      // released; each wait is bounded again.  Nothing is left on the normal path.
+      for (; t < my_n; ++t) {
+        const int i = r + C::LANES * t;
+        mbar_wait(&full[i % C::STAGES], (uint32_t)(i / C::STAGES) & 1u, a.status, kDrainLimitNs);
+      }
+      if (r == 0 && !live) mbar_wait(qbar, 0, a.status, kDrainLimitNs);
     }
   } else if (warp >= C::EPI0) {
     // ------------------------------------------------------ epilogue

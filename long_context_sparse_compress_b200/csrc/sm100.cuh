@@ -58,6 +58,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for the phase with the given parity to complete, for at most
 // `limit_ns`; on time-out set LCSC_DEV_TIMEOUT in *status and return false.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: kernels here run for microseconds
+constexpr uint64_t kDrainLimitNs = 100000000ull;  // 0.1 s: draining copies in flight after a wait gave up
 
 // Non-blocking test of the phase with the given parity.
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
