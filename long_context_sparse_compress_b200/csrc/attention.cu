@@ -245,15 +245,15 @@ __global__ void __launch_bounds__(kThreads) attn_partial_kernel(AttnLaunch a) {
 
 // Merge of the split partials (reference max m_s, sum l_s, unnormalised
 // O_s) and the sink: one pass with a running max, every load of a batch of
-// splits in flight.  grid (B*T, H / 4); block 4 heads x DV/4 threads, four
+// splits in flight.  grid (B*T, H): one head per CTA, so that a single query
+// still spreads its splits' partials over H CTAs; block DV/4 threads, four
 // dims (one float4) per thread.
 template <int DV>
-__global__ void __launch_bounds__(DV) attn_combine_kernel(AttnLaunch a) {
+__global__ void __launch_bounds__(DV / 4) attn_combine_kernel(AttnLaunch a) {
   constexpr int U = 16;         // splits per batch
-  constexpr int TPH = DV / 4;   // threads per head
   const int list = blockIdx.x;
-  const int h = blockIdx.y * 4 + threadIdx.x / TPH;
-  const int d4 = threadIdx.x % TPH;
+  const int h = blockIdx.y;
+  const int d4 = threadIdx.x;
   const float sigma = a.sink ? a.sink[h] : -INFINITY;
   const float* ml = a.part_ml + ((int64_t)list * a.splits * a.H + h) * 2;  // split s at ml[s * H * 2]
   const float4* po = reinterpret_cast<const float4*>(a.part_o + ((int64_t)list * a.splits * a.H + h) * DV) + d4;
@@ -323,7 +323,7 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
   dim3 grid(a.splits, a.H / HPC, a.B * a.T);
   kern<<<grid, kThreads, smem, stream>>>(a);
   if ((e = counted(cudaGetLastError())) != cudaSuccess) return e;
-  attn_combine_kernel<DV><<<dim3(a.B * a.T, a.H / 4), DV, 0, stream>>>(a);
+  attn_combine_kernel<DV><<<dim3(a.B * a.T, a.H), DV / 4, 0, stream>>>(a);
   return counted(cudaGetLastError());
 }
 
@@ -358,7 +358,7 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
     cudaError_t e = launch_attn_mma(a, stream);
     if (e != cudaSuccess) return e;
     if (a.splits == 1) return cudaSuccess;  // one split per query: the kernel wrote the output
-    attn_combine_kernel<512><<<dim3(a.B * a.T, a.H / 4), 512, 0, stream>>>(a);
+    attn_combine_kernel<512><<<dim3(a.B * a.T, a.H), 128, 0, stream>>>(a);
     return counted(cudaGetLastError());
   }
   if (a.kv.f.fmt == LCSC_FMT_F32 && a.D == 128 && a.Dv == 128 && a.H % 8 == 0) {

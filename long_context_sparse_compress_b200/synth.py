@@ -17,9 +17,10 @@ alone.  Values follow the benchmark recipe:
 Layers with caller-given gate logits get per-token logit rows U ~ N(0, 1)
 aligned with the raw rows.  Layers whose sink is the position-0 token get
 that token's raw row as a sink would look: gamma times the unit mean query
-head (plus N(0, 0.01/d) noise), gamma = sqrt(D H), so that its logit is
-about 1 above the others' (a clear share of every head's weight, while its
-values, about sqrt(H) each, keep the outputs near unit scale); when the tail
+head (plus N(0, 0.01/d) noise), gamma = sqrt(D H) / 8: its logit sits
+about 0.125 above the others' and, with values of about sqrt(H) / 8 each,
+it is the row that dominates short contexts while the outputs stay within
+a few units (a query at position 0 returns the row itself); when the tail
 reaches position 0, that tail row is the same row.
 
 Rows that the layer stores as bf16 (raw rows, gate weights, queries) are
@@ -118,7 +119,7 @@ def sequence_inputs(wl, b, seed=SEED, entries=True):
             out["U_idx"] = normal(stream(seed, lay, "U_idx", b), (R, wl.d_I), 1.0)
     if wl.sink_mode == "token":
         u_q = _unit(out["q"].astype(np.float64).mean(axis=(0, 1)))
-        gamma = np.sqrt(wl.D * wl.H)
+        gamma = 0.125 * np.sqrt(wl.D * wl.H)
         x0 = gamma * u_q + normal(stream(seed, lay, "x0_kv", b), (wl.D,), 0.1 * wl.D ** -0.5)
         out["x0_kv"] = as_dtype(wl.x_dtype, x0.astype(np.float32))
         if wl.separate_v:
