@@ -167,6 +167,31 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
   }
   if (warp == kMmaWarp) tmem_alloc(tm_slot, 512);
 
+  // The rows of the first two tiles go to L2 before the query prologue, so
+  // that the loaders' first gathers, issued after it, hit L2: one bulk
+  // prefetch per dense tile of entries, one per gathered entry or window row.
+  if (warp >= kSW && warp < kMmaWarp && tid - kSW * 32 < 2 * kTR) {
+    const int lt = tid - kSW * 32, r = lt % kTR;
+    const int64_t slot = s_lo + lt;
+    const int64_t n_ent_here = s_hi < qr.n_ent_slots ? s_hi : qr.n_ent_slots;
+    const uint32_t rb = (uint32_t)a.kv.f.row_bytes;
+    if (slot < s_hi) {
+      if (slot < qr.n_ent_slots) {
+        if (a.idx) {
+          const int64_t g = a.idx[(int64_t)list * a.k + slot];
+          const int64_t lr = (g >= 0 && g < qr.n_vis) ? a.kv.local(g) : -1;
+          if (lr >= 0) prefetch_l2(a.kv.row(b, lr), rb);
+        } else if (r == 0) {
+          const int64_t cnt = n_ent_here - slot < kTR ? n_ent_here - slot : kTR;
+          prefetch_l2(a.kv.row(b, slot), (uint32_t)cnt * rb);
+        }
+      } else if (slot < qr.n_ent_slots + qr.n_win) {
+        const int64_t cap = a.win_kv.capacity;
+        prefetch_l2(a.win_kv.row(b, (qr.w_lo + (slot - qr.n_ent_slots)) % cap), rb);
+      }
+    }
+  }
+
   // ---- Q (64 x 512) -> f16, K-major swizzled blocks of 64 dims (all threads;
   // bf16 rows: every 16-byte load of a thread in flight at once).  Each head
   // is multiplied by a power of two that puts its largest |q| in

@@ -350,9 +350,10 @@ def make_step(B, T, n_max, ctx_len, x_kv, x_v, x_idx, w_kv, b_kv, w_v, b_v, w_id
 
 
 def set_step_events(step, events):
-    """Attach stage-boundary events (torch.cuda.Event, already created) to a
-    step struct; the returned array must outlive the call."""
-    arr = (c_vp * len(events))(*[e.cuda_event for e in events])
+    """Attach stage-boundary events (torch.cuda.Event, already created; None
+    for a boundary not to record) to a step struct; the returned array must
+    outlive the call."""
+    arr = (c_vp * len(events))(*[None if e is None else e.cuda_event for e in events])
     step.events = ctypes.cast(arr, ctypes.POINTER(c_vp))
     step.n_events = len(events)
     return arr
