@@ -140,9 +140,16 @@ class Layer:
 
     # host-side copies for the end-to-end measurement
     def host_inputs(self):
-        ts = [self.x_kv, self.q, self.ctx_len] + ([self.x_ik, self.q_idx, self.w_idx]
-                                                   if self.wl.kind == "csa" else [])
-        return [(t, t.cpu().pin_memory()) for t in ts]
+        """(device tensor, pinned host copy) of every input a decode step
+        receives: the T new tokens' raw rows (the G - 1 older rows of the
+        closing group arrived with earlier steps and stay on the device, the
+        way a caller keeps a group's rows in a ring written twice so that
+        they are always contiguous), the queries, the indexer queries and
+        weights, and the context lengths."""
+        T = self.wl.T
+        ts = [self.x_kv[:, -T:], self.q, self.ctx_len] + ([self.x_ik[:, -T:], self.q_idx, self.w_idx]
+                                                          if self.wl.kind == "csa" else [])
+        return [(t, t.contiguous().cpu().pin_memory()) for t in ts]
 
     def host_output(self):
         return self.out, torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
@@ -686,7 +693,7 @@ def run_lcsc(args):
                         peak_source=peaks["source"] + " hbm_gbs", **common)
 
     # ---- end to end: pinned host inputs -> device, step, output -> host.
-    # Every step copies all of its inputs in and its outputs out.  The copies
+    # Every step copies the inputs of its new tokens in and its outputs out.  The copies
     # run on a stream of their own: a layer's inputs go up while the layer
     # enqueued before it starts, and each output comes down once its layer
     # is done (with one layer, the copies and the compute run one after the
@@ -735,7 +742,10 @@ def run_lcsc(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "copies": "pinned host buffers on a stream of their own: a layer's inputs upload while the "
                          "layer enqueued before it starts, each output downloads once its layer is done; "
-                         "every copy of a step stays inside that step"}
+                         "every copy of a step stays inside that step",
+               "inputs": "per sequence and layer: the new token's raw rows, the queries, the indexer queries "
+                         "and weights (CSA), the context length; the closing group's G - 1 older raw rows "
+                         "stay on the device from earlier steps"}
 
     if rank != 0:
         return None

@@ -68,7 +68,7 @@ extern "C" {
 #define LCSC_DEV_BAD_INDEX 1       /* an index outside [0, N(p)) was skipped */
 #define LCSC_DEV_BAD_LENGTH 2      /* a ctx_len smaller than T, or past the sizes of the call */
 #define LCSC_DEV_TIMEOUT 4         /* a kernel gave up a bounded wait (no result was written) */
-#define LCSC_DEV_RANGE 8           /* a stored KV row outside the tensor-core attention's range (below) */
+#define LCSC_DEV_RANGE 8           /* reserved: no call of this version raises it */
 
 /* What the sink of a layer is (lcsc_params.sink_mode); "DeepSeek V4
  * Architecture Explained", "How compress-then-sparsify attention works": a
@@ -300,13 +300,13 @@ int32_t lcsc_csa_index_topk_noalloc(const lcsc_params* p, const void* q_idx, con
  *   kv, v (v nullable): stored entries; win_kv, win_v (win_v nullable): the
  *   window rings, which must hold positions max(0, p - w + 1) .. p.
  * Range of the 512-dim FP8 + BF16 path (64 heads; its products run on the
- * tensor cores in f16 with float32 sums): every query is used at any
- * finite bf16 magnitude (each head is scaled by a power of two into the
- * f16 range, and the scale is undone on its logits); a dequantised KV value
- * (E4M3 code x row scale, or a BF16 RoPE dim) is held as f16, so a row
- * whose scale exceeds 65504 / 448 or whose BF16 dims exceed 65504 in
- * magnitude sets LCSC_DEV_RANGE (its result is then not defined), and
- * values below 2^-14 keep f16 subnormal precision.
+ * tensor cores with float32 sums): stored rows enter as stored (E4M3 codes
+ * x E4M3, BF16 RoPE dims x BF16) and the row scale is applied in float32,
+ * so any finite row is used; every query is used at any finite magnitude
+ * (each head is scaled by a power of two, its 448 code dims written as the
+ * sum of two E4M3 numbers, and the scale is undone on its logits).  Query
+ * values below 2^-10 of their head's largest |value| keep an absolute
+ * precision of 2^-17 of it.
  * lcsc_csa_sparse_attn: S = {idx[b][t][j] >= 0} U window (idx (dev):
  *   [B][T][k] int32, e.g. from lcsc_csa_index_topk).
  * lcsc_hca_dense_attn: S = {all g < N(p)} U window. */
