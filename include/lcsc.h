@@ -19,13 +19,14 @@
  *    read before the call returns.
  *  - State the library keeps for the life of the process: a count of the
  *    kernels it has enqueued (lcsc_kernel_launches) and, per device, two
- *    streams and three events of its own, created by the first fused CSA
- *    step on that device (lcsc_csa_decode runs the KV latent's pooling and
- *    the query quantisation on them, joined back to the caller's stream
- *    before the attention and the scoring).  Fused CSA steps on one device share
- *    them, so steps issued on independent caller streams are ordered
- *    against each other's side work; issue independent layers' CSA steps
- *    on one stream, or accept that ordering.  Make the first fused CSA
+ *    streams and three events of its own, created by the first fused step
+ *    on that device (lcsc_csa_decode runs the KV latent's pooling, the
+ *    attention's query images and the query quantisation on them;
+ *    lcsc_hca_decode the query images; each joined back to the caller's
+ *    stream before the attention or the scoring).  Fused steps on one
+ *    device share them, so steps issued on independent caller streams are
+ *    ordered against each other's side work; issue independent layers'
+ *    steps on one stream, or accept that ordering.  Make the first fused
  *    call on a device before any stream capture.  The no-allocation call
  *    below also keeps a fixed array per device.
  *  - Every call enqueues its kernels on `stream` (a cudaStream_t) and

@@ -162,9 +162,12 @@ void plan_attn(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max, bool d
                AttnLaunch* L) {
   const int64_t max_rows = (dense ? n_max : p->top_k) + p->window + (p->sink_mode == LCSC_SINK_TOKEN ? 1 : 0);
   int splits, rps;
+  uint8_t* q_img = nullptr;
   if (p->kv_format == LCSC_FMT_KV && p->head_dim == 512 && p->n_heads == 64) {
-    // tensor-core path: one CTA per (query, split) for all heads, one wave
+    // tensor-core path: one CTA per (query, split) for all heads, one wave;
+    // one query image per (sequence, token)
     attention_splits(max_rows, B * T, 64, sm_count(), &splits, &rps);
+    q_img = cv.take<uint8_t>((size_t)B * T * kAttnQImageBytes);
   } else {
     const int hpc = p->kv_format == LCSC_FMT_F32 ? 8 : 16;
     attention_splits(max_rows, B * T * (p->n_heads / hpc), 32, 2 * sm_count(), &splits, &rps);
@@ -176,6 +179,7 @@ void plan_attn(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max, bool d
     L->rows_per_split = rps;
     L->part_o = po;
     L->part_ml = pml;
+    L->q_img = q_img;
   }
 }
 
@@ -468,7 +472,8 @@ int32_t lcsc_csa_sparse_attn(const lcsc_params* p, const void* q, const lcsc_cac
   if ((st = attn_setup(p, q, kv, v, win_kv, win_v, idx, sink, sink_kv, sink_v, ctx_len, B, T,
                        kv ? kv->capacity : 0, out, lse, cv, ws_bytes, status, &L)))
     return st;
-  cudaError_t e = launch_attention(L, (cudaStream_t)stream);
+  cudaError_t e = launch_attn_prepare(L, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = launch_attention(L, (cudaStream_t)stream);
   return e == cudaSuccess ? LCSC_OK : cuda_fail(e);
 }
 
@@ -484,7 +489,8 @@ int32_t lcsc_hca_dense_attn(const lcsc_params* p, const void* q, const lcsc_cach
   if ((st = attn_setup(p, q, kv, v, win_kv, win_v, nullptr, sink, sink_kv, sink_v, ctx_len, B, T, n_max,
                        out, lse, cv, ws_bytes, status, &L)))
     return st;
-  cudaError_t e = launch_attention(L, (cudaStream_t)stream);
+  cudaError_t e = launch_attn_prepare(L, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = launch_attention(L, (cudaStream_t)stream);
   return e == cudaSuccess ? LCSC_OK : cuda_fail(e);
 }
 
@@ -649,6 +655,7 @@ static int32_t step_impl(const lcsc_params* p, const lcsc_step* s, void* ws, siz
     if ((e = cudaStreamWaitEvent(ss->s2, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
     if ((e = launch_compress(ck, ss->s)) != cudaSuccess) return cuda_fail(e);
     if (sep && (e = launch_compress(cvv, ss->s)) != cudaSuccess) return cuda_fail(e);
+    if ((e = launch_attn_prepare(al, ss->s)) != cudaSuccess) return cuda_fail(e);
     if ((e = cudaEventRecord(ss->join, ss->s)) != cudaSuccess) return cuda_fail(e);
     if ((e = launch_index_quantize(il, ss->s2)) != cudaSuccess) return cuda_fail(e);
     if ((e = cudaEventRecord(ss->join2, ss->s2)) != cudaSuccess) return cuda_fail(e);
@@ -662,9 +669,18 @@ static int32_t step_impl(const lcsc_params* p, const lcsc_step* s, void* ws, siz
     if ((e = mark()) != cudaSuccess) return cuda_fail(e);
     if ((e = cudaStreamWaitEvent(strm, ss->join, 0)) != cudaSuccess) return cuda_fail(e);
   } else {
+    // the attention's query images on a side stream, beside the compression
+    std::lock_guard<std::mutex> lock(g_side_mu);
+    SideStream* ss = nullptr;
+    if ((e = side_stream(&ss)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaEventRecord(ss->fork, strm)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
+    if ((e = launch_attn_prepare(al, ss->s)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaEventRecord(ss->join, ss->s)) != cudaSuccess) return cuda_fail(e);
     if ((e = launch_compress(ck, strm)) != cudaSuccess) return cuda_fail(e);
     if (sep && (e = launch_compress(cvv, strm)) != cudaSuccess) return cuda_fail(e);
     if ((e = mark()) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaStreamWaitEvent(strm, ss->join, 0)) != cudaSuccess) return cuda_fail(e);
   }
   if ((e = launch_attention(al, strm)) != cudaSuccess) return cuda_fail(e);
   if ((e = mark()) != cudaSuccess) return cuda_fail(e);

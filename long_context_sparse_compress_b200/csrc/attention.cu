@@ -352,6 +352,10 @@ void attention_splits(int64_t max_rows, int64_t n_ctas_per_split, int granule, i
   *splits = (int)((max_rows + rps - 1) / rps);
 }
 
+cudaError_t launch_attn_prepare(const AttnLaunch& a, cudaStream_t stream) {
+  return attn_mma_supported(a) ? launch_attn_qimage(a, stream) : cudaSuccess;
+}
+
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
   const bool sep = a.v.data != nullptr;
   if (attn_mma_supported(a)) {

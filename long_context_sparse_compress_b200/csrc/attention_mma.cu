@@ -83,21 +83,25 @@ constexpr int KB_ROPE = kCodeBytes;              // RoPE block inside a tile buf
 constexpr int KBUF = kCodeBytes + kTR * 128;     // 36 KB per buffer
 constexpr int OFF_P = OFF_K + kNB * KBUF;        // 2 buffers x (E4M3 weights 8 KB + bf16 P 8 KB)
 constexpr int PBUF = 2 * kH * 128;
-constexpr int OFF_BAR = OFF_P + 2 * PBUF;        // k_full[3] k_free[3] s_full[2] p_full[2] pv_done[2] drain
-constexpr int kBars = 13;
-constexpr int OFF_ROW = OFF_BAR + kBars * 8;     // int64 [4][64]: row pointers of tiles j % 4
+constexpr int OFF_BAR = OFF_P + 2 * PBUF;  // k_full[3] k_free[3] s_full[2] p_full[2] pv_done[2] drain q_full
+constexpr int kBars = 14;
+constexpr int OFF_QSC = OFF_BAR + kBars * 8;     // float [64]: per-head power-of-two scale of q
+constexpr int OFF_ROW = OFF_QSC + kH * 4;        // int64 [4][64]: row pointers of tiles j % 4
 constexpr int OFF_SCL = OFF_ROW + 4 * kTR * 8;   // float [4][64]: row scales (0: no row)
 constexpr int OFF_MASK = OFF_SCL + 4 * kTR * 4;  // uint32 [4][2]: valid-row bits
 constexpr int OFF_TM = OFF_MASK + 32;
 constexpr int OFF_ABORT = OFF_TM + 4;
 constexpr int OFF_LSTOP = OFF_ABORT + 4;
-constexpr int OFF_QSC = OFF_LSTOP + 4;           // float [64]: per-head amax of q, then its power-of-two scale
-constexpr int SMEM = OFF_QSC + kH * 4 + 1024;
+constexpr int SMEM = OFF_LSTOP + 4 + 1024;
+// The query image a CTA copies in: the query part of this layout (E4M3
+// terms and RoPE dims, 64 KB) followed by the per-head scales.
+constexpr int kQImg = OFF_K;
+static_assert(kQImg + kH * 4 == (int)kAttnQImageBytes, "query image layout");
+static_assert(OFF_QSC % 16 == 0, "bulk copy destination");
 constexpr int kOS = kD + 4;                      // row stride (floats) of the partial O staged in shared memory
 static_assert(OFF_QR % 1024 == 0 && OFF_K % 1024 == 0 && KBUF % 1024 == 0 && OFF_P % 1024 == 0,
               "swizzle atoms need 1024-byte alignment");
 static_assert(kH * kOS * 4 <= OFF_BAR - OFF_K, "the staged partial O fits in the tile and P buffers");
-static_assert(kH * kD * 2 <= OFF_BAR - OFF_K, "the raw query fits in the tile buffers");
 static_assert(SMEM <= 232448, "shared memory per block");
 
 // Byte offset of (row, byte) in a [rows][128 B] block with the 128-byte
@@ -187,80 +191,18 @@ __device__ __forceinline__ float pow2(int e) {
   return __int_as_float((e + 127) << 23);
 }
 
-__global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
+// ---- The query image of one (sequence, token), built once and copied in by
+// every CTA of its row splits.  Per head a power of two 2^-e brings the
+// largest |q| into [128, 256); the 448 code dims become two E4M3 terms
+// (64-byte-swizzled atoms of 64 dims), the 64 RoPE dims bf16 (128-byte
+// swizzle); the image ends with 2^e per head, which the softmax multiplies
+// back into the logits.
+__global__ void __launch_bounds__(kThr) attn_qimage_kernel(const AttnLaunch a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* k_full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);  // [3] a tile's rows have landed
-  uint64_t* k_free = k_full + 3;   // [3] the P V of a tile buffer is done
-  uint64_t* s_full = k_full + 6;   // [2]
-  uint64_t* p_full = k_full + 8;   // [2]
-  uint64_t* pv_done = k_full + 10; // [2]
-  uint64_t* drain = k_full + 12;   // every MMA issued has completed (before TMEM is freed)
-  int64_t* row_s = reinterpret_cast<int64_t*>(sm + OFF_ROW);
-  float* scl_s = reinterpret_cast<float*>(sm + OFF_SCL);
-  uint32_t* mask_s = reinterpret_cast<uint32_t*>(sm + OFF_MASK);
-  uint32_t* tm_slot = reinterpret_cast<uint32_t*>(sm + OFF_TM);
-  volatile int* abort = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
-  volatile int* lstop = reinterpret_cast<volatile int*>(sm + OFF_LSTOP);  // loader-group decision
-  float* qsc_s = reinterpret_cast<float*>(sm + OFF_QSC);
-
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int list = blockIdx.y;
-  const int b = list / a.T, t = list % a.T;
-  const Rows qr = rows_of(a, b, t);
-  if (!qr.ok && tid == 0 && blockIdx.x == 0 && a.status) atomicOr(a.status, LCSC_DEV_BAD_LENGTH);
-  const int64_t total = qr.ok ? qr.n_ent_slots + qr.n_win + qr.n_tok : 0;
-  const int64_t s_lo = (int64_t)blockIdx.x * a.rows_per_split;
-  const int64_t s_hi = s_lo + a.rows_per_split < total ? s_lo + a.rows_per_split : total;
-  const int ntiles = s_hi > s_lo ? (int)((s_hi - s_lo + kTR - 1) / kTR) : 0;
-
-  if (tid < kH) qsc_s[tid] = 0.f;  // per-head amax of q (non-negative: compared as integers)
-  if (tid == 0) {
-    for (int i = 0; i < kNB; ++i) {
-      mbar_init(&k_full[i], kLT + 1);  // every loader's copies + the tile's scales and row mask
-      mbar_init(&k_free[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], kSW);
-      mbar_init(&pv_done[i], 1);
-    }
-    mbar_init(drain, 2);
-    *abort = 0;
-    *lstop = 0;
-    fence_barrier_init();
-  }
-  if (warp == kMmaWarp) tmem_alloc(tm_slot, 512);
-
-  // The rows of the first two tiles go to L2 before the query prologue, so
-  // that the loaders' first gathers, issued after it, hit L2: one bulk
-  // prefetch per dense tile of entries, one per gathered entry or window row.
-  if (warp >= kSW && warp < kPvWarp && tid - kSW * 32 < 2 * kTR) {
-    const int lt = tid - kSW * 32, r = lt % kTR;
-    const int64_t slot = s_lo + lt;
-    const int64_t n_ent_here = s_hi < qr.n_ent_slots ? s_hi : qr.n_ent_slots;
-    const uint32_t rb = (uint32_t)a.kv.f.row_bytes;
-    if (slot < s_hi) {
-      if (slot < qr.n_ent_slots) {
-        if (a.idx) {
-          const int64_t g = a.idx[(int64_t)list * a.k + slot];
-          const int64_t lr = (g >= 0 && g < qr.n_vis) ? a.kv.local(g) : -1;
-          if (lr >= 0) prefetch_l2(a.kv.row(b, lr), rb);
-        } else if (r == 0) {
-          const int64_t cnt = n_ent_here - slot < kTR ? n_ent_here - slot : kTR;
-          prefetch_l2(a.kv.row(b, slot), (uint32_t)cnt * rb);
-        }
-      } else if (slot < qr.n_ent_slots + qr.n_win) {
-        const int64_t cap = a.win_kv.capacity;
-        prefetch_l2(a.win_kv.row(b, (qr.w_lo + (slot - qr.n_ent_slots)) % cap), rb);
-      }
-    }
-  }
-
-  // ---- Q (64 x 512): per head a power of two that brings its largest |q|
-  // into [128, 256); the 448 code dims as two E4M3 terms (64-byte-swizzled
-  // atoms of 64 dims), the 64 RoPE dims as bf16 (128-byte swizzle).  The
-  // softmax multiplies the head's logits back (qsc_s holds 2^e per head).
+  float* qsc_s = reinterpret_cast<float*>(sm + kQImg);  // per-head amax of q, then 2^e
+  const int tid = threadIdx.x, lane = tid % 32;
+  const int list = blockIdx.x;
   constexpr int kQChunks = kH * (kD / 8), kQIter = (kQChunks + kThr - 1) / kThr;
   static_assert(kThr % 64 == 0 && (kD / 8) == 64 && kQChunks % kThr == 0,
                 "the lanes of a warp share one head per chunk round; every thread has kQIter chunks");
@@ -271,15 +213,15 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
     return pow2(-ex);
   };
   const bool q_bf = a.q_dtype == LCSC_DT_BF16;
-  uint4* q_stash = reinterpret_cast<uint4*>(sm + OFF_K);  // raw bf16 chunks between the passes
   auto f32_chunk = [&](int i, float (&v)[8]) {
     const int64_t base = ((int64_t)list * a.H + i / (kD / 8)) * kD + (i % (kD / 8)) * 8;
 #pragma unroll
     for (int j = 0; j < 8; ++j) v[j] = load_elem(a.q, base + j, a.q_dtype);
   };
-  __syncthreads();  // the amax slots are zero
+  if (tid < kH) qsc_s[tid] = 0.f;  // amax slots (non-negative: compared as integers)
+  __syncthreads();
+  uint4 raw[kQIter];  // bf16 queries stay in registers between the passes
   if (q_bf) {
-    uint4 raw[kQIter];
 #pragma unroll
     for (int u = 0; u < kQIter; ++u)
       raw[u] = reinterpret_cast<const uint4*>(a.q)[(int64_t)list * a.H * (kD / 8) + tid + u * kThr];
@@ -292,7 +234,6 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
       for (int j = 0; j < 4; ++j) mb = max(mb, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
       const float mx = warp_max(__uint_as_float(mb << 16));  // one head per warp and round
       if (lane == 0) atomicMax(reinterpret_cast<int*>(qsc_s) + i / (kD / 8), __float_as_int(mx));
-      q_stash[i] = raw[u];
     }
   } else {
     for (int u = 0; u < kQIter; ++u) {
@@ -306,14 +247,14 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
     }
   }
   __syncthreads();
+#pragma unroll
   for (int u = 0; u < kQIter; ++u) {
     const int i = tid + u * kThr;
     const int h = i / (kD / 8), d0 = (i % (kD / 8)) * 8;
     const float f = q_mult(h);
     float v[8];
     if (q_bf) {
-      const uint4 r = q_stash[i];
-      const uint16_t* bf = reinterpret_cast<const uint16_t*>(&r);
+      const uint16_t* bf = reinterpret_cast<const uint16_t*>(&raw[u]);
 #pragma unroll
       for (int j = 0; j < 8; ++j) v[j] = bf16_val(bf[j]) * f;
     } else {
@@ -335,13 +276,72 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
           make_uint4(bf16x2(v[0], v[1]), bf16x2(v[2], v[3]), bf16x2(v[4], v[5]), bf16x2(v[6], v[7]));
     }
   }
-  __syncthreads();  // every multiplier was read (and the stash is dead): the slots now take 2^e
+  __syncthreads();  // every multiplier was read: the slots now take 2^e
   if (tid < kH) qsc_s[tid] = 1.f / q_mult(tid);
-  fence_async_smem();
+  __syncthreads();
+  uint4* dst = reinterpret_cast<uint4*>(a.q_img + (size_t)list * kAttnQImageBytes);
+  const uint4* src = reinterpret_cast<const uint4*>(sm);
+  for (int i = tid; i < (int)(kAttnQImageBytes / 16); i += kThr) dst[i] = src[i];
+}
+
+__global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* k_full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);  // [3] a tile's rows have landed
+  uint64_t* k_free = k_full + 3;   // [3] the P V of a tile buffer is done
+  uint64_t* s_full = k_full + 6;   // [2]
+  uint64_t* p_full = k_full + 8;   // [2]
+  uint64_t* pv_done = k_full + 10; // [2]
+  uint64_t* drain = k_full + 12;   // every MMA issued has completed (before TMEM is freed)
+  uint64_t* q_full = k_full + 13;  // the query image has landed
+  int64_t* row_s = reinterpret_cast<int64_t*>(sm + OFF_ROW);
+  float* scl_s = reinterpret_cast<float*>(sm + OFF_SCL);
+  uint32_t* mask_s = reinterpret_cast<uint32_t*>(sm + OFF_MASK);
+  uint32_t* tm_slot = reinterpret_cast<uint32_t*>(sm + OFF_TM);
+  volatile int* abort = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
+  volatile int* lstop = reinterpret_cast<volatile int*>(sm + OFF_LSTOP);  // loader-group decision
+  float* qsc_s = reinterpret_cast<float*>(sm + OFF_QSC);
+
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int list = blockIdx.y;
+  const int b = list / a.T, t = list % a.T;
+  const Rows qr = rows_of(a, b, t);
+  if (!qr.ok && tid == 0 && blockIdx.x == 0 && a.status) atomicOr(a.status, LCSC_DEV_BAD_LENGTH);
+  const int64_t total = qr.ok ? qr.n_ent_slots + qr.n_win + qr.n_tok : 0;
+  const int64_t s_lo = (int64_t)blockIdx.x * a.rows_per_split;
+  const int64_t s_hi = s_lo + a.rows_per_split < total ? s_lo + a.rows_per_split : total;
+  const int ntiles = s_hi > s_lo ? (int)((s_hi - s_lo + kTR - 1) / kTR) : 0;
+
+  if (tid == 0) {
+    for (int i = 0; i < kNB; ++i) {
+      mbar_init(&k_full[i], kLT + 1);  // every loader's copies + the tile's scales and row mask
+      mbar_init(&k_free[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], kSW);
+      mbar_init(&pv_done[i], 1);
+    }
+    mbar_init(drain, 2);
+    mbar_init(q_full, 1);
+    *abort = 0;
+    *lstop = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) tmem_alloc(tm_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tm_slot;
+  if (tid == 0) {
+    // the query image (attn_qimage_kernel): E4M3 terms, RoPE dims and
+    // per-head scales, in this layout, by two bulk copies; waited for by the
+    // Q K^T issuer and the softmax warps (this thread among them)
+    const uint8_t* img = a.q_img + (size_t)list * kAttnQImageBytes;
+    mbar_arrive_expect_tx(q_full, (uint32_t)kAttnQImageBytes);
+    bulk_load(sm + OFF_QHI, img, kQImg, q_full);
+    bulk_load(qsc_s, img + kQImg, kH * 4, q_full);
+  }
 
   if (warp >= kSW && warp < kPvWarp) {
     // =================================================== loader warps
@@ -546,6 +546,7 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
     };
     if (warp == kMmaWarp) {
       for (int j = 0; j < ntiles; ++j) {
+        if (j == 0 && !warp_wait(q_full, 0, a, abort)) break;
         if (!warp_wait(&k_full[j % kNB], (uint32_t)(j / kNB) & 1u, a, abort)) break;
         if (j >= 2 && !warp_wait(&p_full[j & 1], (uint32_t)((j - 2) >> 1) & 1u, a, abort)) break;
         tc_fence_after();
@@ -575,6 +576,9 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
     // group g; register k: head (k / 2) % 2, group k / 4, column k % 2.
     const int q4 = lane & 3;
     const int hh[2] = {warp * 16 + (lane >> 2), warp * 16 + (lane >> 2) + 8};
+    // the query's per-head scales (and, for warp 0's first thread, the end of
+    // the copy it issued, before the CTA can exit)
+    const bool q_in = warp_wait(q_full, 0, a, abort);
     const uint32_t o_addr = tmem + ((uint32_t)(warp * 32) << 16);
     const uint32_t s_addr = o_addr + (16u << 16);
     float c2[2], m_ref[2], l_part[2], gw[2];
@@ -590,7 +594,7 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
       gw[e] = 1.f;
       o_live[e] = g_set[e] = false;
     }
-    for (int j = 0; j < ntiles; ++j) {
+    for (int j = 0; q_in && j < ntiles; ++j) {
       const int sb = j & 1, slot = j & 3;
       // k_full orders the loaders' row mask and scales before these reads; s_full the TMEM S
       if (!warp_wait(&k_full[j % kNB], (uint32_t)(j / kNB) & 1u, a, abort)) break;
@@ -829,6 +833,14 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
 bool attn_mma_supported(const AttnLaunch& a) {
   return a.kv.f.fmt == LCSC_FMT_KV && a.D == 512 && a.Dv == 512 && a.H == 64 && a.v.data == nullptr &&
          a.kv.f.row_bytes == 576 && a.kv.f.rope == 64 && a.rows_per_split % kTR == 0;
+}
+
+cudaError_t launch_attn_qimage(const AttnLaunch& a, cudaStream_t stream) {
+  constexpr int kImgSmem = (int)kAttnQImageBytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(attn_qimage_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kImgSmem);
+  if (e != cudaSuccess) return e;
+  attn_qimage_kernel<<<a.B * a.T, kThr, kImgSmem, stream>>>(a);
+  return counted(cudaGetLastError());
 }
 
 cudaError_t launch_attn_mma(const AttnLaunch& a, cudaStream_t stream) {

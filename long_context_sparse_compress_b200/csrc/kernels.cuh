@@ -105,6 +105,7 @@ struct AttnLaunch {
   int rows_per_split;
   float* part_o;        // [B*T][splits][H][Dv]
   float* part_ml;       // [B*T][splits][H][2]
+  uint8_t* q_img;       // [B*T][kAttnQImageBytes]: the tensor-core path's query images
   void* out;            // [B][T][H][Dv] q_dtype
   float* lse;           // [B][T][H] or nullptr
   int32_t* status;
@@ -112,9 +113,14 @@ struct AttnLaunch {
 
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream);
 
-// Tensor-core attention (64 heads, 512-d FP8 + BF16 rows, V = K).
+// Tensor-core attention (64 heads, 512-d FP8 + BF16 rows, V = K).  Its
+// query images (launch_attn_qimage, or launch_attn_prepare, which launches
+// it only for this path) must be built before the attention runs.
+constexpr size_t kAttnQImageBytes = 64 * 1024 + 64 * 4;
 bool attn_mma_supported(const AttnLaunch& a);
+cudaError_t launch_attn_qimage(const AttnLaunch& a, cudaStream_t stream);
 cudaError_t launch_attn_mma(const AttnLaunch& a, cudaStream_t stream);
+cudaError_t launch_attn_prepare(const AttnLaunch& a, cudaStream_t stream);
 
 // Merges of entry shards' results (shard.cu).
 struct TopkMergeLaunch {

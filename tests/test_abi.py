@@ -109,14 +109,16 @@ def test_bad_arguments_are_rejected_before_launch(lib):
 
 def _attn_splits(lib, wl, B, T, n_max, dense):
     """The attention's split count, read back from its workspace size: one
-    [B*T][splits][H][Dv] fp32 partial O and one [B*T][splits][H][2] fp32
-    (max, sum) array, each rounded up to 256 bytes."""
+    [B*T][splits][H][Dv] fp32 partial O, one [B*T][splits][H][2] fp32
+    (max, sum) array and the tensor-core path's [B*T] query images of
+    64 KB + 256 B, each rounded up to 256 bytes."""
     p = L.params(wl)
     out = ctypes.c_size_t(0)
     assert lib.lcsc_attn_workspace_size(ctypes.byref(p), B, T, n_max, int(dense), ctypes.byref(out)) == 0
     up = lambda x: (x + 255) // 256 * 256
+    img = up(B * T * (65536 + 256))
     for s in range(1, 4096):
-        if up(B * T * s * wl.H * wl.Dv * 4) + up(B * T * s * wl.H * 2 * 4) == out.value:
+        if up(B * T * s * wl.H * wl.Dv * 4) + up(B * T * s * wl.H * 2 * 4) + img == out.value:
             return s
     raise AssertionError(f"no split count gives {out.value} bytes")
 

@@ -127,14 +127,14 @@ def test_step_twice_is_deterministic(cuda_lib):
     # every sequence completes a group this step (16384 and 6000 are multiples
     # of 4): pooling of the indexer keys and of the KV latent, one cluster per
     # sequence, each storing its rows (2); query quantisation + tensor-core
-    # scoring (2); top-k collect + final (2); attention with several splits
-    # per query + the combine pass (2)
-    ("csa_fp4_decode", 8),
+    # scoring (2); top-k collect + final (2); the attention's query images,
+    # the attention with several splits per query and the combine pass (3)
+    ("csa_fp4_decode", 9),
     # 4096 and 1152 complete a 128-token group: one pooling launch that stores
-    # the entries and window rows itself (three clusters fit); attention over
-    # at most 32 entries + 128 window rows runs one split per query, which
-    # writes the output itself
-    ("hca_decode", 2),
+    # the entries and window rows itself (three clusters fit); the query
+    # images, and attention over at most 32 entries + 128 window rows in one
+    # split per query, which writes the output itself
+    ("hca_decode", 3),
 ])
 def test_library_counts_its_launches(cuda_lib, name, expected):
     from long_context_sparse_compress_b200 import lib as L
