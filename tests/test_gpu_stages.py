@@ -155,6 +155,17 @@ def test_index_topk_many_lists(cuda_lib, fmt, B, T):
     check_index_topk(fmt, lengths, T=T, seed=22)
 
 
+def test_index_topk_whole_lists(cuda_lib):
+    """Four FP8 queries per scoring CTA and one CTA per query group (600
+    lists: chunked prefill's configuration, where each CTA's own histograms
+    give its lists' threshold bins): lists shorter than k, one of exactly k
+    entries, long lists, and a run of equal keys."""
+    rng = np.random.default_rng(23)
+    lengths = [4 * 200 + 1, 4 * 300 + 3, 4 * 20000, 4 * 9000 + 2]
+    lengths += [int(v) for v in rng.integers(4 * 300, 4 * 2500, size=146)]
+    check_index_topk("fp8", lengths, T=4, seed=24)
+
+
 def test_topk_resolves_the_last_digit(cuda_lib):
     """Forty keys whose scores are s0 (1 + 4e-6 j), about seven to a bin of
     the first 24 key bits: the 17th largest falls inside such a bin, so the
