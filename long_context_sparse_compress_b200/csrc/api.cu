@@ -41,18 +41,6 @@ struct Carve {
 
 bool valid_format(int fmt) { return fmt >= LCSC_FMT_F32 && fmt <= LCSC_FMT_FP4; }
 
-// SMs of the current device (for sizing grids that fill it); 148 when the
-// host has no device (sizes then only matter for workspace queries).
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      n <= 0) {
-    cudaGetLastError();
-    return 148;
-  }
-  return n;
-}
-
 int32_t check_params(const lcsc_params* p) {
   if (!p) return LCSC_ERR_INVALID_ARG;
   if (p->m < 1 || p->group_len < p->m || p->group_len > 2 * p->m) return LCSC_ERR_INVALID_ARG;

@@ -577,17 +577,6 @@ bool map_rows(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t row
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
 // Queries per CTA (the MMA's N = 64 per query): four FP8 queries when T
 // allows it, else one.
 int queries_per_cta(const IndexLaunch& a) { return a.keys.f.fmt == LCSC_FMT_FP8 && a.T % 4 == 0 ? 4 : 1; }

@@ -45,6 +45,18 @@ cudaError_t launch_compress(const CompressLaunch& a, cudaStream_t stream);
 cudaError_t launch_encode_rows(const float* rows, int B, int64_t n, int64_t row0,
                                const CacheView& out, cudaStream_t stream);
 
+// SMs of the current device (for sizing grids that fill it); 148 when the
+// host has no device (sizes then only matter for workspace queries).
+inline int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
+
 struct IndexLaunch {
   const void* q_idx;    // [B][T][H_I][d_I] q_dtype
   int q_dtype;
