@@ -86,13 +86,17 @@ struct Cfg {
   static constexpr int KSTEPS = 4 - (FMT == LCSC_FMT_FP4 ? 2 : 0);  // 32 bytes of K per MMA
   // Ring depth: enough bytes in flight to cover DRAM latency, and more than
   // half the shared memory so that a second CTA never shares the SM's TMEM.
-  static constexpr int STAGES = FMT == LCSC_FMT_FP4 ? 20 : (NQ == 1 ? 8 : 6);
+  static constexpr int STAGES = FMT == LCSC_FMT_FP4 ? (NQ == 1 ? 20 : 16) : (NQ == 1 ? 8 : 6);
   // Accumulators in TMEM: the MMA runs up to NACC tiles ahead of the epilogue.
   static constexpr int NACC = NQ == 1 ? 4 : 2;
   // TMA + MMA lanes (warps 0 .. LANES-1) and how many of its own tiles each
   // loads ahead; LANES * DIST < STAGES keeps every wait on an earlier tile.
-  static constexpr int LANES = FMT == LCSC_FMT_FP4 ? 4 : 2;
+  static constexpr int LANES = FMT == LCSC_FMT_FP4 && NQ == 1 ? 4 : 2;
   static constexpr int DIST = STAGES / LANES - 1;
+  // Lane r's tiles i = r, r + LANES, ... use accumulators i % NACC: each
+  // accumulator belongs to one lane, whose waits on it then never fall two
+  // phases behind.
+  static_assert(NACC % LANES == 0, "one lane per accumulator");
   // Epilogue: GROUPS groups of four warps from warp EPI0 on (warp w reads
   // TMEM sub-partition w % 4).  Several queries: group g drains query g of
   // every tile.
@@ -181,24 +185,25 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_TMEM);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int groups = a.T / NQ;
+  const int groups = (a.T + NQ - 1) / NQ;  // the last may hold fewer than NQ queries
   const int b = blockIdx.y / groups;
   const int t0 = (blockIdx.y % groups) * NQ;
+  const int nq_here = a.T - t0 < NQ ? a.T - t0 : NQ;  // queries this group holds
   const int64_t L = a.ctx_len[b];
   const bool ok = length_ok(a, L);
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(sm + C::OFF_HIST);
   const int64_t list0 = (int64_t)b * a.T + t0;
   int64_t nvis[NQ];
 #pragma unroll
-  for (int l = 0; l < NQ; ++l) nvis[l] = ok ? rows_seen(a, L - a.T + t0 + l) : 0;
-  const int64_t n_last = ok ? rows_seen(a, L - a.T + t0 + NQ - 1) : 0;  // rows the group's last query sees
+  for (int l = 0; l < NQ; ++l) nvis[l] = ok && l < nq_here ? rows_seen(a, L - a.T + t0 + l) : 0;
+  const int64_t n_last = ok ? rows_seen(a, L - a.T + t0 + nq_here - 1) : 0;  // rows the group's last query sees
   const int64_t tiles = (n_last + C::TILE - 1) / C::TILE;
   const int64_t per = (tiles + a.chunks - 1) / a.chunks;
   const int64_t tile_lo = C::DYN ? 0 : (int64_t)blockIdx.x * per;
   const int64_t tile_hi = C::DYN ? tiles : (tile_lo + per < tiles ? tile_lo + per : tiles);
   uint32_t* tile_ctr = a.counters + list0 * 8 + 4;  // claimed batches (DYN), zeroed with the histograms
   if (tile_hi <= tile_lo) {  // uniform over the CTA, before any barrier or TMEM use
-    hist_finish(hist_s, false, NQ, a.hist, a.counters, list0, list0, gridDim.x, nvis, a.k, !a.bins_in_collect);
+    hist_finish(hist_s, false, nq_here, a.hist, a.counters, list0, list0, gridDim.x, nvis, a.k, !a.bins_in_collect);
     return;
   }
   for (int i = threadIdx.x; i < NQ * kTopkBins; i += blockDim.x) hist_s[i] = 0u;
@@ -221,8 +226,11 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
   }
   for (int i = threadIdx.x; i < C::N; i += blockDim.x) {
     const int64_t list = (int64_t)b * a.T + t0 + i / 64;
-    float wv = a.w_idx[list * 64 + (i % 64)];
-    if (FMT == LCSC_FMT_FP8) wv *= reinterpret_cast<const float*>(a.q_scale)[list * 64 + (i % 64)];
+    float wv = 0.f;  // a slot past the group's last query scores nothing
+    if (i / 64 < nq_here) {
+      wv = a.w_idx[list * 64 + (i % 64)];
+      if (FMT == LCSC_FMT_FP8) wv *= reinterpret_cast<const float*>(a.q_scale)[list * 64 + (i % 64)];
+    }
     w_s[i] = wv;
   }
   if (warp == 2) tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -481,7 +489,8 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
       uint64_t wq[8];  // (w[8c + 2 (t % 4)], w[8c + 2 (t % 4) + 1]) pairs
 #pragma unroll
       for (int c = 0; c < 8; ++c) wq[c] = pack2(w_s[nq * 64 + 8 * c + 2 * j4], w_s[nq * 64 + 8 * c + 2 * j4 + 1]);
-      const int64_t n_q = ok ? rows_seen(a, L - a.T + t0 + nq) : 0;  // entries the query sees
+      // entries the query sees (none past the group's last query)
+      const int64_t n_q = ok && nq < nq_here ? rows_seen(a, L - a.T + t0 + nq) : 0;
       const int my_row = q4 * 32 + (lane >> 2) + 8 * j4;
       float* score_row = a.scores + ((int64_t)b * a.T + t0 + nq) * a.stride;
       uint32_t* hist_q = hist_s + nq * kTopkBins;
@@ -546,7 +555,7 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
-  hist_finish(hist_s, true, NQ, a.hist, a.counters, list0, list0, gridDim.x, nvis, a.k, !a.bins_in_collect);
+  hist_finish(hist_s, true, nq_here, a.hist, a.counters, list0, list0, gridDim.x, nvis, a.k, !a.bins_in_collect);
 }
 
 // ---------------------------------------------------------------- host side
@@ -577,9 +586,14 @@ bool map_rows(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t row
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Queries per CTA (the MMA's N = 64 per query): four FP8 queries when T
-// allows it, else one.
-int queries_per_cta(const IndexLaunch& a) { return a.keys.f.fmt == LCSC_FMT_FP8 && a.T % 4 == 0 ? 4 : 1; }
+// Queries per CTA (the MMA's N = 64 per query): four FP8 queries when T is
+// a multiple of four (chunked prefill), two FP4 queries whenever T > 1 (the
+// two share one 128-row tile of block scales; an odd T leaves the last group
+// one query), else one.
+int queries_per_cta(const IndexLaunch& a) {
+  if (a.keys.f.fmt == LCSC_FMT_FP8) return a.T % 4 == 0 ? 4 : 1;
+  return a.T > 1 ? 2 : 1;
+}
 
 // CTAs per query group: as many as fit beside the other groups' on the SMs
 // (one CTA per SM), at least one.  One query per CTA claims its tiles at run
@@ -587,7 +601,8 @@ int queries_per_cta(const IndexLaunch& a) { return a.keys.f.fmt == LCSC_FMT_FP8 
 // fit they share the list; a CTA that waits for an SM joins its list late
 // and takes what is left.
 int chunks_per_group(const IndexLaunch& a) {
-  const int64_t ctas = (int64_t)a.B * (a.T / queries_per_cta(a));
+  const int q = queries_per_cta(a);
+  const int64_t ctas = (int64_t)a.B * ((a.T + q - 1) / q);
   if (ctas >= sm_count()) return 1;
   const int fit = (int)(sm_count() / ctas);
   return queries_per_cta(a) == 1 && fit < 2 ? 2 : fit;
@@ -618,7 +633,7 @@ cudaError_t launch_mma(const IndexLaunch& a, cudaStream_t stream) {
   m.shard_row0 = a.keys.row0;
   m.shard_rows = a.keys.rows;
   m.status = a.status;
-  const int groups = a.T / NQ;
+  const int groups = (a.T + NQ - 1) / NQ;
   const int64_t ctas = (int64_t)a.B * groups;
   m.chunks = chunks_per_group(a);
   m.bins_in_collect = index_bins_in_collect(a);
@@ -651,7 +666,8 @@ bool index_mma_supported(const IndexLaunch& a) {
 }
 
 cudaError_t launch_index_mma(const IndexLaunch& a, cudaStream_t stream) {
-  if (a.keys.f.fmt == LCSC_FMT_FP4) return launch_mma<LCSC_FMT_FP4, 1>(a, stream);
+  if (a.keys.f.fmt == LCSC_FMT_FP4)
+    return queries_per_cta(a) == 2 ? launch_mma<LCSC_FMT_FP4, 2>(a, stream) : launch_mma<LCSC_FMT_FP4, 1>(a, stream);
   if (queries_per_cta(a) == 4) return launch_mma<LCSC_FMT_FP8, 4>(a, stream);
   return launch_mma<LCSC_FMT_FP8, 1>(a, stream);
 }
