@@ -446,7 +446,7 @@ def job_throughput(B, T, ws, steps, ms_total):
 
 L2_BYTES = 126 * 2 ** 20
 SUB_WORKLOADS = (workloads.PAIR_DECODE_1M_B1.name, workloads.CSA_DECODE_128K.name,
-                 workloads.CSA_PREFILL_256K.name)
+                 workloads.CSA_PREFILL_256K.name, workloads.PAIR_DECODE_1M_B16_T5.name)
 
 
 def measure_sub(name, dev, peaks, warmup, target_s=0.4, max_steps=5000):
