@@ -151,9 +151,11 @@ void plan_attn(const lcsc_params* p, int64_t B, int64_t T, int64_t n_max, bool d
   const int64_t max_rows = (dense ? n_max : p->top_k) + p->window + (p->sink_mode == LCSC_SINK_TOKEN ? 1 : 0);
   int splits, rps;
   uint8_t* q_img = nullptr;
-  if (p->kv_format == LCSC_FMT_KV && p->head_dim == 512 && p->n_heads == 64) {
-    // tensor-core path: one CTA per (query, split) for all heads, one wave;
-    // one query image per (sequence, token)
+  const bool tc = p->kv_format == LCSC_FMT_KV && p->head_dim == 512 && p->v_dim == 512 && p->n_heads == 64 &&
+                  p->rope_dim == 64;
+  if (tc) {
+    // tensor-core path (attn_mma_supported): one CTA per (query, split) for
+    // all heads, one wave; one query image per (sequence, token)
     attention_splits(max_rows, B * T, 64, sm_count(), &splits, &rps);
     q_img = cv.take<uint8_t>((size_t)B * T * kAttnQImageBytes);
   } else {

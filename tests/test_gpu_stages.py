@@ -259,10 +259,14 @@ def _attn_case(kind, fmt_kv, rng):
 
 
 @pytest.mark.parametrize("kind", ["csa", "hca"])
-@pytest.mark.parametrize("fmt_kv", ["f32", "kv"])
-def test_attention_matches_oracle(cuda_lib, kind, fmt_kv):
+@pytest.mark.parametrize("fmt_kv,q_dtype", [("f32", None), ("kv", None), ("kv", "f32")])
+def test_attention_matches_oracle(cuda_lib, kind, fmt_kv, q_dtype):
+    """fp32 rows (CUDA-core path) and FP8 + BF16 rows (tensor-core path),
+    the latter with bf16 queries and outputs and with fp32 ones."""
     rng = np.random.default_rng(31)
     wl = _attn_case(kind, fmt_kv, rng)
+    if q_dtype:
+        wl = wl.with_(q_dtype=q_dtype)
     T = 2
     lengths = [3000, 30, 1500]                 # one context shorter than the window
     B = len(lengths)
