@@ -352,7 +352,10 @@ def layer_step_bytes(lw):
 def layer_step_flops(lw):
     """Algorithmic flops of one step of a layer, by the operand type of the
     contraction that carries them: {"fp4" / "fp8" / "f32": indexer scoring,
-    "bf16": attention (f16 MMA, the same tensor rate) and the gate GEMM}."""
+    "bf16": attention and the gate GEMM}.  The attention's code dims run as
+    pairs of E4M3 MMAs (two-term query and weights), which together take the
+    time of one bf16 MMA, and its RoPE dims as bf16 MMAs: its flops count at
+    the bf16 rate."""
     out = {}
     T, m = lw.T, lw.m
     pos = [lw.L - T + t for t in range(T)]
