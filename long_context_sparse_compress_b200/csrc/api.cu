@@ -1,5 +1,6 @@
 // The C ABI (include/lcsc.h): argument validation, workspace planning and
 // the launch sequence of every call.  No device memory is allocated here.
+#include <stdlib.h>
 #include <string.h>
 
 #include <atomic>
@@ -13,6 +14,14 @@ namespace lcsc {
 std::atomic<uint64_t> g_kernel_launches{0};
 
 void note_launch() { g_kernel_launches.fetch_add(1, std::memory_order_relaxed); }
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("LCSC_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
 
 namespace {
 

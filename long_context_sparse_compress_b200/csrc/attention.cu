@@ -88,6 +88,7 @@ __device__ __forceinline__ void load_row(const CacheView& cv, int b, int64_t r, 
 // grid: (splits, H / HPC, B*T); block 256.
 template <int KVFMT, int D, int DV, int HPC, bool kSepV>
 __global__ void __launch_bounds__(kThreads) attn_partial_kernel(AttnLaunch a) {
+  grid_dep_wait();
   constexpr int KS = D + 1, VS = DV + 1;
   constexpr int TPH = kThreads / HPC;      // threads per head
   constexpr int OPT = DV / TPH;            // outputs per thread
@@ -250,6 +251,7 @@ __global__ void __launch_bounds__(kThreads) attn_partial_kernel(AttnLaunch a) {
 // dims (one float4) per thread.
 template <int DV>
 __global__ void __launch_bounds__(DV / 4) attn_combine_kernel(AttnLaunch a) {
+  grid_dep_wait();
   constexpr int U = 16;         // splits per batch
   const int list = blockIdx.x;
   const int h = blockIdx.y;
@@ -321,10 +323,8 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.splits, a.H / HPC, a.B * a.T);
-  kern<<<grid, kThreads, smem, stream>>>(a);
-  if ((e = counted(cudaGetLastError())) != cudaSuccess) return e;
-  attn_combine_kernel<DV><<<dim3(a.B * a.T, a.H), DV / 4, 0, stream>>>(a);
-  return counted(cudaGetLastError());
+  if ((e = launch_pdl(kern, grid, dim3(kThreads), smem, stream, a)) != cudaSuccess) return e;
+  return launch_pdl(attn_combine_kernel<DV>, dim3(a.B * a.T, a.H), dim3(DV / 4), 0, stream, a);
 }
 
 }  // namespace
@@ -362,8 +362,7 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
     cudaError_t e = launch_attn_mma(a, stream);
     if (e != cudaSuccess) return e;
     if (a.splits == 1) return cudaSuccess;  // one split per query: the kernel wrote the output
-    attn_combine_kernel<512><<<dim3(a.B * a.T, a.H), 128, 0, stream>>>(a);
-    return counted(cudaGetLastError());
+    return launch_pdl(attn_combine_kernel<512>, dim3(a.B * a.T, a.H), dim3(128), 0, stream, a);
   }
   if (a.kv.f.fmt == LCSC_FMT_F32 && a.D == 128 && a.Dv == 128 && a.H % 8 == 0) {
     if (sep) return launch_attn<LCSC_FMT_F32, 128, 128, 8, true>(a, stream);

@@ -198,6 +198,7 @@ __device__ __forceinline__ float pow2(int e) {
 // swizzle); the image ends with 2^e per head, which the softmax multiplies
 // back into the logits.
 __global__ void __launch_bounds__(kThr) attn_qimage_kernel(const AttnLaunch a) {
+  grid_dep_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* qsc_s = reinterpret_cast<float*>(sm + kQImg);  // per-head amax of q, then 2^e
@@ -285,6 +286,7 @@ __global__ void __launch_bounds__(kThr) attn_qimage_kernel(const AttnLaunch a) {
 }
 
 __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
+  grid_dep_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* k_full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);  // [3] a tile's rows have landed
@@ -839,15 +841,13 @@ cudaError_t launch_attn_qimage(const AttnLaunch& a, cudaStream_t stream) {
   constexpr int kImgSmem = (int)kAttnQImageBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_qimage_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kImgSmem);
   if (e != cudaSuccess) return e;
-  attn_qimage_kernel<<<a.B * a.T, kThr, kImgSmem, stream>>>(a);
-  return counted(cudaGetLastError());
+  return launch_pdl(attn_qimage_kernel, dim3(a.B * a.T), dim3(kThr), kImgSmem, stream, a);
 }
 
 cudaError_t launch_attn_mma(const AttnLaunch& a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(attn_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
-  attn_mma_kernel<<<dim3(a.splits, a.B * a.T), kThr, SMEM, stream>>>(a);
-  return counted(cudaGetLastError());
+  return launch_pdl(attn_mma_kernel, dim3(a.splits, a.B * a.T), dim3(kThr), SMEM, stream, a);
 }
 
 }  // namespace lcsc

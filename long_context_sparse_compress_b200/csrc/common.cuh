@@ -14,6 +14,17 @@ namespace lcsc {
 
 constexpr int kWarp = 32;
 
+// Programmatic dependent launch: the first statement of every kernel of this
+// library.  Returns once the stream's previous grid has completed and its
+// memory operations are visible (at once when the launch had no programmatic
+// dependency), so each grid still completes after all earlier work of its
+// stream and touches no global memory or TMEM before that.  No kernel
+// signals its dependents early (griddepcontrol.launch_dependents): the next
+// grid's launch then starts as this one's last CTA exits, which removes the
+// launch gap without CTAs that wait on an SM for a whole kernel while the
+// other layer's stream could use it (measured slower with two streams).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ----------------------------------------------------------------- row layout
 
 struct RowFmt {

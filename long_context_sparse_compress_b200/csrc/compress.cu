@@ -191,6 +191,7 @@ __device__ __forceinline__ void store_entries(const CompressLaunch& a, const flo
 // masked out of the softmax.
 template <bool kBf16, int DIM, int NC, bool kFused>
 __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E, bool packed) {
+  grid_dep_wait();
   using Elem = typename std::conditional<kBf16, uint16_t, float>::type;
   constexpr int XS = kBf16 ? DIM : DIM + 1;       // x tile row stride (elements; fp32 path)
   constexpr int WS = kBf16 ? NC : NC + 1;         // W chunk row stride (fp32 path)
@@ -514,6 +515,7 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(CompressLaunch a, int E,
 // grid: (ceil((n_new_max + n_win_max) / 8), B); one warp per row.
 template <int VPL>
 __global__ void __launch_bounds__(256) store_kernel(CompressLaunch a) {
+  grid_dep_wait();
   const int b = blockIdx.y;
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
   const int64_t i = (int64_t)blockIdx.x * 8 + warp;
@@ -547,6 +549,7 @@ __global__ void __launch_bounds__(256) store_kernel(CompressLaunch a) {
 template <int VPL>
 __global__ void __launch_bounds__(256) encode_rows_kernel(const float* rows, int64_t n, int64_t row0,
                                                           CacheView out) {
+  grid_dep_wait();
   const int b = blockIdx.y;
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
   const int64_t i = (int64_t)blockIdx.x * 8 + warp;
@@ -577,7 +580,7 @@ cudaError_t launch_pool(const CompressLaunch& a, int E, cudaStream_t stream, boo
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = DIM / NC;
@@ -590,12 +593,15 @@ cudaError_t launch_pool(const CompressLaunch& a, int E, cudaStream_t stream, boo
     max_clusters = 0;
   }
   *fused = (int64_t)grid.x * grid.z <= max_clusters;
-  if (*fused) return counted(cudaLaunchKernelEx(&cfg, kf, a, E, packed));
+  if (*fused) {
+    set_pdl(attr[1]);
+    cfg.numAttrs = 2;
+    return counted(cudaLaunchKernelEx(&cfg, kf, a, E, packed));
+  }
   auto ku = pool_kernel<kBf16, DIM, NC, false>;
   e = cudaFuncSetAttribute(ku, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  ku<<<grid, kThreads, smem, stream>>>(a, E, packed);
-  return counted(cudaGetLastError());
+  return launch_pdl(ku, grid, dim3(kThreads), smem, stream, a, E, packed);
 }
 
 }  // namespace
@@ -620,12 +626,11 @@ cudaError_t launch_compress(const CompressLaunch& a, cudaStream_t stream) {
   if (rows == 0) return cudaSuccess;
   dim3 grid((unsigned)((rows + 7) / 8), a.B);
   switch (a.dim) {
-    case 512: store_kernel<16><<<grid, 256, 0, stream>>>(a); break;
-    case 128: store_kernel<4><<<grid, 256, 0, stream>>>(a); break;
-    case 32: store_kernel<1><<<grid, 256, 0, stream>>>(a); break;
+    case 512: return launch_pdl(store_kernel<16>, grid, dim3(256), 0, stream, a);
+    case 128: return launch_pdl(store_kernel<4>, grid, dim3(256), 0, stream, a);
+    case 32: return launch_pdl(store_kernel<1>, grid, dim3(256), 0, stream, a);
     default: return cudaErrorInvalidValue;
   }
-  return counted(cudaGetLastError());
 }
 
 cudaError_t launch_encode_rows(const float* rows, int B, int64_t n, int64_t row0,
@@ -633,12 +638,11 @@ cudaError_t launch_encode_rows(const float* rows, int B, int64_t n, int64_t row0
   if (n == 0) return cudaSuccess;
   dim3 grid((unsigned)((n + 7) / 8), B);
   switch (out.f.dim) {
-    case 512: encode_rows_kernel<16><<<grid, 256, 0, stream>>>(rows, n, row0, out); break;
-    case 128: encode_rows_kernel<4><<<grid, 256, 0, stream>>>(rows, n, row0, out); break;
-    case 32: encode_rows_kernel<1><<<grid, 256, 0, stream>>>(rows, n, row0, out); break;
+    case 512: return launch_pdl(encode_rows_kernel<16>, grid, dim3(256), 0, stream, rows, n, row0, out);
+    case 128: return launch_pdl(encode_rows_kernel<4>, grid, dim3(256), 0, stream, rows, n, row0, out);
+    case 32: return launch_pdl(encode_rows_kernel<1>, grid, dim3(256), 0, stream, rows, n, row0, out);
     default: return cudaErrorInvalidValue;
   }
-  return counted(cudaGetLastError());
 }
 
 }  // namespace lcsc

@@ -54,6 +54,7 @@ __device__ __forceinline__ int64_t visible(const IndexLaunch& a, int b, int t, b
 // One warp per (b, t, h) row: the query row is stored in the key format.
 template <int VPL>
 __global__ void __launch_bounds__(256) quantize_queries_kernel(IndexLaunch a, bool zero_hist) {
+  grid_dep_wait();
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
   {  // the top-k's counters, and the digit-1 histograms when they are summed in memory, start at zero
     const int64_t lists = (int64_t)a.B * a.T;
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(256) quantize_queries_kernel(IndexLaunch a, bo
 // cores).  grid (ceil(n_max / 64), B*T); block 256 = 64 keys x 4 head groups.
 template <int DI, int HI>
 __global__ void __launch_bounds__(256) score_kernel(IndexLaunch a) {
+  grid_dep_wait();
   constexpr int KEYS = 64;
   constexpr int HG = HI < 4 ? HI : 4;
   constexpr int HPT = HI / HG;
@@ -185,6 +187,7 @@ __device__ __forceinline__ void scan_scores(const float* s, int64_t lo, int64_t 
 // Digit-1 histogram of one slice of a list (scores written by a kernel that
 // did not histogram them); the list's last CTA finds the threshold bin.
 __global__ void __launch_bounds__(512) topk_hist_kernel(IndexLaunch a, int slices) {
+  grid_dep_wait();
   __shared__ uint32_t h[kBins];
   const int list = blockIdx.y;
   const ListInfo li = list_info(a, list, slices);
@@ -199,6 +202,7 @@ __global__ void __launch_bounds__(512) topk_hist_kernel(IndexLaunch a, int slice
 // All slices of a list: scores above the digit-1 threshold bin go to the
 // output, those in it to the candidate list.
 __global__ void __launch_bounds__(512) topk_collect_kernel(IndexLaunch a, int slices, bool set_bins) {
+  grid_dep_wait();
   extern __shared__ float4 slice_s[];  // the slice's scores, one bulk copy
   __shared__ uint64_t bar;
   constexpr int kLocal = 2048;          // candidates gathered in shared memory first
@@ -327,6 +331,7 @@ constexpr size_t kFinalSmem = (size_t)kCandCap * 8;
 // join the collect pass's marks in the bitmap, which is then compacted into
 // the output (index order).
 __global__ void __launch_bounds__(512) topk_final_kernel(IndexLaunch a) {
+  grid_dep_wait();
   __shared__ uint32_t h[kBins];
   __shared__ Thresh th;
   __shared__ uint32_t warp_tot[32];
@@ -487,11 +492,10 @@ cudaError_t launch_index_quantize(const IndexLaunch& a, cudaStream_t stream) {
   // shared memory: the global ones are then never read
   const bool zero_hist = !index_mma_supported(a) || index_bins_in_collect(a) || !index_whole_lists(a);
   switch (a.d_I) {
-    case 128: quantize_queries_kernel<4><<<qgrid, 256, 0, stream>>>(a, zero_hist); break;
-    case 32: quantize_queries_kernel<1><<<qgrid, 256, 0, stream>>>(a, zero_hist); break;
+    case 128: return launch_pdl(quantize_queries_kernel<4>, dim3(qgrid), dim3(256), 0, stream, a, zero_hist);
+    case 32: return launch_pdl(quantize_queries_kernel<1>, dim3(qgrid), dim3(256), 0, stream, a, zero_hist);
     default: return cudaErrorInvalidValue;
   }
-  return counted(cudaGetLastError());
 }
 
 cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream) {
@@ -502,13 +506,11 @@ cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream) {
 
 cudaError_t launch_index_score_only(const IndexLaunch& a, cudaStream_t stream) {
   const int lists = a.B * a.T;
-  if (index_mma_supported(a)) return counted(launch_index_mma(a, stream));
+  if (index_mma_supported(a)) return launch_index_mma(a, stream);
   dim3 sgrid((unsigned)((a.n_max + 63) / 64), lists);
   if (a.keys.f.fmt == LCSC_FMT_F32 && a.d_I == 32 && a.H_I == 4)
-    score_kernel<32, 4><<<sgrid, 256, 0, stream>>>(a);
-  else
-    return cudaErrorInvalidValue;
-  return counted(cudaGetLastError());
+    return launch_pdl(score_kernel<32, 4>, sgrid, dim3(256), 0, stream, a);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_topk(const IndexLaunch& a, cudaStream_t stream) {
@@ -520,20 +522,18 @@ cudaError_t launch_topk(const IndexLaunch& a, cudaStream_t stream) {
   if (slices < 1) slices = 1;
   dim3 tgrid(slices, lists);
   if (!index_mma_supported(a)) {
-    topk_hist_kernel<<<tgrid, 512, 0, stream>>>(a, slices);
-    if ((e = counted(cudaGetLastError())) != cudaSuccess) return e;
+    if ((e = launch_pdl(topk_hist_kernel, tgrid, dim3(512), 0, stream, a, slices)) != cudaSuccess) return e;
   }
   // the collect pass copies each slice into shared memory in one bulk copy
   const int64_t per_max = ((a.n_max + slices - 1) / slices + 31) / 32 * 32;
   const size_t slice_bytes = (size_t)per_max * 4;
   e = cudaFuncSetAttribute(topk_collect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)slice_bytes);
   if (e != cudaSuccess) return e;
-  topk_collect_kernel<<<tgrid, 512, slice_bytes, stream>>>(a, slices, index_bins_in_collect(a));
-  if ((e = counted(cudaGetLastError())) != cudaSuccess) return e;
+  e = launch_pdl(topk_collect_kernel, tgrid, dim3(512), slice_bytes, stream, a, slices, index_bins_in_collect(a));
+  if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(topk_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFinalSmem);
   if (e != cudaSuccess) return e;
-  topk_final_kernel<<<lists, 512, kFinalSmem, stream>>>(a);
-  return counted(cudaGetLastError());
+  return launch_pdl(topk_final_kernel, dim3(lists), dim3(512), kFinalSmem, stream, a);
 }
 
 cudaError_t launch_index_topk(const IndexLaunch& a, cudaStream_t stream) {

@@ -34,6 +34,7 @@
 #include <cudaTypedefs.h>
 
 #include "kernels.cuh"
+#include "launches.h"
 #include "sm100.cuh"
 #include "topk.cuh"
 
@@ -170,6 +171,7 @@ template <int FMT, int NQ>
 __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
     index_mma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                      const MmaArgs a) {
+  grid_dep_wait();
   using C = Cfg<FMT, NQ>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
@@ -640,8 +642,7 @@ cudaError_t launch_mma(const IndexLaunch& a, cudaStream_t stream) {
   auto kern = index_mma_kernel<FMT, NQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(m.chunks, (unsigned)ctas), C::THREADS, C::SMEM, stream>>>(tk, tq, m);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(m.chunks, (unsigned)ctas), dim3(C::THREADS), C::SMEM, stream, tk, tq, m);
 }
 
 }  // namespace

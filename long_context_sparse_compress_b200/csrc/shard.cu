@@ -26,6 +26,7 @@ constexpr int kMergeThreads = 512;
 // the parts' order (index order when the parts are shards in range order and
 // each part's list is index-ordered).
 __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(TopkMergeLaunch a) {
+  grid_dep_wait();
   extern __shared__ uint64_t ck[];  // [n_parts * k] candidate keys (0: none)
   __shared__ uint32_t h[256];
   __shared__ uint32_t warp_tot[32];
@@ -106,6 +107,7 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(TopkMergeLaun
 // row is sum_r e^{lse_r - M} o_r / (e^{sigma - M} + sum_r e^{lse_r - M}).
 template <int DV>
 __global__ void __launch_bounds__(DV) attn_merge_kernel(AttnMergeLaunch a) {
+  grid_dep_wait();
   constexpr int TPH = DV / 4;
   const int list = blockIdx.x;
   const int h = blockIdx.y * 4 + threadIdx.x / TPH;
@@ -164,18 +166,16 @@ cudaError_t launch_topk_merge(const TopkMergeLaunch& a, cudaStream_t stream) {
   const size_t smem = sizeof(uint64_t) * (size_t)a.n_parts * (size_t)a.k;
   cudaError_t e = cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  topk_merge_kernel<<<(unsigned)a.lists, kMergeThreads, smem, stream>>>(a);
-  return counted(cudaGetLastError());
+  return launch_pdl(topk_merge_kernel, dim3((unsigned)a.lists), dim3(kMergeThreads), smem, stream, a);
 }
 
 cudaError_t launch_attn_merge(const AttnMergeLaunch& a, cudaStream_t stream) {
   const dim3 grid((unsigned)a.lists, (unsigned)(a.H / 4));
   switch (a.Dv) {
-    case 512: attn_merge_kernel<512><<<grid, 512, 0, stream>>>(a); break;
-    case 128: attn_merge_kernel<128><<<grid, 128, 0, stream>>>(a); break;
+    case 512: return launch_pdl(attn_merge_kernel<512>, grid, dim3(512), 0, stream, a);
+    case 128: return launch_pdl(attn_merge_kernel<128>, grid, dim3(128), 0, stream, a);
     default: return cudaErrorInvalidValue;
   }
-  return counted(cudaGetLastError());
 }
 
 }  // namespace lcsc
