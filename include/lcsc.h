@@ -30,7 +30,11 @@
  *    call on a device before any stream capture.  The no-allocation call
  *    below also keeps a fixed array per device.
  *  - Every call enqueues its kernels on `stream` (a cudaStream_t) and
- *    returns without synchronising.
+ *    returns without synchronising.  Kernels are launched with programmatic
+ *    stream serialisation and each waits (griddepcontrol.wait) for the
+ *    stream's previous grid before touching memory, so results follow
+ *    stream order as with plain launches; the environment variable
+ *    LCSC_PDL=0, read once per process, launches without the attribute.
  *  - On a non-zero return nothing has been enqueued.
  *  - Data-dependent anomalies found on the device (an index in `idx` that
  *    is out of range, a window ring too small for the query positions) never
