@@ -72,7 +72,7 @@ extern "C" {
 /* Bits OR-ed into *status on the device. */
 #define LCSC_DEV_BAD_INDEX 1       /* an index outside [0, N(p)) was skipped */
 #define LCSC_DEV_BAD_LENGTH 2      /* a ctx_len smaller than T, or past the sizes of the call */
-#define LCSC_DEV_TIMEOUT 4         /* a kernel gave up a bounded wait (no result was written) */
+#define LCSC_DEV_TIMEOUT 4         /* a kernel gave up a bounded wait (the call's results are not valid) */
 #define LCSC_DEV_RANGE 8           /* reserved: no call of this version raises it */
 
 /* What the sink of a layer is (lcsc_params.sink_mode); "DeepSeek V4
@@ -197,6 +197,18 @@ const char* lcsc_status_string(int32_t status);
  * it runs; read the count before and after a region to learn how many
  * launches that region issued. */
 uint64_t lcsc_kernel_launches(void);
+/* For tests of the failure path of the bounded waits (process-wide; affects
+ * calls enqueued after it returns).  limit_ns > 0: the waits of the
+ * tensor-core attention and scoring kernels give up after limit_ns instead
+ * of 2 s.  stall != 0: in each CTA of those kernels one thread first waits on
+ * a barrier that cannot complete at that point (the attention's Q K^T issuer
+ * on the barrier it commits to at its end; the scoring's first lane on the
+ * drain of its first accumulator, which it has not filled), so the wait runs
+ * out, LCSC_DEV_TIMEOUT is set, and every role of the CTA stops, waits for
+ * its copies and MMAs in flight and frees its tensor memory.  (0, 0)
+ * restores the normal behaviour.  Returns LCSC_OK, or LCSC_ERR_INVALID_ARG for a
+ * negative limit. */
+int32_t lcsc_set_wait_test(int64_t limit_ns, int32_t stall);
 /* Bytes of one stored row for a format and dimension (0 if invalid). */
 int64_t lcsc_row_bytes(int32_t format, int32_t dim, int32_t rope_dim);
 

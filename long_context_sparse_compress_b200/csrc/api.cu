@@ -15,6 +15,21 @@ std::atomic<uint64_t> g_kernel_launches{0};
 
 void note_launch() { g_kernel_launches.fetch_add(1, std::memory_order_relaxed); }
 
+namespace {
+std::atomic<int64_t> g_wait_limit_ns{0};
+std::atomic<int32_t> g_wait_stall{0};
+}  // namespace
+
+void set_wait_test(int64_t limit_ns, int32_t stall) {
+  g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+  g_wait_stall.store(stall, std::memory_order_relaxed);
+}
+
+WaitTest wait_test() {
+  const int64_t l = g_wait_limit_ns.load(std::memory_order_relaxed);
+  return WaitTest{l > 0 ? (uint64_t)l : kDefaultWaitNs, g_wait_stall.load(std::memory_order_relaxed) != 0};
+}
+
 bool pdl_enabled() {
   static const bool on = [] {
     const char* v = std::getenv("LCSC_PDL");
@@ -203,6 +218,12 @@ int32_t lcsc_abi_version(void) { return LCSC_ABI_VERSION; }
 int32_t lcsc_last_cuda_error(void) { return g_last_cuda_error; }
 
 uint64_t lcsc_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }
+
+int32_t lcsc_set_wait_test(int64_t limit_ns, int32_t stall) {
+  if (limit_ns < 0) return LCSC_ERR_INVALID_ARG;
+  lcsc::set_wait_test(limit_ns, stall);
+  return LCSC_OK;
+}
 
 const char* lcsc_status_string(int32_t s) {
   switch (s) {

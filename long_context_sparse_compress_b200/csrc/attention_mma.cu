@@ -51,6 +51,8 @@
 namespace lcsc {
 namespace {
 
+static_assert(kDefaultWaitNs == sm100::kWaitLimitNs, "one default limit for the bounded waits");
+
 using namespace sm100;
 
 constexpr int kH = 64;       // heads (MMA M)
@@ -179,7 +181,7 @@ __device__ __forceinline__ Rows rows_of(const AttnLaunch& a, int b, int t) {
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const AttnLaunch& a,
                                           volatile int* abort) {
   if (*abort) return false;
-  bool ok = mbar_wait(bar, parity, a.status);
+  bool ok = mbar_wait(bar, parity, a.status, a.waits.limit_ns);
   ok = __all_sync(0xffffffffu, ok);
   if (!ok && (threadIdx.x & 31) == 0) *abort = 1;
   return ok;
@@ -477,7 +479,8 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
         // between group barriers)
         if (lt == 0) {
           bool ok = !*abort;
-          if (ok && j >= 1) ok = mbar_wait(&k_free[(j + 2) % kNB], (uint32_t)((j - 1) / kNB) & 1u, a.status);
+          if (ok && j >= 1)
+            ok = mbar_wait(&k_free[(j + 2) % kNB], (uint32_t)((j - 1) / kNB) & 1u, a.status, a.waits.limit_ns);
           if (!ok) *abort = 1;
           *lstop = ok ? 0 : 1;
         }
@@ -547,7 +550,11 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
       tc_commit(&k_free[j % kNB]);
     };
     if (warp == kMmaWarp) {
-      for (int j = 0; j < ntiles; ++j) {
+      // A test of the failure path (lcsc_set_wait_test): first wait on the
+      // drain barrier, which cannot complete before this warp's own commit
+      // below, so the wait runs out and the CTA aborts.
+      const bool go = !a.waits.stall || warp_wait(drain, 0u, a, abort);
+      for (int j = 0; go && j < ntiles; ++j) {
         if (j == 0 && !warp_wait(q_full, 0, a, abort)) break;
         if (!warp_wait(&k_full[j % kNB], (uint32_t)(j / kNB) & 1u, a, abort)) break;
         if (j >= 2 && !warp_wait(&p_full[j & 1], (uint32_t)((j - 2) >> 1) & 1u, a, abort)) break;
@@ -795,6 +802,9 @@ __global__ void __maxnreg__(128) attn_mma_kernel(const AttnLaunch a) {
       a.part_ml[pidx * 2 + 1] = l_h;
     }
   }
+  // the query image's copies have landed before the CTA can end (they have on
+  // every path but an abort that came before them; bounded)
+  if (tid == 0) mbar_wait(q_full, 0, nullptr, kDrainLimitNs);
   tc_fence_before();
   __syncthreads();
   {  // O of this split, [64 heads][512] contiguous: coalesced stores by every thread, of the
@@ -847,7 +857,9 @@ cudaError_t launch_attn_qimage(const AttnLaunch& a, cudaStream_t stream) {
 cudaError_t launch_attn_mma(const AttnLaunch& a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(attn_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
-  return launch_pdl(attn_mma_kernel, dim3(a.splits, a.B * a.T), dim3(kThr), SMEM, stream, a);
+  AttnLaunch la = a;
+  la.waits = wait_test();
+  return launch_pdl(attn_mma_kernel, dim3(a.splits, a.B * a.T), dim3(kThr), SMEM, stream, la);
 }
 
 }  // namespace lcsc

@@ -60,6 +60,8 @@ struct MmaArgs {
   bool bins_in_collect;    // several CTAs per list: the collect pass sets the threshold bins
   int64_t shard_row0, shard_rows;  // keys of an entry shard: entries [row0, row0 + rows) in rows 0 ..
   int32_t* status;
+  uint64_t wait_ns;        // limit of the bounded waits
+  bool stall;              // a test of the failure path (lcsc_set_wait_test)
 };
 
 // A context length the call can serve (an unsharded call must have been sized
@@ -285,7 +287,7 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
       auto load = [&](int i, int64_t tile) {  // TMA of (local) tile i, global tile `tile`, into stage i % STAGES
         const int s = i % C::STAGES;
         const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u, a.status)) {
+        if (!mbar_wait(&empty[s], ph ^ 1u, a.status, a.wait_ns)) {
           live = false;
           return;
         }
@@ -308,7 +310,7 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
         load(r + C::LANES * my_n, tile);
       };
       for (int t = 0; t < C::DIST && more && live; ++t) load_next();
-      live = live && mbar_wait(qbar, 0, a.status);
+      live = live && mbar_wait(qbar, 0, a.status, a.wait_ns);
       tc_fence_after();
       const uint32_t q_addr = smem_u32(sm + C::OFF_Q);
       if (live && r == 0 && FMT == LCSC_FMT_FP4) {
@@ -328,8 +330,12 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
       }
       // the other lanes start once the query scales are in TMEM
       if (r == 0) tc_commit(sfb_bar);
-      else live = live && mbar_wait(sfb_bar, 0, a.status);
+      else live = live && mbar_wait(sfb_bar, 0, a.status, a.wait_ns);
       tc_fence_after();
+      // A test of the failure path (lcsc_set_wait_test): the first lane
+      // waits for the drain of its first accumulator, which it has not
+      // filled, so the wait runs out and the lane stops.
+      if (a.stall && r == 0) live = live && mbar_wait(&acce[0], 0u, a.status, a.wait_ns);
       const uint32_t idesc = FMT == LCSC_FMT_FP4 ? idesc_mxf4nvf4(128, C::N) : idesc_dense(0, 0, 128, C::N);
       int last = -1;
       int t = 0;  // this lane's first tile whose copies were not yet consumed
@@ -343,8 +349,8 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
         const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
         const int ab = i % C::NACC;
         const uint32_t au = (uint32_t)(i / C::NACC) & 1u;
-        if (!mbar_wait(&full[s], ph, a.status)) break;
-        if (!mbar_wait(&acce[ab], au ^ 1u, a.status)) break;
+        if (!mbar_wait(&full[s], ph, a.status, a.wait_ns)) break;
+        if (!mbar_wait(&acce[ab], au ^ 1u, a.status, a.wait_ns)) break;
         tc_fence_after();
         const uint32_t a_addr = smem_u32(sm + C::OFF_A + s * C::A_BYTES);
         const uint32_t d = tmem + ab * C::N;
@@ -369,7 +375,7 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
         last = i;
       }
       if (last >= 0)  // the accumulator of the last tile is complete before TMEM is freed
-        mbar_wait(&accf[last % C::NACC], (uint32_t)(last / C::NACC) & 1u, a.status);
+        mbar_wait(&accf[last % C::NACC], (uint32_t)(last / C::NACC) & 1u, a.status, a.wait_ns);
       // After a wait gave up: the copies this lane issued and did not consume
       // (and the query's, on lane 0) land before the CTA's shared memory is
       // released; each wait is bounded again.  Nothing is left on the normal path.
@@ -423,7 +429,9 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
           if (d) continue;
           if (tl % C::BL == 0) {  // the lane's next claim
             const int cb = tl / C::BL;
-            if (!mbar_wait(&clm_bar[r * C::RING + cb % C::RING], (uint32_t)(cb / C::RING) & 1u, a.status)) break;
+            if (!mbar_wait(&clm_bar[r * C::RING + cb % C::RING], (uint32_t)(cb / C::RING) & 1u, a.status,
+                           a.wait_ns))
+              break;
             c = clm_s[r * C::RING + cb % C::RING];
           }
           gtile = (int64_t)c * C::BL + tl % C::BL;
@@ -445,7 +453,7 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
         const int ab = i % C::NACC;
         const int64_t g = gtile * 128 + row;
         const float sk = FMT == LCSC_FMT_FP8 ? kscale[g] : 1.f;
-        if (!mbar_wait(&accf[ab], (uint32_t)(i / C::NACC) & 1u, a.status)) break;
+        if (!mbar_wait(&accf[ab], (uint32_t)(i / C::NACC) & 1u, a.status, a.wait_ns)) break;
         tc_fence_after();
         uint32_t r0[32], r1[32];
         const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) + ab * C::N;
@@ -527,7 +535,7 @@ __global__ void __launch_bounds__(Cfg<FMT, NQ>::THREADS, 1)
         const int ab = i % C::NACC;
         const int64_t g = (tile_lo + i) * 128 + my_row;
         const float sk = FMT == LCSC_FMT_FP8 ? kscale[g] : 1.f;
-        if (!mbar_wait(&accf[ab], (uint32_t)(i / C::NACC) & 1u, a.status)) break;
+        if (!mbar_wait(&accf[ab], (uint32_t)(i / C::NACC) & 1u, a.status, a.wait_ns)) break;
         tc_fence_after();
         const uint32_t base = tmem + ((uint32_t)(q4 * 32) << 16) + ab * C::N + nq * 64;
         // the query's 64 columns of this sub-partition's rows go to
@@ -635,6 +643,9 @@ cudaError_t launch_mma(const IndexLaunch& a, cudaStream_t stream) {
   m.shard_row0 = a.keys.row0;
   m.shard_rows = a.keys.rows;
   m.status = a.status;
+  const WaitTest wt = wait_test();
+  m.wait_ns = wt.limit_ns;
+  m.stall = wt.stall;
   const int groups = (a.T + NQ - 1) / NQ;
   const int64_t ctas = (int64_t)a.B * groups;
   m.chunks = chunks_per_group(a);

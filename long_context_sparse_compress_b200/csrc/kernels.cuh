@@ -57,6 +57,17 @@ inline int sm_count() {
   return n;
 }
 
+// The bounded waits of the tensor-core kernels: their limit (2 s unless a
+// test of the failure path shortened it) and whether one thread of each CTA
+// first waits on a barrier that cannot complete (lcsc_set_wait_test).
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+struct WaitTest {
+  uint64_t limit_ns;
+  bool stall;
+};
+void set_wait_test(int64_t limit_ns, int32_t stall);
+WaitTest wait_test();
+
 struct IndexLaunch {
   const void* q_idx;    // [B][T][H_I][d_I] q_dtype
   int q_dtype;
@@ -118,6 +129,7 @@ struct AttnLaunch {
   float* part_o;        // [B*T][splits][H][Dv]
   float* part_ml;       // [B*T][splits][H][2]
   uint8_t* q_img;       // [B*T][kAttnQImageBytes]: the tensor-core path's query images
+  WaitTest waits;       // set by the tensor-core launcher
   void* out;            // [B][T][H][Dv] q_dtype
   float* lse;           // [B][T][H] or nullptr
   int32_t* status;

@@ -58,6 +58,7 @@ _SIGS = {
     "lcsc_last_cuda_error": (c_i32, []),
     "lcsc_status_string": (ctypes.c_char_p, [c_i32]),
     "lcsc_kernel_launches": (ctypes.c_uint64, []),
+    "lcsc_set_wait_test": (c_i32, [c_i64, c_i32]),
     "lcsc_row_bytes": (c_i64, [c_i32, c_i32, c_i32]),
     "lcsc_compress_workspace_size": (c_i32, [c_vp, c_i64, c_i64, c_vp]),
     "lcsc_csa_compress": (c_i32, [c_vp, c_i32, c_vp, c_i64, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp,
@@ -111,6 +112,13 @@ def load(path=LIB_PATH):
 def kernel_launches():
     """Kernels the library has enqueued since it was loaded (host-side count)."""
     return int(load().lcsc_kernel_launches())
+
+
+def set_wait_test(limit_ns=0, stall=False):
+    """Bounded-wait limit of the tensor-core kernels and the stall of one
+    thread per CTA, for tests of the failure path; (0, False) restores the
+    normal behaviour."""
+    check(load().lcsc_set_wait_test(int(limit_ns), 1 if stall else 0))
 
 
 def check(status):

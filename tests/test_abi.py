@@ -46,6 +46,12 @@ def test_abi_version_and_strings(lib):
     assert lib.lcsc_row_bytes(L.FMT["f32"], 128, 0) == 512
 
 
+def test_wait_test_switch_is_host_only(lib):
+    assert lib.lcsc_set_wait_test(-1, 0) == 1  # LCSC_ERR_INVALID_ARG
+    assert lib.lcsc_set_wait_test(5_000_000, 1) == 0
+    assert lib.lcsc_set_wait_test(0, 0) == 0
+
+
 def test_workspace_sizes_are_host_only(lib):
     p = L.params(W.PAIR_DECODE_1M_B16.layer("csa"))
     out = ctypes.c_size_t(0)

@@ -201,7 +201,10 @@ def test_topk_resolves_the_last_digit(cuda_lib):
     assert set(out_idx.cpu().numpy()[0, 0].tolist()) == set(pos[23:].tolist())
 
 
-def check_index_topk(fmt, lengths, T, seed):
+def check_index_topk(fmt, lengths, T, seed, stalled=False):
+    """Scores and top-k of a seeded case against the oracle.  ``stalled``:
+    the bounded waits were set to run out (lcsc_set_wait_test); the call must
+    then report LCSC_DEV_TIMEOUT and end without a CUDA error."""
     rng = np.random.default_rng(seed)
     if fmt == "f32":
         wl = W.CSA_DECODE_4K_F32.with_(k=64)
@@ -230,6 +233,9 @@ def check_index_topk(fmt, lengths, T, seed):
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     L.index_topk(p, dev(qi, TORCH_DT[wl.q_dtype]), dev(wi), keys, ctx, n_cap, out_idx, out_sc, status=status)
     torch.cuda.synchronize()
+    if stalled:
+        assert status.item() & L.DEV_TIMEOUT
+        return
     assert status.item() == 0
     oi, osc = out_idx.cpu().numpy(), out_sc.cpu().numpy()
     for b in range(B):
@@ -263,6 +269,12 @@ def _attn_case(kind, fmt_kv, rng):
 def test_attention_matches_oracle(cuda_lib, kind, fmt_kv, q_dtype):
     """fp32 rows (CUDA-core path) and FP8 + BF16 rows (tensor-core path),
     the latter with bf16 queries and outputs and with fp32 ones."""
+    check_attention(kind, fmt_kv, q_dtype)
+
+
+def check_attention(kind, fmt_kv, q_dtype, stalled=False):
+    """One seeded sparse (CSA) or dense (HCA) attention call against the
+    oracle.  ``stalled``: as in check_index_topk."""
     rng = np.random.default_rng(31)
     wl = _attn_case(kind, fmt_kv, rng)
     if q_dtype:
@@ -314,6 +326,9 @@ def test_attention_matches_oracle(cuda_lib, kind, fmt_kv, q_dtype):
         L.dense_attn(p, dev(q, TORCH_DT[wl.q_dtype]), kv, v, wk, wv, dev(sink), ctx, n_cap, out, lse,
                      status=status)
     torch.cuda.synchronize()
+    if stalled:
+        assert status.item() & L.DEV_TIMEOUT
+        return
     assert status.item() == 0
     o_gpu, lse_gpu = out.float().cpu().numpy(), lse.cpu().numpy()
     for b in range(B):
