@@ -139,37 +139,46 @@ class Layer:
         L.decode_step(self.p, self.step, self.wl.kind == "csa", self.ws, self.status, stream)
 
     # host-side copies for the end-to-end measurement
-    def host_inputs(self):
-        """(device tensor, pinned host copy) of every input a decode step
-        receives: the T new tokens' raw rows (the G - 1 older rows of the
-        closing group arrived with earlier steps and stay on the device, the
-        way a caller keeps a group's rows in a ring written twice so that
-        they are always contiguous), the queries, the indexer queries and
-        weights, and the context lengths."""
-        T = self.wl.T
-        ts = [self.x_kv[:, -T:], self.q, self.ctx_len] + ([self.x_ik[:, -T:], self.q_idx, self.w_idx]
-                                                          if self.wl.kind == "csa" else [])
-        return [(t, t.contiguous().cpu().pin_memory()) for t in ts]
-
-    def host_output(self):
-        return self.out, torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
-
     def io_slot(self):
         """A second set of the step's per-step device inputs and outputs (the
         caches, weights and workspace are shared) with a step struct over
         them, for the double-buffered end-to-end loop: (step, [(device input,
-        pinned host input)], (device output, pinned host output))."""
+        pinned host input)], (device output, pinned host output)).  The inputs
+        a decode step receives: the T new tokens' raw rows (the G - 1 older
+        rows of the closing group arrived with earlier steps and stay on the
+        device, the way a caller keeps a group's rows in a ring written twice
+        so that they are always contiguous), the queries, the indexer queries
+        and weights, and the context lengths.  The dense ones (queries, their
+        indexer queries and weights, lengths) share one device buffer and one
+        pinned host buffer at 16-byte aligned offsets, so that they travel in
+        one copy; the raw rows are a strided slice of each sequence's rows
+        and travel in a copy of their own."""
         clone = lambda t: None if t is None else t.clone()
+        csa = self.wl.kind == "csa"
+        dense = [self.q, self.ctx_len] + ([self.q_idx, self.w_idx] if csa else [])
+        sizes = [t.numel() * t.element_size() for t in dense]
+        offs = [sum((n + 15) // 16 * 16 for n in sizes[:i]) for i in range(len(sizes))]
+        total = offs[-1] + (sizes[-1] + 15) // 16 * 16
+        dbuf = torch.empty(total, dtype=torch.uint8, device=self.dev)
+        hbuf = torch.zeros(total, dtype=torch.uint8).pin_memory()
+        views = []
+        for t, o, n in zip(dense, offs, sizes):
+            dv = dbuf[o:o + n].view(t.dtype).view(t.shape)
+            dv.copy_(t)
+            hbuf[o:o + n].view(t.dtype).view(t.shape).copy_(t.cpu())
+            views.append(dv)
+        q, ctx = views[0], views[1]
+        q_idx, w_idx = (views[2], views[3]) if csa else (None, None)
         x_kv, x_ik = clone(self.x_kv), clone(self.x_ik)
-        q, q_idx, w_idx, ctx = clone(self.q), clone(self.q_idx), clone(self.w_idx), clone(self.ctx_len)
         out, lse, sel = torch.empty_like(self.out), torch.empty_like(self.lse), clone(self.sel)
         step = L.make_step(self.wl.B, self.wl.T, self.n_max, ctx, x_kv, None, x_ik, self.w_kv, self.b_kv, None,
                            None, self.w_ik, self.b_ik, self.kv, None, self.idx, self.win, None, q, q_idx, w_idx,
                            self.sink, out, lse, sel, None)
         T = self.wl.T
-        dev = [x_kv[:, -T:], q, ctx] + ([x_ik[:, -T:], q_idx, w_idx] if self.wl.kind == "csa" else [])
-        host = [h for _, h in self.host_inputs()]
-        return step, list(zip(dev, host)), (out, torch.empty(out.shape, dtype=out.dtype).pin_memory())
+        rows = [(x_kv[:, -T:], self.x_kv[:, -T:].contiguous().cpu().pin_memory())]
+        if csa:
+            rows.append((x_ik[:, -T:], self.x_ik[:, -T:].contiguous().cpu().pin_memory()))
+        return step, [(dbuf, hbuf)] + rows, (out, torch.empty(out.shape, dtype=out.dtype).pin_memory())
 
 
 class StepRunner:
@@ -785,8 +794,10 @@ def run_lcsc(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "copies": "pinned host buffers, two sets of per-step device buffers used in turn: step s+1's "
                          "inputs upload on one copy stream while step s computes, step s's outputs download on a "
-                         "second while step s+1 computes; every step's uploads and downloads are inside the "
-                         "timed region, which ends when the last step's outputs are on the host",
+                         "second while step s+1 computes; per layer and step one copy of the dense inputs "
+                         "(queries, indexer queries and weights, lengths in one buffer), one of each layer's raw "
+                         "rows and one of the output; every step's uploads and downloads are inside the timed "
+                         "region, which ends when the last step's outputs are on the host",
                "inputs": "per sequence and layer: the new token's raw rows, the queries, the indexer queries "
                          "and weights (CSA), the context length; the closing group's G - 1 older raw rows "
                          "stay on the device from earlier steps"}
