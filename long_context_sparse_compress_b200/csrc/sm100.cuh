@@ -91,7 +91,7 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
-// 2D tile load, no multicast: box at (x, y) -> smem, completion on `bar`.
+// 2D tile load into this CTA's own shared memory: box at (x, y) -> smem, completion on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, int32_t x, int32_t y,
                                             uint64_t* bar) {
   asm volatile(
